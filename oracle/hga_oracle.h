@@ -1,0 +1,25 @@
+/* Plain fp64 CPU oracle for the HGA per-segment attention step.
+ * TEST INFRASTRUCTURE ONLY: used by the tests, the smoke check and the CPU
+ * baseline of the benchmark; never by the product library.  See hga_oracle.c
+ * for the definitions and layouts. */
+#ifndef OHGA_ORACLE_H
+#define OHGA_ORACLE_H
+#include <stdint.h>
+
+typedef struct {
+  int B, Hq, Hkv, d, blk, S, nblk, topk;
+} ohga_dims;
+
+void ohga_block_summaries(const ohga_dims* D, const double* k_hist, double* summ);
+void ohga_query_means(const ohga_dims* D, const double* q, double* qm);
+void ohga_block_scores(const ohga_dims* D, const double* qm, const double* summ, double* score);
+void ohga_select_topk(const ohga_dims* D, const double* score, int32_t* idx);
+void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
+                   const double* k_hist, const double* v_hist, const int32_t* idx, int h0, int h1, double* o,
+                   double* lse);
+void ohga_attn_bwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
+                   const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o, int h0, int h1,
+                   double* dq, double* dk, double* dv);
+void ohga_dense_causal_fwd(int B, int T, int Hq, int Hkv, int d, const double* q, const double* k, const double* v,
+                           double* o, double* lse);
+#endif
