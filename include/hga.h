@@ -1,0 +1,226 @@
+/*
+ * hga.h -- C ABI of libhga.so, the B200 (sm_100a) kernels of the HGA
+ * per-segment attention step.
+ *
+ * Source of the method: "Low-VRAM Long-Context Fine-Tuning: Hierarchical
+ * Global Attention and Segmented Backpropagation in Practice" (sns.style; the
+ * ja/de/ko editions share one text, the fr edition is a rewrite):
+ *   Background (背景と概要 / Hintergrund / 배경): a long sequence is cut into
+ *     segments; only the active segment is differentiable and kept on the GPU;
+ *     the history KV is offloaded to system RAM (or NVMe); each query block
+ *     attends to a bounded, exact set of history tokens rather than the dense
+ *     history, so per-token cost stays roughly constant.
+ *   Deep analysis (深掘り分析 / Tiefenanalyse / 심층 분석): per-block summaries
+ *     stay resident in VRAM and grow slowly with the context.
+ *   fr edition, Contexte: history tokens are loaded dynamically and precisely
+ *     per query block; Analyse approfondie: the KV of finished segments is
+ *     offloaded right away and decoupled from the active graph.
+ * The article leaves the summary, the score, K and the block size open.  This
+ * library fixes them as follows (the plainest reading the text supports):
+ *   summary[b,h,n]  = mean over the block's tokens of K_hist[b,t,h,:] (fp32)
+ *   score[b,h,i,n]  = max over the query heads hq of KV head h of
+ *                     mean_{t in query block i}(Q[b,t,hq,:]) . summary / sqrt(d)
+ *   selection       = the min(K, n_hist_blocks) highest scores, equal scores
+ *                     resolved to the lower block index, listed in ascending
+ *                     block order, unused slots = -1
+ *   attention       = softmax over [tokens of the selected history blocks] U
+ *                     [segment tokens at positions <= the query's], scale
+ *                     1/sqrt(d), fp32 statistics
+ *   backward        = dQ, dK_seg, dV_seg of <O, dO>; the history, the summaries
+ *                     and the selection get no gradient.
+ *
+ * Notation: B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0, query head hq
+ * uses KV head hq / (Hq/Hkv)), d head dim, `block` tokens per history block and
+ * per query block, S segment tokens (S % block == 0), Nqb = S / block.
+ *
+ * Layouts (row-major, token-major as QKV projections produce them):
+ *   q, o, d_o           [B, S, Hq, d]          dtype
+ *   k_seg, v_seg        [B, S, Hkv, d]         dtype
+ *   k_hist, v_hist      [B, n_kv_blocks*block, Hkv, d] dtype; block n = tokens
+ *                       [n*block, (n+1)*block)
+ *   summ                [B, Hkv, n_hist_blocks, d] fp32
+ *   idx                 [B, Hkv, Nqb, topk]    int32
+ *   lse                 [B, Hq, S]             fp32 (natural log)
+ *   dq                  [B, S, Hq, d]          fp32
+ *   dk_seg, dv_seg      [B, S, Hkv, d]         fp32
+ *
+ * Conventions:
+ *   - Ownership: the caller owns every buffer (device memory unless stated).
+ *     The library allocates no device or pinned memory; scratch space is
+ *     passed in by the caller (hga_attn_bwd_workspace_size).
+ *   - Asynchrony: every call enqueues work on `stream` and returns; errors in
+ *     arguments are reported before anything is enqueued.  hga_fetch_blocks is
+ *     the exception: it waits (bounded by timeout_ms) for a small index copy.
+ *   - Device-side faults that a kernel can detect (an out-of-range idx entry,
+ *     an expired pipeline wait) set a per-device flag instead of trapping;
+ *     hga_device_status() synchronizes the stream and reports and clears it.
+ *   - Paths: bf16 with d == 128 and block == 128 and an even group size runs
+ *     on the tcgen05 tensor-core kernels; every other supported shape (fp32,
+ *     d in {64,128}, block in {16,32,64,128}) runs on CUDA-core kernels.  Both
+ *     are GPU code; there is no CPU path.
+ *   - Thread safety: calls are independent; hga_last_error() is thread-local.
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HGA_API __attribute__((visibility("default")))
+#else
+#define HGA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HGA_OK = 0,
+  HGA_ERR_INVALID_ARG = 1, /* null pointer, bad enum, bad size */
+  HGA_ERR_SHAPE = 2,       /* dimensions outside the supported set */
+  HGA_ERR_UNSUPPORTED = 3, /* valid request this build does not implement */
+  HGA_ERR_INDEX = 4,       /* a kernel met an out-of-range block index */
+  HGA_ERR_TIMEOUT = 5,     /* a bounded wait expired (host or device) */
+  HGA_ERR_CUDA = 6         /* a CUDA runtime call failed; see hga_last_error */
+} hga_status;
+
+typedef enum { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype;
+
+/* Shape of one attention step.  n_hist_blocks: history blocks that exist
+ * (what selection ranks); topk: K. */
+typedef struct {
+  int B, Hq, Hkv, d, block, S, n_hist_blocks, topk;
+  hga_dtype dtype;
+} hga_dims;
+
+/* A CUDA stream (cudaStream_t); NULL = legacy default stream. */
+typedef struct CUstream_st* hga_stream_t;
+/* A CUDA event (cudaEvent_t). */
+typedef struct CUevent_st* hga_event_t;
+
+/* Human-readable name of a status code (static string). */
+HGA_API const char* hga_status_string(hga_status s);
+/* Details of the last failure in this thread (static per-thread buffer). */
+HGA_API const char* hga_last_error(void);
+
+/* Synchronizes `stream`, then reports (and clears) the device-side error flag
+ * of the current device: HGA_ERR_INDEX if a kernel saw an idx entry outside
+ * [-1, n_kv_blocks), HGA_ERR_TIMEOUT if a pipeline wait expired, else HGA_OK. */
+HGA_API hga_status hga_device_status(hga_stream_t stream);
+
+/*
+ * Block summaries (article, Deep analysis: resident per-block summaries).
+ *   summ[b,h,n,:] = (1/block) * sum_{t<block} k_hist[b, n*block+t, h, :]
+ * for blocks n in [blk_begin, blk_end) of a history of dims->n_hist_blocks
+ * blocks; other entries of summ are left untouched, so summaries can be added
+ * as blocks enter the history.  k_hist: dtype; summ: fp32 device buffer
+ * [B, Hkv, n_hist_blocks, d].  Accumulation in fp32.
+ * Errors: HGA_ERR_INVALID_ARG (null pointers, bad range), HGA_ERR_SHAPE.
+ */
+HGA_API hga_status hga_block_summaries(const hga_dims* dims, const void* k_hist, int blk_begin, int blk_end, float* summ,
+                               hga_stream_t stream);
+
+/*
+ * Per-query-block history selection (article, Background: bounded exact
+ * history set per query block; fr Contexte: precise historical tokens per
+ * query block).  For every (b, KV head h, query block i):
+ *   qm[g]     = mean over the block's `block` rows of q[b, row, h*G+g, :] (fp32)
+ *   score[n]  = max_g (qm[g] . summ[b,h,n,:]) / sqrt(d)                   (fp32)
+ *   idx[b,h,i,:] = the K_eff = min(topk, n_hist_blocks) best n (ties to the
+ *                  lower n), ascending, then -1 up to topk.
+ * scores_or_null (optional, fp32 [B,Hkv,Nqb,topk]) receives the selected
+ * blocks' scores in the same order (-inf for padding).
+ * Limits: n_hist_blocks <= 4096.
+ * Errors: HGA_ERR_INVALID_ARG, HGA_ERR_SHAPE.
+ */
+HGA_API hga_status hga_select_topk(const hga_dims* dims, const void* q_seg, const float* summ, int32_t* idx,
+                           float* scores_or_null, hga_stream_t stream);
+
+/*
+ * Attention forward over [selected history blocks] U [causal segment]
+ * (article, Background: exact attention over a bounded history set; only
+ * the active segment is computed on).  For query row p of head hq (KV head h,
+ * query block i = p / block), keys J = tokens of blocks idx[b,h,i,:] (entries
+ * >= 0) of k_hist/v_hist, plus segment tokens 0..p:
+ *   s_j = q.k_j / sqrt(d);  O = sum_j softmax(s)_j v_j;  lse = log sum_j exp(s_j)
+ * k_hist/v_hist hold n_kv_blocks blocks: the history itself (n_kv_blocks =
+ * n_hist_blocks) or a staging pool filled by hga_fetch_blocks (idx then holds
+ * pool slots).  o has the input dtype; lse fp32.
+ * Errors: HGA_ERR_INVALID_ARG, HGA_ERR_SHAPE (host checks); an idx entry
+ * outside [-1, n_kv_blocks) is skipped and flags HGA_ERR_INDEX on the device.
+ */
+HGA_API hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                        const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, void* o,
+                        float* lse, hga_stream_t stream);
+
+/* Bytes of device scratch hga_attn_bwd needs for these dims (256-byte
+ * aligned start required). */
+HGA_API size_t hga_attn_bwd_workspace_size(const hga_dims* dims);
+
+/*
+ * Attention backward for the active segment only (article, Background and
+ * fr Analyse approfondie: only the active segment is differentiable; history
+ * KV is detached).  With P the forward softmax (recomputed from lse),
+ * dP_j = dO.v_j, Dr = dO.O:
+ *   dS_j  = P_j (dP_j - Dr)
+ *   dq    = sum_{j in J} dS_j k_j / sqrt(d)                 (history + segment)
+ *   dk_seg[j] = sum over rows and the G heads of dS_j q / sqrt(d)  (segment j)
+ *   dv_seg[j] = sum over rows and the G heads of P_j dO            (segment j)
+ * No gradient is produced for k_hist, v_hist, summaries or idx.
+ * o and lse are the forward outputs; d_o has the input dtype; dq, dk_seg and
+ * dv_seg are fp32 and fully overwritten.  ws: device scratch of at least
+ * hga_attn_bwd_workspace_size(dims) bytes, owned by the caller; its contents
+ * need no initialisation and are undefined afterwards.
+ * Errors: as hga_attn_fwd, plus HGA_ERR_INVALID_ARG for a short workspace.
+ */
+HGA_API hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                        const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o,
+                        const float* lse, const void* d_o, float* dq, float* dk_seg, float* dv_seg, void* ws,
+                        size_t ws_bytes, hga_stream_t stream);
+
+/*
+ * Targeted loading of the selected history (fr edition, Contexte: dynamic
+ * loading of precise historical tokens per query block; Background: history
+ * KV lives in system RAM).  host_k/host_v: pinned host memory (cudaHostAlloc)
+ * of one layer's history tier [B, host_capacity_blocks*block, Hkv, d] in
+ * dtype, of which the first n_hist_blocks blocks are valid.  idx_dev:
+ * device idx from hga_select_topk.  The call
+ *   1. copies idx to the host on copy_stream (after the work already queued on
+ *      compute_stream) and waits for it, at most timeout_ms;
+ *   2. forms the sorted set of distinct selected blocks (at most pool_slots);
+ *   3. on copy_stream, copies each of those blocks' K and V (all B and Hkv)
+ *      from host to the device pool (pool_k/pool_v [B, pool_slots*block, Hkv,
+ *      d]), and writes idx_pool_dev = idx with each block number replaced by its
+ *      pool slot (-1 kept);
+ *   4. records `done` on copy_stream; compute work that reads the pool must
+ *      wait on it (cudaStreamWaitEvent).
+ * host_idx_scratch: pinned host buffer of B*Hkv*Nqb*topk int32 owned by the
+ * caller; it must stay untouched until `done` (the pool idx is uploaded from
+ * it).  *n_unique_out receives the number of distinct blocks fetched.
+ * Errors: HGA_ERR_TIMEOUT (idx copy did not finish in time), HGA_ERR_INDEX
+ * (an idx entry out of range), HGA_ERR_INVALID_ARG (more distinct blocks than
+ * pool_slots, null pointers), HGA_ERR_CUDA.
+ */
+HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,
+                            const int32_t* idx_dev,
+                            int32_t* host_idx_scratch, void* pool_k, void* pool_v, int pool_slots,
+                            int32_t* idx_pool_dev, int* n_unique_out, hga_stream_t compute_stream,
+                            hga_stream_t copy_stream, hga_event_t done, int timeout_ms);
+
+/*
+ * Segment-end offload (fr edition, Analyse approfondie: the KV of a finished
+ * segment is offloaded right away).  Copies the segment's K and V (device,
+ * [B, S, Hkv, d]) into the pinned host tier at history block `at_block`
+ * (host_k/host_v [B, capacity_blocks*block, Hkv, d]) on `stream`, one copy per
+ * (batch, tensor).  The summaries of the new blocks are computed on the device
+ * with hga_block_summaries.  Errors: HGA_ERR_INVALID_ARG, HGA_ERR_SHAPE.
+ */
+HGA_API hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
+                               void* host_v, int capacity_blocks, int at_block, hga_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HGA_H */

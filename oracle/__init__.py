@@ -63,7 +63,7 @@ def _lib():
         lib.ohga_query_means.argtypes = [D, P, P]
         lib.ohga_block_scores.argtypes = [D, P, P, P]
         lib.ohga_select_topk.argtypes = [D, P, P]
-        lib.ohga_attn_fwd.argtypes = [D, P, P, P, P, P, P, I, I, P, P]
+        lib.ohga_attn_fwd.argtypes = [D, P, P, P, P, P, P, I, I, P, P, P]
         lib.ohga_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, I, I, P, P, P]
         lib.ohga_dense_causal_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P]
         _LIB = lib
@@ -140,15 +140,20 @@ def _attn_inputs(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx):
     return Dc, q, k_seg, v_seg, k_hist, v_hist, idx
 
 
-def attn_fwd(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx, kv_heads=None):
-    """O [B,S,Hq,d] and LSE [B,Hq,S] for KV heads in range(kv_heads) (default all).
-    Rows of query heads outside the range are left as NaN."""
+def attn_fwd(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx, kv_heads=None, rows=None):
+    """O [B,S,Hq,d] and LSE [B,Hq,S] for KV heads in range(kv_heads) (default
+    all) and segment positions ``rows`` (default all).  Entries not computed
+    are left as NaN."""
     Dc, q, k_seg, v_seg, k_hist, v_hist, idx = _attn_inputs(D, q, k_seg, v_seg, k_hist, v_hist, idx)
     h0, h1 = (0, D.Hkv) if kv_heads is None else (kv_heads.start, kv_heads.stop)
+    mask = None
+    if rows is not None:
+        mask = np.zeros(D.S, dtype=np.int8)
+        mask[np.asarray(rows)] = 1
     o = np.full((D.B, D.S, D.Hq, D.d), np.nan)
     lse = np.full((D.B, D.Hq, D.S), np.nan)
     _lib().ohga_attn_fwd(ctypes.byref(Dc.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist), _ptr(v_hist),
-                         _ptr(idx), h0, h1, _ptr(o), _ptr(lse))
+                         _ptr(idx), h0, h1, None if mask is None else _ptr(mask), _ptr(o), _ptr(lse))
     return o, lse
 
 

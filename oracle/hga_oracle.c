@@ -206,9 +206,11 @@ static void row_attention(int d, const double* qrow, int nk, const double** keys
   *lse = m + log(z);
 }
 
+/* row_mask (optional, length S): only segment positions p with row_mask[p]
+ * != 0 are computed. */
 void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
-                   const double* k_hist, const double* v_hist, const int32_t* idx, int h0, int h1, double* o,
-                   double* lse) {
+                   const double* k_hist, const double* v_hist, const int32_t* idx, int h0, int h1,
+                   const int8_t* row_mask, double* o, double* lse) {
   const int G = D->Hq / D->Hkv;
   const int maxk = D->topk * D->blk + D->S;
 #pragma omp parallel
@@ -222,6 +224,7 @@ void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, con
         for (int p = 0; p < D->S; ++p) {
           const int h = hq / G;
           if (!in_range(h, h0, h1)) continue;
+          if (row_mask && !row_mask[p]) continue;
           const int nk = gather_keys(D, b, h, p / D->blk, p, k_seg, v_seg, k_hist, v_hist, idx, keys, vals);
           row_attention(D->d, q + tok_off(b, p, D->S, hq, D->Hq, D->d), nk, keys, vals,
                         o + tok_off(b, p, D->S, hq, D->Hq, D->d), &lse[((size_t)b * D->Hq + hq) * D->S + p], s_buf,

@@ -15,8 +15,8 @@ void ohga_query_means(const ohga_dims* D, const double* q, double* qm);
 void ohga_block_scores(const ohga_dims* D, const double* qm, const double* summ, double* score);
 void ohga_select_topk(const ohga_dims* D, const double* score, int32_t* idx);
 void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
-                   const double* k_hist, const double* v_hist, const int32_t* idx, int h0, int h1, double* o,
-                   double* lse);
+                   const double* k_hist, const double* v_hist, const int32_t* idx, int h0, int h1,
+                   const int8_t* row_mask, double* o, double* lse);
 void ohga_attn_bwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
                    const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o, int h0, int h1,
                    double* dq, double* dk, double* dv);

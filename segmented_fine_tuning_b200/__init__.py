@@ -1,0 +1,12 @@
+"""B200-native HGA per-segment attention step.
+
+The compute lives in libhga.so (hand-written sm_100a kernels behind a C ABI,
+include/hga.h).  This package is its thin binding plus the buffer plumbing of
+one attention step (``step.AttentionStep``) and of the full segmented pass
+(``segmented.SegmentedPass``).
+"""
+from ._binding import (  # noqa: F401
+    Dims, HgaError, LIB_PATH, hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd, hga_block_summaries,
+    hga_device_status, hga_fetch_blocks, hga_offload_segment, hga_select_topk, hga_selftest_umma,
+    hga_status_string, load_library,
+)

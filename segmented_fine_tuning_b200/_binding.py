@@ -1,0 +1,242 @@
+"""ctypes binding of libhga.so: argument marshalling only.
+
+Every function has the name of the C entry point it wraps (include/hga.h) and
+takes torch tensors where the C call takes device (or pinned host) pointers.
+Each step of the HGA attention computation runs in the library's CUDA
+kernels; nothing here computes.  A missing library is an ImportError, a
+failing call an HgaError: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhga.so")
+
+HGA_OK = 0
+STATUS_NAMES = {0: "HGA_OK", 1: "HGA_ERR_INVALID_ARG", 2: "HGA_ERR_SHAPE", 3: "HGA_ERR_UNSUPPORTED",
+                4: "HGA_ERR_INDEX", 5: "HGA_ERR_TIMEOUT", 6: "HGA_ERR_CUDA"}
+HGA_F32, HGA_BF16 = 0, 1
+
+
+class HgaError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {detail}")
+
+
+class hga_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
+                ("block", ctypes.c_int), ("S", ctypes.c_int), ("n_hist_blocks", ctypes.c_int),
+                ("topk", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+@dataclass(frozen=True)
+class Dims:
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    block: int
+    S: int
+    n_hist_blocks: int
+    topk: int
+    dtype: str = "bf16"  # "bf16" or "f32"
+
+    @property
+    def nqb(self) -> int:
+        return self.S // self.block
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    def c(self) -> hga_dims:
+        return hga_dims(self.B, self.Hq, self.Hkv, self.d, self.block, self.S, self.n_hist_blocks, self.topk,
+                        HGA_BF16 if self.dtype == "bf16" else HGA_F32)
+
+    def with_history(self, n_hist_blocks: int) -> "Dims":
+        return Dims(self.B, self.Hq, self.Hkv, self.d, self.block, self.S, n_hist_blocks, self.topk, self.dtype)
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_D = ctypes.POINTER(hga_dims)
+
+# (name, restype, argtypes) for every entry point of include/hga.h and
+# include/hga_selftest.h.
+_SIGNATURES = [
+    ("hga_status_string", ctypes.c_char_p, [_I]),
+    ("hga_last_error", ctypes.c_char_p, []),
+    ("hga_device_status", _I, [_P]),
+    ("hga_block_summaries", _I, [_D, _P, _I, _I, _P, _P]),
+    ("hga_select_topk", _I, [_D, _P, _P, _P, _P, _P]),
+    ("hga_attn_fwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
+    ("hga_attn_bwd_workspace_size", ctypes.c_size_t, [_D]),
+    ("hga_attn_bwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("hga_fetch_blocks", _I, [_D, _P, _P, _I, _P, _P, _P, _P, _I, _P, ctypes.POINTER(ctypes.c_int), _P, _P, _P,
+                              _I]),
+    ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
+    ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
+]
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python segmented_fine_tuning_b200/build.py`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, res, args in _SIGNATURES:
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != HGA_OK:
+        raise HgaError(status, where, load_library().hga_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return stream
+
+
+def _expect(t: torch.Tensor, shape, dtype, name: str, device=True):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype} != {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def hga_status_string(status: int) -> str:
+    return load_library().hga_status_string(status).decode()
+
+
+def hga_device_status(stream=None) -> None:
+    _check(load_library().hga_device_status(_stream(stream)), "hga_device_status")
+
+
+def hga_block_summaries(dims: Dims, k_hist, blk_begin: int, blk_end: int, summ, stream=None) -> None:
+    _expect(k_hist, (dims.B, dims.n_hist_blocks * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "k_hist")
+    _expect(summ, (dims.B, dims.Hkv, dims.n_hist_blocks, dims.d), torch.float32, "summ")
+    _check(load_library().hga_block_summaries(ctypes.byref(dims.c()), _ptr(k_hist), blk_begin, blk_end, _ptr(summ),
+                                              _stream(stream)), "hga_block_summaries")
+
+
+def hga_select_topk(dims: Dims, q_seg, summ, idx, scores=None, stream=None) -> None:
+    _expect(q_seg, (dims.B, dims.S, dims.Hq, dims.d), dims.torch_dtype, "q_seg")
+    _expect(summ, (dims.B, dims.Hkv, dims.n_hist_blocks, dims.d), torch.float32, "summ")
+    _expect(idx, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx")
+    if scores is not None:
+        _expect(scores, idx.shape, torch.float32, "scores")
+    _check(load_library().hga_select_topk(ctypes.byref(dims.c()), _ptr(q_seg), _ptr(summ), _ptr(idx), _ptr(scores),
+                                          _stream(stream)), "hga_select_topk")
+
+
+def _attn_shapes(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx):
+    _expect(q, (dims.B, dims.S, dims.Hq, dims.d), dims.torch_dtype, "q")
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(v_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "v_seg")
+    if n_kv_blocks > 0:
+        _expect(k_hist, (dims.B, n_kv_blocks * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "k_hist")
+        _expect(v_hist, (dims.B, n_kv_blocks * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "v_hist")
+    _expect(idx, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx")
+
+
+def hga_attn_fwd(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, o, lse, stream=None) -> None:
+    _attn_shapes(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx)
+    _expect(o, q.shape, dims.torch_dtype, "o")
+    _expect(lse, (dims.B, dims.Hq, dims.S), torch.float32, "lse")
+    _check(load_library().hga_attn_fwd(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist),
+                                       _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse), _stream(stream)),
+           "hga_attn_fwd")
+
+
+def hga_attn_bwd_workspace_size(dims: Dims) -> int:
+    return int(load_library().hga_attn_bwd_workspace_size(ctypes.byref(dims.c())))
+
+
+def hga_attn_bwd(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, o, lse, d_o, dq, dk_seg,
+                 dv_seg, ws, stream=None) -> None:
+    _attn_shapes(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx)
+    _expect(o, q.shape, dims.torch_dtype, "o")
+    _expect(d_o, q.shape, dims.torch_dtype, "d_o")
+    _expect(lse, (dims.B, dims.Hq, dims.S), torch.float32, "lse")
+    _expect(dq, q.shape, torch.float32, "dq")
+    _expect(dk_seg, k_seg.shape, torch.float32, "dk_seg")
+    _expect(dv_seg, v_seg.shape, torch.float32, "dv_seg")
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous CUDA tensor")
+    _check(load_library().hga_attn_bwd(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist),
+                                       _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq),
+                                       _ptr(dk_seg), _ptr(dv_seg), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _stream(stream)), "hga_attn_bwd")
+
+
+def hga_fetch_blocks(dims: Dims, host_k, host_v, host_capacity_blocks: int, idx_dev, host_idx_scratch, pool_k,
+                     pool_v, pool_slots: int, idx_pool_dev, compute_stream, copy_stream, done: torch.cuda.Event,
+                     timeout_ms: int = 10000) -> int:
+    """Returns the number of distinct history blocks fetched into the pool."""
+    shape = (dims.B, host_capacity_blocks * dims.block, dims.Hkv, dims.d)
+    _expect(host_k, shape, dims.torch_dtype, "host_k", device=False)
+    _expect(host_v, shape, dims.torch_dtype, "host_v", device=False)
+    if not (host_k.is_pinned() and host_v.is_pinned() and host_idx_scratch.is_pinned()):
+        raise ValueError("host tier and idx scratch must be pinned host memory")
+    _expect(idx_dev, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx_dev")
+    _expect(host_idx_scratch, idx_dev.shape, torch.int32, "host_idx_scratch", device=False)
+    _expect(pool_k, (dims.B, pool_slots * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "pool_k")
+    _expect(pool_v, pool_k.shape, dims.torch_dtype, "pool_v")
+    _expect(idx_pool_dev, idx_dev.shape, torch.int32, "idx_pool_dev")
+    n_unique = ctypes.c_int(0)
+    _check(load_library().hga_fetch_blocks(ctypes.byref(dims.c()), _ptr(host_k), _ptr(host_v), host_capacity_blocks,
+                                           _ptr(idx_dev), _ptr(host_idx_scratch), _ptr(pool_k), _ptr(pool_v),
+                                           pool_slots, _ptr(idx_pool_dev), ctypes.byref(n_unique),
+                                           _stream(compute_stream), _stream(copy_stream), done.cuda_event,
+                                           timeout_ms), "hga_fetch_blocks")
+    return n_unique.value
+
+
+def hga_offload_segment(dims: Dims, k_seg, v_seg, host_k, host_v, capacity_blocks: int, at_block: int,
+                        stream=None) -> None:
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(v_seg, k_seg.shape, dims.torch_dtype, "v_seg")
+    shape = (dims.B, capacity_blocks * dims.block, dims.Hkv, dims.d)
+    _expect(host_k, shape, dims.torch_dtype, "host_k", device=False)
+    _expect(host_v, shape, dims.torch_dtype, "host_v", device=False)
+    _check(load_library().hga_offload_segment(ctypes.byref(dims.c()), _ptr(k_seg), _ptr(v_seg), _ptr(host_k),
+                                              _ptr(host_v), capacity_blocks, at_block, _stream(stream)),
+           "hga_offload_segment")
+
+
+def hga_selftest_umma(form: int, a, b, d, stream=None) -> None:
+    _expect(a, (128, 128), torch.bfloat16, "a")
+    _expect(b, (128, 128), torch.bfloat16, "b")
+    _expect(d, (128, 128), torch.float32, "d")
+    _check(load_library().hga_selftest_umma(form, _ptr(a), _ptr(b), _ptr(d), _stream(stream)), "hga_selftest_umma")

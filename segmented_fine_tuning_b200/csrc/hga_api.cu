@@ -1,0 +1,402 @@
+// C ABI of libhga.so: argument checks, tensor-map encoding, kernel dispatch,
+// and the host side of the history tier (fetch of selected blocks, segment
+// offload).  Declarations and the method's definition: include/hga.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <chrono>
+#include <mutex>
+#include <thread>
+#include <vector>
+
+#include "../../include/hga.h"
+#include "../../include/hga_selftest.h"
+#include "hga_kernels.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+hga_status fail(hga_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+hga_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(HGA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// Per-device error flag written by the kernels (see hga_device_status).
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_mu;
+
+hga_status device_err_ptr(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HGA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error flag)");
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return HGA_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+hga_status get_encoder(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(HGA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *fn = cached;
+  return HGA_OK;
+}
+
+// bf16 tensor [B, T, H, 128] with a {64, 1, 128, 1} box, 128-byte swizzle.
+hga_status encode_tokens(CUtensorMap* m, const void* base, int B, int T, int H) {
+  EncodeTiledFn enc;
+  hga_status s = get_encoder(&enc);
+  if (s != HGA_OK) return s;
+  const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)H * 128 * 2, (cuuint64_t)T * H * 128 * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HGA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HGA_OK;
+}
+
+// ---------------------------------------------------------------- checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hga_status check_dims(const hga_dims* d, hga::Shape* out) {
+  if (!d) return fail(HGA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->dtype != HGA_F32 && d->dtype != HGA_BF16) return fail(HGA_ERR_INVALID_ARG, "bad dtype %d", (int)d->dtype);
+  if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->S < 1 || d->n_hist_blocks < 0 || d->topk < 1)
+    return fail(HGA_ERR_SHAPE, "non-positive dimension");
+  if (d->Hq % d->Hkv) return fail(HGA_ERR_SHAPE, "Hq (%d) not a multiple of Hkv (%d)", d->Hq, d->Hkv);
+  if (d->d != 64 && d->d != 128) return fail(HGA_ERR_SHAPE, "head dim %d not in {64,128}", d->d);
+  if (d->block != 16 && d->block != 32 && d->block != 64 && d->block != 128)
+    return fail(HGA_ERR_SHAPE, "block %d not in {16,32,64,128}", d->block);
+  if (d->S % d->block) return fail(HGA_ERR_SHAPE, "S (%d) not a multiple of block (%d)", d->S, d->block);
+  if (d->topk > hga::kMaxTopk) return fail(HGA_ERR_SHAPE, "topk %d > %d", d->topk, hga::kMaxTopk);
+  const double tokens = (double)d->B * ((double)d->n_hist_blocks * d->block + d->S) * d->Hq * d->d;
+  if (tokens > 4.0e12) return fail(HGA_ERR_SHAPE, "problem too large");
+  out->B = d->B; out->Hq = d->Hq; out->Hkv = d->Hkv; out->d = d->d; out->blk = d->block; out->S = d->S;
+  out->nblk = d->n_hist_blocks; out->topk = d->topk; out->bf16 = (d->dtype == HGA_BF16);
+  return HGA_OK;
+}
+
+template <typename... P>
+bool any_null(P... p) {
+  return ((p == nullptr) || ...);
+}
+
+hga_status check_attn_ptrs(const hga::Shape& s, int n_kv_blocks, const void* q, const void* ks, const void* vs,
+                           const void* kh, const void* vh, const int32_t* idx) {
+  if (any_null(q, ks, vs, idx)) return fail(HGA_ERR_INVALID_ARG, "NULL input pointer");
+  if (n_kv_blocks < 0) return fail(HGA_ERR_INVALID_ARG, "n_kv_blocks < 0");
+  if (n_kv_blocks > 0 && any_null(kh, vh)) return fail(HGA_ERR_INVALID_ARG, "NULL history pointer");
+  if (!aligned16(q) || !aligned16(ks) || !aligned16(vs) || (n_kv_blocks > 0 && (!aligned16(kh) || !aligned16(vh))))
+    return fail(HGA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  (void)s;
+  return HGA_OK;
+}
+
+hga_status build_maps(const hga::Shape& s, int nkv, const void* q, const void* d_o, const void* ks, const void* vs,
+                      const void* kh, const void* vh, hga::TcMaps* m) {
+  hga_status r;
+  if ((r = encode_tokens(&m->q, q, s.B, s.S, s.Hq)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->d_o, d_o ? d_o : q, s.B, s.S, s.Hq)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->ks, ks, s.B, s.S, s.Hkv)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->vs, vs, s.B, s.S, s.Hkv)) != HGA_OK) return r;
+  // With no history the history maps are never read; point them at the segment.
+  if ((r = encode_tokens(&m->kh, nkv > 0 ? kh : ks, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->vh, nkv > 0 ? vh : vs, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv)) != HGA_OK) return r;
+  return HGA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char* hga_status_string(hga_status s) {
+  switch (s) {
+    case HGA_OK: return "HGA_OK";
+    case HGA_ERR_INVALID_ARG: return "HGA_ERR_INVALID_ARG";
+    case HGA_ERR_SHAPE: return "HGA_ERR_SHAPE";
+    case HGA_ERR_UNSUPPORTED: return "HGA_ERR_UNSUPPORTED";
+    case HGA_ERR_INDEX: return "HGA_ERR_INDEX";
+    case HGA_ERR_TIMEOUT: return "HGA_ERR_TIMEOUT";
+    case HGA_ERR_CUDA: return "HGA_ERR_CUDA";
+  }
+  return "HGA_ERR_UNKNOWN";
+}
+
+const char* hga_last_error(void) { return g_last_error; }
+
+hga_status hga_device_status(hga_stream_t stream) {
+  int* flag;
+  hga_status s = device_err_ptr(&flag);
+  if (s != HGA_OK) return s;
+  int host = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&host, flag, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error flag");
+  if (host == 0) return HGA_OK;
+  e = cudaMemsetAsync(flag, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error flag");
+  if (host & hga::kDevErrIndex) return fail(HGA_ERR_INDEX, "a kernel met an idx entry outside [-1, n_kv_blocks)");
+  return fail(HGA_ERR_TIMEOUT, "a kernel pipeline wait expired");
+}
+
+hga_status hga_block_summaries(const hga_dims* dims, const void* k_hist, int blk_begin, int blk_end, float* summ,
+                               hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (blk_begin < 0 || blk_end > s.nblk || blk_begin > blk_end)
+    return fail(HGA_ERR_INVALID_ARG, "block range [%d,%d) outside [0,%d)", blk_begin, blk_end, s.nblk);
+  if (blk_end == blk_begin) return HGA_OK;
+  if (any_null(k_hist, summ)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k_hist)) return fail(HGA_ERR_INVALID_ARG, "k_hist must be 16-byte aligned");
+  cudaError_t e = hga::launch_block_summaries(s, k_hist, blk_begin, blk_end, summ,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "block summaries launch");
+}
+
+hga_status hga_select_topk(const hga_dims* dims, const void* q_seg, const float* summ, int32_t* idx,
+                           float* scores_or_null, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (s.nblk > hga::kMaxSelectBlocks)
+    return fail(HGA_ERR_SHAPE, "n_hist_blocks %d > %d", s.nblk, hga::kMaxSelectBlocks);
+  if (any_null(q_seg, idx) || (s.nblk > 0 && summ == nullptr)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q_seg)) return fail(HGA_ERR_INVALID_ARG, "q must be 16-byte aligned");
+  cudaError_t e = hga::launch_select_topk(s, q_seg, summ, idx, scores_or_null, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "select launch");
+}
+
+hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                        const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, void* o,
+                        float* lse, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if ((r = check_attn_ptrs(s, n_kv_blocks, q, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
+  if (any_null(o, lse)) return fail(HGA_ERR_INVALID_ARG, "NULL output pointer");
+  int* err;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (hga::tc_supported(s)) {
+    hga::TcMaps m;
+    if ((r = build_maps(s, n_kv_blocks, q, nullptr, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
+    e = hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, st);
+  } else {
+    e = hga::launch_attn_fwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse, err, st);
+  }
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "attention forward launch");
+}
+
+size_t hga_attn_bwd_workspace_size(const hga_dims* dims) {
+  if (!dims) return 0;
+  return round256((size_t)dims->B * dims->Hq * dims->S * sizeof(float));
+}
+
+hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                        const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o,
+                        const float* lse, const void* d_o, float* dq, float* dk_seg, float* dv_seg, void* ws,
+                        size_t ws_bytes, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if ((r = check_attn_ptrs(s, n_kv_blocks, q, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
+  if (any_null(o, lse, d_o, dq, dk_seg, dv_seg, ws)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(o) || !aligned16(d_o) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk_seg) ||
+      !aligned16(dv_seg))
+    return fail(HGA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(HGA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (ws_bytes < hga_attn_bwd_workspace_size(dims))
+    return fail(HGA_ERR_INVALID_ARG, "workspace %zu bytes < %zu", ws_bytes, hga_attn_bwd_workspace_size(dims));
+  int* err;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* Dr = static_cast<float*>(ws);
+  cudaError_t e = hga::launch_bwd_preprocess(s, o, d_o, Dr, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward preprocess launch");
+  if (hga::tc_supported(s)) {
+    hga::TcMaps m;
+    if ((r = build_maps(s, n_kv_blocks, q, d_o, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
+    e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, err, st);
+  } else {
+    e = hga::launch_attn_bwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, lse, Dr, d_o, dq, dk_seg,
+                                  dv_seg, err, st);
+  }
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "attention backward launch");
+}
+
+hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,
+                            const int32_t* idx_dev,
+                            int32_t* host_idx_scratch, void* pool_k, void* pool_v, int pool_slots,
+                            int32_t* idx_pool_dev, int* n_unique_out, hga_stream_t compute_stream,
+                            hga_stream_t copy_stream, hga_event_t done, int timeout_ms) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(host_k, host_v, idx_dev, host_idx_scratch, pool_k, pool_v, idx_pool_dev, done))
+    return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (pool_slots < 0) return fail(HGA_ERR_INVALID_ARG, "pool_slots < 0");
+  if (host_capacity_blocks < dims->n_hist_blocks)
+    return fail(HGA_ERR_INVALID_ARG, "host tier holds %d blocks < n_hist_blocks %d", host_capacity_blocks,
+                dims->n_hist_blocks);
+  cudaStream_t cst = reinterpret_cast<cudaStream_t>(compute_stream);
+  cudaStream_t xst = reinterpret_cast<cudaStream_t>(copy_stream);
+  const size_t n_idx = (size_t)s.B * s.Hkv * s.nqb() * s.topk;
+  cudaEvent_t ready = nullptr, landed = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&landed, cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    if (ready) cudaEventDestroy(ready);
+    return cuda_fail(e, "event create");
+  }
+  struct Guard {
+    cudaEvent_t a, b;
+    ~Guard() { cudaEventDestroy(a); cudaEventDestroy(b); }
+  } guard{ready, landed};
+  // 1. idx -> host, after the selection queued on the compute stream.
+  if ((e = cudaEventRecord(ready, cst)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaStreamWaitEvent(xst, ready, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, xst)) !=
+      cudaSuccess)
+    return cuda_fail(e, "idx copy to host");
+  if ((e = cudaEventRecord(landed, xst)) != cudaSuccess) return cuda_fail(e, "event record");
+  const auto t0 = std::chrono::steady_clock::now();
+  while (true) {
+    e = cudaEventQuery(landed);
+    if (e == cudaSuccess) break;
+    if (e != cudaErrorNotReady) return cuda_fail(e, "waiting for idx");
+    if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms))
+      return fail(HGA_ERR_TIMEOUT, "idx copy did not complete within %d ms", timeout_ms);
+    std::this_thread::yield();
+  }
+  // 2. distinct selected blocks, ascending -> pool slots.
+  std::vector<int32_t> slot_of(s.nblk > 0 ? s.nblk : 1, -1);
+  for (size_t k = 0; k < n_idx; ++k) {
+    const int n = host_idx_scratch[k];
+    if (n == -1) continue;
+    if (n < 0 || n >= s.nblk) return fail(HGA_ERR_INDEX, "idx entry %d outside [-1, %d)", n, s.nblk);
+    slot_of[n] = 0;
+  }
+  int n_unique = 0;
+  for (int n = 0; n < s.nblk; ++n)
+    if (slot_of[n] == 0) slot_of[n] = n_unique++;
+  if (n_unique > pool_slots)
+    return fail(HGA_ERR_INVALID_ARG, "%d distinct blocks selected, pool holds %d", n_unique, pool_slots);
+  // 3. host -> pool copies, one per run of consecutive blocks, per batch and tensor.
+  const size_t es = s.bf16 ? 2 : 4;
+  const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
+  for (int n = 0; n < s.nblk;) {
+    if (slot_of[n] < 0) {
+      ++n;
+      continue;
+    }
+    int run = 1;
+    while (n + run < s.nblk && slot_of[n + run] >= 0) ++run;
+    for (int b = 0; b < s.B; ++b) {
+      const size_t src = ((size_t)b * host_capacity_blocks + n) * blk_bytes;
+      const size_t dst = ((size_t)b * pool_slots + slot_of[n]) * blk_bytes;
+      if ((e = cudaMemcpyAsync(static_cast<char*>(pool_k) + dst, static_cast<const char*>(host_k) + src,
+                               run * blk_bytes, cudaMemcpyHostToDevice, xst)) != cudaSuccess)
+        return cuda_fail(e, "K block copy");
+      if ((e = cudaMemcpyAsync(static_cast<char*>(pool_v) + dst, static_cast<const char*>(host_v) + src,
+                               run * blk_bytes, cudaMemcpyHostToDevice, xst)) != cudaSuccess)
+        return cuda_fail(e, "V block copy");
+    }
+    n += run;
+  }
+  // 4. idx rewritten to pool slots (in the pinned scratch), then uploaded.
+  for (size_t k = 0; k < n_idx; ++k) {
+    const int n = host_idx_scratch[k];
+    host_idx_scratch[k] = n < 0 ? -1 : slot_of[n];
+  }
+  if ((e = cudaMemcpyAsync(idx_pool_dev, host_idx_scratch, n_idx * sizeof(int32_t), cudaMemcpyHostToDevice, xst)) !=
+      cudaSuccess)
+    return cuda_fail(e, "pool idx upload");
+  if ((e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(done), xst)) != cudaSuccess)
+    return cuda_fail(e, "event record");
+  if (n_unique_out) *n_unique_out = n_unique;
+  return HGA_OK;
+}
+
+hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
+                               void* host_v, int capacity_blocks, int at_block, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(k_seg, v_seg, host_k, host_v)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  const int nseg = s.nqb();
+  if (at_block < 0 || at_block + nseg > capacity_blocks)
+    return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the tier's %d", at_block, at_block + nseg,
+                capacity_blocks);
+  const size_t es = s.bf16 ? 2 : 4;
+  const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int b = 0; b < s.B; ++b) {
+    const size_t dst = ((size_t)b * capacity_blocks + at_block) * blk_bytes;
+    const size_t src = (size_t)b * nseg * blk_bytes;
+    cudaError_t e = cudaMemcpyAsync(static_cast<char*>(host_k) + dst, static_cast<const char*>(k_seg) + src,
+                                    nseg * blk_bytes, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(host_v) + dst, static_cast<const char*>(v_seg) + src, nseg * blk_bytes,
+                          cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "segment offload copy");
+  }
+  return HGA_OK;
+}
+
+hga_status hga_selftest_umma(int form, const void* a, const void* b, float* d, hga_stream_t stream) {
+  if (form < 0 || form > 3) return fail(HGA_ERR_INVALID_ARG, "form %d not in 0..3", form);
+  if (any_null(a, b, d) || !aligned16(a) || !aligned16(b)) return fail(HGA_ERR_INVALID_ARG, "bad pointer");
+  CUtensorMap ma, mb;
+  hga_status r;
+  if ((r = encode_tokens(&ma, a, 1, 128, 1)) != HGA_OK) return r;
+  if ((r = encode_tokens(&mb, b, 1, 128, 1)) != HGA_OK) return r;
+  int* err;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  cudaError_t e = hga::launch_selftest_umma(form, ma, mb, a, d, err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "selftest launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,353 @@
+// Tensor-core (tcgen05) forward of the HGA attention step, bf16 in, fp32
+// accumulate, for d = 128 and 128-token blocks.
+//
+// Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention
+// and Segmented Backpropagation in Practice", Background: each query block
+// attends, exactly, to a bounded set of history tokens (the top-K blocks picked
+// by summary score) plus the causal part of the active segment.
+//
+// Work unit (one CTA): batch b, KV head h, query block i, and a PAIR of query
+// heads of h.  Both heads share the KV head and the query block, hence the
+// same tile list: the K_eff selected history blocks followed by segment blocks
+// 0..i (the last one, the diagonal, is causally masked).  Every K/V tile that
+// TMA brings into shared memory feeds two 128x128x128 products.
+//
+// Roles (384 threads, 1 CTA per SM):
+//   warps 0-3   softmax for head 0 of the pair (one query row per thread)
+//   warps 4-7   softmax for head 1
+//   warp  8     TMA producer: Q tiles once, then K_j, V_j into a 5-slot ring
+//   warp  9     MMA issuer (one thread): S_t = Q_t K_j^T, O_t += P_t V_j
+// Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns each, fp32.
+// The softmax writes P (bf16) back into the S columns it has just read, and
+// the PV product takes P straight from tensor memory.
+//
+// Online softmax in base 2 with a lazily updated reference maximum: the
+// running reference m only moves (and O is rescaled in tensor memory) when a
+// row's new maximum exceeds it by more than 8, so that P <= 2^8 stays exact
+// in fp32/bf16 range while most tiles skip the rescale.
+// MMA order per tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  Because tcgen05
+// operations of one thread complete in order, the commit that announces
+// S_t(j+1) also guarantees that PV_t(j) is done, which frees P_t and makes O_t
+// safe to rescale.
+#include "hga_kernels.h"
+#include "hga_ptx.cuh"
+
+namespace hga {
+namespace {
+
+constexpr int kBM = 128;                      // query rows per tile
+constexpr int kBN = 128;                      // keys per tile
+constexpr int kD = 128;                       // head dim
+constexpr int kTileBytes = kBM * kD * 2;      // 32 KB bf16 tile
+constexpr int kHalf = kTileBytes / 2;         // one 64-column TMA box
+constexpr int kStages = 5;                    // K/V ring slots
+constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
+
+struct FwdCtl {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t mma_done;
+  uint32_t tmem;
+  int abort;
+  int nt;
+  int tiles[kMaxTiles];  // >= 0: history block; < 0: segment block -(t+1)
+};
+
+constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kStages * kTileBytes + sizeof(FwdCtl);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct FwdArgs {
+  int B, Hq, Hkv, S, nkv, topk, nqb, G;
+  float sl2;  // log2(e) / sqrt(d)
+  const int32_t* idx;
+  __nv_bfloat16* o;
+  float* lse;
+  int* err;
+};
+
+__global__ void __launch_bounds__(384, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
+                  const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kh,
+                  const __grid_constant__ CUtensorMap tm_vh, const FwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* sQ = sm;                                // 2 Q tiles
+  uint8_t* sRing = sm + 2 * kTileBytes;            // kStages K/V tiles
+  FwdCtl* ctl = reinterpret_cast<FwdCtl*>(sRing + kStages * kTileBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Longest work first: query block i descending with blockIdx.
+  const int npair = a.G >> 1;
+  const int per_i = a.B * a.Hkv * npair;
+  const int i = a.nqb - 1 - (int)(blockIdx.x / per_i);
+  const int rem = (int)(blockIdx.x % per_i);
+  const int b = rem / (a.Hkv * npair);
+  const int kvh = (rem / npair) % a.Hkv;
+  const int hq0 = kvh * a.G + 2 * (rem % npair);
+
+  if (warp == 0) {
+    const int32_t* row = a.idx + (((size_t)b * a.Hkv + kvh) * a.nqb + i) * a.topk;
+    int nh = 0;
+    for (int base = 0; base < a.topk; base += 32) {
+      const int r = base + lane;
+      const int n = (r < a.topk) ? __ldg(row + r) : -1;
+      const bool ok = (n >= 0 && n < a.nkv);
+      if (r < a.topk && !ok && n != -1) flag_error(a.err, kDevErrIndex);
+      const unsigned m = __ballot_sync(0xffffffffu, ok);
+      if (ok) ctl->tiles[nh + __popc(m & ((1u << lane) - 1u))] = n;
+      nh += __popc(m);
+    }
+    for (int jb = lane; jb <= i; jb += 32) ctl->tiles[nh + jb] = -(jb + 1);
+    if (lane == 0) {
+      ctl->nt = nh + i + 1;
+      ctl->abort = 0;
+      mbar_init(&ctl->q_full, 1);
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(&ctl->kv_full[s], 1);
+        mbar_init(&ctl->kv_empty[s], 1);
+      }
+      for (int t = 0; t < 2; ++t) {
+        mbar_init(&ctl->s_full[t], 1);
+        mbar_init(&ctl->p_full[t], 128);
+        mbar_init(&ctl->o_full[t], 1);
+      }
+      mbar_init(&ctl->mma_done, 1);
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(&ctl->tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem;
+  const int nt = ctl->nt;
+  volatile int* abort = &ctl->abort;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_kh);
+      prefetch_tmap(&tm_vh);
+      prefetch_tmap(&tm_ks);
+      prefetch_tmap(&tm_vs);
+      mbar_expect_tx(&ctl->q_full, 2 * kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_4d(&tm_q, &ctl->q_full, sQ + t * kTileBytes + hh * kHalf, hh * 64, hq0 + t, i * kBM, b);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int tile = ctl->tiles[j];
+        const bool hist = tile >= 0;
+        const int row0 = (hist ? tile : (-tile - 1)) * kBN;
+        bool ok = true;
+        for (int w = 0; w < 2 && ok; ++w) {
+          const int pos = 2 * j + w;
+          const int s = pos % kStages;
+          if (!mbar_wait(&ctl->kv_empty[s], ((pos / kStages) & 1) ^ 1, abort, a.err)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* m = hist ? (w ? &tm_vh : &tm_kh) : (w ? &tm_vs : &tm_ks);
+          mbar_expect_tx(&ctl->kv_full[s], kTileBytes);
+          tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes, 0, kvh, row0, b);
+          tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes + kHalf, 64, kvh, row0, b);
+          issued = pos + 1;
+        }
+        if (!ok) break;
+      }
+      // Never leave the CTA with copies in flight: wait (bounded) for the
+      // last loads issued into each slot and for Q.
+      volatile int no_abort = 0;
+      mbar_wait(&ctl->q_full, 0, &no_abort, a.err);
+      for (int pos = issued - kStages > 0 ? issued - kStages : 0; pos < issued; ++pos)
+        mbar_wait(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, &no_abort, a.err);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);  // Q, K both K-major
+      constexpr uint32_t kIdO = idesc_bf16(kBM, kD, false, true);    // P (tmem) x V (MN-major)
+      const uint32_t sq = smem_u32(sQ), sr = smem_u32(sRing);
+      auto issue_S = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          umma_ss(tmem + t * 128, sdesc_sw128(sq + t * kTileBytes + off, 16, 1024),
+                  sdesc_sw128(sr + s * kTileBytes + off, 16, 1024), kIdS, kk > 0);
+        }
+      };
+      auto issue_PV = [&](int t, int s, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // P chunk c (keys 32c..32c+31) sits at S columns [32c, 32c+16).
+          const uint32_t pcol = (kk >> 1) * 32 + (kk & 1) * 8;
+          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + pcol, sdesc_sw128(sr + s * kTileBytes + kk * 2048, kHalf, 1024),
+                  kIdO, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_full = [&](int pos) {
+        return mbar_wait(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, abort, a.err);
+      };
+      bool ok = mbar_wait(&ctl->q_full, 0, abort, a.err) && wait_full(0);
+      if (ok) {
+        tc_fence_after();
+        issue_S(0, 0);
+        umma_commit(&ctl->s_full[0]);
+        issue_S(1, 0);
+        umma_commit(&ctl->s_full[1]);
+        umma_commit(&ctl->kv_empty[0]);
+        for (int j = 0; j < nt; ++j) {
+          const int sV = (2 * j + 1) % kStages;
+          const int sK = (2 * j + 2) % kStages;
+          const bool more = j + 1 < nt;
+          if (!wait_full(2 * j + 1)) break;
+          if (!mbar_wait(&ctl->p_full[0], j & 1, abort, a.err)) break;
+          tc_fence_after();
+          issue_PV(0, sV, j > 0);
+          if (more) {
+            if (!wait_full(2 * j + 2)) break;
+            tc_fence_after();
+            issue_S(0, sK);
+            umma_commit(&ctl->s_full[0]);
+          } else {
+            umma_commit(&ctl->o_full[0]);
+          }
+          if (!mbar_wait(&ctl->p_full[1], j & 1, abort, a.err)) break;
+          tc_fence_after();
+          issue_PV(1, sV, j > 0);
+          umma_commit(&ctl->kv_empty[sV]);
+          if (more) {
+            issue_S(1, sK);
+            umma_commit(&ctl->s_full[1]);
+            umma_commit(&ctl->kv_empty[sK]);
+          } else {
+            umma_commit(&ctl->o_full[1]);
+          }
+        }
+      }
+      // All issued MMAs must finish before tensor memory is released.
+      umma_commit(&ctl->mma_done);
+      volatile int no_abort = 0;
+      mbar_wait(&ctl->mma_done, 0, &no_abort, a.err);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    const float sl2 = a.sl2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t v[32];
+    for (int j = 0; j < nt; ++j) {
+      if (!mbar_wait(&ctl->s_full[t], j & 1, abort, a.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = (j == nt - 1);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        HGA_TMEM_LD32_WAIT(tS + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (!diag || c * 32 + e <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
+      }
+      mx *= sl2;
+      if (mx > m_ref + kRescaleThreshold) {
+        const float alpha = ex2_approx(m_ref - mx);
+        l *= alpha;
+        if (j > 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            HGA_TMEM_LD32_WAIT(tO + c * 32, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            HGA_TMEM_ST32(tO + c * 32, v);
+          }
+        }
+        m_ref = mx;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        HGA_TMEM_LD32_WAIT(tS + c * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const bool k0 = !diag || c * 32 + e <= r;
+          const bool k1 = !diag || c * 32 + e + 1 <= r;
+          const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(v[e]), sl2, -m_ref)) : 0.f;
+          const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), sl2, -m_ref)) : 0.f;
+          l += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        HGA_TMEM_ST16(tS + c * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ctl->p_full[t]);
+    }
+    if (ok && mbar_wait(&ctl->o_full[t], 0, abort, a.err)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const int p = i * kBM + r;
+      const int hq = hq0 + t;
+      __nv_bfloat16* orow = a.o + (((size_t)b * a.S + p) * a.Hq + hq) * kD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        HGA_TMEM_LD32_WAIT(tO + c * 32, v);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * qd + 0]) * inv_l, __uint_as_float(v[8 * qd + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(v[8 * qd + 2]) * inv_l, __uint_as_float(v[8 * qd + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(v[8 * qd + 4]) * inv_l, __uint_as_float(v[8 * qd + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(v[8 * qd + 6]) * inv_l, __uint_as_float(v[8 * qd + 7]) * inv_l);
+          dst[qd] = w;
+        }
+      }
+      a.lse[((size_t)b * a.Hq + hq) * a.S + p] = (m_ref + log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool tc_supported(const Shape& s) {
+  return s.bf16 && s.d == kD && s.blk == kBM && (s.G() % 2) == 0 && s.topk <= kMaxTopk &&
+         s.nqb() <= kMaxQueryBlocks;
+}
+
+cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
+                               int* err, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  FwdArgs a;
+  a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
+  a.sl2 = 1.4426950408889634f / sqrtf((float)kD);
+  a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err;
+  const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
+  fwd_tc_kernel<<<grid, 384, kSmemBytes, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
+  return cudaGetLastError();
+}
+
+}  // namespace hga

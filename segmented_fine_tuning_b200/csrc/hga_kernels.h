@@ -1,0 +1,59 @@
+// Internal launch interface between the C-ABI layer (hga_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hga {
+
+// Bits of the per-device error flag.
+enum : int { kDevErrIndex = 1, kDevErrTimeout = 2 };
+
+struct Shape {
+  int B, Hq, Hkv, d, blk, S, nblk, topk;
+  bool bf16;
+  int G() const { return Hq / Hkv; }
+  int nqb() const { return S / blk; }
+};
+
+// Largest K and history length the selection kernel handles in one CTA.
+constexpr int kMaxTopk = 64;
+constexpr int kMaxSelectBlocks = 4096;
+// Longest segment (in query blocks) the tensor-core kernels handle.
+constexpr int kMaxQueryBlocks = 128;
+
+cudaError_t launch_block_summaries(const Shape& s, const void* k_hist, int b0, int b1, float* summ,
+                                   cudaStream_t st);
+cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
+                               cudaStream_t st);
+// D[b,hq,p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k]  (fp32)
+cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st);
+
+// CUDA-core attention (any supported shape, fp32 or bf16).
+cudaError_t launch_attn_fwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
+                                 const void* k_hist, const void* v_hist, int nkv, const int32_t* idx, void* o,
+                                 float* lse, int* err, cudaStream_t st);
+cudaError_t launch_attn_bwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
+                                 const void* k_hist, const void* v_hist, int nkv, const int32_t* idx,
+                                 const float* lse, const float* Dr, const void* d_o, float* dq, float* dk,
+                                 float* dv, int* err, cudaStream_t st);
+
+// Tensor-core attention (bf16, d = 128, block = 128, even G).  Tensor maps:
+// q/d_o [B,S,Hq,128], k/v seg [B,S,Hkv,128], k/v hist [B,nkv*128,Hkv,128],
+// all with a 64 x 1 x 128 x 1 box and 128-byte swizzle.
+struct TcMaps {
+  CUtensorMap q, d_o, ks, vs, kh, vh;
+};
+bool tc_supported(const Shape& s);
+cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
+                               int* err, cudaStream_t st);
+cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
+                               const float* Dr, float* dq, float* dk, float* dv, int* err, cudaStream_t st);
+
+// Tensor-core operand-layout self test (see hga_selftest.h).
+cudaError_t launch_selftest_umma(int form, const CUtensorMap& ma, const CUtensorMap& mb, const void* a_raw,
+                                 float* d, int* err, cudaStream_t st);
+
+}  // namespace hga

@@ -1,0 +1,293 @@
+// HBM-bound kernels of the HGA step: block summaries, per-query-block
+// selection (scores + top-K), and the backward preprocessing row dot.
+//
+// Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention and
+// Segmented Backpropagation in Practice" -- Deep analysis (resident per-block
+// summaries), Background (bounded exact history set per query block).  The
+// summary is the mean of a block's keys, the score the group-max of
+// query-block-mean . summary / sqrt(d), ties to the lower block index.
+#include <float.h>
+
+#include "hga_kernels.h"
+#include "hga_ptx.cuh"
+
+namespace hga {
+namespace {
+
+template <typename T>
+struct Vec;  // 16-byte vector of T, widened to float
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float* out) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* out) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      out[2 * k] = __uint_as_float(w[k] << 16);
+      out[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+
+// ------------------------------------------------------------ summaries
+// CTA = (history block n, column chunk of 32 vectors, batch b).  Each warp
+// reads whole 32-vector stretches of token rows (coalesced 512 B for bf16),
+// 8 warps cover 8 rows per pass; partials are combined in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k, int T_tok, int Hkv, int d, int blk,
+                                                        int nblk, int b0, float* __restrict__ summ) {
+  constexpr int V = Vec<T>::N;
+  const int n = b0 + blockIdx.x;
+  const int b = blockIdx.z;
+  const int cols = Hkv * d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int col = (blockIdx.y * 32 + lane) * V;
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  if (col < cols) {
+    const T* base = k + ((size_t)b * T_tok + (size_t)n * blk) * cols + col;
+    int t = warp;
+#pragma unroll 4
+    for (; t < blk; t += 8) {
+      float x[V];
+      Vec<T>::load(base + (size_t)t * cols, x);
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] += x[e];
+    }
+  }
+  __shared__ float part[8][32 * 8];
+#pragma unroll
+  for (int e = 0; e < V; ++e) part[warp][lane * V + e] = acc[e];
+  __syncthreads();
+  for (int x = threadIdx.x; x < 32 * V; x += 256) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += part[w][x];
+    const int c = blockIdx.y * 32 * V + x;
+    if (c < cols) {
+      const int h = c / d, kk = c % d;
+      summ[(((size_t)b * Hkv + h) * nblk + n) * d + kk] = s * (1.0f / blk);
+    }
+  }
+}
+
+// ------------------------------------------------------------ selection
+// Ordered 64-bit key: larger score first, then lower block index first.
+__device__ __forceinline__ unsigned long long sel_key(float s, int n) {
+  uint32_t u = __float_as_uint(s + 0.0f);  // -0 -> +0 so that they tie
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)n);
+}
+
+// CTA = (query block i, KV head h, batch b).  256 threads.
+//  1. qm[g][:] = mean of the block's rows of Q for the G query heads of h
+//     (the G heads of a KV head are contiguous in a token row).
+//  2. score[n] = max_g qm[g] . summ[b,h,n] / sqrt(d): one warp per block n.
+//  3. bitonic sort of (score, index) keys, descending; first K_eff kept,
+//     then listed in ascending block order.
+template <typename T>
+__global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, const float* __restrict__ summ, int S,
+                                                     int Hq, int Hkv, int d, int blk, int nblk, int topk,
+                                                     float inv_sqrt_d, int32_t* __restrict__ idx,
+                                                     float* __restrict__ scores) {
+  constexpr int V = Vec<T>::N;
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = Hq / Hkv;
+  const int nqb = S / blk;
+  const int cols = G * d;
+  int npow = 1;
+  while (npow < nblk) npow <<= 1;
+  float* qm = reinterpret_cast<float*>(sel_smem);                              // [G*d]
+  float* part = qm + cols + (cols & 1);                                        // [256*V]
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part + 256 * V);  // [npow]
+  __shared__ int chosen[kMaxTopk];
+  const int tid = threadIdx.x;
+
+  // 1. query means: thread = (row phase r0, vector vt); rows r0, r0+rpp, ...
+  //    are summed per thread, the rpp partials are then combined.
+  const int tpr = cols / V;  // vectors per row (d is a multiple of 8)
+  for (int c0 = 0; c0 < tpr; c0 += 256) {
+    const int width = min(256, tpr - c0);
+    const int rpp = 256 / width;
+    const int vt = c0 + tid % width, r0 = tid / width;
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    if (r0 < rpp) {
+      const T* base = q + (((size_t)b * S + (size_t)i * blk) * Hq + (size_t)h * G) * d + (size_t)vt * V;
+      const size_t rs = (size_t)Hq * d;
+#pragma unroll 8
+      for (int t = r0; t < blk; t += rpp) {
+        float x[V];
+        Vec<T>::load(base + t * rs, x);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += x[e];
+      }
+#pragma unroll
+      for (int e = 0; e < V; ++e) part[r0 * width * V + (vt - c0) * V + e] = acc[e];
+    }
+    __syncthreads();
+    for (int x = tid; x < width * V; x += 256) {
+      float s = 0.f;
+      for (int r = 0; r < rpp; ++r) s += part[r * width * V + x];
+      qm[c0 * V + x] = s * (1.0f / blk);
+    }
+    __syncthreads();
+  }
+
+  // 2. scores -> keys
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int n = warp; n < npow; n += 8) {
+    if (n >= nblk) {
+      if (lane == 0) keys[n] = 0ull;
+      continue;
+    }
+    const float* sv = summ + (((size_t)b * Hkv + h) * nblk + n) * d;
+    float best = -FLT_MAX;
+    for (int g = 0; g < G; ++g) {
+      float part = 0.f;
+      for (int kk = lane; kk < d; kk += 32) part += qm[g * d + kk] * __ldg(sv + kk);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      best = fmaxf(best, part);
+    }
+    if (lane == 0) keys[n] = sel_key(best * inv_sqrt_d, n);
+  }
+  __syncthreads();
+
+  // 3. bitonic sort, descending
+  for (int size = 2; size <= npow; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int x = tid; x < npow; x += 256) {
+        const int y = x ^ stride;
+        if (y > x) {
+          const bool desc = ((x & size) == 0);
+          const unsigned long long a = keys[x], c = keys[y];
+          if (desc ? (a < c) : (a > c)) {
+            keys[x] = c;
+            keys[y] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int keff = topk < nblk ? topk : nblk;
+  if (tid < keff) chosen[tid] = (int)(0xFFFFFFFFu - (uint32_t)(keys[tid] & 0xFFFFFFFFull));
+  __syncthreads();
+  const size_t row = (((size_t)b * Hkv + h) * nqb + i) * topk;
+  if (tid < topk) {
+    if (tid < keff) {
+      const int n = chosen[tid];
+      int rank = 0;
+      for (int u = 0; u < keff; ++u) rank += chosen[u] < n;
+      idx[row + rank] = n;
+      if (scores) {
+        // recover the score from the key (inverse of the ordering map)
+        uint32_t u = (uint32_t)(keys[tid] >> 32);
+        u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+        scores[row + rank] = __uint_as_float(u);
+      }
+    } else {
+      idx[row + tid] = -1;
+      if (scores) scores[row + tid] = -INFINITY;
+    }
+  }
+}
+
+// ------------------------------------------------------------ bwd preprocess
+// One warp per (b, p, hq) row: D = sum_k dO * O in fp32.
+template <typename T>
+__global__ void __launch_bounds__(256) preprocess_kernel(const T* __restrict__ o, const T* __restrict__ d_o, int S,
+                                                         int Hq, int d, int rows, float* __restrict__ Dr) {
+  constexpr int V = Vec<T>::N;
+  const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  // rows are enumerated token-major: warp = (b*S + p)*Hq + hq
+  const size_t off = (size_t)warp * d;
+  float s = 0.f;
+  for (int c = lane * V; c < d; c += 32 * V) {
+    float x[V], y[V];
+    Vec<T>::load(o + off + c, x);
+    Vec<T>::load(d_o + off + c, y);
+#pragma unroll
+    for (int e = 0; e < V; ++e) s += x[e] * y[e];
+  }
+#pragma unroll
+  for (int k = 16; k > 0; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
+  if (lane == 0) {
+    const int hq = warp % Hq;
+    const int bp = warp / Hq;
+    const int b = bp / S, p = bp % S;
+    Dr[((size_t)b * Hq + hq) * S + p] = s;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_block_summaries(const Shape& s, const void* k_hist, int b0, int b1, float* summ,
+                                   cudaStream_t st) {
+  if (b1 <= b0) return cudaSuccess;
+  const int V = s.bf16 ? 8 : 4;
+  const int cols = s.Hkv * s.d;
+  dim3 grid(b1 - b0, (cols + 32 * V - 1) / (32 * V), s.B);
+  const int T_tok = s.nblk * s.blk;
+  if (s.bf16)
+    summaries_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k_hist), T_tok, s.Hkv,
+                                                          s.d, s.blk, s.nblk, b0, summ);
+  else
+    summaries_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(k_hist), T_tok, s.Hkv, s.d, s.blk,
+                                                  s.nblk, b0, summ);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
+                               cudaStream_t st) {
+  int npow = 1;
+  while (npow < s.nblk) npow <<= 1;
+  const int cols = s.G() * s.d;
+  const size_t smem = (size_t)(cols + (cols & 1) + 256 * (s.bf16 ? 8 : 4)) * sizeof(float) + (size_t)npow * 8;
+  dim3 grid(s.nqb(), s.Hkv, s.B);
+  const float isd = 1.0f / sqrtf((float)s.d);
+  cudaError_t e;
+  if (s.bf16) {
+    auto kern = select_kernel<__nv_bfloat16>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk,
+                                  s.topk, isd, idx, scores);
+  } else {
+    auto kern = select_kernel<float>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    kern<<<grid, 256, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk, s.topk,
+                                  isd, idx, scores);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st) {
+  const int rows = s.B * s.S * s.Hq;
+  const int grid = (rows + 7) / 8;
+  if (s.bf16)
+    preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                           static_cast<const __nv_bfloat16*>(d_o), s.S, s.Hq, s.d,
+                                                           rows, Dr);
+  else
+    preprocess_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(o), static_cast<const float*>(d_o), s.S,
+                                                   s.Hq, s.d, rows, Dr);
+  return cudaGetLastError();
+}
+
+}  // namespace hga

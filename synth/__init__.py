@@ -87,10 +87,14 @@ def round_f32(x: np.ndarray) -> np.ndarray:
 
 def f32_to_bf16_bits(x32: np.ndarray) -> np.ndarray:
     """float32 -> bfloat16 bit patterns (uint16), round to nearest even.
-    Inputs are finite by construction."""
-    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = u + 0x7FFF + ((u >> 16) & 1)
-    return (u >> 16).astype(np.uint16)
+    Inputs are finite by construction, so the 32-bit sum cannot overflow
+    (the largest finite pattern is 0xFF7FFFFF)."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32)
+    r = (u >> 16) & 1
+    r += 0x7FFF
+    r += u
+    r >>= 16
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:

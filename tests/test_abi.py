@@ -1,0 +1,113 @@
+"""The C ABI library: it loads without a GPU, exports every entry point that
+include/*.h declares, and rejects bad arguments on the host before any CUDA
+call."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from segmented_fine_tuning_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        for m in re.finditer(r"^\s*(?:HGA_API\s+)?(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+(hga_[a-z0-9_]+)\s*\(", txt, re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from segmented_fine_tuning_b200 import build
+    build.build()
+    return _binding.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 11, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_binding_covers_every_symbol():
+    bound = {n for n, _, _ in _binding._SIGNATURES}
+    assert set(_declared_functions()) <= bound
+
+
+def test_status_strings(lib):
+    for code, name in _binding.STATUS_NAMES.items():
+        assert lib.hga_status_string(code).decode() == name
+
+
+def _dims(**kw):
+    base = dict(B=1, Hq=4, Hkv=2, d=128, block=128, S=256, n_hist_blocks=4, topk=2, dtype=1)
+    base.update(kw)
+    return _binding.hga_dims(**base)
+
+
+BAD_DIMS = [
+    dict(Hq=3),          # Hq % Hkv
+    dict(d=96),          # head dim
+    dict(block=48),      # block size
+    dict(S=200),         # S % block
+    dict(topk=0),        # K >= 1
+    dict(topk=65),       # K <= 64
+    dict(B=0),
+    dict(n_hist_blocks=-1),
+]
+
+
+@pytest.mark.parametrize("kw", BAD_DIMS)
+def test_bad_shapes_rejected_on_host(lib, kw):
+    d = _dims(**kw)
+    p = ctypes.c_void_p(16)
+    st = lib.hga_attn_fwd(ctypes.byref(d), p, p, p, p, p, 4, p, p, p, None)
+    assert st == 2, (kw, st, lib.hga_last_error())
+    assert lib.hga_last_error()
+
+
+def test_null_and_invalid_arguments(lib):
+    d = _dims()
+    p = ctypes.c_void_p(16)
+    assert lib.hga_attn_fwd(None, p, p, p, p, p, 4, p, p, p, None) == 1
+    assert lib.hga_attn_fwd(ctypes.byref(d), None, p, p, p, p, 4, p, p, p, None) == 1
+    assert lib.hga_attn_fwd(ctypes.byref(d), p, p, p, None, p, 4, p, p, p, None) == 1   # history missing
+    assert lib.hga_attn_fwd(ctypes.byref(d), ctypes.c_void_p(18), p, p, p, p, 4, p, p, p, None) == 1  # misaligned
+    assert lib.hga_block_summaries(ctypes.byref(d), p, 0, 9, p, None) == 1   # range past n_hist_blocks
+    assert lib.hga_block_summaries(ctypes.byref(d), p, 3, 1, p, None) == 1
+    assert lib.hga_select_topk(ctypes.byref(_dims(n_hist_blocks=5000)), p, p, p, None, None) == 2
+    # workspace too small
+    ws = lib.hga_attn_bwd_workspace_size(ctypes.byref(d))
+    assert ws >= 4 * 4 * 256 and ws % 256 == 0
+    assert lib.hga_attn_bwd(ctypes.byref(d), p, p, p, p, p, 4, p, p, p, p, p, p, p, ctypes.c_void_p(256), ws - 1,
+                            None) == 1
+    assert lib.hga_selftest_umma(7, p, p, p, None) == 1
+    assert lib.hga_offload_segment(ctypes.byref(d), p, p, p, p, 4, 3, None) == 1  # 2 blocks at 3 > capacity 4
+
+
+def test_binding_rejects_wrong_shapes():
+    import torch
+    D = _binding.Dims(1, 4, 2, 128, 128, 256, 4, 2, "bf16")
+    q = torch.zeros((1, 256, 4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        _binding.hga_attn_fwd(D, q, q, q, q, q, 4, q, q, q)
+
+
+def test_oracle_and_library_share_nothing():
+    """The CUDA sources and the oracle neither include nor import each other."""
+    csrc = glob.glob(os.path.join(ROOT, "segmented_fine_tuning_b200", "**", "*"), recursive=True)
+    for f in csrc:
+        if f.endswith((".cu", ".cuh", ".h", ".py")):
+            txt = open(f).read()
+            assert "oracle" not in re.sub(r"#.*|//.*", "", txt).lower() or f.endswith("build.py"), f
+    for f in glob.glob(os.path.join(ROOT, "oracle", "*")):
+        if f.endswith((".c", ".h", ".py")):
+            assert "segmented_fine_tuning_b200" not in open(f).read(), f

@@ -1,0 +1,260 @@
+"""GPU parity: every kernel of the HGA step through the C ABI against the fp64
+oracle, on the seeded synthetic workloads and on edge cases.
+
+Tolerances: selection bit-exact except at oracle near-ties (K-th vs (K+1)-th
+score closer than 1e-3 relative; the alternative must still be a valid top-K);
+fp32 workloads max abs 1e-4; bf16 workloads max abs 2e-2 and relative L2 1e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from hga_testutil import (BF16_ABS, BF16_REL, F32_ABS, assert_close, check_selection, dims_of, to_dev, to_host)
+from segmented_fine_tuning_b200 import (Dims, HgaError, hga_attn_fwd, hga_block_summaries, hga_device_status,
+                                        hga_select_topk, hga_selftest_umma)
+from segmented_fine_tuning_b200.step import AttentionStep
+
+pytestmark = pytest.mark.gpu
+
+
+def _odims(w: synth.Workload, nblk=None):
+    return oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk if nblk is None else nblk, w.topk)
+
+
+def _tols(w):
+    return (F32_ABS, None) if w.dtype == "f32" else (BF16_ABS, BF16_REL)
+
+
+def _gpu_step(w: synth.Workload, x: synth.Inputs, backward=True):
+    D = dims_of(w)
+    dev = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    st = AttentionStep(D)
+    st.select(dev["q"], dev["k_hist"])
+    st.forward(dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"])
+    if backward:
+        st.backward(dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], dev["d_o"])
+    torch.cuda.synchronize()
+    hga_device_status()
+    return st, dev
+
+
+# ------------------------------------------------------------------ tensor-core operand layouts
+
+@pytest.mark.parametrize("form", [0, 1, 2, 3])
+def test_selftest_umma_forms(form):
+    g = torch.Generator().manual_seed(form)
+    a = torch.randn(128, 128, generator=g).to(torch.bfloat16)
+    b = torch.randn(128, 128, generator=g).to(torch.bfloat16)
+    d = torch.zeros(128, 128, dtype=torch.float32, device="cuda")
+    hga_selftest_umma(form, a.cuda(), b.cuda(), d)
+    torch.cuda.synchronize()
+    hga_device_status()
+    A, Bm = a.double(), b.double()
+    want = A @ Bm.T if form in (0, 3) else A @ Bm
+    err = (d.cpu().double() - want).abs().max().item()
+    assert err < 1e-3, f"form {form}: max abs err {err}"
+
+
+# ------------------------------------------------------------------ summaries and selection
+
+SEL_CASES = [
+    synth.TINY_F32,
+    synth.Workload("small-bf16-G4", 1, 8, 2, 128, 128, 512, 9, 3, "bf16", 21, structured_keys=True),
+    synth.Workload("d64-bf16-blk64-G1", 2, 3, 3, 64, 64, 256, 7, 5, "bf16", 22),
+    synth.Workload("k-exceeds-history", 1, 4, 2, 128, 128, 256, 3, 8, "bf16", 23),
+    synth.QWEN3_8B_LAYER,
+    synth.PREFILL_131K,
+]
+
+
+@pytest.mark.parametrize("w", SEL_CASES, ids=lambda w: w.name.split(":")[0])
+def test_summaries_and_selection(w):
+    x = synth.draw(w)
+    D = dims_of(w)
+    q, kh = to_dev(x.q), to_dev(x.k_hist)
+    summ = torch.zeros((w.B, w.Hkv, w.nblk, w.d), dtype=torch.float32, device="cuda")
+    idx = torch.empty((w.B, w.Hkv, w.nqb, w.topk), dtype=torch.int32, device="cuda")
+    scores = torch.empty(idx.shape, dtype=torch.float32, device="cuda")
+    hga_block_summaries(D, kh, 0, w.nblk, summ)
+    hga_select_topk(D, q, summ, idx, scores)
+    torch.cuda.synchronize()
+    od = _odims(w)
+    summ_ref = oracle.block_summaries(od, x.k_hist.f64)
+    s = to_host(summ)
+    assert np.abs(s - summ_ref).max() <= 1e-6 * max(1.0, np.abs(summ_ref).max())
+    idx_ref, score_ref = oracle.select(od, x.q.f64, x.k_hist.f64)
+    near = oracle.near_tie_positions(od, score_ref)
+    n_acc = check_selection(D, idx.cpu().numpy(), idx_ref, score_ref, near)
+    print(f"{w.name}: near-tie positions {int(near.sum())}, accepted differences {n_acc}")
+    # the reported scores are the selected blocks' scores
+    sg = scores.cpu().numpy()
+    ig = idx.cpu().numpy()
+    ref_sel = np.take_along_axis(score_ref, np.maximum(ig, 0), axis=-1)
+    ok = ig >= 0
+    assert np.abs(sg[ok] - ref_sel[ok]).max() <= 1e-4 * max(1.0, np.abs(score_ref).max())
+    assert np.all(np.isneginf(sg[~ok]))
+
+
+def test_summaries_partial_range_leaves_rest():
+    w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 6, 2, "bf16", 24)
+    x = synth.draw(w)
+    D = dims_of(w)
+    summ = torch.full((1, 2, 6, 128), 7.0, device="cuda")
+    hga_block_summaries(D, to_dev(x.k_hist), 2, 4, summ)
+    torch.cuda.synchronize()
+    s = summ.cpu().numpy()
+    ref = oracle.block_summaries(_odims(w), x.k_hist.f64)
+    assert np.all(s[:, :, [0, 1, 4, 5]] == 7.0)
+    assert np.abs(s[:, :, 2:4] - ref[:, :, 2:4]).max() < 1e-6
+
+
+def test_select_q_zero_tie_rule():
+    """Q = 0: every score is exactly 0; the tie rule picks blocks 0..K-1."""
+    w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 10, 4, "bf16", 25)
+    x = synth.draw(w)
+    D = dims_of(w)
+    q = torch.zeros((1, 256, 4, 128), dtype=torch.bfloat16, device="cuda")
+    summ = torch.empty((1, 2, 10, 128), device="cuda")
+    idx = torch.empty((1, 2, 2, 4), dtype=torch.int32, device="cuda")
+    hga_block_summaries(D, to_dev(x.k_hist), 0, 10, summ)
+    hga_select_topk(D, q, summ, idx)
+    torch.cuda.synchronize()
+    assert np.all(idx.cpu().numpy() == np.arange(4))
+
+
+# ------------------------------------------------------------------ attention forward + backward
+
+ATTN_CASES = [
+    synth.TINY_F32,                                                                              # fp32, SIMT
+    synth.Workload("tc-small: Hq4/Hkv2 S384 hist5 K3", 1, 4, 2, 128, 128, 384, 5, 3, "bf16", 31),
+    synth.Workload("tc-G2-B2: Hq4/Hkv2 S256 hist4 K2", 2, 4, 2, 128, 128, 256, 4, 2, "bf16", 32,
+                   structured_keys=True),
+    synth.Workload("tc-no-history: S512", 1, 4, 1, 128, 128, 512, 0, 4, "bf16", 33),
+    synth.Workload("tc-K>hist: hist2 K5", 1, 8, 2, 128, 128, 256, 2, 5, "bf16", 34),
+    synth.Workload("tc-K1: hist6 K1", 1, 4, 2, 128, 128, 256, 6, 1, "bf16", 35),
+    synth.Workload("simt-bf16-d64-blk64-G3", 1, 6, 2, 64, 64, 192, 5, 2, "bf16", 36),
+    synth.Workload("simt-f32-d128-blk32", 1, 2, 2, 128, 32, 96, 6, 3, "f32", 37),
+]
+
+
+@pytest.mark.parametrize("w", ATTN_CASES, ids=lambda w: w.name.split(":")[0])
+def test_attention_small(w):
+    x = synth.draw(w)
+    st, _ = _gpu_step(w, x)
+    od = _odims(w)
+    idx_ref, score_ref = oracle.select(od, x.q.f64, x.k_hist.f64)
+    idx = st.idx.cpu().numpy()
+    check_selection(dims_of(w), idx, idx_ref, score_ref, oracle.near_tie_positions(od, score_ref))
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
+    o_ref, lse_ref = oracle.attn_fwd(od, *args)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(od, *args, x.d_o.f64)
+    ma, rl = _tols(w)
+    assert_close("O", to_host(st.o), o_ref, ma, rl)
+    assert_close("LSE", to_host(st.lse), lse_ref, ma, rl)
+    assert_close("dQ", to_host(st.dq), dq_ref, ma, rl)
+    assert_close("dK", to_host(st.dk), dk_ref, ma, rl)
+    assert_close("dV", to_host(st.dv), dv_ref, ma, rl)
+
+
+def test_dense_equivalence_full():
+    """K = every history block: HGA equals dense causal attention; checked
+    against the oracle's own dense path too, at full size."""
+    w = synth.DENSE_EQUIV
+    x = synth.draw(w)
+    st, _ = _gpu_step(w, x)
+    idx = st.idx.cpu().numpy()
+    assert np.all(idx == np.arange(w.nblk))
+    od = _odims(w)
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
+    o_ref, lse_ref = oracle.attn_fwd(od, *args)
+    assert_close("O", to_host(st.o), o_ref, BF16_ABS, BF16_REL)
+    assert_close("LSE", to_host(st.lse), lse_ref, BF16_ABS, BF16_REL)
+    # dense identity on sampled rows
+    H = w.nblk * w.blk
+    qf = np.concatenate([np.zeros((1, H, w.Hq, w.d)), x.q.f64], 1)
+    kf = np.concatenate([x.k_hist.f64, x.k_seg.f64], 1)
+    vf = np.concatenate([x.v_hist.f64, x.v_seg.f64], 1)
+    o_dense, _ = oracle.dense_causal_fwd(qf[:, :, :4], kf[:, :, :1], vf[:, :, :1])
+    assert_close("O vs dense (head group 0)", to_host(st.o)[:, :, :4], o_dense[:, H:], BF16_ABS, BF16_REL)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(od, *args, x.d_o.f64)
+    assert_close("dQ", to_host(st.dq), dq_ref, BF16_ABS, BF16_REL)
+    assert_close("dK", to_host(st.dk), dk_ref, BF16_ABS, BF16_REL)
+    assert_close("dV", to_host(st.dv), dv_ref, BF16_ABS, BF16_REL)
+
+
+def test_qwen3_8b_layer_sampled():
+    """Full-size Qwen3-8B-shaped layer (the benchmark launch): selection over
+    all heads; O/LSE/dQ/dK/dV for KV heads 0 and 7 (all their query heads)."""
+    w = synth.QWEN3_8B_LAYER
+    x = synth.draw(w)
+    st, _ = _gpu_step(w, x)
+    od = _odims(w)
+    idx_ref, score_ref = oracle.select(od, x.q.f64, x.k_hist.f64)
+    idx = st.idx.cpu().numpy()
+    check_selection(dims_of(w), idx, idx_ref, score_ref, oracle.near_tie_positions(od, score_ref))
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
+    for h in (0, 7):
+        o_ref, lse_ref = oracle.attn_fwd(od, *args, kv_heads=range(h, h + 1))
+        dq_ref, dk_ref, dv_ref = oracle.attn_bwd(od, *args, x.d_o.f64, kv_heads=range(h, h + 1))
+        hs = slice(4 * h, 4 * h + 4)
+        assert_close(f"O h{h}", to_host(st.o)[:, :, hs], o_ref[:, :, hs], BF16_ABS, BF16_REL)
+        assert_close(f"LSE h{h}", to_host(st.lse)[:, hs], lse_ref[:, hs], BF16_ABS, BF16_REL)
+        assert_close(f"dQ h{h}", to_host(st.dq)[:, :, hs], dq_ref[:, :, hs], BF16_ABS, BF16_REL)
+        assert_close(f"dK h{h}", to_host(st.dk)[:, :, h], dk_ref[:, :, h], BF16_ABS, BF16_REL)
+        assert_close(f"dV h{h}", to_host(st.dv)[:, :, h], dv_ref[:, :, h], BF16_ABS, BF16_REL)
+
+
+def test_prefill_131k_sampled():
+    """131K-token prefill, forward only: selection over all heads; O/LSE of two
+    rows per query block for KV heads 0 and 5."""
+    w = synth.PREFILL_131K
+    x = synth.draw(w)
+    st, _ = _gpu_step(w, x, backward=False)
+    od = _odims(w)
+    idx_ref, score_ref = oracle.select(od, x.q.f64, x.k_hist.f64)
+    idx = st.idx.cpu().numpy()
+    check_selection(dims_of(w), idx, idx_ref, score_ref, oracle.near_tie_positions(od, score_ref))
+    rows = sorted({i * w.blk + r for i in range(w.nqb) for r in (0, 127 - (i % 7) * 9)})
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
+    for h in (0, 5):
+        o_ref, lse_ref = oracle.attn_fwd(od, *args, kv_heads=range(h, h + 1), rows=rows)
+        hs = slice(4 * h, 4 * h + 4)
+        assert_close(f"O h{h}", to_host(st.o)[:, rows][:, :, hs], o_ref[:, rows][:, :, hs], BF16_ABS, BF16_REL)
+        assert_close(f"LSE h{h}", to_host(st.lse)[:, hs][:, :, rows], lse_ref[:, hs][:, :, rows], BF16_ABS,
+                     BF16_REL)
+
+
+def test_out_of_range_index_is_flagged_not_faulted():
+    """A bad block index in idx is skipped by the kernels and reported."""
+    w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 4, 2, "bf16", 38)
+    x = synth.draw(w)
+    D = dims_of(w)
+    dev = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist")}
+    idx = torch.tensor([0, 9], dtype=torch.int32).repeat(1, 2, 2, 1).contiguous().cuda()
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((1, 4, 256), device="cuda")
+    hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], 4, idx, o, lse)
+    with pytest.raises(HgaError) as ei:
+        hga_device_status()
+    assert ei.value.status == 4
+    hga_device_status()  # flag cleared
+    # the valid part was still computed: equals attention with idx [0, -1]
+    idx2 = torch.tensor([0, -1], dtype=torch.int32).repeat(1, 2, 2, 1).contiguous().cuda()
+    o2 = torch.empty_like(o)
+    lse2 = torch.empty_like(lse)
+    hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], 4, idx2, o2, lse2)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
+def test_repeat_runs_bit_identical_forward():
+    w = synth.Workload("t", 1, 8, 2, 128, 128, 512, 6, 3, "bf16", 39, structured_keys=True)
+    x = synth.draw(w)
+    st1, dev = _gpu_step(w, x, backward=False)
+    o1, lse1, idx1 = st1.o.clone(), st1.lse.clone(), st1.idx.clone()
+    st1.select(dev["q"], dev["k_hist"])
+    st1.forward(dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"])
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, st1.idx) and torch.equal(o1, st1.o) and torch.equal(lse1, st1.lse)

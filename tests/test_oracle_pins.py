@@ -269,6 +269,10 @@ def test_kv_head_subset_is_exact_restriction():
     o1, lse1 = oracle.attn_fwd(D, q, ks, vs, kh, vh, idx, kv_heads=range(1, 2))
     np.testing.assert_array_equal(o1[:, :, 2:], o[:, :, 2:])
     assert np.all(np.isnan(o1[:, :, :2]))
+    o2, lse2 = oracle.attn_fwd(D, q, ks, vs, kh, vh, idx, rows=[0, 5, 7])
+    np.testing.assert_array_equal(o2[:, [0, 5, 7]], o[:, [0, 5, 7]])
+    np.testing.assert_array_equal(lse2[:, :, [0, 5, 7]], lse[:, :, [0, 5, 7]])
+    assert np.all(np.isnan(o2[:, [1, 2, 3, 4, 6]]))
     g = oracle.attn_bwd(D, q, ks, vs, kh, vh, idx, do)
     g1 = oracle.attn_bwd(D, q, ks, vs, kh, vh, idx, do, kv_heads=range(1, 2))
     np.testing.assert_array_equal(g1[0][:, :, 2:], g[0][:, :, 2:])
