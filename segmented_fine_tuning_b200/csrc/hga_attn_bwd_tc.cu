@@ -229,7 +229,8 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     uint32_t sv[32], dv[32];
     for (int j = 0; j < nt; ++j) {
-      if (!mbar_wait(&ctl->sdp_full, j & 1, abort, a.err)) {
+      // tcgen05.ld/st are warp-collective: branches around them are warp-uniform.
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full, j & 1, abort, a.err))) {
         ok = false;
         break;
       }
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(&ctl->ds_full);
     }
-    if (ok && mbar_wait(&ctl->dq_full, 0, abort, a.err)) {
+    if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dq_full, 0, abort, a.err))) {
       tc_fence_after();
       float* out = a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + 64 * e;
 #pragma unroll
@@ -425,7 +426,10 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t sv[32], dv[32];
     for (int it = 0; it < n; ++it) {
       const int s = it % kQStages;
-      if (!mbar_wait(&ctl->sdp_full, it & 1, abort, a.err)) {
+      // The row statistics arrive with the Q/dO stage: observe that stage's
+      // barrier directly (its phase is complete by now) before reading them.
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full, it & 1, abort, a.err) &&
+                                       mbar_wait(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err))) {
         ok = false;
         break;
       }
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(&ctl->pds_full);
     }
-    if (ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err)) {
+    if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err))) {
       tc_fence_after();
       const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + 64 * e;
 #pragma unroll

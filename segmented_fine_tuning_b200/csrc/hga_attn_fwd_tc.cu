@@ -250,7 +250,9 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     uint32_t v[32];
     for (int j = 0; j < nt; ++j) {
-      if (!mbar_wait(&ctl->s_full[t], j & 1, abort, a.err)) {
+      // tcgen05.ld/st are warp-collective: every branch around them is
+      // decided for the whole warp.
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[t], j & 1, abort, a.err))) {
         ok = false;
         break;
       }
@@ -265,8 +267,10 @@ __global__ void __launch_bounds__(384, 1)
           if (!diag || c * 32 + e <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
       }
       mx *= sl2;
-      if (mx > m_ref + kRescaleThreshold) {
-        const float alpha = ex2_approx(m_ref - mx);
+      const bool need = mx > m_ref + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, need)) {
+        // Rows that keep their reference use alpha = 1.
+        const float alpha = need ? ex2_approx(m_ref - mx) : 1.0f;
         l *= alpha;
         if (j > 0) {
 #pragma unroll
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(384, 1)
             HGA_TMEM_ST32(tO + c * 32, v);
           }
         }
-        m_ref = mx;
+        if (need) m_ref = mx;
       }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(&ctl->p_full[t]);
     }
-    if (ok && mbar_wait(&ctl->o_full[t], 0, abort, a.err)) {
+    if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->o_full[t], 0, abort, a.err))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const int p = i * kBM + r;

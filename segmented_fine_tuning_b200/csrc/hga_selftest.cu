@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(160, 1) selftest_umma_kernel(const __grid_cons
   }
   if (warp < 4) {
     volatile int no_abort = 0;
-    if (mbar_wait(&ctl->done, 0, &no_abort, err)) {
+    if (__all_sync(0xffffffffu, mbar_wait(&ctl->done, 0, &no_abort, err))) {
       tc_fence_after();
       const int r = warp * 32 + lane;
       uint32_t v[32];

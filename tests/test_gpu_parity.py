@@ -158,6 +158,33 @@ def test_attention_small(w):
     assert_close("dV", to_host(st.dv), dv_ref, ma, rl)
 
 
+def test_rescale_rows_diverge():
+    """A history block late in the tile list dominates only the even query
+    rows: their running maximum jumps mid-way (the O rescale path) while the
+    odd rows of the same warps keep theirs."""
+    w = synth.Workload("rescale: Hq2/Hkv1 S256 hist4 K2", 1, 2, 1, 128, 128, 256, 4, 2, "bf16", 40)
+    x = synth.draw(w)
+    q = x.q.f64.copy()
+    kh = x.k_hist.f64.copy()
+    q[:, ::2, :, :] = 0.0
+    q[:, ::2, :, 0] = 10.0          # even rows: q = 10 e0
+    kh[:, 3 * 128:4 * 128, :, 0] = 10.0  # block 3 keys: k0 = 10 -> logit ~8.8 nats for even rows
+    x.q = synth._store(q, "bf16")
+    x.k_hist = synth._store(kh, "bf16")
+    st, _ = _gpu_step(w, x)
+    idx = st.idx.cpu().numpy()
+    assert np.all(idx[..., 1] == 3) and np.all(idx[..., 0] < 3)
+    od = _odims(w)
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
+    o_ref, lse_ref = oracle.attn_fwd(od, *args)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(od, *args, x.d_o.f64)
+    assert_close("O", to_host(st.o), o_ref, BF16_ABS, BF16_REL)
+    assert_close("LSE", to_host(st.lse), lse_ref, BF16_ABS, BF16_REL)
+    assert_close("dQ", to_host(st.dq), dq_ref, BF16_ABS, BF16_REL)
+    assert_close("dK", to_host(st.dk), dk_ref, BF16_ABS, BF16_REL)
+    assert_close("dV", to_host(st.dv), dv_ref, BF16_ABS, BF16_REL)
+
+
 def test_dense_equivalence_full():
     """K = every history block: HGA equals dense causal attention; checked
     against the oracle's own dense path too, at full size."""
