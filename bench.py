@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the HGA per-segment attention step on B200.
+
+Workload: one Qwen3-8B-shaped attention layer in bf16 -- 32 query / 8 KV
+heads, d = 128, history 14,336 tokens (112 blocks of 128), active segment
+2,048 tokens (16 query blocks), top-K = 16 -- with seeded synthetic inputs.
+One step = every kernel of the hot path over that layer: block summaries,
+top-K selection, attention forward, backward preprocess, dK/dV, dQ.
+
+Metric: attention fwd+bwd tokens/s per layer (segment tokens / step time),
+summed over the GPUs (each GPU runs its own independent layer: replicas).
+Timing: CUDA events on the launching stream around every kernel; L2 is
+flushed (256 MiB write) between steps, outside the timed events.
+
+Extra keys: roofline of the dominant kernel, per-kernel breakdown, e2e
+(the same step through the public API with host buffers: pinned H2D of the
+segment's inputs, history blocks fetched from a pinned host tier by
+hga_fetch_blocks, D2H of the per-row log-sum-exp), cpu_baseline (the fp64
+oracle on a bounded sample, on this host's cores), and SM clocks sampled
+during the timed region.
+
+--impl reference times the fp64 CPU oracle (the reference arm) on the same
+workload: each step is a bounded sample (selection for every head, forward
+and backward for one KV head), scaled to the metric's unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "HGA attn fwd+bwd tokens/s per layer on 1 B200; % of bf16 tensor peak / HBM BW"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ("summaries", "select", "fwd", "bwd_pre", "bwd_dkdv", "bwd_dq")
+KERNEL_SOURCES = {"fwd": "hga_attn_fwd_tc.cu", "bwd_dq": "hga_attn_bwd_tc.cu", "bwd_dkdv": "hga_attn_bwd_tc.cu",
+                  "summaries": "hga_select.cu", "select": "hga_select.cu", "bwd_pre": "hga_select.cu"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload_config(w: synth.Workload, l2_note: str):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "block": w.blk,
+            "segment_tokens": w.S, "history_blocks": w.nblk, "topk": w.topk, "l2": l2_note}
+
+
+# ---------------------------------------------------------------- work model
+
+def work_model(w: synth.Workload, keff_sum_per_head: float):
+    """Algorithmic work of one step.  Attention counts only the (query, key)
+    pairs the method computes: per query head, history pairs = sum over query
+    rows of K_eff*block, segment pairs = S(S+1)/2.  Forward 4d FLOP per pair;
+    backward 4d per history pair (dP, dQ) and 8d per segment pair (dP, dQ, dK,
+    dV); of those, the dQ kernel does dP and dQ for every pair, the dK/dV
+    kernel dK and dV for segment pairs."""
+    d = w.d
+    hist_pairs = keff_sum_per_head * w.blk * w.blk  # per head: sum_i K_eff(i) * blk rows * blk keys
+    seg_pairs = w.S * (w.S + 1) / 2
+    H = w.Hq * w.B
+    flops = {
+        "fwd": 4 * d * (hist_pairs + seg_pairs) * H,
+        "bwd_dq": 4 * d * (hist_pairs + seg_pairs) * H,
+        "bwd_dkdv": 4 * d * seg_pairs * H,
+    }
+    es = 2 if w.dtype == "bf16" else 4
+    bytes_ = {
+        "summaries": w.B * w.nblk * w.blk * w.Hkv * d * es + w.B * w.Hkv * w.nblk * d * 4,
+        "select": w.B * w.S * w.Hq * d * es + w.B * w.Hkv * w.nblk * d * 4 + w.B * w.Hkv * w.nqb * w.topk * 4,
+        "bwd_pre": 2 * w.B * w.S * w.Hq * d * es + w.B * w.Hq * w.S * 4,
+    }
+    return flops, bytes_
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML unavailable: report no clocks
+            self._nvml = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nvml:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def to_dev(t: synth.Tensor, device):
+    if t.dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(t.store).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(t.store)).to(device)
+
+
+def to_pinned(t: synth.Tensor):
+    if t.dtype == "bf16":
+        x = torch.from_numpy(np.ascontiguousarray(t.store).view(np.int16)).view(torch.bfloat16)
+    else:
+        x = torch.from_numpy(np.ascontiguousarray(t.store))
+    return x.pin_memory()
+
+
+def source_sha(fname: str) -> str:
+    with open(os.path.join(ROOT, "segmented_fine_tuning_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when
+    the kernel's source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_sha") != source_sha(KERNEL_SOURCES[kernel]):
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- device leg
+
+def run_device(args, rank, world, device):
+    import segmented_fine_tuning_b200 as hga
+    from segmented_fine_tuning_b200.step import AttentionStep
+
+    w = synth.QWEN3_8B_LAYER
+    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
+    x = synth.draw(w)
+    dev = {n: to_dev(getattr(x, n), device) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    st = AttentionStep(D, device)
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def step(evs=None):
+        def mark(k):
+            if evs is not None:
+                evs[k].record(stream)
+        mark(0)
+        hga.hga_block_summaries(D, dev["k_hist"], 0, D.n_hist_blocks, st.summ, stream)
+        mark(1)
+        hga.hga_select_topk(D, dev["q"], st.summ, st.idx, None, stream)
+        mark(2)
+        hga.hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], D.n_hist_blocks,
+                         st.idx, st.o, st.lse, stream)
+        mark(3)
+        hga.hga_attn_bwd_preprocess(D, st.o, dev["d_o"], st.ws, stream)
+        mark(4)
+        hga.hga_attn_bwd_dkdv(D, dev["q"], dev["k_seg"], dev["v_seg"], st.lse, dev["d_o"], st.ws, st.dk, st.dv,
+                              stream)
+        mark(5)
+        hga.hga_attn_bwd_dq(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"],
+                            D.n_hist_blocks, st.idx, st.lse, dev["d_o"], st.ws, st.dq, stream)
+        mark(6)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    hga.hga_device_status(stream)
+    keff_sum = float((st.idx >= 0).sum().item()) / (w.B * w.Hkv)  # sum over query blocks, per KV head
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            step(evs[k])
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    hga.hga_device_status(stream)
+
+    per_kernel = {name: [] for name in KERNELS}
+    step_ms = []
+    for e in evs:
+        step_ms.append(e[0].elapsed_time(e[6]))
+        for j, name in enumerate(KERNELS):
+            per_kernel[name].append(e[j].elapsed_time(e[j + 1]))
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * w.S / (ms_per_step / 1e3)
+
+    peaks, peak_src = load_peaks()
+    flops, bytes_ = work_model(w, keff_sum)
+    kern = {}
+    for name in KERNELS:
+        ms = float(np.mean(per_kernel[name]))
+        entry = {"ms": round(ms, 4)}
+        if name in flops:
+            tf = flops[name] / (ms / 1e3) / 1e12
+            entry.update({"tflops": round(tf, 1), "frac_bf16_peak": round(tf / peaks["bf16_tflops"], 3)})
+        if name in bytes_:
+            gbs = bytes_[name] / (ms / 1e3) / 1e9
+            entry.update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)})
+        kern[name] = entry
+    dom = max(("fwd", "bwd_dq", "bwd_dkdv"), key=lambda n: kern[n]["ms"])
+    dom_ms = kern[dom]["ms"]
+    achieved = flops[dom] / (dom_ms / 1e3) / 1e12
+    traffic = committed_traffic(dom)
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+                "peak_source": f"{peak_src} dense bf16 (burst)",
+                "algorithmic_flop_per_launch": flops[dom]}
+    fwd_bwd_flops = flops["fwd"] + flops["bwd_dq"] + flops["bwd_dkdv"]
+    attn_ms = kern["fwd"]["ms"] + kern["bwd_dq"]["ms"] + kern["bwd_dkdv"]["ms"]
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); block-structured keys)",
+        "config": workload_config(w, "flushed between steps (256 MiB write, outside the timed events)"),
+        "roofline": roofline,
+        "attention_fwd_bwd": {"tflops": round(fwd_bwd_flops / (attn_ms / 1e3) / 1e12, 1),
+                              "frac_bf16_peak": round(fwd_bwd_flops / (attn_ms / 1e3) / 1e12 /
+                                                      peaks["bf16_tflops"], 3),
+                              "algorithmic_gflop": round(fwd_bwd_flops / 1e9, 2)},
+        "kernels": kern,
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+    }
+    return out, (w, x, D, dev, st)
+
+
+def run_e2e(args, ctx, device):
+    """The same step through the public API with host buffers: the segment's
+    Q, K, V, dO copied from pinned host memory, the selected history blocks
+    fetched from a pinned host tier, and the per-row log-sum-exp read back."""
+    import segmented_fine_tuning_b200 as hga
+    w, x, D, dev, st = ctx
+    stream = torch.cuda.current_stream(device)
+    copy_stream = torch.cuda.Stream(device)
+    host = {n: to_pinned(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "d_o")}
+    tier_k, tier_v = to_pinned(x.k_hist), to_pinned(x.v_hist)
+    idx_scratch = torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory()
+    lse_host = torch.empty(tuple(st.lse.shape), dtype=torch.float32).pin_memory()
+    pool_k = torch.empty_like(dev["k_hist"])
+    pool_v = torch.empty_like(dev["v_hist"])
+    idx_pool = torch.empty_like(st.idx)
+    # the history's summaries are resident on the device (computed once, when
+    # the blocks entered the history)
+    hga.hga_block_summaries(D, dev["k_hist"], 0, D.n_hist_blocks, st.summ, stream)
+    seg = {n: torch.empty_like(dev[n]) for n in host}
+    done = torch.cuda.Event()
+    done.record(copy_stream)  # materialise the event handle
+    blk_bytes = w.blk * w.Hkv * w.d * 2 * 2  # K and V of one block
+    fetched = []
+
+    def step():
+        for n in host:
+            seg[n].copy_(host[n], non_blocking=True)
+        hga.hga_select_topk(D, seg["q"], st.summ, st.idx, None, stream)
+        nu = hga.hga_fetch_blocks(D, tier_k, tier_v, D.n_hist_blocks, st.idx, idx_scratch, pool_k, pool_v,
+                                  D.n_hist_blocks, idx_pool, stream, copy_stream, done)
+        fetched.append(nu)
+        stream.wait_event(done)
+        hga.hga_attn_fwd(D, seg["q"], seg["k_seg"], seg["v_seg"], pool_k, pool_v, D.n_hist_blocks, idx_pool, st.o,
+                         st.lse, stream)
+        hga.hga_attn_bwd(D, seg["q"], seg["k_seg"], seg["v_seg"], pool_k, pool_v, D.n_hist_blocks, idx_pool, st.o,
+                         st.lse, seg["d_o"], st.dq, st.dk, st.dv, st.ws, stream)
+        lse_host.copy_(st.lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    fetched.clear()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = args.steps
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    hga.hga_device_status(stream)
+    ms = e0.elapsed_time(e1) / n
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + np.mean(fetched) * blk_bytes \
+        + idx_pool.numel() * 4
+    d2h = idx_scratch.numel() * 4 + lse_host.numel() * 4
+    return {"value": round(w.S / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "fetched_blocks_per_step": float(np.mean(fetched)), "path": "pinned host tier + hga_fetch_blocks"}
+
+
+# ---------------------------------------------------------------- oracle legs
+
+def oracle_sample(w: synth.Workload, x, kv_heads):
+    """One bounded sample of the workload on the fp64 oracle: selection for
+    every head, then forward and backward for the given KV heads."""
+    import oracle
+    od = oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk)
+    q, kh = x["q"], x["k_hist"]
+    idx, _ = oracle.select(od, q, kh)
+    args = (q, x["k_seg"], x["v_seg"], kh, x["v_hist"], idx)
+    oracle.attn_fwd(od, *args, kv_heads=kv_heads)
+    oracle.attn_bwd(od, *args, x["d_o"], kv_heads=kv_heads)
+
+
+def cpu_cores():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+
+
+def run_cpu_baseline(w, x_inputs, budget_s=12.0):
+    x = {n: getattr(x_inputs, n).f64 for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    t0 = time.perf_counter()
+    done = 0
+    while done < w.Hkv and (time.perf_counter() - t0) < budget_s:
+        oracle_sample(w, x, range(done, done + 1))
+        done += 1
+    el = time.perf_counter() - t0
+    return {"value": round(w.S * (done / w.Hkv) / el, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"fp64 oracle: selection for all heads + fwd and bwd for {done} of {w.Hkv} KV heads "
+                      f"({done * w.G} of {w.Hq} query heads) in {el:.1f} s, scaled to the full layer"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    w = synth.QWEN3_8B_LAYER
+    xi = synth.draw(w)
+    x = {n: getattr(xi, n).f64 for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    for _ in range(args.warmup):
+        oracle_sample(w, x, range(0, 1))
+    times = []
+    for k in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_sample(w, x, range(k % w.Hkv, k % w.Hkv + 1))
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    value = w.S * (1 / w.Hkv) / (ms / 1e3)
+    sample = (f"each step: fp64 oracle selection for all heads + fwd and bwd for 1 of {w.Hkv} KV heads "
+              f"(4 query heads), scaled to the full layer (x{w.Hkv})")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+            "config": workload_config(w, "n/a (CPU)"),
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("hga", "reference"), default="hga")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "hga":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    try:
+        out, ctx = run_device(args, rank, world, device)
+        if not args.no_e2e:
+            e2e = run_e2e(args, ctx, device)
+            if world > 1:
+                t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=device)
+                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+                e2e["ms_per_step"] = round(float(t.item()), 4)
+                e2e["value"] = round(world * ctx[0].S / (e2e["ms_per_step"] / 1e3), 1)
+            out["e2e"] = e2e
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = run_cpu_baseline(ctx[0], ctx[1])
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -181,6 +181,27 @@ HGA_API hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void*
                         size_t ws_bytes, hga_stream_t stream);
 
 /*
+ * The three stages of hga_attn_bwd as separate calls (same arguments, same
+ * results), for callers that schedule or time them individually.  ws is the
+ * same caller-owned scratch; its first B*Hq*S floats hold Dr = rowsum(dO * O)
+ * [B, Hq, S] between the stages.
+ *   hga_attn_bwd_preprocess: Dr from o and d_o.
+ *   hga_attn_bwd_dkdv:       dk_seg, dv_seg (fully overwritten), needs Dr.
+ *   hga_attn_bwd_dq:         dq (fully overwritten), needs Dr.
+ * dkdv and dq read only inputs and Dr, so they may run concurrently on two
+ * streams once the preprocess has completed.
+ */
+HGA_API hga_status hga_attn_bwd_preprocess(const hga_dims* dims, const void* o, const void* d_o, void* ws,
+                                           size_t ws_bytes, hga_stream_t stream);
+HGA_API hga_status hga_attn_bwd_dkdv(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                                     const float* lse, const void* d_o, const void* ws, size_t ws_bytes,
+                                     float* dk_seg, float* dv_seg, hga_stream_t stream);
+HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                                   const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx,
+                                   const float* lse, const void* d_o, const void* ws, size_t ws_bytes, float* dq,
+                                   hga_stream_t stream);
+
+/*
  * Targeted loading of the selected history (fr edition, Contexte: dynamic
  * loading of precise historical tokens per query block; Background: history
  * KV lives in system RAM).  host_k/host_v: pinned host memory (cudaHostAlloc)

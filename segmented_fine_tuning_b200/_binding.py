@@ -78,6 +78,9 @@ _SIGNATURES = [
     ("hga_attn_fwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     ("hga_attn_bwd_workspace_size", ctypes.c_size_t, [_D]),
     ("hga_attn_bwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("hga_attn_bwd_preprocess", _I, [_D, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("hga_attn_bwd_dkdv", _I, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P]),
+    ("hga_attn_bwd_dq", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     ("hga_fetch_blocks", _I, [_D, _P, _P, _I, _P, _P, _P, _P, _I, _P, ctypes.POINTER(ctypes.c_int), _P, _P, _P,
                               _I]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
@@ -198,6 +201,46 @@ def hga_attn_bwd(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, 
                                        _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq),
                                        _ptr(dk_seg), _ptr(dv_seg), _ptr(ws), ws.numel() * ws.element_size(),
                                        _stream(stream)), "hga_attn_bwd")
+
+
+def _ws(ws):
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous CUDA tensor")
+    return _ptr(ws), ws.numel() * ws.element_size()
+
+
+def hga_attn_bwd_preprocess(dims: Dims, o, d_o, ws, stream=None) -> None:
+    _expect(o, (dims.B, dims.S, dims.Hq, dims.d), dims.torch_dtype, "o")
+    _expect(d_o, o.shape, dims.torch_dtype, "d_o")
+    wp, wb = _ws(ws)
+    _check(load_library().hga_attn_bwd_preprocess(ctypes.byref(dims.c()), _ptr(o), _ptr(d_o), wp, wb,
+                                                  _stream(stream)), "hga_attn_bwd_preprocess")
+
+
+def hga_attn_bwd_dkdv(dims: Dims, q, k_seg, v_seg, lse, d_o, ws, dk_seg, dv_seg, stream=None) -> None:
+    _expect(q, (dims.B, dims.S, dims.Hq, dims.d), dims.torch_dtype, "q")
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(v_seg, k_seg.shape, dims.torch_dtype, "v_seg")
+    _expect(lse, (dims.B, dims.Hq, dims.S), torch.float32, "lse")
+    _expect(d_o, q.shape, dims.torch_dtype, "d_o")
+    _expect(dk_seg, k_seg.shape, torch.float32, "dk_seg")
+    _expect(dv_seg, k_seg.shape, torch.float32, "dv_seg")
+    wp, wb = _ws(ws)
+    _check(load_library().hga_attn_bwd_dkdv(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(lse),
+                                            _ptr(d_o), wp, wb, _ptr(dk_seg), _ptr(dv_seg), _stream(stream)),
+           "hga_attn_bwd_dkdv")
+
+
+def hga_attn_bwd_dq(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, lse, d_o, ws, dq,
+                    stream=None) -> None:
+    _attn_shapes(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx)
+    _expect(lse, (dims.B, dims.Hq, dims.S), torch.float32, "lse")
+    _expect(d_o, q.shape, dims.torch_dtype, "d_o")
+    _expect(dq, q.shape, torch.float32, "dq")
+    wp, wb = _ws(ws)
+    _check(load_library().hga_attn_bwd_dq(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist),
+                                          _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(lse), _ptr(d_o), wp, wb, _ptr(dq),
+                                          _stream(stream)), "hga_attn_bwd_dq")
 
 
 def hga_fetch_blocks(dims: Dims, host_k, host_v, host_capacity_blocks: int, idx_dev, host_idx_scratch, pool_k,

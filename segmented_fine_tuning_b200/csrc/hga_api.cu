@@ -235,36 +235,86 @@ size_t hga_attn_bwd_workspace_size(const hga_dims* dims) {
   return round256((size_t)dims->B * dims->Hq * dims->S * sizeof(float));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Shared checks and dispatch of the backward stages (parts: hga::kBwdDq |
+// hga::kBwdDkdv; preprocess when `pre` is set).
+hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg, const void* k_hist,
+                   const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o, const float* lse,
+                   const void* d_o, float* dq, float* dk_seg, float* dv_seg, const void* ws, size_t ws_bytes,
+                   bool pre, int parts, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(ws)) return fail(HGA_ERR_INVALID_ARG, "NULL workspace");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(HGA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (ws_bytes < hga_attn_bwd_workspace_size(dims))
+    return fail(HGA_ERR_INVALID_ARG, "workspace %zu bytes < %zu", ws_bytes, hga_attn_bwd_workspace_size(dims));
+  if (pre && (any_null(o, d_o) || !aligned16(o) || !aligned16(d_o)))
+    return fail(HGA_ERR_INVALID_ARG, "o and d_o must be non-NULL and 16-byte aligned");
+  if (parts) {
+    if ((r = check_attn_ptrs(s, (parts & hga::kBwdDq) ? n_kv_blocks : 0, q, k_seg, v_seg, k_hist, v_hist,
+                             (parts & hga::kBwdDq) ? idx : reinterpret_cast<const int32_t*>(q))) != HGA_OK)
+      return r;
+    if (any_null(lse, d_o) || !aligned16(lse) || !aligned16(d_o))
+      return fail(HGA_ERR_INVALID_ARG, "lse and d_o must be non-NULL and 16-byte aligned");
+    if ((parts & hga::kBwdDq) && (any_null(dq) || !aligned16(dq)))
+      return fail(HGA_ERR_INVALID_ARG, "dq must be non-NULL and 16-byte aligned");
+    if ((parts & hga::kBwdDkdv) && (any_null(dk_seg, dv_seg) || !aligned16(dk_seg) || !aligned16(dv_seg)))
+      return fail(HGA_ERR_INVALID_ARG, "dk_seg/dv_seg must be non-NULL and 16-byte aligned");
+  }
+  int* err;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* Dr = static_cast<float*>(const_cast<void*>(ws));
+  cudaError_t e;
+  if (pre && (e = hga::launch_bwd_preprocess(s, o, d_o, Dr, st)) != cudaSuccess)
+    return cuda_fail(e, "backward preprocess launch");
+  if (!parts) return HGA_OK;
+  if (hga::tc_supported(s)) {
+    hga::TcMaps m;
+    if ((r = build_maps(s, n_kv_blocks, q, d_o, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
+    e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, parts, err, st);
+  } else {
+    e = hga::launch_attn_bwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, lse, Dr, d_o, dq, dk_seg,
+                                  dv_seg, parts, err, st);
+  }
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "attention backward launch");
+}
+
+}  // namespace
+
+extern "C" {
+
 hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
                         const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o,
                         const float* lse, const void* d_o, float* dq, float* dk_seg, float* dv_seg, void* ws,
                         size_t ws_bytes, hga_stream_t stream) {
-  hga::Shape s;
-  hga_status r = check_dims(dims, &s);
-  if (r != HGA_OK) return r;
-  if ((r = check_attn_ptrs(s, n_kv_blocks, q, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
-  if (any_null(o, lse, d_o, dq, dk_seg, dv_seg, ws)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
-  if (!aligned16(o) || !aligned16(d_o) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk_seg) ||
-      !aligned16(dv_seg))
-    return fail(HGA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(HGA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  if (ws_bytes < hga_attn_bwd_workspace_size(dims))
-    return fail(HGA_ERR_INVALID_ARG, "workspace %zu bytes < %zu", ws_bytes, hga_attn_bwd_workspace_size(dims));
-  int* err;
-  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float* Dr = static_cast<float*>(ws);
-  cudaError_t e = hga::launch_bwd_preprocess(s, o, d_o, Dr, st);
-  if (e != cudaSuccess) return cuda_fail(e, "backward preprocess launch");
-  if (hga::tc_supported(s)) {
-    hga::TcMaps m;
-    if ((r = build_maps(s, n_kv_blocks, q, d_o, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
-    e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, err, st);
-  } else {
-    e = hga::launch_attn_bwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, lse, Dr, d_o, dq, dk_seg,
-                                  dv_seg, err, st);
-  }
-  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "attention backward launch");
+  return run_bwd(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse, d_o, dq, dk_seg, dv_seg, ws,
+                 ws_bytes, true, hga::kBwdDq | hga::kBwdDkdv, stream);
+}
+
+hga_status hga_attn_bwd_preprocess(const hga_dims* dims, const void* o, const void* d_o, void* ws, size_t ws_bytes,
+                                   hga_stream_t stream) {
+  return run_bwd(dims, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, o, nullptr, d_o, nullptr, nullptr,
+                 nullptr, ws, ws_bytes, true, 0, stream);
+}
+
+hga_status hga_attn_bwd_dkdv(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                             const float* lse, const void* d_o, const void* ws, size_t ws_bytes, float* dk_seg,
+                             float* dv_seg, hga_stream_t stream) {
+  return run_bwd(dims, q, k_seg, v_seg, nullptr, nullptr, 0, nullptr, nullptr, lse, d_o, nullptr, dk_seg, dv_seg,
+                 ws, ws_bytes, false, hga::kBwdDkdv, stream);
+}
+
+hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                           const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx,
+                           const float* lse, const void* d_o, const void* ws, size_t ws_bytes, float* dq,
+                           hga_stream_t stream) {
+  return run_bwd(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, nullptr, lse, d_o, dq, nullptr, nullptr,
+                 ws, ws_bytes, false, hga::kBwdDq, stream);
 }
 
 hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,

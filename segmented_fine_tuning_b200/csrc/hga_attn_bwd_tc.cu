@@ -492,7 +492,8 @@ __global__ void __launch_bounds__(320, 1)
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
-                               const float* Dr, float* dq, float* dk, float* dv, int* err, cudaStream_t st) {
+                               const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
+                               cudaStream_t st) {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDqSmem)) !=
       cudaSuccess)
@@ -505,13 +506,19 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const i
   a.scale = 1.0f / sqrtf((float)kD);
   a.sl2 = kLog2e * a.scale;
   a.idx = idx; a.lse = lse; a.Dr = Dr; a.dq = dq; a.dk = dk; a.dv = dv; a.err = err;
-  const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * kD * sizeof(float);
-  if ((e = cudaMemsetAsync(dk, 0, kv_bytes, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(dv, 0, kv_bytes, st)) != cudaSuccess) return e;
-  dkdv_tc_kernel<<<s.B * s.Hq * s.nqb(), 320, kDkvSmem, st>>>(m.q, m.d_o, m.ks, m.vs, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dq_tc_kernel<<<s.B * s.Hq * s.nqb(), 320, kDqSmem, st>>>(m.q, m.d_o, m.ks, m.vs, m.kh, m.vh, a);
-  return cudaGetLastError();
+  if (parts & kBwdDkdv) {
+    // Per-head partials are added into the outputs: start from zero.
+    const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * kD * sizeof(float);
+    if ((e = cudaMemsetAsync(dk, 0, kv_bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dv, 0, kv_bytes, st)) != cudaSuccess) return e;
+    dkdv_tc_kernel<<<s.B * s.Hq * s.nqb(), 320, kDkvSmem, st>>>(m.q, m.d_o, m.ks, m.vs, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (parts & kBwdDq) {
+    dq_tc_kernel<<<s.B * s.Hq * s.nqb(), 320, kDqSmem, st>>>(m.q, m.d_o, m.ks, m.vs, m.kh, m.vh, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace hga

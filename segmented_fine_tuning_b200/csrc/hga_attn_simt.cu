@@ -233,13 +233,18 @@ void fwd_simt(const SimtArgs& a, const void* q, const void* ks, const void* vs, 
 
 template <int DPL, typename T>
 void bwd_simt(const SimtArgs& a, const void* q, const void* ks, const void* vs, const void* kh, const void* vh,
-              const float* lse, const float* Dr, const void* d_o, float* dq, float* dk, float* dv, cudaStream_t st) {
-  const int rows = a.B * a.Hq * a.S;
-  dq_simt_kernel<DPL, T><<<(rows + 7) / 8, 256, 0, st>>>(a, (const T*)q, (const T*)ks, (const T*)vs, (const T*)kh,
-                                                         (const T*)vh, (const T*)d_o, lse, Dr, dq);
-  const int krows = a.B * a.Hkv * a.S;
-  dkdv_simt_kernel<DPL, T><<<(krows + 7) / 8, 256, 0, st>>>(a, (const T*)q, (const T*)ks, (const T*)vs,
-                                                            (const T*)d_o, lse, Dr, dk, dv);
+              const float* lse, const float* Dr, const void* d_o, float* dq, float* dk, float* dv, int parts,
+              cudaStream_t st) {
+  if (parts & kBwdDq) {
+    const int rows = a.B * a.Hq * a.S;
+    dq_simt_kernel<DPL, T><<<(rows + 7) / 8, 256, 0, st>>>(a, (const T*)q, (const T*)ks, (const T*)vs,
+                                                           (const T*)kh, (const T*)vh, (const T*)d_o, lse, Dr, dq);
+  }
+  if (parts & kBwdDkdv) {
+    const int krows = a.B * a.Hkv * a.S;
+    dkdv_simt_kernel<DPL, T><<<(krows + 7) / 8, 256, 0, st>>>(a, (const T*)q, (const T*)ks, (const T*)vs,
+                                                              (const T*)d_o, lse, Dr, dk, dv);
+  }
 }
 
 }  // namespace
@@ -261,14 +266,14 @@ cudaError_t launch_attn_fwd_simt(const Shape& s, const void* q, const void* k_se
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
                                  const void* k_hist, const void* v_hist, int nkv, const int32_t* idx,
                                  const float* lse, const float* Dr, const void* d_o, float* dq, float* dk,
-                                 float* dv, int* err, cudaStream_t st) {
+                                 float* dv, int parts, int* err, cudaStream_t st) {
   const SimtArgs a = make_args(s, nkv, idx, err);
   if (s.d == 64) {
-    if (s.bf16) bwd_simt<2, __nv_bfloat16>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, st);
-    else bwd_simt<2, float>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, st);
+    if (s.bf16) bwd_simt<2, __nv_bfloat16>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, parts, st);
+    else bwd_simt<2, float>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, parts, st);
   } else {
-    if (s.bf16) bwd_simt<4, __nv_bfloat16>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, st);
-    else bwd_simt<4, float>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, st);
+    if (s.bf16) bwd_simt<4, __nv_bfloat16>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, parts, st);
+    else bwd_simt<4, float>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, parts, st);
   }
   return cudaGetLastError();
 }

@@ -31,6 +31,9 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
 // D[b,hq,p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k]  (fp32)
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st);
 
+// Backward parts (bit mask): dQ and dK/dV are independent once Dr exists.
+enum : int { kBwdDq = 1, kBwdDkdv = 2 };
+
 // CUDA-core attention (any supported shape, fp32 or bf16).
 cudaError_t launch_attn_fwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
                                  const void* k_hist, const void* v_hist, int nkv, const int32_t* idx, void* o,
@@ -38,7 +41,7 @@ cudaError_t launch_attn_fwd_simt(const Shape& s, const void* q, const void* k_se
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
                                  const void* k_hist, const void* v_hist, int nkv, const int32_t* idx,
                                  const float* lse, const float* Dr, const void* d_o, float* dq, float* dk,
-                                 float* dv, int* err, cudaStream_t st);
+                                 float* dv, int parts, int* err, cudaStream_t st);
 
 // Tensor-core attention (bf16, d = 128, block = 128, even G).  Tensor maps:
 // q/d_o [B,S,Hq,128], k/v seg [B,S,Hkv,128], k/v hist [B,nkv*128,Hkv,128],
@@ -50,7 +53,8 @@ bool tc_supported(const Shape& s);
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
                                int* err, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
-                               const float* Dr, float* dq, float* dk, float* dv, int* err, cudaStream_t st);
+                               const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
+                               cudaStream_t st);
 
 // Tensor-core operand-layout self test (see hga_selftest.h).
 cudaError_t launch_selftest_umma(int form, const CUtensorMap& ma, const CUtensorMap& mb, const void* a_raw,

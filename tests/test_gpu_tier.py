@@ -1,0 +1,106 @@
+"""Host KV tier: targeted loading of the selected history blocks from pinned
+host memory (hga_fetch_blocks) and the segment-end offload
+(hga_offload_segment), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from hga_testutil import dims_of, to_dev
+from segmented_fine_tuning_b200 import (HgaError, hga_attn_bwd, hga_attn_fwd, hga_device_status, hga_fetch_blocks,
+                                        hga_offload_segment)
+from segmented_fine_tuning_b200.step import AttentionStep
+
+pytestmark = pytest.mark.gpu
+
+
+def _pinned(t: synth.Tensor):
+    return torch.from_numpy(np.ascontiguousarray(t.store).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+
+@pytest.mark.parametrize("capacity_extra", [0, 3])
+def test_fetch_into_pool_matches_resident_history(capacity_extra):
+    w = synth.Workload("tier: Hq8/Hkv2 S512 hist20 K3", 1, 8, 2, 128, 128, 512, 20, 3, "bf16", 41,
+                       structured_keys=True)
+    x = synth.draw(w)
+    D = dims_of(w)
+    dev = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    st = AttentionStep(D)
+    st.run(dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], dev["d_o"])
+    torch.cuda.synchronize()
+    o_ref, lse_ref, dq_ref = st.o.clone(), st.lse.clone(), st.dq.clone()
+    dk_ref, dv_ref = st.dk.clone(), st.dv.clone()
+
+    cap = w.nblk + capacity_extra
+    tier_k = torch.zeros((1, cap * 128, 2, 128), dtype=torch.bfloat16).pin_memory()
+    tier_v = torch.zeros_like(tier_k).pin_memory()
+    tier_k[:, : w.nblk * 128] = _pinned(x.k_hist)
+    tier_v[:, : w.nblk * 128] = _pinned(x.v_hist)
+    scratch = torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory()
+    n_sel = len(set(st.idx.cpu().numpy().ravel().tolist()) - {-1})
+    pool_slots = n_sel + 1
+    pool_k = torch.full((1, pool_slots * 128, 2, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    pool_v = torch.full_like(pool_k, float("nan"))
+    idx_pool = torch.empty_like(st.idx)
+    copy_stream = torch.cuda.Stream()
+    done = torch.cuda.Event()
+    done.record(copy_stream)
+    nu = hga_fetch_blocks(D, tier_k, tier_v, cap, st.idx, scratch, pool_k, pool_v, pool_slots, idx_pool,
+                          torch.cuda.current_stream(), copy_stream, done)
+    torch.cuda.current_stream().wait_event(done)
+    assert nu == n_sel
+    # pool slot s holds the s-th smallest selected block
+    sel = sorted(set(st.idx.cpu().numpy().ravel().tolist()) - {-1})
+    ip = idx_pool.cpu().numpy()
+    ig = st.idx.cpu().numpy()
+    assert np.array_equal(np.where(ig >= 0, np.searchsorted(sel, np.maximum(ig, 0)), -1), ip)
+    o = torch.empty_like(st.o)
+    lse = torch.empty_like(st.lse)
+    hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], pool_k, pool_v, pool_slots, idx_pool, o, lse)
+    dq, dk, dv = torch.empty_like(st.dq), torch.empty_like(st.dk), torch.empty_like(st.dv)
+    hga_attn_bwd(D, dev["q"], dev["k_seg"], dev["v_seg"], pool_k, pool_v, pool_slots, idx_pool, o, lse,
+                 dev["d_o"], dq, dk, dv, st.ws)
+    torch.cuda.synchronize()
+    hga_device_status()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref) and torch.equal(dq, dq_ref)
+    # dK/dV accumulate per-head partials with atomics: equal up to summation order
+    assert torch.allclose(dk, dk_ref, rtol=0, atol=1e-5) and torch.allclose(dv, dv_ref, rtol=0, atol=1e-5)
+
+
+def test_fetch_rejects_small_pool_and_bad_index():
+    w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 6, 3, "bf16", 42)
+    D = dims_of(w)
+    idx = torch.tensor([[0, 2, 4], [1, 3, 5]], dtype=torch.int32).reshape(1, 1, 2, 3).repeat(1, 2, 1, 1).cuda()
+    tier = torch.zeros((1, 6 * 128, 2, 128), dtype=torch.bfloat16).pin_memory()
+    scratch = torch.empty((1, 2, 2, 3), dtype=torch.int32).pin_memory()
+    pool = torch.empty((1, 4 * 128, 2, 128), dtype=torch.bfloat16, device="cuda")
+    ip = torch.empty_like(idx)
+    cs = torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    ev.record(cs)
+    with pytest.raises(HgaError) as e:
+        hga_fetch_blocks(D, tier, tier, 6, idx, scratch, pool, pool, 4, ip, torch.cuda.current_stream(), cs, ev)
+    assert e.value.status == 1
+    bad = idx.clone()
+    bad[0, 0, 0, 0] = 17
+    pool6 = torch.empty((1, 6 * 128, 2, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(HgaError) as e:
+        hga_fetch_blocks(D, tier, tier, 6, bad, scratch, pool6, pool6, 6, ip, torch.cuda.current_stream(), cs, ev)
+    assert e.value.status == 4
+    torch.cuda.synchronize()
+
+
+def test_offload_segment_into_tier():
+    w = synth.Workload("t", 2, 4, 2, 128, 128, 256, 3, 2, "bf16", 43)
+    x = synth.draw(w)
+    D = dims_of(w)
+    ks, vs = to_dev(x.k_seg), to_dev(x.v_seg)
+    cap = 8
+    tk = torch.zeros((2, cap * 128, 2, 128), dtype=torch.bfloat16).pin_memory()
+    tv = torch.zeros_like(tk).pin_memory()
+    hga_offload_segment(D, ks, vs, tk, tv, cap, 5)
+    torch.cuda.synchronize()
+    assert torch.equal(tk[:, 5 * 128: 7 * 128], ks.cpu()) and torch.equal(tv[:, 5 * 128: 7 * 128], vs.cpu())
+    assert torch.count_nonzero(tk[:, : 5 * 128]) == 0 and torch.count_nonzero(tk[:, 7 * 128:]) == 0
+    with pytest.raises(HgaError):
+        hga_offload_segment(D, ks, vs, tk, tv, cap, 7)
