@@ -181,6 +181,36 @@ HGA_API hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void*
                         size_t ws_bytes, hga_stream_t stream);
 
 /*
+ * hga_attn_bwd for callers that cannot allocate device memory.  The article
+ * has no counterpart to this call; it exists for integration.
+ *
+ * Some callers cannot call cudaMalloc at the point where they run the
+ * backward: code that runs under a framework-owned memory pool (an allocator
+ * that owns every device byte and forbids outside allocations), host code
+ * driving a pre-planned memory budget, or a plugin that only receives the
+ * tensors it reads and writes.  Such a caller has no workspace to pass.  This
+ * variant takes the same inputs and outputs as hga_attn_bwd, minus ws and
+ * ws_bytes, and keeps its scratch (Dr = rowsum(dO * O), B*Hq*S floats) in a
+ * fixed array inside the library instead.
+ *
+ * Limit: B*Hq*S <= 1,048,576 (a 4 MiB array, held on every GPU that loads
+ * the library until the process exits).  Larger problems return
+ * HGA_ERR_SHAPE; use hga_attn_bwd with a caller-owned workspace for them.
+ * The call allocates nothing (no cudaMalloc or allocating library routine).
+ * Set-up: the first call on each device looks up the array's device address
+ * with the device current; make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents (the
+ * stage that reads it first overwrites every element it reads, so nothing
+ * needs clearing); two calls that overlap on the GPU (different streams, no
+ * ordering between them) race on it.
+ * Results, errors and asynchrony otherwise as hga_attn_bwd.
+ */
+HGA_API hga_status hga_attn_bwd_noalloc(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                                        const void* k_hist, const void* v_hist, int n_kv_blocks,
+                                        const int32_t* idx, const void* o, const float* lse, const void* d_o,
+                                        float* dq, float* dk_seg, float* dv_seg, hga_stream_t stream);
+
+/*
  * The three stages of hga_attn_bwd as separate calls (same arguments, same
  * results), for callers that schedule or time them individually.  ws is the
  * same caller-owned scratch; its first B*Hq*S floats hold Dr = rowsum(dO * O)

@@ -78,6 +78,7 @@ _SIGNATURES = [
     ("hga_attn_fwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     ("hga_attn_bwd_workspace_size", ctypes.c_size_t, [_D]),
     ("hga_attn_bwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("hga_attn_bwd_noalloc", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     ("hga_attn_bwd_preprocess", _I, [_D, _P, _P, _P, ctypes.c_size_t, _P]),
     ("hga_attn_bwd_dkdv", _I, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P]),
     ("hga_attn_bwd_dq", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
@@ -201,6 +202,25 @@ def hga_attn_bwd(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, 
                                        _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq),
                                        _ptr(dk_seg), _ptr(dv_seg), _ptr(ws), ws.numel() * ws.element_size(),
                                        _stream(stream)), "hga_attn_bwd")
+
+
+def hga_attn_bwd_noalloc(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, o, lse, d_o, dq,
+                         dk_seg, dv_seg, stream=None) -> None:
+    """hga_attn_bwd without a workspace argument, for callers that cannot
+    allocate device memory: the library keeps the scratch in a fixed 4 MiB
+    array per device (B*Hq*S <= 2**20).  Calls that overlap on the GPU race on
+    that array."""
+    _attn_shapes(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx)
+    _expect(o, q.shape, dims.torch_dtype, "o")
+    _expect(d_o, q.shape, dims.torch_dtype, "d_o")
+    _expect(lse, (dims.B, dims.Hq, dims.S), torch.float32, "lse")
+    _expect(dq, q.shape, torch.float32, "dq")
+    _expect(dk_seg, k_seg.shape, torch.float32, "dk_seg")
+    _expect(dv_seg, v_seg.shape, torch.float32, "dv_seg")
+    _check(load_library().hga_attn_bwd_noalloc(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg),
+                                               _ptr(k_hist), _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse),
+                                               _ptr(d_o), _ptr(dq), _ptr(dk_seg), _ptr(dv_seg), _stream(stream)),
+           "hga_attn_bwd_noalloc")
 
 
 def _ws(ws):

@@ -317,6 +317,64 @@ hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const void* k_se
                  ws, ws_bytes, false, hga::kBwdDq, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- backward without a caller workspace
+// For callers that cannot allocate device memory (a framework-owned pool that
+// forbids outside allocations, a fixed memory plan, a plugin that only sees
+// its inputs and outputs): the backward's scratch lives in this fixed array.
+// 1,048,576 floats = 4 MiB, the Dr row statistics of B*Hq*S <= 2^20 rows.
+// Every GPU that loads the library holds it until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;
+static __device__ __align__(256) float g_bwd_scratch[kNoAllocScratchFloats];
+
+// In host code g_bwd_scratch names a host-side stand-in, not device memory:
+// the device address is looked up once per device, with that device current.
+float* g_bwd_scratch_ptr[kMaxDevices] = {nullptr};
+
+hga_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HGA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_bwd_scratch_ptr[dev]) {
+    float* p = nullptr;
+    e = cudaGetSymbolAddress((void**)&p, g_bwd_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(backward scratch)");
+    g_bwd_scratch_ptr[dev] = p;
+  }
+  *out = g_bwd_scratch_ptr[dev];
+  return HGA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+hga_status hga_attn_bwd_noalloc(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                                const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx,
+                                const void* o, const float* lse, const void* d_o, float* dq, float* dk_seg,
+                                float* dv_seg, hga_stream_t stream) {
+  if (!dims) return fail(HGA_ERR_INVALID_ARG, "dims is NULL");
+  const size_t rows = (size_t)(dims->B > 0 ? dims->B : 0) * (size_t)(dims->Hq > 0 ? dims->Hq : 0) *
+                      (size_t)(dims->S > 0 ? dims->S : 0);
+  if (rows > kNoAllocScratchFloats)
+    return fail(HGA_ERR_SHAPE,
+                "B*Hq*S = %zu exceeds the %zu rows of the built-in backward scratch; call hga_attn_bwd with a "
+                "caller-owned workspace instead",
+                rows, kNoAllocScratchFloats);
+  float* scratch = nullptr;
+  hga_status r = noalloc_scratch(&scratch);
+  if (r != HGA_OK) return r;
+  // Dr is written in full by the preprocess stage before any stage reads it,
+  // so the previous call's contents need no clearing.
+  return run_bwd(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse, d_o, dq, dk_seg, dv_seg, scratch,
+                 kNoAllocScratchFloats * sizeof(float), true, hga::kBwdDq | hga::kBwdDkdv, stream);
+}
+
 hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,
                             const int32_t* idx_dev,
                             int32_t* host_idx_scratch, void* pool_k, void* pool_v, int pool_slots,

@@ -1,0 +1,78 @@
+"""hga_attn_bwd_noalloc: the backward for callers that cannot allocate device
+memory (a framework-owned pool that forbids outside allocations, a fixed
+memory plan, a plugin that only receives its inputs and outputs).  Its
+scratch is a fixed array inside the library instead of a caller workspace.
+
+Checked through the C ABI against hga_attn_bwd with a caller-owned
+workspace, within the bf16 tolerance of the parity tests (max abs 2e-2,
+relative L2 1e-2; in practice the two agree to the atomics' summation order),
+on two calls in a row with different inputs, so the second call runs on the
+array the first one left behind.  This file is collected last; it passes
+alone in a fresh process and after the other tests."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from hga_testutil import BF16_ABS, BF16_REL, F32_ABS, assert_close, dims_of, to_dev, to_host
+from segmented_fine_tuning_b200 import (HgaError, hga_attn_bwd, hga_attn_bwd_noalloc, hga_attn_fwd,
+                                        hga_block_summaries, hga_device_status, hga_select_topk)
+from segmented_fine_tuning_b200 import _binding
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # tensor-core path
+    (synth.Workload("noalloc-tc: Hq8/Hkv2 S512 hist6 K3", 1, 8, 2, 128, 128, 512, 6, 3, "bf16", 51,
+                    structured_keys=True), (BF16_ABS, BF16_REL)),
+    # CUDA-core path (fp32)
+    (synth.TINY_F32, (F32_ABS, None)),
+]
+
+
+def _forward(w, seed):
+    x = synth.draw(w, seed=seed)
+    D = dims_of(w)
+    t = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    summ = torch.empty((w.B, w.Hkv, w.nblk, w.d), device="cuda")
+    idx = torch.empty((w.B, w.Hkv, w.nqb, w.topk), dtype=torch.int32, device="cuda")
+    o = torch.empty_like(t["q"])
+    lse = torch.empty((w.B, w.Hq, w.S), device="cuda")
+    hga_block_summaries(D, t["k_hist"], 0, w.nblk, summ)
+    hga_select_topk(D, t["q"], summ, idx)
+    hga_attn_fwd(D, t["q"], t["k_seg"], t["v_seg"], t["k_hist"], t["v_hist"], w.nblk, idx, o, lse)
+    return D, t, idx, o, lse
+
+
+@pytest.mark.parametrize("w,tol", CASES, ids=lambda c: c.name.split(":")[0] if hasattr(c, "name") else "")
+def test_noalloc_backward_matches_workspace_backward_twice(w, tol):
+    for call, seed in enumerate((w.seed + 100, w.seed + 200)):
+        D, t, idx, o, lse = _forward(w, seed)
+        outs = {}
+        for variant in ("workspace", "noalloc"):
+            dq = torch.full_like(t["q"], float("nan"), dtype=torch.float32)
+            dk = torch.full_like(t["k_seg"], float("nan"), dtype=torch.float32)
+            dv = torch.full_like(t["v_seg"], float("nan"), dtype=torch.float32)
+            if variant == "workspace":
+                ws = torch.empty((_binding.hga_attn_bwd_workspace_size(D),), dtype=torch.uint8, device="cuda")
+                hga_attn_bwd(D, t["q"], t["k_seg"], t["v_seg"], t["k_hist"], t["v_hist"], w.nblk, idx, o, lse,
+                             t["d_o"], dq, dk, dv, ws)
+            else:
+                hga_attn_bwd_noalloc(D, t["q"], t["k_seg"], t["v_seg"], t["k_hist"], t["v_hist"], w.nblk, idx, o,
+                                     lse, t["d_o"], dq, dk, dv)
+            torch.cuda.synchronize()
+            hga_device_status()
+            outs[variant] = (to_host(dq), to_host(dk), to_host(dv))
+        for name, a, b in zip(("dQ", "dK", "dV"), outs["noalloc"], outs["workspace"]):
+            assert np.all(np.isfinite(a)), f"call {call}: {name} not fully written"
+            assert_close(f"call {call} {name}", a, b, *tol)
+
+
+def test_noalloc_rejects_sizes_beyond_the_array():
+    D = _binding.Dims(1, 64, 8, 128, 128, 32768, 0, 4, "bf16")  # B*Hq*S = 2^21 rows > 2^20
+    lib = _binding.load_library()
+    p = torch.empty(16, device="cuda").data_ptr()
+    st = lib.hga_attn_bwd_noalloc(__import__("ctypes").byref(D.c()), p, p, p, None, None, 0, p, p, p, p, p, p, p,
+                                  None)
+    assert st == 2
+    assert "caller-owned workspace" in lib.hga_last_error().decode()
