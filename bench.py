@@ -351,6 +351,79 @@ def run_e2e(args, ctx, device):
             "fetched_blocks_per_step": float(np.mean(fetched)), "path": "pinned host tier + hga_fetch_blocks"}
 
 
+# ---------------------------------------------------------------- segmented pass
+
+def h2d_probe(device, nbytes=1 << 30, reps=5):
+    """Pinned host -> device copy bandwidth (GB/s), the roofline of the fetch."""
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    st = torch.cuda.current_stream(device)
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        dst.copy_(src, non_blocking=True)
+        e1.record(st)
+        torch.cuda.synchronize(device)
+        best = max(best, nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    return best
+
+
+def run_segmented(args, device):
+    """The full segmented pass: 36 Qwen3-8B-shaped layers over a 16,384-token
+    sequence as 8 segments of 2,048 (history in a pinned host tier, selected
+    blocks fetched per (layer, segment), summaries appended on the device).
+    Inputs: the 8 segments of layer 0 drawn with the workload's recipe and
+    reused for every layer (the kernels' speed does not depend on values;
+    selection, and so fetch volume, is representative).  One step = one pass."""
+    import segmented_fine_tuning_b200 as hga
+    from segmented_fine_tuning_b200.segmented import SegmentedPass
+    w = synth.QWEN3_8B_LAYER
+    L, NS = synth.SEGMENTED_LAYERS, synth.SEGMENTED_SEGMENTS
+    seg = hga.Dims(1, w.Hq, w.Hkv, w.d, w.blk, w.S, 0, w.topk, "bf16")
+    xs = [synth.draw_segment(w, 0, s) for s in range(NS)]
+    dev = [tuple(to_dev(t, device) for t in (x.q, x.k_seg, x.v_seg, x.d_o)) for x in xs]
+    sp = SegmentedPass(seg, L, NS, device)
+    stream = torch.cuda.current_stream(device)
+
+    def one_pass():
+        for s in range(NS):
+            sp.run_segment(s, [dev[s]] * L)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize(device)
+    hga.hga_device_status(stream)
+    sp.fetched_blocks.clear()
+    times = []
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            one_pass()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(e0.elapsed_time(e1))
+    hga.hga_device_status(stream)
+    ms = float(np.mean(times))
+    tokens = NS * w.S
+    fetched = float(np.mean(sp.fetched_blocks))
+    blk_bytes = w.blk * w.Hkv * w.d * 2 * 2
+    h2d_bytes = fetched * blk_bytes * L * (NS - 1)
+    probe = h2d_probe(device)
+    return {"metric": "HGA full segmented pass tokens/s per layer (fwd+bwd, history fetched from a pinned host tier)",
+            "value": round(tokens * L / (ms / 1e3), 1), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (layer 0's 8 segments reused for all layers)",
+            "config": {"workload": "segmented pass: 36 Qwen3-8B-shaped layers x 8 segments of 2,048 tokens, "
+                                   "history +16 blocks of 128 per segment, K16, pinned host tier",
+                       "layers": L, "segments": NS, "segment_tokens": w.S, "topk": w.topk},
+            "fetch": {"blocks_per_layer_step": round(fetched, 1), "h2d_bytes_per_pass": int(h2d_bytes),
+                      "h2d_probe_gbs": round(probe, 1),
+                      "fetch_time_at_probe_ms": round(h2d_bytes / (probe * 1e9) * 1e3, 2)},
+            "gpu_launches": int(L * NS * 6 + L * NS), "clocks": clk.summary()}
+
+
 # ---------------------------------------------------------------- oracle legs
 
 def oracle_sample(w: synth.Workload, x, kv_heads):
@@ -419,6 +492,9 @@ def main():
     ap.add_argument("--impl", choices=("hga", "reference"), default="hga")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=("layer", "segmented"), default="layer",
+                    help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
+                         "8-segment pass with the pinned host tier")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3
@@ -439,6 +515,11 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     try:
+        if args.workload == "segmented":
+            out = run_segmented(args, device)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+            return
         out, ctx = run_device(args, rank, world, device)
         if not args.no_e2e:
             e2e = run_e2e(args, ctx, device)

@@ -38,7 +38,9 @@
  *   k_seg, v_seg        [B, S, Hkv, d]         dtype
  *   k_hist, v_hist      [B, n_kv_blocks*block, Hkv, d] dtype; block n = tokens
  *                       [n*block, (n+1)*block)
- *   summ                [B, Hkv, n_hist_blocks, d] fp32
+ *   summ                [B, n_hist_blocks, Hkv, d] fp32 (block-major, so a growing
+ *                       history appends: the first n blocks of a larger array
+ *                       are a valid summary array of n blocks when B == 1)
  *   idx                 [B, Hkv, Nqb, topk]    int32
  *   lse                 [B, Hq, S]             fp32 (natural log)
  *   dq                  [B, S, Hq, d]          fp32
@@ -112,22 +114,35 @@ HGA_API hga_status hga_device_status(hga_stream_t stream);
 
 /*
  * Block summaries (article, Deep analysis: resident per-block summaries).
- *   summ[b,h,n,:] = (1/block) * sum_{t<block} k_hist[b, n*block+t, h, :]
+ *   summ[b,n,h,:] = (1/block) * sum_{t<block} k_hist[b, n*block+t, h, :]
  * for blocks n in [blk_begin, blk_end) of a history of dims->n_hist_blocks
  * blocks; other entries of summ are left untouched, so summaries can be added
  * as blocks enter the history.  k_hist: dtype; summ: fp32 device buffer
- * [B, Hkv, n_hist_blocks, d].  Accumulation in fp32.
+ * [B, n_hist_blocks, Hkv, d].  Accumulation in fp32.
  * Errors: HGA_ERR_INVALID_ARG (null pointers, bad range), HGA_ERR_SHAPE.
  */
 HGA_API hga_status hga_block_summaries(const hga_dims* dims, const void* k_hist, int blk_begin, int blk_end, float* summ,
                                hga_stream_t stream);
 
 /*
+ * Summaries of a finished segment's blocks, as they enter the history
+ * (article, Deep analysis: summaries stay resident and grow with the context;
+ * fr Analyse approfondie: the segment's KV leaves the active window).
+ *   summ[b, at_block + t, h, :] = (1/block) * sum_{u<block} k_seg[b, t*block+u, h, :]
+ * for the S/block blocks t of the segment.  Here dims->n_hist_blocks is the
+ * capacity (in blocks) of the summ array [B, n_hist_blocks, Hkv, d];
+ * at_block + S/block must not exceed it.  Other entries are untouched.
+ * Errors: HGA_ERR_INVALID_ARG (null pointers, range), HGA_ERR_SHAPE.
+ */
+HGA_API hga_status hga_segment_summaries(const hga_dims* dims, const void* k_seg, int at_block, float* summ,
+                                         hga_stream_t stream);
+
+/*
  * Per-query-block history selection (article, Background: bounded exact
  * history set per query block; fr Contexte: precise historical tokens per
  * query block).  For every (b, KV head h, query block i):
  *   qm[g]     = mean over the block's `block` rows of q[b, row, h*G+g, :] (fp32)
- *   score[n]  = max_g (qm[g] . summ[b,h,n,:]) / sqrt(d)                   (fp32)
+ *   score[n]  = max_g (qm[g] . summ[b,n,h,:]) / sqrt(d)                   (fp32)
  *   idx[b,h,i,:] = the K_eff = min(topk, n_hist_blocks) best n (ties to the
  *                  lower n), ascending, then -1 up to topk.
  * scores_or_null (optional, fp32 [B,Hkv,Nqb,topk]) receives the selected
@@ -266,7 +281,7 @@ HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, co
  * [B, S, Hkv, d]) into the pinned host tier at history block `at_block`
  * (host_k/host_v [B, capacity_blocks*block, Hkv, d]) on `stream`, one copy per
  * (batch, tensor).  The summaries of the new blocks are computed on the device
- * with hga_block_summaries.  Errors: HGA_ERR_INVALID_ARG, HGA_ERR_SHAPE.
+ * with hga_segment_summaries.  Errors: HGA_ERR_INVALID_ARG, HGA_ERR_SHAPE.
  */
 HGA_API hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
                                void* host_v, int capacity_blocks, int at_block, hga_stream_t stream);

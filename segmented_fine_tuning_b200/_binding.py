@@ -74,6 +74,7 @@ _SIGNATURES = [
     ("hga_last_error", ctypes.c_char_p, []),
     ("hga_device_status", _I, [_P]),
     ("hga_block_summaries", _I, [_D, _P, _I, _I, _P, _P]),
+    ("hga_segment_summaries", _I, [_D, _P, _I, _P, _P]),
     ("hga_select_topk", _I, [_D, _P, _P, _P, _P, _P]),
     ("hga_attn_fwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     ("hga_attn_bwd_workspace_size", ctypes.c_size_t, [_D]),
@@ -149,14 +150,28 @@ def hga_device_status(stream=None) -> None:
 
 def hga_block_summaries(dims: Dims, k_hist, blk_begin: int, blk_end: int, summ, stream=None) -> None:
     _expect(k_hist, (dims.B, dims.n_hist_blocks * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "k_hist")
-    _expect(summ, (dims.B, dims.Hkv, dims.n_hist_blocks, dims.d), torch.float32, "summ")
+    _expect(summ, (dims.B, dims.n_hist_blocks, dims.Hkv, dims.d), torch.float32, "summ")
     _check(load_library().hga_block_summaries(ctypes.byref(dims.c()), _ptr(k_hist), blk_begin, blk_end, _ptr(summ),
                                               _stream(stream)), "hga_block_summaries")
 
 
+def hga_segment_summaries(dims: Dims, k_seg, at_block: int, summ, stream=None) -> None:
+    """dims.n_hist_blocks is the capacity (blocks) of the summ array."""
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(summ, (dims.B, dims.n_hist_blocks, dims.Hkv, dims.d), torch.float32, "summ")
+    _check(load_library().hga_segment_summaries(ctypes.byref(dims.c()), _ptr(k_seg), at_block, _ptr(summ),
+                                                _stream(stream)), "hga_segment_summaries")
+
+
 def hga_select_topk(dims: Dims, q_seg, summ, idx, scores=None, stream=None) -> None:
     _expect(q_seg, (dims.B, dims.S, dims.Hq, dims.d), dims.torch_dtype, "q_seg")
-    _expect(summ, (dims.B, dims.Hkv, dims.n_hist_blocks, dims.d), torch.float32, "summ")
+    if summ is None or summ.dim() != 4 or summ.shape[1] < dims.n_hist_blocks or \
+            tuple(summ.shape[2:]) != (dims.Hkv, dims.d) or summ.shape[0] != dims.B:
+        raise ValueError(f"summ: expected [B, >= n_hist_blocks, Hkv, d], got {None if summ is None else tuple(summ.shape)}")
+    if summ.dtype != torch.float32 or not summ.is_contiguous() or not summ.is_cuda:
+        raise ValueError("summ must be a contiguous fp32 CUDA tensor")
+    if dims.B > 1 and summ.shape[1] != dims.n_hist_blocks:
+        raise ValueError("with B > 1 the summ array must hold exactly n_hist_blocks blocks")
     _expect(idx, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx")
     if scores is not None:
         _expect(scores, idx.shape, torch.float32, "scores")

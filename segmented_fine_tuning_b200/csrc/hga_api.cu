@@ -190,9 +190,24 @@ hga_status hga_block_summaries(const hga_dims* dims, const void* k_hist, int blk
   if (blk_end == blk_begin) return HGA_OK;
   if (any_null(k_hist, summ)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(k_hist)) return fail(HGA_ERR_INVALID_ARG, "k_hist must be 16-byte aligned");
-  cudaError_t e = hga::launch_block_summaries(s, k_hist, blk_begin, blk_end, summ,
-                                              reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = hga::launch_block_summaries(s, k_hist, s.nblk * s.blk, blk_begin, blk_begin, blk_end - blk_begin,
+                                              summ, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "block summaries launch");
+}
+
+hga_status hga_segment_summaries(const hga_dims* dims, const void* k_seg, int at_block, float* summ,
+                                 hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (at_block < 0 || at_block + s.nqb() > s.nblk)
+    return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the summary array's %d", at_block, at_block + s.nqb(),
+                s.nblk);
+  if (any_null(k_seg, summ)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k_seg)) return fail(HGA_ERR_INVALID_ARG, "k_seg must be 16-byte aligned");
+  cudaError_t e = hga::launch_block_summaries(s, k_seg, s.S, 0, at_block, s.nqb(), summ,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "segment summaries launch");
 }
 
 hga_status hga_select_topk(const hga_dims* dims, const void* q_seg, const float* summ, int32_t* idx,

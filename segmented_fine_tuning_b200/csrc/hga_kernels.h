@@ -24,8 +24,10 @@ constexpr int kMaxSelectBlocks = 4096;
 // Longest segment (in query blocks) the tensor-core kernels handle.
 constexpr int kMaxQueryBlocks = 128;
 
-cudaError_t launch_block_summaries(const Shape& s, const void* k_hist, int b0, int b1, float* summ,
-                                   cudaStream_t st);
+// Summaries of `nblocks` blocks: source blocks src_b0.. of k_src (T_src tokens
+// per batch) -> destination blocks dst_b0.. of summ [B, s.nblk, Hkv, d].
+cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src, int src_b0, int dst_b0, int nblocks,
+                                   float* summ, cudaStream_t st);
 cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
                                cudaStream_t st);
 // D[b,hq,p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k]  (fp32)

@@ -39,14 +39,17 @@ struct Vec<__nv_bfloat16> {
 };
 
 // ------------------------------------------------------------ summaries
-// CTA = (history block n, column chunk of 32 vectors, batch b).  Each warp
-// reads whole 32-vector stretches of token rows (coalesced 512 B for bf16),
-// 8 warps cover 8 rows per pass; partials are combined in shared memory.
+// CTA = (block n, column chunk of 32 vectors, batch b).  Each warp reads whole
+// 32-vector stretches of token rows (coalesced 512 B for bf16), 8 warps cover
+// 8 rows per pass; partials are combined in shared memory.  Source block
+// src_b0 + n of k (T_src tokens per batch) -> destination block dst_b0 + n of
+// summ [B, nblk_dst, Hkv, d].
 template <typename T>
-__global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k, int T_tok, int Hkv, int d, int blk,
-                                                        int nblk, int b0, float* __restrict__ summ) {
+__global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k, int T_src, int Hkv, int d, int blk,
+                                                        int src_b0, int dst_b0, int nblk_dst,
+                                                        float* __restrict__ summ) {
   constexpr int V = Vec<T>::N;
-  const int n = b0 + blockIdx.x;
+  const int n = blockIdx.x;
   const int b = blockIdx.z;
   const int cols = Hkv * d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -55,7 +58,7 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k,
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
   if (col < cols) {
-    const T* base = k + ((size_t)b * T_tok + (size_t)n * blk) * cols + col;
+    const T* base = k + ((size_t)b * T_src + (size_t)(src_b0 + n) * blk) * cols + col;
     int t = warp;
 #pragma unroll 4
     for (; t < blk; t += 8) {
@@ -70,14 +73,11 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k,
   for (int e = 0; e < V; ++e) part[warp][lane * V + e] = acc[e];
   __syncthreads();
   for (int x = threadIdx.x; x < 32 * V; x += 256) {
-    float s = 0.f;
+    float sacc = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += part[w][x];
-    const int c = blockIdx.y * 32 * V + x;
-    if (c < cols) {
-      const int h = c / d, kk = c % d;
-      summ[(((size_t)b * Hkv + h) * nblk + n) * d + kk] = s * (1.0f / blk);
-    }
+    for (int w = 0; w < 8; ++w) sacc += part[w][x];
+    const int c = blockIdx.y * 32 * V + x;  // = h*d + channel: contiguous in the block-major layout
+    if (c < cols) summ[((size_t)b * nblk_dst + dst_b0 + n) * cols + c] = sacc * (1.0f / blk);
   }
 }
 
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, co
       if (lane == 0) keys[n] = 0ull;
       continue;
     }
-    const float* sv = summ + (((size_t)b * Hkv + h) * nblk + n) * d;
+    const float* sv = summ + (((size_t)b * nblk + n) * Hkv + h) * d;
     float best = -FLT_MAX;
     for (int g = 0; g < G; ++g) {
       float part = 0.f;
@@ -236,19 +236,18 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const T* __restrict__ o
 
 }  // namespace
 
-cudaError_t launch_block_summaries(const Shape& s, const void* k_hist, int b0, int b1, float* summ,
-                                   cudaStream_t st) {
-  if (b1 <= b0) return cudaSuccess;
+cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src, int src_b0, int dst_b0, int nblocks,
+                                   float* summ, cudaStream_t st) {
+  if (nblocks <= 0) return cudaSuccess;
   const int V = s.bf16 ? 8 : 4;
   const int cols = s.Hkv * s.d;
-  dim3 grid(b1 - b0, (cols + 32 * V - 1) / (32 * V), s.B);
-  const int T_tok = s.nblk * s.blk;
+  dim3 grid(nblocks, (cols + 32 * V - 1) / (32 * V), s.B);
   if (s.bf16)
-    summaries_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k_hist), T_tok, s.Hkv,
-                                                          s.d, s.blk, s.nblk, b0, summ);
+    summaries_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k_src), T_src, s.Hkv,
+                                                          s.d, s.blk, src_b0, dst_b0, s.nblk, summ);
   else
-    summaries_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(k_hist), T_tok, s.Hkv, s.d, s.blk,
-                                                  s.nblk, b0, summ);
+    summaries_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(k_src), T_src, s.Hkv, s.d, s.blk, src_b0,
+                                                  dst_b0, s.nblk, summ);
   return cudaGetLastError();
 }
 

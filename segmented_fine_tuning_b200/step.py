@@ -20,7 +20,7 @@ class AttentionStep:
         self.dims = dims
         D = dims
         dt = D.torch_dtype
-        self.summ = torch.empty((D.B, D.Hkv, D.n_hist_blocks, D.d), dtype=torch.float32, device=device)
+        self.summ = torch.empty((D.B, D.n_hist_blocks, D.Hkv, D.d), dtype=torch.float32, device=device)
         self.idx = torch.empty((D.B, D.Hkv, D.nqb, D.topk), dtype=torch.int32, device=device)
         self.o = torch.empty((D.B, D.S, D.Hq, D.d), dtype=dt, device=device)
         self.lse = torch.empty((D.B, D.Hq, D.S), dtype=torch.float32, device=device)

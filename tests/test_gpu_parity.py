@@ -74,7 +74,7 @@ def test_summaries_and_selection(w):
     x = synth.draw(w)
     D = dims_of(w)
     q, kh = to_dev(x.q), to_dev(x.k_hist)
-    summ = torch.zeros((w.B, w.Hkv, w.nblk, w.d), dtype=torch.float32, device="cuda")
+    summ = torch.zeros((w.B, w.nblk, w.Hkv, w.d), dtype=torch.float32, device="cuda")
     idx = torch.empty((w.B, w.Hkv, w.nqb, w.topk), dtype=torch.int32, device="cuda")
     scores = torch.empty(idx.shape, dtype=torch.float32, device="cuda")
     hga_block_summaries(D, kh, 0, w.nblk, summ)
@@ -82,7 +82,7 @@ def test_summaries_and_selection(w):
     torch.cuda.synchronize()
     od = _odims(w)
     summ_ref = oracle.block_summaries(od, x.k_hist.f64)
-    s = to_host(summ)
+    s = to_host(summ).transpose(0, 2, 1, 3)  # block-major -> oracle layout [B, Hkv, nblk, d]
     assert np.abs(s - summ_ref).max() <= 1e-6 * max(1.0, np.abs(summ_ref).max())
     idx_ref, score_ref = oracle.select(od, x.q.f64, x.k_hist.f64)
     near = oracle.near_tie_positions(od, score_ref)
@@ -101,10 +101,10 @@ def test_summaries_partial_range_leaves_rest():
     w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 6, 2, "bf16", 24)
     x = synth.draw(w)
     D = dims_of(w)
-    summ = torch.full((1, 2, 6, 128), 7.0, device="cuda")
+    summ = torch.full((1, 6, 2, 128), 7.0, device="cuda")
     hga_block_summaries(D, to_dev(x.k_hist), 2, 4, summ)
     torch.cuda.synchronize()
-    s = summ.cpu().numpy()
+    s = summ.cpu().numpy().transpose(0, 2, 1, 3)
     ref = oracle.block_summaries(_odims(w), x.k_hist.f64)
     assert np.all(s[:, :, [0, 1, 4, 5]] == 7.0)
     assert np.abs(s[:, :, 2:4] - ref[:, :, 2:4]).max() < 1e-6
@@ -116,7 +116,7 @@ def test_select_q_zero_tie_rule():
     x = synth.draw(w)
     D = dims_of(w)
     q = torch.zeros((1, 256, 4, 128), dtype=torch.bfloat16, device="cuda")
-    summ = torch.empty((1, 2, 10, 128), device="cuda")
+    summ = torch.empty((1, 10, 2, 128), device="cuda")
     idx = torch.empty((1, 2, 2, 4), dtype=torch.int32, device="cuda")
     hga_block_summaries(D, to_dev(x.k_hist), 0, 10, summ)
     hga_select_topk(D, q, summ, idx)

@@ -34,7 +34,7 @@ def _forward(w, seed):
     x = synth.draw(w, seed=seed)
     D = dims_of(w)
     t = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
-    summ = torch.empty((w.B, w.Hkv, w.nblk, w.d), device="cuda")
+    summ = torch.empty((w.B, w.nblk, w.Hkv, w.d), device="cuda")
     idx = torch.empty((w.B, w.Hkv, w.nqb, w.topk), dtype=torch.int32, device="cuda")
     o = torch.empty_like(t["q"])
     lse = torch.empty((w.B, w.Hq, w.S), device="cuda")
