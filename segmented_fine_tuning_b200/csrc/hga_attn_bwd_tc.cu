@@ -13,19 +13,26 @@
 //   dK = dS^T Q / sqrt(d),   dV = P^T dO   (segment keys, summed over heads)
 //
 // Kernel 1 (dq_tc_kernel), one CTA per (b, query head, query block i), walks
-// the same tile list as the forward (selected history blocks, then segment
-// blocks 0..i).  Tensor memory: S double buffer | dP | dQ.  Per tile:
-// S = Q K^T, dP = dO V^T (tensor core); dS (CUDA cores, two warpgroups, 64
-// key columns each) is written as bf16 over the S columns it came from;
-// dQ += dS K with dS read from tensor memory.  S runs two tiles ahead and dP
-// one tile ahead of the dS pass.
+// the forward's tile list (selected history blocks, then segment blocks
+// 0..i).  Tensor memory: S double buffer | dP | dQ (128 columns each).  Per
+// tile: S = Q K^T and dP = dO V^T (M 128 queries, N 128 keys); dS (two
+// warpgroups, 64 key columns each) is written as bf16 over the S columns it
+// came from; dQ += dS K takes dS from tensor memory.  S runs two tiles ahead;
+// dP's buffer is released as soon as the dS pass has loaded it, so dP(j+1)
+// overlaps the dS math of tile j.
+//
+// Kernel 2 works in 64-query sub-tiles so that tensor memory holds two
+// sub-tiles of S^T and dP^T at once: while the CUDA cores turn sub-tile u into
+// P^T and dS^T, the tensor core finishes the products of sub-tile u-1 and
+// computes S^T and dP^T of sub-tile u+1.
 //
 // Kernel 2 (dkdv_tc_kernel), one CTA per (b, KV head, segment key block jb,
-// query head of the group), walks query blocks i >= jb.  It computes the
-// transposed products (keys in tensor-memory lanes): S^T = K Q^T,
-// dP^T = V dO^T, then P^T and dS^T in place as bf16, and accumulates
-// dV += P^T dO, dK += dS^T Q in tensor memory.  Each CTA adds its head's
-// partial dK/dV to the fp32 outputs with vector atomics.
+// query head of the group), walks query blocks i >= jb, each as two 64-query
+// halves, with the transposed products (keys in tensor-memory lanes):
+// S^T = K Q^T, dP^T = V dO^T (M 128 keys, N 64 queries), P^T and dS^T in
+// place as bf16, dV += P^T dO and dK += dS^T Q (K = 64 queries) accumulated
+// in tensor memory.  Each CTA adds its head's partial dK/dV to the fp32
+// outputs with vector atomics.
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
 
@@ -35,25 +42,16 @@ namespace {
 constexpr int kB = 128;  // rows / keys per tile
 constexpr int kD = 128;
 constexpr int kTileBytes = kB * kD * 2;
-constexpr int kHalf = kTileBytes / 2;
+constexpr int kHalf = kTileBytes / 2;        // one 64-channel TMA box: 128 rows x 128 B
+constexpr int kSubRows = 64;                 // rows of a sub-tile
+constexpr int kSubOff = kSubRows * 128;      // byte offset of the second 64-row half inside a box
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// ============================================================== dQ kernel
-constexpr int kKStages = 3, kVStages = 2;
-
-struct DqCtl {
-  uint64_t qdo_full;
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t sdp_full, ds_full, dq_full, mma_done;
-  uint32_t tmem;
-  int abort;
-  int nt;
-  int tiles[kMaxTiles];
-};
-constexpr size_t kDqSmem = 1024 + (2 + kKStages + kVStages) * kTileBytes + sizeof(DqCtl);
-static_assert(kDqSmem <= 232448, "shared memory budget");
+// A bf16 chunk of 32 elements packed as 16 columns sits at the first 16 of
+// the 32 fp32 columns it was computed from; k-step kk (16 elements) of a
+// 64-element sub-tile therefore starts at column (kk / 2) * 32 + (kk % 2) * 8.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 
 struct BwdArgs {
   int B, Hq, Hkv, S, nkv, topk, nqb, G;
@@ -68,6 +66,32 @@ struct BwdArgs {
   int* err;
 };
 
+// ============================================================== dQ kernel
+constexpr int kKStages = 3, kVStages = 2;
+
+struct DqCtl {
+  uint64_t qdo_full;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t sdp_full[2], ds_full[2];
+  uint64_t dp_free;
+  uint64_t dq_full, mma_done;
+  uint32_t tmem;
+  int abort;
+  int nt;
+  int tiles[kMaxTiles];
+};
+constexpr size_t kDqSmem = 1024 + (2 + kKStages + kVStages) * kTileBytes + sizeof(DqCtl);
+static_assert(kDqSmem <= 232448, "shared memory budget");
+
+// Tensor-memory columns of the dQ kernel: S double buffer, dP, dQ.
+constexpr uint32_t kDqS = 0, kDqP = 256, kDqAcc = 384;
+
+// dQ kernel: full 128-key tiles (N = 128 products: half the shared-memory
+// re-reads of A per FLOP compared with 64-key halves).  S is double-buffered
+// and runs two tiles ahead.  dP has one buffer, but the dS pass releases it as
+// soon as it has loaded its columns (dp_free), so dP(j+1) is computed while
+// dS(j) is being formed; dQ(j) follows dS(j).
 __global__ void __launch_bounds__(320, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
@@ -83,7 +107,7 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_i = a.B * a.Hq;
-  const int i = a.nqb - 1 - (int)(blockIdx.x / per_i);
+  const int i = a.nqb - 1 - (int)(blockIdx.x / per_i);  // longest tile lists first
   const int rem = (int)(blockIdx.x % per_i);
   const int b = rem / a.Hq, hq = rem % a.Hq;
   const int kvh = hq / a.G;
@@ -107,8 +131,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&ctl->qdo_full, 1);
       for (int s = 0; s < kKStages; ++s) { mbar_init(&ctl->k_full[s], 1); mbar_init(&ctl->k_empty[s], 1); }
       for (int s = 0; s < kVStages; ++s) { mbar_init(&ctl->v_full[s], 1); mbar_init(&ctl->v_empty[s], 1); }
-      mbar_init(&ctl->sdp_full, 1);
-      mbar_init(&ctl->ds_full, 256);
+      for (int x = 0; x < 2; ++x) { mbar_init(&ctl->sdp_full[x], 1); mbar_init(&ctl->ds_full[x], 256); }
+      mbar_init(&ctl->dp_free, 256);
       mbar_init(&ctl->dq_full, 1);
       mbar_init(&ctl->mma_done, 1);
       fence_mbar_init();
@@ -125,6 +149,7 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort = &ctl->abort;
 
   if (warp == 8) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_expect_tx(&ctl->qdo_full, 2 * kTileBytes);
       for (int hh = 0; hh < 2; ++hh) {
@@ -158,60 +183,71 @@ __global__ void __launch_bounds__(320, 1)
         mbar_wait(&ctl->v_full[j % kVStages], (j / kVStages) & 1, &no_abort, a.err);
     }
   } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(kB, kB, false, false);
-      constexpr uint32_t kIdQ = idesc_bf16(kB, kD, false, true);
-      const uint32_t sq = smem_u32(sQ), sdo = smem_u32(sDO), sk = smem_u32(sK), sv = smem_u32(sV);
-      auto kmajor = [&](uint32_t A, uint32_t Bm, uint32_t d_col) {
+      constexpr uint32_t kIdS = idesc_bf16(kB, kB, false, false);  // [128 q x 128 keys] = Q K^T, dO V^T
+      constexpr uint32_t kIdQ = idesc_bf16(kB, kD, false, true);   // dQ += dS (tmem) K (MN-major)
+      // Descriptors built once; k-steps and ring slots are constant adds.
+      const uint64_t dQd = sdesc_sw128(smem_u32(sQ), 16, 1024), dOd = sdesc_sw128(smem_u32(sDO), 16, 1024);
+      const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024), dVk = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dKmn = sdesc_sw128(smem_u32(sK), kHalf, 1024);  // K as the MN-major B of dQ += dS K
+      auto wait_k = [=](int j) { return mbar_wait(&ctl->k_full[j % kKStages], (j / kKStages) & 1, abort, a.err); };
+      auto wait_v = [=](int j) { return mbar_wait(&ctl->v_full[j % kVStages], (j / kVStages) & 1, abort, a.err); };
+      auto issue_s = [=](int j) {  // S(j) = Q K_j^T into buffer j % 2
+        const uint64_t kb = dKk + sdesc_units((j % kKStages) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_ss(tmem + d_col, sdesc_sw128(A + off, 16, 1024), sdesc_sw128(Bm + off, 16, 1024), kIdS, kk > 0);
+          const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
+          umma_ss(tmem + kDqS + (j & 1) * 128, dQd + off, kb + off, kIdS, kk > 0);
         }
       };
-      auto wait_k = [&](int j) { return mbar_wait(&ctl->k_full[j % kKStages], (j / kKStages) & 1, abort, a.err); };
-      auto wait_v = [&](int j) { return mbar_wait(&ctl->v_full[j % kVStages], (j / kVStages) & 1, abort, a.err); };
+      auto issue_dp = [=](int j) {  // dP(j) = dO V_j^T
+        const uint64_t vb = dVk + sdesc_units((j % kVStages) * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
+          umma_ss(tmem + kDqP, dOd + off, vb + off, kIdS, kk > 0);
+        }
+        umma_commit(&ctl->sdp_full[j & 1]);           // S(j) was issued earlier: both ready
+        umma_commit(&ctl->v_empty[j % kVStages]);     // V_j's only reader
+      };
       bool ok = mbar_wait(&ctl->qdo_full, 0, abort, a.err) && wait_k(0) && wait_v(0);
       if (ok) {
         tc_fence_after();
-        kmajor(sq, sk, 0);                       // S(0) -> buffer 0
-        kmajor(sdo, sv, 256);                    // dP(0)
-        umma_commit(&ctl->sdp_full);
-        umma_commit(&ctl->v_empty[0]);
+        issue_s(0);
+        issue_dp(0);
         if (nt > 1) {
           ok = wait_k(1);
           if (ok) {
             tc_fence_after();
-            kmajor(sq, sk + (1 % kKStages) * kTileBytes, 128);  // S(1) -> buffer 1
+            issue_s(1);
           }
         }
       }
       for (int j = 0; ok && j < nt; ++j) {
-        if (!mbar_wait(&ctl->ds_full, j & 1, abort, a.err)) break;
-        tc_fence_after();
-        const uint32_t sb = (uint32_t)(j & 1) * 128;
-        const uint32_t kslot = sk + (j % kKStages) * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kB / 16; ++kk) {
-          const uint32_t pcol = (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_ts(tmem + 384, tmem + sb + pcol, sdesc_sw128(kslot + kk * 2048, kHalf, 1024), kIdQ,
-                  (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&ctl->k_empty[j % kKStages]);
         if (j + 1 < nt) {
-          if (!wait_v(j + 1)) break;
+          // dP(j+1) as soon as the dS pass has read dP(j)
+          if (!mbar_wait(&ctl->dp_free, j & 1, abort, a.err) || !wait_v(j + 1)) break;
           tc_fence_after();
-          kmajor(sdo, sv + ((j + 1) % kVStages) * kTileBytes, 256);
-          umma_commit(&ctl->sdp_full);
-          umma_commit(&ctl->v_empty[(j + 1) % kVStages]);
+          issue_dp(j + 1);
         }
+        if (!mbar_wait(&ctl->ds_full[j & 1], (j >> 1) & 1, abort, a.err)) break;
+        tc_fence_after();
+        const uint64_t kb = dKmn + sdesc_units((j % kKStages) * kTileBytes);
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kB / 16; ++kk)
+          umma_ts(tmem + kDqAcc, tmem + kDqS + (j & 1) * 128 + packed_col(kk), kb + sdesc_units(kk * 2048), kIdQ,
+                  kk > 0 ? 1u : acc0);
+        umma_commit(&ctl->k_empty[j % kKStages]);  // K_j's last reader
         if (j + 2 < nt) {
           if (!wait_k(j + 2)) break;
           tc_fence_after();
-          kmajor(sq, sk + ((j + 2) % kKStages) * kTileBytes, sb);
+          issue_s(j + 2);  // into buffer j % 2, after dQ(j) read dS(j) from it
         }
         if (j == nt - 1) umma_commit(&ctl->dq_full);
       }
+      // All issued MMAs must finish before tensor memory is released.
       umma_commit(&ctl->mma_done);
       volatile int no_abort = 0;
       mbar_wait(&ctl->mma_done, 0, &no_abort, a.err);
@@ -219,7 +255,7 @@ __global__ void __launch_bounds__(320, 1)
   } else {
     // ------------------------------------------------------------ dS pass
     const int e = warp >> 2, wq = warp & 3;
-    const int r = wq * 32 + lane;
+    const int r = wq * 32 + lane;  // query row within block i
     const int p = i * kB + r;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const size_t rrow = ((size_t)b * a.Hq + hq) * a.S + p;
@@ -227,47 +263,51 @@ __global__ void __launch_bounds__(320, 1)
     const float Dv = __ldg(a.Dr + rrow);
     const float sl2 = a.sl2;
     bool ok = true;
-    uint32_t sv[32], dv[32];
+    uint32_t sd[128];  // S columns [64e, 64e+64) of this row, then dP columns [64e, 64e+64)
     for (int j = 0; j < nt; ++j) {
+      const int x = j & 1;
       // tcgen05.ld/st are warp-collective: branches around them are warp-uniform.
-      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full, j & 1, abort, a.err))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full[x], (j >> 1) & 1, abort, a.err))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      tmem_ld64x2_wait(tmem + lane_off + kDqS + x * 128 + 64 * e, tmem + lane_off + kDqP + 64 * e, sd);
+      tc_fence_before();
+      mbar_arrive(&ctl->dp_free);  // dP(j) is in registers: the tensor core may overwrite it
       const bool diag = (j == nt - 1);
-      const uint32_t sb = (uint32_t)(j & 1) * 128;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * e + cc;
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + sb + c * 32, sv);
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + 256 + c * 32, dv);
         uint32_t pk[16];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const bool k0 = !diag || c * 32 + x <= r;
-          const bool k1 = !diag || c * 32 + x + 1 <= r;
-          const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(sv[x]), sl2, -lse2)) : 0.f;
-          const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(sv[x + 1]), sl2, -lse2)) : 0.f;
-          pk[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[x]) - Dv), p1 * (__uint_as_float(dv[x + 1]) - Dv));
+        for (int xx = 0; xx < 32; xx += 2) {
+          const int key = 64 * e + 32 * cc + xx;  // key column within the tile
+          const bool k0 = !diag || key <= r;
+          const bool k1 = !diag || key + 1 <= r;
+          const float s0 = __uint_as_float(sd[32 * cc + xx]), s1 = __uint_as_float(sd[32 * cc + xx + 1]);
+          const float p0 = k0 ? ex2_approx(fmaf(s0, sl2, -lse2)) : 0.f;
+          const float p1 = k1 ? ex2_approx(fmaf(s1, sl2, -lse2)) : 0.f;
+          pk[xx >> 1] = pack_bf16x2(p0 * (__uint_as_float(sd[64 + 32 * cc + xx]) - Dv),
+                                    p1 * (__uint_as_float(sd[64 + 32 * cc + xx + 1]) - Dv));
         }
-        HGA_TMEM_ST16(tmem + lane_off + sb + c * 32, pk);
+        HGA_TMEM_ST16(tmem + lane_off + kDqS + x * 128 + 64 * e + 32 * cc, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ctl->ds_full);
+      mbar_arrive(&ctl->ds_full[x]);
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dq_full, 0, abort, a.err))) {
       tc_fence_after();
       float* out = a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + 64 * e;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + 384 + 64 * e + 32 * cc, sv);
+        uint32_t v[32];
+        HGA_TMEM_LD32_WAIT(tmem + lane_off + kDqAcc + 64 * e + 32 * cc, v);
         float4* dst = reinterpret_cast<float4*>(out + 32 * cc);
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-          dst[x] = make_float4(__uint_as_float(sv[4 * x]) * a.scale, __uint_as_float(sv[4 * x + 1]) * a.scale,
-                               __uint_as_float(sv[4 * x + 2]) * a.scale, __uint_as_float(sv[4 * x + 3]) * a.scale);
+        for (int xx = 0; xx < 8; ++xx)
+          dst[xx] = make_float4(__uint_as_float(v[4 * xx]) * a.scale, __uint_as_float(v[4 * xx + 1]) * a.scale,
+                                __uint_as_float(v[4 * xx + 2]) * a.scale, __uint_as_float(v[4 * xx + 3]) * a.scale);
       }
     }
   }
@@ -286,7 +326,8 @@ constexpr int kQStages = 2;
 struct DkvCtl {
   uint64_t kv_full;
   uint64_t qd_full[kQStages], qd_empty[kQStages];
-  uint64_t sdp_full, pds_full, dkv_full, mma_done;
+  uint64_t sdp_full[2], pds_full[2];
+  uint64_t dkv_full, mma_done;
   uint32_t tmem;
   int abort;
 };
@@ -296,6 +337,9 @@ struct __align__(16) RowStats {
 };
 constexpr size_t kDkvSmem = 1024 + (2 + 2 * kQStages) * kTileBytes + kQStages * sizeof(RowStats) + sizeof(DkvCtl);
 static_assert(kDkvSmem <= 232448, "shared memory budget");
+
+// Tensor-memory columns of the dK/dV kernel.
+constexpr uint32_t kKvS = 0, kKvP = 128, kKvDK = 256, kKvDV = 384;
 
 __global__ void __launch_bounds__(320, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -318,14 +362,14 @@ __global__ void __launch_bounds__(320, 1)
   const int b = rem / a.Hq, hq = rem % a.Hq;
   const int kvh = hq / a.G;
   const int n = a.nqb - jb;  // query blocks jb..nqb-1
+  const int nsub = 2 * n;
 
   if (warp == 0) {
     if (lane == 0) {
       ctl->abort = 0;
       mbar_init(&ctl->kv_full, 1);
       for (int s = 0; s < kQStages; ++s) { mbar_init(&ctl->qd_full[s], 1); mbar_init(&ctl->qd_empty[s], 1); }
-      mbar_init(&ctl->sdp_full, 1);
-      mbar_init(&ctl->pds_full, 256);
+      for (int x = 0; x < 2; ++x) { mbar_init(&ctl->sdp_full[x], 1); mbar_init(&ctl->pds_full[x], 256); }
       mbar_init(&ctl->dkv_full, 1);
       mbar_init(&ctl->mma_done, 1);
       fence_mbar_init();
@@ -341,6 +385,7 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort = &ctl->abort;
 
   if (warp == 8) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_expect_tx(&ctl->kv_full, 2 * kTileBytes);
       for (int hh = 0; hh < 2; ++hh) {
@@ -368,49 +413,62 @@ __global__ void __launch_bounds__(320, 1)
         mbar_wait(&ctl->qd_full[it % kQStages], (it / kQStages) & 1, &no_abort, a.err);
     }
   } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdT = idesc_bf16(kB, kB, false, false);  // K Q^T, V dO^T
-      constexpr uint32_t kIdG = idesc_bf16(kB, kD, false, true);   // P^T dO, dS^T Q
-      const uint32_t sk = smem_u32(sK), sv = smem_u32(sV), sq = smem_u32(sQ), sdo = smem_u32(sDO);
-      auto kmajor = [&](uint32_t A, uint32_t Bm, uint32_t d_col) {
+      constexpr uint32_t kIdT = idesc_bf16(kB, kSubRows, false, false);  // [128 keys x 64 queries]
+      constexpr uint32_t kIdG = idesc_bf16(kB, kD, false, true);         // dV += P^T dO_half, dK += dS^T Q_half
+      // Descriptors built once; k-steps, query halves and stages are constant adds.
+      const uint64_t dKd = sdesc_sw128(smem_u32(sK), 16, 1024), dVd = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024), dOk = sdesc_sw128(smem_u32(sDO), 16, 1024);
+      const uint64_t dQmn = sdesc_sw128(smem_u32(sQ), kHalf, 1024), dOmn = sdesc_sw128(smem_u32(sDO), kHalf, 1024);
+      // S^T and dP^T of sub-tile u (query block jb + u/2, query half u%2) into buffer u%2.
+      auto issue_sdp = [=](int u) -> bool {
+        const int it = u >> 1, h = u & 1, s = it % kQStages;
+        if (h == 0) {
+          if (!mbar_wait(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err)) return false;
+          tc_fence_after();
+        }
+        const uint32_t so = sdesc_units(s * kTileBytes + h * kSubOff);
+        const uint64_t qb = dQk + so, ob = dOk + so;
+        const uint32_t ts = tmem + kKvS + h * 64, tp = tmem + kKvP + h * 64;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_ss(tmem + d_col, sdesc_sw128(A + off, 16, 1024), sdesc_sw128(Bm + off, 16, 1024), kIdT, kk > 0);
+          const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
+          umma_ss(ts, dKd + off, qb + off, kIdT, kk > 0);
         }
-      };
-      auto tsmma = [&](uint32_t a_col, uint32_t Bm, uint32_t d_col, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < kB / 16; ++kk) {
-          const uint32_t pcol = (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_ts(tmem + d_col, tmem + a_col + pcol, sdesc_sw128(Bm + kk * 2048, kHalf, 1024), kIdG,
-                  (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
+          umma_ss(tp, dVd + off, ob + off, kIdT, kk > 0);
         }
+        umma_commit(&ctl->sdp_full[h]);
+        return true;
       };
-      bool ok = mbar_wait(&ctl->kv_full, 0, abort, a.err) && mbar_wait(&ctl->qd_full[0], 0, abort, a.err);
+      bool ok = mbar_wait(&ctl->kv_full, 0, abort, a.err);
       if (ok) {
         tc_fence_after();
-        kmajor(sk, sq, 0);
-        kmajor(sv, sdo, 128);
-        umma_commit(&ctl->sdp_full);
+        ok = issue_sdp(0) && issue_sdp(1);
       }
-      for (int it = 0; ok && it < n; ++it) {
-        const int s = it % kQStages;
-        if (!mbar_wait(&ctl->pds_full, it & 1, abort, a.err)) break;
+      for (int u = 0; ok && u < nsub; ++u) {
+        const int it = u >> 1, h = u & 1, s = it % kQStages;
+        if (!mbar_wait(&ctl->pds_full[h], (u >> 1) & 1, abort, a.err)) break;
         tc_fence_after();
-        tsmma(0, sdo + s * kTileBytes, 384, it > 0);    // dV += P^T dO
-        tsmma(128, sq + s * kTileBytes, 256, it > 0);   // dK += dS^T Q
-        umma_commit(&ctl->qd_empty[s]);
-        if (it + 1 < n) {
-          const int s1 = (it + 1) % kQStages;
-          if (!mbar_wait(&ctl->qd_full[s1], ((it + 1) / kQStages) & 1, abort, a.err)) break;
-          tc_fence_after();
-          kmajor(sk, sq + s1 * kTileBytes, 0);
-          kmajor(sv, sdo + s1 * kTileBytes, 128);
-          umma_commit(&ctl->sdp_full);
-        } else {
-          umma_commit(&ctl->dkv_full);
+        const uint32_t so = sdesc_units(s * kTileBytes + h * kSubOff);
+        const uint64_t qb = dQmn + so, ob = dOmn + so;
+        const uint32_t acc0 = u > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kSubRows / 16; ++kk)  // dV += P^T dO_half
+          umma_ts(tmem + kKvDV, tmem + kKvS + h * 64 + packed_col(kk), ob + sdesc_units(kk * 2048), kIdG,
+                  kk > 0 ? 1u : acc0);
+#pragma unroll
+        for (int kk = 0; kk < kSubRows / 16; ++kk)  // dK += dS^T Q_half
+          umma_ts(tmem + kKvDK, tmem + kKvP + h * 64 + packed_col(kk), qb + sdesc_units(kk * 2048), kIdG,
+                  kk > 0 ? 1u : acc0);
+        if (h == 1) umma_commit(&ctl->qd_empty[s]);
+        if (u + 2 < nsub) {
+          if (!issue_sdp(u + 2)) break;
         }
+        if (u == nsub - 1) umma_commit(&ctl->dkv_full);
       }
       umma_commit(&ctl->mma_done);
       volatile int no_abort = 0;
@@ -423,12 +481,12 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float sl2 = a.sl2;
     bool ok = true;
-    uint32_t sv[32], dv[32];
-    for (int it = 0; it < n; ++it) {
-      const int s = it % kQStages;
+    uint32_t sd[64];  // 32 S^T columns then 32 dP^T columns of this thread's key row
+    for (int u = 0; u < nsub; ++u) {
+      const int it = u >> 1, h = u & 1, s = it % kQStages;
       // The row statistics arrive with the Q/dO stage: observe that stage's
       // barrier directly (its phase is complete by now) before reading them.
-      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full, it & 1, abort, a.err) &&
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full[h], (u >> 1) & 1, abort, a.err) &&
                                        mbar_wait(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err))) {
         ok = false;
         break;
@@ -436,46 +494,43 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const bool diag = (it == 0);
       const RowStats& rs = stats[s];
+      tmem_ld32x2_wait(tmem + lane_off + kKvS + h * 64 + 32 * e, tmem + lane_off + kKvP + h * 64 + 32 * e, sd);
+      const int q0 = 64 * h + 32 * e;  // query column of sd[0] within block i
+      uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * e + cc;
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + c * 32, sv);
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + 128 + c * 32, dv);
-        uint32_t pp[16], pd[16];
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const int q0 = c * 32 + x;  // query column within block i
-          const bool k0 = !diag || q0 >= r;
-          const bool k1 = !diag || q0 + 1 >= r;
-          const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(sv[x]), sl2, -rs.lse[q0] * kLog2e)) : 0.f;
-          const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(sv[x + 1]), sl2, -rs.lse[q0 + 1] * kLog2e)) : 0.f;
-          pp[x >> 1] = pack_bf16x2(p0, p1);
-          pd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(dv[x]) - rs.D[q0]),
-                                   p1 * (__uint_as_float(dv[x + 1]) - rs.D[q0 + 1]));
-        }
-        HGA_TMEM_ST16(tmem + lane_off + c * 32, pp);
-        HGA_TMEM_ST16(tmem + lane_off + 128 + c * 32, pd);
+      for (int x = 0; x < 32; x += 2) {
+        const int q = q0 + x;
+        const bool k0 = !diag || q >= r;
+        const bool k1 = !diag || q + 1 >= r;
+        const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(sd[x]), sl2, -rs.lse[q] * kLog2e)) : 0.f;
+        const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(sd[x + 1]), sl2, -rs.lse[q + 1] * kLog2e)) : 0.f;
+        pp[x >> 1] = pack_bf16x2(p0, p1);
+        pd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(sd[32 + x]) - rs.D[q]),
+                                 p1 * (__uint_as_float(sd[33 + x]) - rs.D[q + 1]));
       }
+      HGA_TMEM_ST16(tmem + lane_off + kKvS + h * 64 + 32 * e, pp);
+      HGA_TMEM_ST16(tmem + lane_off + kKvP + h * 64 + 32 * e, pd);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ctl->pds_full);
+      mbar_arrive(&ctl->pds_full[h]);
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err))) {
       tc_fence_after();
       const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + 64 * e;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + 256 + 64 * e + 32 * cc, sv);
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + 384 + 64 * e + 32 * cc, dv);
-        float4* gk = reinterpret_cast<float4*>(a.dk + off + 32 * cc);
-        float4* gv = reinterpret_cast<float4*>(a.dv + off + 32 * cc);
+        uint32_t gk[32], gv[32];
+        HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDK + 64 * e + 32 * cc, gk);
+        HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDV + 64 * e + 32 * cc, gv);
+        float4* pk4 = reinterpret_cast<float4*>(a.dk + off + 32 * cc);
+        float4* pv4 = reinterpret_cast<float4*>(a.dv + off + 32 * cc);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          atomicAdd(gk + x, make_float4(__uint_as_float(sv[4 * x]) * a.scale, __uint_as_float(sv[4 * x + 1]) * a.scale,
-                                        __uint_as_float(sv[4 * x + 2]) * a.scale,
-                                        __uint_as_float(sv[4 * x + 3]) * a.scale));
-          atomicAdd(gv + x, make_float4(__uint_as_float(dv[4 * x]), __uint_as_float(dv[4 * x + 1]),
-                                        __uint_as_float(dv[4 * x + 2]), __uint_as_float(dv[4 * x + 3])));
+          atomicAdd(pk4 + x, make_float4(__uint_as_float(gk[4 * x]) * a.scale, __uint_as_float(gk[4 * x + 1]) * a.scale,
+                                         __uint_as_float(gk[4 * x + 2]) * a.scale,
+                                         __uint_as_float(gk[4 * x + 3]) * a.scale));
+          atomicAdd(pv4 + x, make_float4(__uint_as_float(gv[4 * x]), __uint_as_float(gv[4 * x + 1]),
+                                         __uint_as_float(gv[4 * x + 2]), __uint_as_float(gv[4 * x + 3])));
         }
       }
     }

@@ -175,25 +175,32 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);  // Q, K both K-major
       constexpr uint32_t kIdO = idesc_bf16(kBM, kD, false, true);    // P (tmem) x V (MN-major)
-      const uint32_t sq = smem_u32(sQ), sr = smem_u32(sRing);
-      auto issue_S = [&](int t, int s) {
+      // Descriptors are built once; every k-step and ring slot is a constant
+      // add to the start-address field, so the issuing thread spends a few
+      // cycles per tcgen05.mma instead of rebuilding descriptors.
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);          // Q tiles, K-major
+      const uint64_t dK = sdesc_sw128(smem_u32(sRing), 16, 1024);       // ring as K tiles, K-major
+      const uint64_t dV = sdesc_sw128(smem_u32(sRing), kHalf, 1024);    // ring as V tiles, MN-major
+      auto issue_S = [=](int t, int s) {
+        const uint64_t a0 = dQ + sdesc_units(t * kTileBytes), b0 = dK + sdesc_units(s * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_ss(tmem + t * 128, sdesc_sw128(sq + t * kTileBytes + off, 16, 1024),
-                  sdesc_sw128(sr + s * kTileBytes + off, 16, 1024), kIdS, kk > 0);
+          const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
+          umma_ss(tmem + t * 128, a0 + off, b0 + off, kIdS, kk > 0);
         }
       };
-      auto issue_PV = [&](int t, int s, bool acc) {
+      auto issue_PV = [=](int t, int s, bool acc) {
+        const uint64_t b0 = dV + sdesc_units(s * kTileBytes);
+        const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           // P chunk c (keys 32c..32c+31) sits at S columns [32c, 32c+16).
           const uint32_t pcol = (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + pcol, sdesc_sw128(sr + s * kTileBytes + kk * 2048, kHalf, 1024),
-                  kIdO, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + pcol, b0 + sdesc_units(kk * 2048), kIdO,
+                  kk > 0 ? 1u : acc0);
         }
       };
-      auto wait_full = [&](int pos) {
+      auto wait_full = [=](int pos) {
         return mbar_wait(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, abort, a.err);
       };
       bool ok = mbar_wait(&ctl->q_full, 0, abort, a.err) && wait_full(0);
@@ -248,7 +255,7 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = a.sl2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t v[32];
+    uint32_t v[128];
     for (int j = 0; j < nt; ++j) {
       // tcgen05.ld/st are warp-collective: every branch around them is
       // decided for the whole warp.
@@ -257,46 +264,51 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      const bool diag = (j == nt - 1);
-      float mx = -INFINITY;
+      // The whole S row in one pass: 128 columns, one wait.
+      tmem_ld128_wait(tS, v);
+      if (j == nt - 1) {
+        // diagonal segment tile: keys after the query's own position are masked
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        HGA_TMEM_LD32_WAIT(tS + c * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (!diag || c * 32 + e <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
+        for (int e = 0; e < 128; ++e)
+          if (e > r) v[e] = 0xFF800000u;  // -inf
       }
-      mx *= sl2;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int e = 0; e < 128; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(v[e]));
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       const bool need = mx > m_ref + kRescaleThreshold;
-      if (__any_sync(0xffffffffu, need)) {
-        // Rows that keep their reference use alpha = 1.
-        const float alpha = need ? ex2_approx(m_ref - mx) : 1.0f;
+      const bool any_need = __any_sync(0xffffffffu, need);
+      float alpha = 1.0f;  // rows that keep their reference use alpha = 1
+      if (need) {
+        alpha = ex2_approx(m_ref - mx);
         l *= alpha;
-        if (j > 0) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            HGA_TMEM_LD32_WAIT(tO + c * 32, v);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            HGA_TMEM_ST32(tO + c * 32, v);
-          }
-        }
-        if (need) m_ref = mx;
+        m_ref = mx;
       }
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        HGA_TMEM_LD32_WAIT(tS + c * 32, v);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const bool k0 = !diag || c * 32 + e <= r;
-          const bool k1 = !diag || c * 32 + e + 1 <= r;
-          const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(v[e]), sl2, -m_ref)) : 0.f;
-          const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), sl2, -m_ref)) : 0.f;
-          l += p0 + p1;
+          const float p0 = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -m_ref));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -m_ref));
+          l4[(e >> 1) & 3] += p0 + p1;
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         HGA_TMEM_ST16(tS + c * 32, pk);
+      }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      if (any_need && j > 0) {
+        // O_t holds the sum up to tile j-1 (PV_t(j-1) completed before S_t(j)
+        // was announced): bring it to the new reference.
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          HGA_TMEM_ST32(tO + c * 32, ov);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -310,15 +322,16 @@ __global__ void __launch_bounds__(384, 1)
       __nv_bfloat16* orow = a.o + (((size_t)b * a.S + p) * a.Hq + hq) * kD;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        HGA_TMEM_LD32_WAIT(tO + c * 32, v);
+        uint32_t ov[32];
+        HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
         for (int qd = 0; qd < 4; ++qd) {
           uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[8 * qd + 0]) * inv_l, __uint_as_float(v[8 * qd + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(v[8 * qd + 2]) * inv_l, __uint_as_float(v[8 * qd + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(v[8 * qd + 4]) * inv_l, __uint_as_float(v[8 * qd + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(v[8 * qd + 6]) * inv_l, __uint_as_float(v[8 * qd + 7]) * inv_l);
+          w.x = pack_bf16x2(__uint_as_float(ov[8 * qd + 0]) * inv_l, __uint_as_float(ov[8 * qd + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(ov[8 * qd + 2]) * inv_l, __uint_as_float(ov[8 * qd + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(ov[8 * qd + 4]) * inv_l, __uint_as_float(ov[8 * qd + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(ov[8 * qd + 6]) * inv_l, __uint_as_float(ov[8 * qd + 7]) * inv_l);
           dst[qd] = w;
         }
       }
