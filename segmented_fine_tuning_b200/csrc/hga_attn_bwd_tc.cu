@@ -32,7 +32,7 @@
 // S^T = K Q^T, dP^T = V dO^T (M 128 keys, N 64 queries), P^T and dS^T in
 // place as bf16, dV += P^T dO and dK += dS^T Q (K = 64 queries) accumulated
 // in tensor memory.  Each CTA adds its head's partial dK/dV to the fp32
-// outputs with vector atomics.
+// outputs with vector reductions (red.global.add.v4.f32).
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
 
@@ -502,11 +502,12 @@ __global__ void __launch_bounds__(320, 1)
         const int q = q0 + x;
         const bool k0 = !diag || q >= r;
         const bool k1 = !diag || q + 1 >= r;
-        const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(sd[x]), sl2, -rs.lse[q] * kLog2e)) : 0.f;
-        const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(sd[x + 1]), sl2, -rs.lse[q + 1] * kLog2e)) : 0.f;
+        const float2 lq = *reinterpret_cast<const float2*>(&rs.lse[q]);  // same for every key row: broadcast
+        const float2 dq2 = *reinterpret_cast<const float2*>(&rs.D[q]);
+        const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(sd[x]), sl2, -lq.x * kLog2e)) : 0.f;
+        const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(sd[x + 1]), sl2, -lq.y * kLog2e)) : 0.f;
         pp[x >> 1] = pack_bf16x2(p0, p1);
-        pd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(sd[32 + x]) - rs.D[q]),
-                                 p1 * (__uint_as_float(sd[33 + x]) - rs.D[q + 1]));
+        pd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(sd[32 + x]) - dq2.x), p1 * (__uint_as_float(sd[33 + x]) - dq2.y));
       }
       HGA_TMEM_ST16(tmem + lane_off + kKvS + h * 64 + 32 * e, pp);
       HGA_TMEM_ST16(tmem + lane_off + kKvP + h * 64 + 32 * e, pd);
@@ -522,15 +523,14 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t gk[32], gv[32];
         HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDK + 64 * e + 32 * cc, gk);
         HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDV + 64 * e + 32 * cc, gv);
-        float4* pk4 = reinterpret_cast<float4*>(a.dk + off + 32 * cc);
-        float4* pv4 = reinterpret_cast<float4*>(a.dv + off + 32 * cc);
+        float* pk4 = a.dk + off + 32 * cc;
+        float* pv4 = a.dv + off + 32 * cc;
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          atomicAdd(pk4 + x, make_float4(__uint_as_float(gk[4 * x]) * a.scale, __uint_as_float(gk[4 * x + 1]) * a.scale,
-                                         __uint_as_float(gk[4 * x + 2]) * a.scale,
-                                         __uint_as_float(gk[4 * x + 3]) * a.scale));
-          atomicAdd(pv4 + x, make_float4(__uint_as_float(gv[4 * x]), __uint_as_float(gv[4 * x + 1]),
-                                         __uint_as_float(gv[4 * x + 2]), __uint_as_float(gv[4 * x + 3])));
+          red_add_v4(pk4 + 4 * x, __uint_as_float(gk[4 * x]) * a.scale, __uint_as_float(gk[4 * x + 1]) * a.scale,
+                     __uint_as_float(gk[4 * x + 2]) * a.scale, __uint_as_float(gk[4 * x + 3]) * a.scale);
+          red_add_v4(pv4 + 4 * x, __uint_as_float(gv[4 * x]), __uint_as_float(gv[4 * x + 1]),
+                     __uint_as_float(gv[4 * x + 2]), __uint_as_float(gv[4 * x + 3]));
         }
       }
     }
