@@ -47,6 +47,9 @@ constexpr int kSubRows = 64;                 // rows of a sub-tile
 constexpr int kSubOff = kSubRows * 128;      // byte offset of the second 64-row half inside a box
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kLog2e = 1.4426950408889634f;
+// Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
+// instead of the ex2 unit.
+constexpr uint32_t kBwdPolyPairs = 0x5252u;
 
 // A bf16 chunk of 32 elements packed as 16 columns sits at the first 16 of
 // the 32 fp32 columns it was computed from; k-step kk (16 elements) of a
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(320, 1)
     const size_t rrow = ((size_t)b * a.Hq + hq) * a.S + p;
     const float lse2 = __ldg(a.lse + rrow) * kLog2e;
     const float Dv = __ldg(a.Dr + rrow);
-    const float sl2 = a.sl2;
+    const float2 s2 = make_float2(a.sl2, a.sl2), nl = make_float2(-lse2, -lse2), D2 = make_float2(Dv, Dv);
     bool ok = true;
     uint32_t sd[128];  // S columns [64e, 64e+64) of this row, then dP columns [64e, 64e+64)
     for (int j = 0; j < nt; ++j) {
@@ -282,13 +285,17 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int xx = 0; xx < 32; xx += 2) {
           const int key = 64 * e + 32 * cc + xx;  // key column within the tile
-          const bool k0 = !diag || key <= r;
-          const bool k1 = !diag || key + 1 <= r;
-          const float s0 = __uint_as_float(sd[32 * cc + xx]), s1 = __uint_as_float(sd[32 * cc + xx + 1]);
-          const float p0 = k0 ? ex2_approx(fmaf(s0, sl2, -lse2)) : 0.f;
-          const float p1 = k1 ? ex2_approx(fmaf(s1, sl2, -lse2)) : 0.f;
-          pk[xx >> 1] = pack_bf16x2(p0 * (__uint_as_float(sd[64 + 32 * cc + xx]) - Dv),
-                                    p1 * (__uint_as_float(sd[64 + 32 * cc + xx + 1]) - Dv));
+          const float2 x = fma2(make_float2(__uint_as_float(sd[32 * cc + xx]), __uint_as_float(sd[32 * cc + xx + 1])),
+                                s2, nl);
+          float2 pr = exp2_pair(x, (kBwdPolyPairs >> (xx >> 1)) & 1u);
+          if (diag) {
+            pr.x = key <= r ? pr.x : 0.f;
+            pr.y = key + 1 <= r ? pr.y : 0.f;
+          }
+          const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[64 + 32 * cc + xx]),
+                                                      __uint_as_float(sd[64 + 32 * cc + xx + 1])),
+                                          D2));
+          pk[xx >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         HGA_TMEM_ST16(tmem + lane_off + kDqS + x * 128 + 64 * e + 32 * cc, pk);
       }
@@ -479,7 +486,7 @@ __global__ void __launch_bounds__(320, 1)
     const int e = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;  // key row within block jb
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const float sl2 = a.sl2;
+    const float2 s2 = make_float2(a.sl2, a.sl2), nlog2e = make_float2(-kLog2e, -kLog2e);
     bool ok = true;
     uint32_t sd[64];  // 32 S^T columns then 32 dP^T columns of this thread's key row
     for (int u = 0; u < nsub; ++u) {
@@ -500,14 +507,18 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int x = 0; x < 32; x += 2) {
         const int q = q0 + x;
-        const bool k0 = !diag || q >= r;
-        const bool k1 = !diag || q + 1 >= r;
         const float2 lq = *reinterpret_cast<const float2*>(&rs.lse[q]);  // same for every key row: broadcast
         const float2 dq2 = *reinterpret_cast<const float2*>(&rs.D[q]);
-        const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(sd[x]), sl2, -lq.x * kLog2e)) : 0.f;
-        const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(sd[x + 1]), sl2, -lq.y * kLog2e)) : 0.f;
-        pp[x >> 1] = pack_bf16x2(p0, p1);
-        pd[x >> 1] = pack_bf16x2(p0 * (__uint_as_float(sd[32 + x]) - dq2.x), p1 * (__uint_as_float(sd[33 + x]) - dq2.y));
+        const float2 arg = fma2(make_float2(__uint_as_float(sd[x]), __uint_as_float(sd[x + 1])), s2,
+                                mul2(lq, nlog2e));
+        float2 pr = exp2_pair(arg, (kBwdPolyPairs >> (x >> 1)) & 1u);
+        if (diag) {
+          pr.x = q >= r ? pr.x : 0.f;
+          pr.y = q + 1 >= r ? pr.y : 0.f;
+        }
+        pp[x >> 1] = pack_bf16x2(pr.x, pr.y);
+        const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[32 + x]), __uint_as_float(sd[33 + x])), dq2));
+        pd[x >> 1] = pack_bf16x2(ds.x, ds.y);
       }
       HGA_TMEM_ST16(tmem + lane_off + kKvS + h * 64 + 32 * e, pp);
       HGA_TMEM_ST16(tmem + lane_off + kKvP + h * 64 + 32 * e, pd);

@@ -43,6 +43,9 @@ constexpr int kHalf = kTileBytes / 2;         // one 64-column TMA box
 constexpr int kStages = 5;                    // K/V ring slots
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+// Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
+// instead of the ex2 unit, which the softmax would otherwise saturate.
+constexpr uint32_t kFwdPolyPairs = 0x5252u;
 
 struct FwdCtl {
   uint64_t q_full;
@@ -274,8 +277,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int e = 0; e < 128; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(v[e]));
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+      for (int e = 0; e < 128; e += 2)
+        m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+      const float mx = max3f(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
       const bool need = mx > m_ref + kRescaleThreshold;
       const bool any_need = __any_sync(0xffffffffu, need);
       float alpha = 1.0f;  // rows that keep their reference use alpha = 1
@@ -284,20 +288,21 @@ __global__ void __launch_bounds__(384, 1)
         l *= alpha;
         m_ref = mx;
       }
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 s2 = make_float2(sl2, sl2), nm = make_float2(-m_ref, -m_ref);
+      float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e]), sl2, -m_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(v[c * 32 + e + 1]), sl2, -m_ref));
-          l4[(e >> 1) & 3] += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+          const float2 x = fma2(make_float2(__uint_as_float(v[c * 32 + e]), __uint_as_float(v[c * 32 + e + 1])), s2, nm);
+          const float2 p = exp2_pair(x, (kFwdPolyPairs >> (e >> 1)) & 1u);
+          l2[(e >> 1) & 1] = add2(l2[(e >> 1) & 1], p);
+          pk[e >> 1] = pack_bf16x2(p.x, p.y);
         }
         HGA_TMEM_ST16(tS + c * 32, pk);
       }
-      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
       if (any_need && j > 0) {
         // O_t holds the sum up to tile j-1 (PV_t(j-1) completed before S_t(j)
         // was announced): bring it to the new reference.

@@ -295,6 +295,59 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair: on the FMA pipe (exp2_poly2) when `poly`, else on the ex2
+// unit.  `poly` is a compile-time constant at every call site.
+__device__ __forceinline__ float2 exp2_pair(float2 x, bool poly);
+
+// Three-input maximum (one instruction).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two lanes on the FMA pipe, to share the exponential work of the
+// softmax passes between this and the ex2 unit.  Range reduction x = n + f,
+// n = round(x) (adding 1.5 * 2^23 rounds to an integer in the low mantissa
+// bits), f in [-1/2, 1/2]; 2^f from the degree-3 polynomial of least maximum
+// relative error on that interval (coefficients from Lawson's algorithm, see
+// fit_exp2_poly.py beside this file; max relative error 7.5e-5, far below
+// the bf16 rounding the result is used at); 2^n is added to the exponent
+// field with an integer add.  Inputs are clamped at -126 so the exponent
+// field never underflows: 2^x for x <= -126 (and -inf) comes out as about
+// 1.2e-38 instead of 0.
+constexpr float kExp2C0 = 0x1.fff692p-1f, kExp2C1 = 0x1.62f31cp-1f, kExp2C2 = 0x1.f0de3cp-3f,
+                kExp2C3 = 0x1.c3f754p-5f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = add2(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = add2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = add2(x, make_float2(-n.x, -n.y));
+  float2 p = fma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = fma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = fma2(p, f, make_float2(kExp2C0, kExp2C0));
+  // the low bits of t hold n (two's complement); shifting them into the
+  // exponent field drops the constant's own bits
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float2 exp2_pair(float2 x, bool poly) {
+  if (poly) return exp2_poly2(x);
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
 // Packs two floats into a bf16x2 word: lo -> bits [0,16), hi -> bits [16,32).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k,
   if (col < cols) {
     const T* base = k + ((size_t)b * T_src + (size_t)(src_b0 + n) * blk) * cols + col;
     int t = warp;
-#pragma unroll 4
+    // up to 16 rows per warp (blk <= 128): all loads in flight at once
+#pragma unroll 16
     for (; t < blk; t += 8) {
       float x[V];
       Vec<T>::load(base + (size_t)t * cols, x);
@@ -89,17 +90,24 @@ __device__ __forceinline__ unsigned long long sel_key(float s, int n) {
   return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)n);
 }
 
-// CTA = (query block i, KV head h, batch b).  256 threads.
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelU = 4;  // blocks per warp per scoring round
+
+// CTA = (query block i, KV head h, batch b).  512 threads.
 //  1. qm[g][:] = mean of the block's rows of Q for the G query heads of h
 //     (the G heads of a KV head are contiguous in a token row).
-//  2. score[n] = max_g qm[g] . summ[b,h,n] / sqrt(d): one warp per block n.
+//  2. score[n] = max_g qm[g] . summ[b,n,h] / sqrt(d).  A warp scores kSelU
+//     blocks per round: their summary channels are loaded before any
+//     arithmetic (the first round's before step 1), and the G * kSelU dot
+//     products are reduced across the warp together.
 //  3. bitonic sort of (score, index) keys, descending; first K_eff kept,
 //     then listed in ascending block order.
 template <typename T>
-__global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, const float* __restrict__ summ, int S,
-                                                     int Hq, int Hkv, int d, int blk, int nblk, int topk,
-                                                     float inv_sqrt_d, int32_t* __restrict__ idx,
-                                                     float* __restrict__ scores) {
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict__ q, const float* __restrict__ summ,
+                                                             int S, int Hq, int Hkv, int d, int blk, int nblk, int topk,
+                                                             float inv_sqrt_d, int32_t* __restrict__ idx,
+                                                             float* __restrict__ scores) {
   constexpr int V = Vec<T>::N;
   extern __shared__ __align__(16) unsigned char sel_smem[];
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -108,18 +116,33 @@ __global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, co
   const int cols = G * d;
   int npow = 1;
   while (npow < nblk) npow <<= 1;
-  float* qm = reinterpret_cast<float*>(sel_smem);                              // [G*d]
-  float* part = qm + cols + (cols & 1);                                        // [256*V]
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part + 256 * V);  // [npow]
+  float* qm = reinterpret_cast<float*>(sel_smem);                                        // [G*d]
+  float* part = qm + cols + (cols & 1);                                                  // [kSelThreads*V]
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part + kSelThreads * V);  // [npow]
   __shared__ int chosen[kMaxTopk];
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int cpl = d >> 5;  // summary channels per lane (d is 64 or 128)
+
+  // first scoring round's summary channels, in flight during step 1
+  float sv[kSelU][4];
+  auto load_round = [&](int n0) {
+#pragma unroll
+    for (int u = 0; u < kSelU; ++u) {
+      const int n = n0 + u;
+      const float* src = summ + (((size_t)b * nblk + (n < nblk ? n : 0)) * Hkv + h) * d + lane;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sv[u][m] = (n < nblk && m < cpl) ? __ldg(src + 32 * m) : 0.f;
+    }
+  };
+  load_round(warp * kSelU);
 
   // 1. query means: thread = (row phase r0, vector vt); rows r0, r0+rpp, ...
   //    are summed per thread, the rpp partials are then combined.
   const int tpr = cols / V;  // vectors per row (d is a multiple of 8)
-  for (int c0 = 0; c0 < tpr; c0 += 256) {
-    const int width = min(256, tpr - c0);
-    const int rpp = 256 / width;
+  for (int c0 = 0; c0 < tpr; c0 += kSelThreads) {
+    const int width = min(kSelThreads, tpr - c0);
+    const int rpp = kSelThreads / width;
     const int vt = c0 + tid % width, r0 = tid / width;
     float acc[V];
 #pragma unroll
@@ -138,7 +161,7 @@ __global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, co
       for (int e = 0; e < V; ++e) part[r0 * width * V + (vt - c0) * V + e] = acc[e];
     }
     __syncthreads();
-    for (int x = tid; x < width * V; x += 256) {
+    for (int x = tid; x < width * V; x += kSelThreads) {
       float s = 0.f;
       for (int r = 0; r < rpp; ++r) s += part[r * width * V + x];
       qm[c0 * V + x] = s * (1.0f / blk);
@@ -147,29 +170,39 @@ __global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, co
   }
 
   // 2. scores -> keys
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int n = warp; n < npow; n += 8) {
-    if (n >= nblk) {
-      if (lane == 0) keys[n] = 0ull;
-      continue;
-    }
-    const float* sv = summ + (((size_t)b * nblk + n) * Hkv + h) * d;
-    float best = -FLT_MAX;
-    for (int g = 0; g < G; ++g) {
-      float part = 0.f;
-      for (int kk = lane; kk < d; kk += 32) part += qm[g * d + kk] * __ldg(sv + kk);
+  for (int n0 = warp * kSelU; n0 < npow; n0 += kSelWarps * kSelU) {
+    if (n0 != warp * kSelU) load_round(n0);
+    float best[kSelU];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      best = fmaxf(best, part);
+    for (int u = 0; u < kSelU; ++u) best[u] = -FLT_MAX;
+    for (int g = 0; g < G; ++g) {
+      float qv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) qv[m] = m < cpl ? qm[g * d + lane + 32 * m] : 0.f;
+      float dot[kSelU];
+#pragma unroll
+      for (int u = 0; u < kSelU; ++u)
+        dot[u] = (qv[0] * sv[u][0] + qv[1] * sv[u][1]) + (qv[2] * sv[u][2] + qv[3] * sv[u][3]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int u = 0; u < kSelU; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+      }
+#pragma unroll
+      for (int u = 0; u < kSelU; ++u) best[u] = fmaxf(best[u], dot[u]);
     }
-    if (lane == 0) keys[n] = sel_key(best * inv_sqrt_d, n);
+#pragma unroll
+    for (int u = 0; u < kSelU; ++u) {
+      const int n = n0 + u;
+      if (lane == u && n < npow) keys[n] = n < nblk ? sel_key(best[u] * inv_sqrt_d, n) : 0ull;
+    }
   }
   __syncthreads();
 
   // 3. bitonic sort, descending
   for (int size = 2; size <= npow; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int x = tid; x < npow; x += 256) {
+      for (int x = tid; x < npow; x += kSelThreads) {
         const int y = x ^ stride;
         if (y > x) {
           const bool desc = ((x & size) == 0);
@@ -207,30 +240,54 @@ __global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ q, co
 }
 
 // ------------------------------------------------------------ bwd preprocess
-// One warp per (b, p, hq) row: D = sum_k dO * O in fp32.
+// D = sum_k dO * O in fp32 per (b, p, hq) row.  A row is read by d/V lanes
+// (16-byte vectors), so a warp covers 32V/d rows per pass; kPreRows passes are
+// loaded before any arithmetic to keep enough bytes in flight.
+constexpr int kPreRows = 4;
 template <typename T>
 __global__ void __launch_bounds__(256) preprocess_kernel(const T* __restrict__ o, const T* __restrict__ d_o, int S,
                                                          int Hq, int d, int rows, float* __restrict__ Dr) {
   constexpr int V = Vec<T>::N;
-  const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  // rows are enumerated token-major: warp = (b*S + p)*Hq + hq
-  const size_t off = (size_t)warp * d;
-  float s = 0.f;
-  for (int c = lane * V; c < d; c += 32 * V) {
-    float x[V], y[V];
-    Vec<T>::load(o + off + c, x);
-    Vec<T>::load(d_o + off + c, y);
+  const int lpr = d / V;    // lanes per row
+  const int rpw = 32 / lpr;  // rows per warp per pass
+  const int gw = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / lpr, cl = lane % lpr;
+  const int row0 = gw * rpw * kPreRows + sub;
+  float x[kPreRows][V], y[kPreRows][V];
 #pragma unroll
-    for (int e = 0; e < V; ++e) s += x[e] * y[e];
+  for (int r = 0; r < kPreRows; ++r) {
+    const int row = row0 + r * rpw;
+    if (row < rows) {
+      // rows are enumerated token-major: row = (b*S + p)*Hq + hq
+      Vec<T>::load(o + (size_t)row * d + cl * V, x[r]);
+      Vec<T>::load(d_o + (size_t)row * d + cl * V, y[r]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < V; ++e) x[r][e] = y[r][e] = 0.f;
+    }
   }
+  float acc[kPreRows];
 #pragma unroll
-  for (int k = 16; k > 0; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
-  if (lane == 0) {
-    const int hq = warp % Hq;
-    const int bp = warp / Hq;
-    const int b = bp / S, p = bp % S;
-    Dr[((size_t)b * Hq + hq) * S + p] = s;
+  for (int r = 0; r < kPreRows; ++r) {
+    acc[r] = 0.f;
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[r] = fmaf(x[r][e], y[r][e], acc[r]);
+  }
+  for (int k = lpr >> 1; k > 0; k >>= 1) {
+#pragma unroll
+    for (int r = 0; r < kPreRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], k);
+  }
+  if (cl == 0) {
+#pragma unroll
+    for (int r = 0; r < kPreRows; ++r) {
+      const int row = row0 + r * rpw;
+      if (row < rows) {
+        const int hq = row % Hq;
+        const int bp = row / Hq;
+        const int b = bp / S, p = bp % S;
+        Dr[((size_t)b * Hq + hq) * S + p] = acc[r];
+      }
+    }
   }
 }
 
@@ -256,7 +313,7 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
   int npow = 1;
   while (npow < s.nblk) npow <<= 1;
   const int cols = s.G() * s.d;
-  const size_t smem = (size_t)(cols + (cols & 1) + 256 * (s.bf16 ? 8 : 4)) * sizeof(float) + (size_t)npow * 8;
+  const size_t smem = (size_t)(cols + (cols & 1) + kSelThreads * (s.bf16 ? 8 : 4)) * sizeof(float) + (size_t)npow * 8;
   dim3 grid(s.nqb(), s.Hkv, s.B);
   const float isd = 1.0f / sqrtf((float)s.d);
   cudaError_t e;
@@ -264,13 +321,13 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
     auto kern = select_kernel<__nv_bfloat16>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
-    kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk,
+    kern<<<grid, kSelThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk,
                                   s.topk, isd, idx, scores);
   } else {
     auto kern = select_kernel<float>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
-    kern<<<grid, 256, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk, s.topk,
+    kern<<<grid, kSelThreads, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk, s.topk,
                                   isd, idx, scores);
   }
   return cudaGetLastError();
@@ -278,7 +335,8 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
 
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st) {
   const int rows = s.B * s.S * s.Hq;
-  const int grid = (rows + 7) / 8;
+  const int rows_per_cta = 8 * (32 * (s.bf16 ? 8 : 4) / s.d) * kPreRows;
+  const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
   if (s.bf16)
     preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
                                                            static_cast<const __nv_bfloat16*>(d_o), s.S, s.Hq, s.d,
