@@ -99,7 +99,7 @@ class ClockSampler:
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples, self.reasons = [], set()
         self.period = period_s
         self._stop = threading.Event()
@@ -185,11 +185,16 @@ def committed_traffic(kernel: str):
 
 # ---------------------------------------------------------------- device leg
 
+# Device workloads of `--workload`: the headline layer step, and the two
+# parity workloads (dense-equivalence, 131K prefill forward) timed the same way.
+DEVICE_WORKLOADS = {"layer": synth.QWEN3_8B_LAYER, "dense": synth.DENSE_EQUIV, "prefill": synth.PREFILL_131K}
+
+
 def run_device(args, rank, world, device):
     import segmented_fine_tuning_b200 as hga
     from segmented_fine_tuning_b200.step import AttentionStep
 
-    w = synth.QWEN3_8B_LAYER
+    w = DEVICE_WORKLOADS[args.workload]
     D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
     x = synth.draw(w)
     dev = {n: to_dev(getattr(x, n), device) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
@@ -209,13 +214,16 @@ def run_device(args, rank, world, device):
         hga.hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], D.n_hist_blocks,
                          st.idx, st.o, st.lse, stream)
         mark(3)
-        hga.hga_attn_bwd_preprocess(D, st.o, dev["d_o"], st.ws, stream)
+        if not w.fwd_only:
+            hga.hga_attn_bwd_preprocess(D, st.o, dev["d_o"], st.ws, stream)
         mark(4)
-        hga.hga_attn_bwd_dkdv(D, dev["q"], dev["k_seg"], dev["v_seg"], st.lse, dev["d_o"], st.ws, st.dk, st.dv,
-                              stream)
+        if not w.fwd_only:
+            hga.hga_attn_bwd_dkdv(D, dev["q"], dev["k_seg"], dev["v_seg"], st.lse, dev["d_o"], st.ws, st.dk, st.dv,
+                                  stream)
         mark(5)
-        hga.hga_attn_bwd_dq(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"],
-                            D.n_hist_blocks, st.idx, st.lse, dev["d_o"], st.ws, st.dq, stream)
+        if not w.fwd_only:
+            hga.hga_attn_bwd_dq(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"],
+                                D.n_hist_blocks, st.idx, st.lse, dev["d_o"], st.ws, st.dq, stream)
         mark(6)
 
     for _ in range(args.warmup):
@@ -265,7 +273,10 @@ def run_device(args, rank, world, device):
             gbs = bytes_[name] / (ms / 1e3) / 1e9
             entry.update({"gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)})
         kern[name] = entry
-    dom = max(("fwd", "bwd_dq", "bwd_dkdv"), key=lambda n: kern[n]["ms"])
+    if w.fwd_only:
+        for name in ("bwd_pre", "bwd_dkdv", "bwd_dq"):
+            kern.pop(name)
+    dom = max([n for n in ("fwd", "bwd_dq", "bwd_dkdv") if n in kern], key=lambda n: kern[n]["ms"])
     dom_ms = kern[dom]["ms"]
     achieved = flops[dom] / (dom_ms / 1e3) / 1e12
     traffic = committed_traffic(dom)
@@ -273,20 +284,21 @@ def run_device(args, rank, world, device):
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
                 "peak_source": f"{peak_src} dense bf16 (burst)",
                 "algorithmic_flop_per_launch": flops[dom]}
-    fwd_bwd_flops = flops["fwd"] + flops["bwd_dq"] + flops["bwd_dkdv"]
-    attn_ms = kern["fwd"]["ms"] + kern["bwd_dq"]["ms"] + kern["bwd_dkdv"]["ms"]
+    attn = [n for n in ("fwd", "bwd_dq", "bwd_dkdv") if n in kern]
+    fwd_bwd_flops = sum(flops[n] for n in attn)
+    attn_ms = sum(kern[n]["ms"] for n in attn)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); block-structured keys)",
         "config": workload_config(w, "flushed between steps (256 MiB write, outside the timed events)"),
         "roofline": roofline,
-        "attention_fwd_bwd": {"tflops": round(fwd_bwd_flops / (attn_ms / 1e3) / 1e12, 1),
+        ("attention_fwd" if w.fwd_only else "attention_fwd_bwd"): {"tflops": round(fwd_bwd_flops / (attn_ms / 1e3) / 1e12, 1),
                               "frac_bf16_peak": round(fwd_bwd_flops / (attn_ms / 1e3) / 1e12 /
                                                       peaks["bf16_tflops"], 3),
                               "algorithmic_gflop": round(fwd_bwd_flops / 1e9, 2)},
         "kernels": kern,
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": (3 if w.fwd_only else 6) * args.steps,
         "clocks": clk.summary(),
     }
     return out, (w, x, D, dev, st)
@@ -492,10 +504,13 @@ def main():
     ap.add_argument("--impl", choices=("hga", "reference"), default="hga")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=("layer", "segmented"), default="layer",
+    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill"), default="layer",
                     help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
-                         "8-segment pass with the pinned host tier")
+                         "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
+                         "the 131K prefill forward, device-timed only")
     args = ap.parse_args()
+    if args.workload in ("dense", "prefill"):
+        args.no_e2e = args.no_cpu_baseline = True
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3
 

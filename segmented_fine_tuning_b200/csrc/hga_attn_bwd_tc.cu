@@ -48,8 +48,10 @@ constexpr int kSubOff = kSubRows * 128;      // byte offset of the second 64-row
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kLog2e = 1.4426950408889634f;
 // Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
-// instead of the ex2 unit.
-constexpr uint32_t kBwdPolyPairs = 0x5252u;
+// (exp2_poly2) instead of the ex2 unit.  Measured on B200 with this
+// kernel's two warps per scheduler: every split tried (4, 6 or 8 of 16
+// pairs) was slower than none, so all pairs use the ex2 unit.
+constexpr uint32_t kBwdPolyPairs = 0x0u;
 
 // A bf16 chunk of 32 elements packed as 16 columns sits at the first 16 of
 // the 32 fp32 columns it was computed from; k-step kk (16 elements) of a

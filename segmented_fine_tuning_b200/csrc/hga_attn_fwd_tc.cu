@@ -44,8 +44,10 @@ constexpr int kStages = 5;                    // K/V ring slots
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 // Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
-// instead of the ex2 unit, which the softmax would otherwise saturate.
-constexpr uint32_t kFwdPolyPairs = 0x5252u;
+// (exp2_poly2) instead of the ex2 unit.  Measured on B200 with this
+// kernel's two warps per scheduler: every split tried (4, 6 or 8 of 16
+// pairs) was slower than none, so all pairs use the ex2 unit.
+constexpr uint32_t kFwdPolyPairs = 0x0u;
 
 struct FwdCtl {
   uint64_t q_full;

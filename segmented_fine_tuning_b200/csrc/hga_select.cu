@@ -93,6 +93,7 @@ __device__ __forceinline__ unsigned long long sel_key(float s, int n) {
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelU = 4;  // blocks per warp per scoring round
+constexpr int kSelRankMax = 256;  // largest padded block count ranked by counting
 
 // CTA = (query block i, KV head h, batch b).  512 threads.
 //  1. qm[g][:] = mean of the block's rows of Q for the G query heads of h
@@ -101,8 +102,8 @@ constexpr int kSelU = 4;  // blocks per warp per scoring round
 //     blocks per round: their summary channels are loaded before any
 //     arithmetic (the first round's before step 1), and the G * kSelU dot
 //     products are reduced across the warp together.
-//  3. bitonic sort of (score, index) keys, descending; first K_eff kept,
-//     then listed in ascending block order.
+//  3. top K_eff of the (score, index) keys by rank counting or a bitonic
+//     sort, then listed in ascending block order.
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict__ q, const float* __restrict__ summ,
                                                              int S, int Hq, int Hkv, int d, int blk, int nblk, int topk,
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
   float* part = qm + cols + (cols & 1);                                                  // [kSelThreads*V]
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(part + kSelThreads * V);  // [npow]
   __shared__ int chosen[kMaxTopk];
+  __shared__ unsigned long long chosen_key[kMaxTopk];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int cpl = d >> 5;  // summary channels per lane (d is 64 or 128)
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
     if (r0 < rpp) {
       const T* base = q + (((size_t)b * S + (size_t)i * blk) * Hq + (size_t)h * G) * d + (size_t)vt * V;
       const size_t rs = (size_t)Hq * d;
-#pragma unroll 8
+#pragma unroll 16
       for (int t = r0; t < blk; t += rpp) {
         float x[V];
         Vec<T>::load(base + t * rs, x);
@@ -199,25 +201,42 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
   }
   __syncthreads();
 
-  // 3. bitonic sort, descending
-  for (int size = 2; size <= npow; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int x = tid; x < npow; x += kSelThreads) {
-        const int y = x ^ stride;
-        if (y > x) {
-          const bool desc = ((x & size) == 0);
-          const unsigned long long a = keys[x], c = keys[y];
-          if (desc ? (a < c) : (a > c)) {
-            keys[x] = c;
-            keys[y] = a;
+  // 3. top K_eff.  Up to kSelRankMax blocks: every block counts the keys
+  //    above its own (keys are distinct), no sort needed; beyond that a
+  //    bitonic sort, descending.
+  const int keff = topk < nblk ? topk : nblk;
+  if (npow <= kSelRankMax) {
+    for (int n = tid; n < nblk; n += kSelThreads) {
+      const unsigned long long kn = keys[n];
+      int rank = 0;
+      for (int m = 0; m < nblk; ++m) rank += keys[m] > kn;
+      if (rank < keff) {
+        chosen[rank] = n;
+        chosen_key[rank] = kn;
+      }
+    }
+  } else {
+    for (int size = 2; size <= npow; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int x = tid; x < npow; x += kSelThreads) {
+          const int y = x ^ stride;
+          if (y > x) {
+            const bool desc = ((x & size) == 0);
+            const unsigned long long a = keys[x], c = keys[y];
+            if (desc ? (a < c) : (a > c)) {
+              keys[x] = c;
+              keys[y] = a;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
+    }
+    if (tid < keff) {
+      chosen[tid] = (int)(0xFFFFFFFFu - (uint32_t)(keys[tid] & 0xFFFFFFFFull));
+      chosen_key[tid] = keys[tid];
     }
   }
-  const int keff = topk < nblk ? topk : nblk;
-  if (tid < keff) chosen[tid] = (int)(0xFFFFFFFFu - (uint32_t)(keys[tid] & 0xFFFFFFFFull));
   __syncthreads();
   const size_t row = (((size_t)b * Hkv + h) * nqb + i) * topk;
   if (tid < topk) {
@@ -228,7 +247,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
       idx[row + rank] = n;
       if (scores) {
         // recover the score from the key (inverse of the ordering map)
-        uint32_t u = (uint32_t)(keys[tid] >> 32);
+        uint32_t u = (uint32_t)(chosen_key[tid] >> 32);
         u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
         scores[row + rank] = __uint_as_float(u);
       }
