@@ -259,65 +259,54 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
 }
 
 // ------------------------------------------------------------ bwd preprocess
-// D = sum_k dO * O in fp32 per (b, p, hq) row.  CTA = 16 tokens x 16 query
-// heads (256 rows; S is a multiple of 16, so a tile never crosses a batch).
-// A row is read by d/V lanes with 16-byte loads, kPreBatch rows per lane
-// group are loaded before any arithmetic; the 256 results are transposed in
-// shared memory so that Dr [B, Hq, S] is written as 64-byte runs of 16
-// consecutive positions per head.
-constexpr int kPreTok = 16, kPreHeads = 16, kPreBatch = 8;
+// D = sum_k dO * O in fp32 per (b, p, hq) row.  A row is read by d/V lanes
+// (16-byte vectors), so a warp covers 32V/d rows per pass; kPreRows passes are
+// loaded before any arithmetic to keep enough bytes in flight.
+constexpr int kPreRows = 4;
 template <typename T>
 __global__ void __launch_bounds__(256) preprocess_kernel(const T* __restrict__ o, const T* __restrict__ d_o, int S,
-                                                         int Hq, int d, float* __restrict__ Dr) {
+                                                         int Hq, int d, int rows, float* __restrict__ Dr) {
   constexpr int V = Vec<T>::N;
-  __shared__ float res[kPreHeads][kPreTok + 1];
-  const int lpr = d / V;     // lanes per row
+  const int lpr = d / V;    // lanes per row
   const int rpw = 32 / lpr;  // rows per warp per pass
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int sub = lane / lpr, cl = lane % lpr;
-  const int tok0 = blockIdx.x * kPreTok;  // global token (b*S + p) of the tile's first row
-  const int hq0 = blockIdx.y * kPreHeads;
-  const int rows_per_pass = 8 * rpw;
-  const int npass = kPreTok * kPreHeads / rows_per_pass;
-  for (int p0 = 0; p0 < npass; p0 += kPreBatch) {
-    float x[kPreBatch][V], y[kPreBatch][V];
+  const int row0 = gw * rpw * kPreRows + sub;
+  float x[kPreRows][V], y[kPreRows][V];
 #pragma unroll
-    for (int r = 0; r < kPreBatch; ++r) {
-      const int lr = (p0 + r) * rows_per_pass + warp * rpw + sub;  // local row: token lr / 16, head lr % 16
-      const int hq = hq0 + lr % kPreHeads;
-      if (p0 + r < npass && hq < Hq) {
-        const size_t off = ((size_t)(tok0 + lr / kPreHeads) * Hq + hq) * d + cl * V;
-        Vec<T>::load(o + off, x[r]);
-        Vec<T>::load(d_o + off, y[r]);
-      } else {
+  for (int r = 0; r < kPreRows; ++r) {
+    const int row = row0 + r * rpw;
+    if (row < rows) {
+      // rows are enumerated token-major: row = (b*S + p)*Hq + hq
+      Vec<T>::load(o + (size_t)row * d + cl * V, x[r]);
+      Vec<T>::load(d_o + (size_t)row * d + cl * V, y[r]);
+    } else {
 #pragma unroll
-        for (int e = 0; e < V; ++e) x[r][e] = y[r][e] = 0.f;
-      }
-    }
-    float acc[kPreBatch];
-#pragma unroll
-    for (int r = 0; r < kPreBatch; ++r) {
-      acc[r] = 0.f;
-#pragma unroll
-      for (int e = 0; e < V; ++e) acc[r] = fmaf(x[r][e], y[r][e], acc[r]);
-    }
-    for (int k = lpr >> 1; k > 0; k >>= 1) {
-#pragma unroll
-      for (int r = 0; r < kPreBatch; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], k);
-    }
-    if (cl == 0) {
-#pragma unroll
-      for (int r = 0; r < kPreBatch; ++r) {
-        const int lr = (p0 + r) * rows_per_pass + warp * rpw + sub;
-        if (p0 + r < npass) res[lr % kPreHeads][lr / kPreHeads] = acc[r];
-      }
+      for (int e = 0; e < V; ++e) x[r][e] = y[r][e] = 0.f;
     }
   }
-  __syncthreads();
-  const int h = threadIdx.x / kPreTok, t = threadIdx.x % kPreTok;
-  if (h < kPreHeads && hq0 + h < Hq) {
-    const int b = tok0 / S, p = tok0 % S + t;
-    Dr[((size_t)b * Hq + hq0 + h) * S + p] = res[h][t];
+  float acc[kPreRows];
+#pragma unroll
+  for (int r = 0; r < kPreRows; ++r) {
+    acc[r] = 0.f;
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[r] = fmaf(x[r][e], y[r][e], acc[r]);
+  }
+  for (int k = lpr >> 1; k > 0; k >>= 1) {
+#pragma unroll
+    for (int r = 0; r < kPreRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], k);
+  }
+  if (cl == 0) {
+#pragma unroll
+    for (int r = 0; r < kPreRows; ++r) {
+      const int row = row0 + r * rpw;
+      if (row < rows) {
+        const int hq = row % Hq;
+        const int bp = row / Hq;
+        const int b = bp / S, p = bp % S;
+        Dr[((size_t)b * Hq + hq) * S + p] = acc[r];
+      }
+    }
   }
 }
 
@@ -364,14 +353,16 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
 }
 
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st) {
-  // S is a multiple of the block size (>= 16), so tiles of 16 tokens cover B*S exactly.
-  dim3 grid(s.B * s.S / kPreTok, (s.Hq + kPreHeads - 1) / kPreHeads);
+  const int rows = s.B * s.S * s.Hq;
+  const int rows_per_cta = 8 * (32 * (s.bf16 ? 8 : 4) / s.d) * kPreRows;
+  const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
   if (s.bf16)
     preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                           static_cast<const __nv_bfloat16*>(d_o), s.S, s.Hq, s.d, Dr);
+                                                           static_cast<const __nv_bfloat16*>(d_o), s.S, s.Hq, s.d,
+                                                           rows, Dr);
   else
     preprocess_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(o), static_cast<const float*>(d_o), s.S,
-                                                   s.Hq, s.d, Dr);
+                                                   s.Hq, s.d, rows, Dr);
   return cudaGetLastError();
 }
 
