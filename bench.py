@@ -64,6 +64,23 @@ def workload_config(w: synth.Workload, l2_note: str):
             "segment_tokens": w.S, "history_blocks": w.nblk, "topk": w.topk, "l2": l2_note}
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest x over the ranks of the default process group (every rank
+    calls it with its own x; identity for a single process)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own replica of the step."""
+    return world * tokens_per_step / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- work model
 
 def work_model(w: synth.Workload, keff_sum_per_head: float):
@@ -252,13 +269,9 @@ def run_device(args, rank, world, device):
         step_ms.append(e[0].elapsed_time(e[6]))
         for j, name in enumerate(KERNELS):
             per_kernel[name].append(e[j].elapsed_time(e[j + 1]))
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, device)
     ms_per_step = total_ms / args.steps
-    value = world * w.S / (ms_per_step / 1e3)
+    value = job_throughput(world, w.S, ms_per_step)
 
     peaks, peak_src = load_peaks()
     flops, bytes_ = work_model(w, keff_sum)
@@ -539,10 +552,8 @@ def main():
         if not args.no_e2e:
             e2e = run_e2e(args, ctx, device)
             if world > 1:
-                t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=device)
-                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-                e2e["ms_per_step"] = round(float(t.item()), 4)
-                e2e["value"] = round(world * ctx[0].S / (e2e["ms_per_step"] / 1e3), 1)
+                e2e["ms_per_step"] = round(max_over_ranks(e2e["ms_per_step"], world, device), 4)
+                e2e["value"] = round(job_throughput(world, ctx[0].S, e2e["ms_per_step"]), 1)
             out["e2e"] = e2e
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = run_cpu_baseline(ctx[0], ctx[1])
