@@ -397,7 +397,8 @@ def h2d_probe(device, nbytes=1 << 30, reps=5):
 def run_segmented(args, device):
     """The full segmented pass: 36 Qwen3-8B-shaped layers over a 16,384-token
     sequence as 8 segments of 2,048 (history in a pinned host tier, selected
-    blocks fetched per (layer, segment), summaries appended on the device).
+    blocks fetched per (layer, segment) unless already resident in the
+    layer's device block cache, summaries appended on the device).
     Inputs: the 8 segments of layer 0 drawn with the workload's recipe and
     reused for every layer (the kernels' speed does not depend on values;
     selection, and so fetch volume, is representative).  One step = one pass."""
@@ -412,6 +413,7 @@ def run_segmented(args, device):
     stream = torch.cuda.current_stream(device)
 
     def one_pass():
+        sp.new_sequence()  # each pass is a new sequence: nothing resident carries over
         for s in range(NS):
             sp.run_segment(s, [dev[s]] * L)
 
@@ -420,6 +422,7 @@ def run_segmented(args, device):
     torch.cuda.synchronize(device)
     hga.hga_device_status(stream)
     sp.fetched_blocks.clear()
+    sp.selected_blocks.clear()
     times = []
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         for _ in range(args.steps):
@@ -433,6 +436,7 @@ def run_segmented(args, device):
     ms = float(np.mean(times))
     tokens = NS * w.S
     fetched = float(np.mean(sp.fetched_blocks))
+    selected = float(np.mean(sp.selected_blocks))
     blk_bytes = w.blk * w.Hkv * w.d * 2 * 2
     h2d_bytes = fetched * blk_bytes * L * (NS - 1)
     probe = h2d_probe(device)
@@ -443,7 +447,9 @@ def run_segmented(args, device):
             "config": {"workload": "segmented pass: 36 Qwen3-8B-shaped layers x 8 segments of 2,048 tokens, "
                                    "history +16 blocks of 128 per segment, K16, pinned host tier",
                        "layers": L, "segments": NS, "segment_tokens": w.S, "topk": w.topk},
-            "fetch": {"blocks_per_layer_step": round(fetched, 1), "h2d_bytes_per_pass": int(h2d_bytes),
+            "fetch": {"blocks_selected_per_layer_step": round(selected, 1),
+                      "blocks_copied_per_layer_step": round(fetched, 1),
+                      "device_block_cache_slots_per_layer": sp.pool_slots, "h2d_bytes_per_pass": int(h2d_bytes),
                       "h2d_probe_gbs": round(probe, 1),
                       "fetch_time_at_probe_ms": round(h2d_bytes / (probe * 1e9) * 1e3, 2)},
             "gpu_launches": int(L * NS * 6 + L * NS), "clocks": clk.summary()}

@@ -276,6 +276,62 @@ HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, co
                             hga_stream_t copy_stream, hga_event_t done, int timeout_ms);
 
 /*
+ * Device block cache: history blocks stay in a layer's device pool across
+ * calls, so a block selected again (by the next segment, or by the backward
+ * of the same segment) is not copied over the host link again.  The pages'
+ * Outlook names faster VRAM <-> RAM <-> NVMe transfer as the open problem;
+ * the history tier's blocks never change once offloaded, so a resident copy
+ * stays valid.
+ *
+ * hga_block_cache is host memory owned by the caller and kept across calls:
+ *   slot_of_block  [host_capacity_blocks] int32: pool slot holding block n, or -1
+ *   block_of_slot  [pool_slots] int32: block held by slot, or -1
+ *   last_use       [pool_slots] int64: tick of the last call that needed the slot
+ *   tick           calls planned so far
+ * hga_block_cache_reset empties it (needed when the tier or pool is reused for
+ * another sequence).  Both functions are host-only (no GPU work).
+ *
+ * hga_block_cache_plan: need[0..n_need) are distinct block numbers in
+ * [0, host_capacity_blocks), ascending.  Each gets a slot: a resident block
+ * keeps its own (a hit); a missing block takes an empty slot, else the least
+ * recently used slot whose block this call does not need (ties: the lowest
+ * slot).  slot_out[k] is need[k]'s slot; miss_out[0..*n_miss) lists the
+ * missing blocks (ascending), the ones to copy.  The cache records the
+ * assignment and advances its tick.  Errors: HGA_ERR_INVALID_ARG (NULL
+ * pointers, out-of-range or unsorted need, more distinct blocks than slots;
+ * the cache is then unchanged).
+ */
+typedef struct {
+  int32_t* slot_of_block;
+  int32_t* block_of_slot;
+  int64_t* last_use;
+  int host_capacity_blocks;
+  int pool_slots;
+  int64_t tick;
+} hga_block_cache;
+
+HGA_API hga_status hga_block_cache_reset(hga_block_cache* cache);
+HGA_API hga_status hga_block_cache_plan(hga_block_cache* cache, const int32_t* need, int n_need, int32_t* slot_out,
+                                        int32_t* miss_out, int* n_miss);
+
+/*
+ * hga_fetch_blocks through a device block cache: as hga_fetch_blocks, except
+ * that the pool (pool_k/pool_v [B, cache->pool_slots*block, Hkv, d]) keeps its
+ * contents between calls and only the selected blocks that are not resident
+ * are copied (hga_block_cache_plan decides).  idx_pool_dev receives idx with
+ * block numbers replaced by their slots.  *n_unique_out: distinct selected
+ * blocks; *n_fetched_out: blocks copied by this call.  The copies run on
+ * copy_stream after the work already queued on compute_stream, so a slot is
+ * never overwritten while earlier kernels may still read it.  host tier
+ * capacity: cache->host_capacity_blocks.  Errors as hga_fetch_blocks.
+ */
+HGA_API hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, const void* host_v,
+                                           const int32_t* idx_dev, int32_t* host_idx_scratch, void* pool_k,
+                                           void* pool_v, hga_block_cache* cache, int32_t* idx_pool_dev,
+                                           int* n_unique_out, int* n_fetched_out, hga_stream_t compute_stream,
+                                           hga_stream_t copy_stream, hga_event_t done, int timeout_ms);
+
+/*
  * Segment-end offload (fr edition, Analyse approfondie: the KV of a finished
  * segment is offloaded right away).  Copies the segment's K and V (device,
  * [B, S, Hkv, d]) into the pinned host tier at history block `at_block`

@@ -9,6 +9,8 @@ failing call an HgaError: there is no fallback path.
 from __future__ import annotations
 
 import ctypes
+
+import numpy as np
 import os
 from dataclasses import dataclass
 
@@ -63,9 +65,16 @@ class Dims:
         return Dims(self.B, self.Hq, self.Hkv, self.d, self.block, self.S, n_hist_blocks, self.topk, self.dtype)
 
 
+class hga_block_cache(ctypes.Structure):
+    _fields_ = [("slot_of_block", ctypes.POINTER(ctypes.c_int32)), ("block_of_slot", ctypes.POINTER(ctypes.c_int32)),
+                ("last_use", ctypes.POINTER(ctypes.c_int64)), ("host_capacity_blocks", ctypes.c_int),
+                ("pool_slots", ctypes.c_int), ("tick", ctypes.c_int64)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _D = ctypes.POINTER(hga_dims)
+_C = ctypes.POINTER(hga_block_cache)
 
 # (name, restype, argtypes) for every entry point of include/hga.h and
 # include/hga_selftest.h.
@@ -85,6 +94,10 @@ _SIGNATURES = [
     ("hga_attn_bwd_dq", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     ("hga_fetch_blocks", _I, [_D, _P, _P, _I, _P, _P, _P, _P, _I, _P, ctypes.POINTER(ctypes.c_int), _P, _P, _P,
                               _I]),
+    ("hga_block_cache_reset", _I, [_C]),
+    ("hga_block_cache_plan", _I, [_C, _P, _I, _P, _P, ctypes.POINTER(ctypes.c_int)]),
+    ("hga_fetch_blocks_cached", _I, [_D, _P, _P, _P, _P, _P, _P, _C, _P, ctypes.POINTER(ctypes.c_int),
+                                     ctypes.POINTER(ctypes.c_int), _P, _P, _P, _I]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
     ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
 ]
@@ -299,6 +312,68 @@ def hga_fetch_blocks(dims: Dims, host_k, host_v, host_capacity_blocks: int, idx_
                                            _stream(compute_stream), _stream(copy_stream), done.cuda_event,
                                            timeout_ms), "hga_fetch_blocks")
     return n_unique.value
+
+
+class BlockCache:
+    """Host-side state of one layer's device block cache (hga_block_cache):
+    which history block each pool slot holds, and when each slot was last
+    needed.  The arrays are numpy buffers kept alive by this object."""
+
+    def __init__(self, host_capacity_blocks: int, pool_slots: int):
+        self.slot_of_block = np.full(max(1, host_capacity_blocks), -1, dtype=np.int32)
+        self.block_of_slot = np.full(max(1, pool_slots), -1, dtype=np.int32)
+        self.last_use = np.full(max(1, pool_slots), -1, dtype=np.int64)
+        self.c = hga_block_cache(self.slot_of_block.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                 self.block_of_slot.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                 self.last_use.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                 host_capacity_blocks, pool_slots, 0)
+        self.reset()
+
+    @property
+    def host_capacity_blocks(self) -> int:
+        return self.c.host_capacity_blocks
+
+    @property
+    def pool_slots(self) -> int:
+        return self.c.pool_slots
+
+    def reset(self) -> None:
+        _check(load_library().hga_block_cache_reset(ctypes.byref(self.c)), "hga_block_cache_reset")
+
+    def plan(self, need):
+        """(slots for `need`, the blocks to copy) -- see hga_block_cache_plan."""
+        need = np.ascontiguousarray(need, dtype=np.int32)
+        slot = np.empty(max(1, need.size), dtype=np.int32)
+        miss = np.empty(max(1, need.size), dtype=np.int32)
+        n_miss = ctypes.c_int(0)
+        _check(load_library().hga_block_cache_plan(ctypes.byref(self.c), need.ctypes.data, int(need.size),
+                                                   slot.ctypes.data, miss.ctypes.data, ctypes.byref(n_miss)),
+               "hga_block_cache_plan")
+        return slot[:need.size].copy(), miss[:n_miss.value].copy()
+
+
+def hga_fetch_blocks_cached(dims: Dims, host_k, host_v, idx_dev, host_idx_scratch, pool_k, pool_v,
+                            cache: BlockCache, idx_pool_dev, compute_stream, copy_stream, done: torch.cuda.Event,
+                            timeout_ms: int = 10000):
+    """Returns (distinct selected blocks, blocks copied by this call)."""
+    shape = (dims.B, cache.host_capacity_blocks * dims.block, dims.Hkv, dims.d)
+    _expect(host_k, shape, dims.torch_dtype, "host_k", device=False)
+    _expect(host_v, shape, dims.torch_dtype, "host_v", device=False)
+    if not (host_k.is_pinned() and host_v.is_pinned() and host_idx_scratch.is_pinned()):
+        raise ValueError("host tier and idx scratch must be pinned host memory")
+    _expect(idx_dev, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx_dev")
+    _expect(host_idx_scratch, idx_dev.shape, torch.int32, "host_idx_scratch", device=False)
+    _expect(pool_k, (dims.B, cache.pool_slots * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "pool_k")
+    _expect(pool_v, pool_k.shape, dims.torch_dtype, "pool_v")
+    _expect(idx_pool_dev, idx_dev.shape, torch.int32, "idx_pool_dev")
+    n_unique, n_fetched = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load_library().hga_fetch_blocks_cached(ctypes.byref(dims.c()), _ptr(host_k), _ptr(host_v), _ptr(idx_dev),
+                                                  _ptr(host_idx_scratch), _ptr(pool_k), _ptr(pool_v),
+                                                  ctypes.byref(cache.c), _ptr(idx_pool_dev), ctypes.byref(n_unique),
+                                                  ctypes.byref(n_fetched), _stream(compute_stream),
+                                                  _stream(copy_stream), done.cuda_event, timeout_ms),
+           "hga_fetch_blocks_cached")
+    return n_unique.value, n_fetched.value
 
 
 def hga_offload_segment(dims: Dims, k_seg, v_seg, host_k, host_v, capacity_blocks: int, at_block: int,

@@ -483,6 +483,158 @@ hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void
   return HGA_OK;
 }
 
+hga_status hga_block_cache_reset(hga_block_cache* c) {
+  if (any_null(c) || c->host_capacity_blocks < 0 || c->pool_slots < 0 ||
+      (c->host_capacity_blocks > 0 && c->slot_of_block == nullptr) ||
+      (c->pool_slots > 0 && (c->block_of_slot == nullptr || c->last_use == nullptr)))
+    return fail(HGA_ERR_INVALID_ARG, "block cache: NULL arrays or negative sizes");
+  for (int n = 0; n < c->host_capacity_blocks; ++n) c->slot_of_block[n] = -1;
+  for (int k = 0; k < c->pool_slots; ++k) {
+    c->block_of_slot[k] = -1;
+    c->last_use[k] = -1;
+  }
+  c->tick = 0;
+  return HGA_OK;
+}
+
+hga_status hga_block_cache_plan(hga_block_cache* c, const int32_t* need, int n_need, int32_t* slot_out,
+                                int32_t* miss_out, int* n_miss) {
+  if (any_null(c, n_miss) || n_need < 0 || (n_need > 0 && any_null(need, slot_out, miss_out)))
+    return fail(HGA_ERR_INVALID_ARG, "block cache plan: NULL pointer or negative count");
+  if (n_need > c->pool_slots)
+    return fail(HGA_ERR_INVALID_ARG, "%d distinct blocks needed, pool holds %d", n_need, c->pool_slots);
+  for (int k = 0; k < n_need; ++k) {
+    if (need[k] < 0 || need[k] >= c->host_capacity_blocks)
+      return fail(HGA_ERR_INVALID_ARG, "needed block %d outside [0, %d)", need[k], c->host_capacity_blocks);
+    if (k > 0 && need[k] <= need[k - 1]) return fail(HGA_ERR_INVALID_ARG, "needed blocks not ascending");
+  }
+  const int64_t now = c->tick + 1;
+  // hits first: they pin their slots for this call
+  for (int k = 0; k < n_need; ++k) {
+    const int slot = c->slot_of_block[need[k]];
+    slot_out[k] = slot;
+    if (slot >= 0) c->last_use[slot] = now;
+  }
+  // misses: an empty slot, else the least recently used slot not needed now
+  int nm = 0;
+  for (int k = 0; k < n_need; ++k) {
+    if (slot_out[k] >= 0) continue;
+    int best = -1;
+    for (int x = 0; x < c->pool_slots; ++x) {
+      if (c->last_use[x] == now) continue;  // needed by this call
+      if (c->block_of_slot[x] < 0) {
+        best = x;
+        break;
+      }
+      if (best < 0 || c->last_use[x] < c->last_use[best]) best = x;
+    }
+    // n_need <= pool_slots guarantees a slot that this call has not claimed
+    const int old = c->block_of_slot[best];
+    if (old >= 0) c->slot_of_block[old] = -1;
+    c->block_of_slot[best] = need[k];
+    c->slot_of_block[need[k]] = best;
+    c->last_use[best] = now;
+    slot_out[k] = best;
+    miss_out[nm++] = need[k];
+  }
+  c->tick = now;
+  *n_miss = nm;
+  return HGA_OK;
+}
+
+hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, const void* host_v,
+                                   const int32_t* idx_dev, int32_t* host_idx_scratch, void* pool_k, void* pool_v,
+                                   hga_block_cache* cache, int32_t* idx_pool_dev, int* n_unique_out,
+                                   int* n_fetched_out, hga_stream_t compute_stream, hga_stream_t copy_stream,
+                                   hga_event_t done, int timeout_ms) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(host_k, host_v, idx_dev, host_idx_scratch, pool_k, pool_v, cache, idx_pool_dev, done))
+    return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  const int cap = cache->host_capacity_blocks, pool_slots = cache->pool_slots;
+  if (cap < dims->n_hist_blocks)
+    return fail(HGA_ERR_INVALID_ARG, "host tier holds %d blocks < n_hist_blocks %d", cap, dims->n_hist_blocks);
+  cudaStream_t cst = reinterpret_cast<cudaStream_t>(compute_stream);
+  cudaStream_t xst = reinterpret_cast<cudaStream_t>(copy_stream);
+  const size_t n_idx = (size_t)s.B * s.Hkv * s.nqb() * s.topk;
+  cudaEvent_t ready = nullptr, landed = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&landed, cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    if (ready) cudaEventDestroy(ready);
+    return cuda_fail(e, "event create");
+  }
+  struct Guard {
+    cudaEvent_t a, b;
+    ~Guard() { cudaEventDestroy(a); cudaEventDestroy(b); }
+  } guard{ready, landed};
+  // 1. idx -> host, after the work queued on the compute stream (which also
+  //    orders every later pool write after the kernels that read the pool).
+  if ((e = cudaEventRecord(ready, cst)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaStreamWaitEvent(xst, ready, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
+  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, xst)) !=
+      cudaSuccess)
+    return cuda_fail(e, "idx copy to host");
+  if ((e = cudaEventRecord(landed, xst)) != cudaSuccess) return cuda_fail(e, "event record");
+  const auto t0 = std::chrono::steady_clock::now();
+  while (true) {
+    e = cudaEventQuery(landed);
+    if (e == cudaSuccess) break;
+    if (e != cudaErrorNotReady) return cuda_fail(e, "waiting for idx");
+    if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms))
+      return fail(HGA_ERR_TIMEOUT, "idx copy did not complete within %d ms", timeout_ms);
+    std::this_thread::yield();
+  }
+  // 2. distinct selected blocks, ascending; cache plan.
+  std::vector<char> used(s.nblk > 0 ? s.nblk : 1, 0);
+  for (size_t k = 0; k < n_idx; ++k) {
+    const int n = host_idx_scratch[k];
+    if (n == -1) continue;
+    if (n < 0 || n >= s.nblk) return fail(HGA_ERR_INDEX, "idx entry %d outside [-1, %d)", n, s.nblk);
+    used[n] = 1;
+  }
+  std::vector<int32_t> need;
+  for (int n = 0; n < s.nblk; ++n)
+    if (used[n]) need.push_back(n);
+  std::vector<int32_t> slot(need.size() + 1), miss(need.size() + 1);
+  int n_miss = 0;
+  if ((r = hga_block_cache_plan(cache, need.data(), (int)need.size(), slot.data(), miss.data(), &n_miss)) != HGA_OK)
+    return r;
+  // 3. host -> pool copies of the misses, merged where blocks and slots are both consecutive.
+  const size_t es = s.bf16 ? 2 : 4;
+  const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
+  for (int k = 0; k < n_miss;) {
+    const int n0 = miss[k], s0 = cache->slot_of_block[n0];
+    int run = 1;
+    while (k + run < n_miss && miss[k + run] == n0 + run && cache->slot_of_block[n0 + run] == s0 + run) ++run;
+    for (int b = 0; b < s.B; ++b) {
+      const size_t src = ((size_t)b * cap + n0) * blk_bytes;
+      const size_t dst = ((size_t)b * pool_slots + s0) * blk_bytes;
+      if ((e = cudaMemcpyAsync(static_cast<char*>(pool_k) + dst, static_cast<const char*>(host_k) + src,
+                               run * blk_bytes, cudaMemcpyHostToDevice, xst)) != cudaSuccess)
+        return cuda_fail(e, "K block copy");
+      if ((e = cudaMemcpyAsync(static_cast<char*>(pool_v) + dst, static_cast<const char*>(host_v) + src,
+                               run * blk_bytes, cudaMemcpyHostToDevice, xst)) != cudaSuccess)
+        return cuda_fail(e, "V block copy");
+    }
+    k += run;
+  }
+  // 4. idx rewritten to slots (in the pinned scratch), then uploaded.
+  for (size_t k = 0; k < n_idx; ++k) {
+    const int n = host_idx_scratch[k];
+    host_idx_scratch[k] = n < 0 ? -1 : cache->slot_of_block[n];
+  }
+  if ((e = cudaMemcpyAsync(idx_pool_dev, host_idx_scratch, n_idx * sizeof(int32_t), cudaMemcpyHostToDevice, xst)) !=
+      cudaSuccess)
+    return cuda_fail(e, "pool idx upload");
+  if ((e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(done), xst)) != cudaSuccess)
+    return cuda_fail(e, "event record");
+  if (n_unique_out) *n_unique_out = (int)need.size();
+  if (n_fetched_out) *n_fetched_out = n_miss;
+  return HGA_OK;
+}
+
 hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
                                void* host_v, int capacity_blocks, int at_block, hga_stream_t stream) {
   hga::Shape s;

@@ -10,8 +10,10 @@ finished segment's KV is offloaded right away.
 
 Per segment s (history = segments 0..s-1, 16 blocks each at 2,048 tokens):
   forward,  layers 0..L-1:  select (resident summaries) -> fetch the distinct
-                            selected blocks from the layer's pinned host tier
-                            into the layer's device pool -> attention forward
+                            selected blocks that are not already in the
+                            layer's device pool from its pinned host tier (a
+                            block cache: slots are reused least recently used
+                            first) -> attention forward
   backward, layers L-1..0:  attention backward on the same pool (kept from the
                             forward; no second fetch)
   segment end, every layer: summaries of the segment's blocks appended to the
@@ -25,12 +27,15 @@ from __future__ import annotations
 
 import torch
 
-from ._binding import (Dims, hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd, hga_fetch_blocks,
-                       hga_offload_segment, hga_segment_summaries, hga_select_topk)
+from ._binding import (BlockCache, Dims, hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
+                       hga_fetch_blocks_cached, hga_offload_segment, hga_segment_summaries, hga_select_topk)
 
 
 class SegmentedPass:
-    def __init__(self, seg: Dims, n_layers: int, n_segments: int, device="cuda", fetch_timeout_ms: int = 10000):
+    def __init__(self, seg: Dims, n_layers: int, n_segments: int, device="cuda", fetch_timeout_ms: int = 10000,
+                 pool_slots: int | None = None):
+        """pool_slots: device pool (cache) size per layer in blocks; by default
+        the largest history, so no block is fetched twice in one sequence."""
         if seg.B != 1:
             raise ValueError("the segmented pass drives one sequence (B = 1)")
         self.seg, self.L, self.NS = seg, n_layers, n_segments
@@ -41,9 +46,11 @@ class SegmentedPass:
         self.timeout = fetch_timeout_ms
         dt = seg.torch_dtype
         H, d, blk = seg.Hkv, seg.d, seg.block
-        pool_blocks = max(1, self.max_hist)
+        pool_blocks = max(1, self.max_hist if pool_slots is None else pool_slots)
+        self.pool_slots = pool_blocks
         self.tier_k, self.tier_v, self.summ, self.pool_k, self.pool_v = [], [], [], [], []
         self.idx, self.idx_pool, self.scratch, self.o, self.lse, self.done = [], [], [], [], [], []
+        self.cache = []
         for _ in range(n_layers):
             self.tier_k.append(torch.empty((1, self.cap * blk, H, d), dtype=dt).pin_memory())
             self.tier_v.append(torch.empty((1, self.cap * blk, H, d), dtype=dt).pin_memory())
@@ -57,6 +64,7 @@ class SegmentedPass:
             self.lse.append(torch.empty((1, seg.Hq, seg.S), dtype=torch.float32, device=self.device))
             ev = torch.cuda.Event()
             self.done.append(ev)
+            self.cache.append(BlockCache(self.cap, pool_blocks))
         self.dq = torch.empty((1, seg.S, seg.Hq, d), dtype=torch.float32, device=self.device)
         self.dk = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
         self.dv = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
@@ -65,13 +73,20 @@ class SegmentedPass:
         self.offloaded = torch.cuda.Event()
         for ev in self.done:
             ev.record(self.copy_stream)  # materialise the handles
-        self.fetched_blocks = []
+        self.fetched_blocks = []   # blocks copied per (layer, segment) fetch
+        self.selected_blocks = []  # distinct blocks selected per (layer, segment)
+
+    def new_sequence(self) -> None:
+        """Start another sequence: its history tier replaces the previous one,
+        so nothing resident in the pools is valid any more."""
+        for c in self.cache:
+            c.reset()
 
     def dims(self, s: int) -> Dims:
         return self.seg.with_history(s * self.nqb)
 
     def n_kv(self, s: int) -> int:
-        return max(1, self.max_hist) if s > 0 else 0
+        return self.pool_slots if s > 0 else 0
 
     # ------------------------------------------------------------ steps
     def forward(self, s: int, l: int, q, k_seg, v_seg):
@@ -79,12 +94,13 @@ class SegmentedPass:
         st = torch.cuda.current_stream(self.device)
         hga_select_topk(D, q, self.summ[l], self.idx[l], None, st)
         if s > 0:
-            nu = hga_fetch_blocks(D, self.tier_k[l], self.tier_v[l], self.cap, self.idx[l], self.scratch[l],
-                                  self.pool_k[l], self.pool_v[l], self.max_hist, self.idx_pool[l], st,
-                                  self.copy_stream, self.done[l], self.timeout)
-            self.fetched_blocks.append(nu)
+            nu, nf = hga_fetch_blocks_cached(D, self.tier_k[l], self.tier_v[l], self.idx[l], self.scratch[l],
+                                             self.pool_k[l], self.pool_v[l], self.cache[l], self.idx_pool[l], st,
+                                             self.copy_stream, self.done[l], self.timeout)
+            self.selected_blocks.append(nu)
+            self.fetched_blocks.append(nf)
             st.wait_event(self.done[l])
-            hga_attn_fwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.max_hist, self.idx_pool[l],
+            hga_attn_fwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.pool_slots, self.idx_pool[l],
                          self.o[l], self.lse[l], st)
         else:
             hga_attn_fwd(D, q, k_seg, v_seg, None, None, 0, self.idx[l], self.o[l], self.lse[l], st)
@@ -94,7 +110,7 @@ class SegmentedPass:
         D = self.dims(s)
         st = torch.cuda.current_stream(self.device)
         if s > 0:
-            hga_attn_bwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.max_hist, self.idx_pool[l],
+            hga_attn_bwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.pool_slots, self.idx_pool[l],
                          self.o[l], self.lse[l], d_o, self.dq, self.dk, self.dv, self.ws, st)
         else:
             hga_attn_bwd(D, q, k_seg, v_seg, None, None, 0, self.idx[l], self.o[l], self.lse[l], d_o, self.dq,

@@ -7,8 +7,8 @@ import torch
 
 import synth
 from hga_testutil import dims_of, to_dev
-from segmented_fine_tuning_b200 import (HgaError, hga_attn_bwd, hga_attn_fwd, hga_device_status, hga_fetch_blocks,
-                                        hga_offload_segment)
+from segmented_fine_tuning_b200 import (BlockCache, HgaError, hga_attn_bwd, hga_attn_fwd, hga_device_status,
+                                        hga_fetch_blocks, hga_fetch_blocks_cached, hga_offload_segment)
 from segmented_fine_tuning_b200.step import AttentionStep
 
 pytestmark = pytest.mark.gpu
@@ -104,3 +104,66 @@ def test_offload_segment_into_tier():
     assert torch.count_nonzero(tk[:, : 5 * 128]) == 0 and torch.count_nonzero(tk[:, 7 * 128:]) == 0
     with pytest.raises(HgaError):
         hga_offload_segment(D, ks, vs, tk, tv, cap, 7)
+
+
+def test_cached_fetch_reuses_resident_blocks_and_evicts():
+    """hga_fetch_blocks_cached: a repeated selection copies nothing; a new
+    selection through a pool that cannot hold both copies only the missing
+    blocks, evicting the least recently used; the forward over the pool
+    equals the forward over the resident history each time."""
+    w = synth.Workload("tier-cache: Hq8/Hkv2 S512 hist20 K3", 1, 8, 2, 128, 128, 512, 20, 3, "bf16", 44,
+                       structured_keys=True)
+    x = synth.draw(w)
+    D = dims_of(w)
+    dev = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist")}
+    st = AttentionStep(D)
+    st.select(dev["q"], dev["k_hist"])
+    rng = np.random.default_rng(5)
+    idx2 = np.sort(np.stack([rng.choice(w.nblk, w.topk, replace=False) for _ in range(2 * 4)]), axis=1)
+    idx2 = torch.from_numpy(idx2.astype(np.int32).reshape(1, 2, 4, w.topk)).cuda()
+    refs = []
+    for idx in (st.idx, idx2):
+        o, lse = torch.empty_like(st.o), torch.empty_like(st.lse)
+        hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk, idx, o, lse)
+        refs.append((o, lse))
+    cap = w.nblk
+    tier_k = _pinned(x.k_hist)
+    tier_v = _pinned(x.v_hist)
+    scratch = torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory()
+    sets = [set(i.cpu().numpy().ravel().tolist()) - {-1} for i in (st.idx, idx2)]
+    slots = max(len(sets[0]), len(sets[1]))
+    cache = BlockCache(cap, slots)
+    pool_k = torch.full((1, slots * 128, 2, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    pool_v = torch.full_like(pool_k, float("nan"))
+    ip = torch.empty_like(st.idx)
+    cs = torch.cuda.Stream()
+    done = torch.cuda.Event()
+    done.record(cs)
+
+    def run(idx):
+        nu, nf = hga_fetch_blocks_cached(D, tier_k, tier_v, idx, scratch, pool_k, pool_v, cache, ip,
+                                         torch.cuda.current_stream(), cs, done)
+        torch.cuda.current_stream().wait_event(done)
+        o, lse = torch.empty_like(st.o), torch.empty_like(st.lse)
+        hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], pool_k, pool_v, slots, ip, o, lse)
+        torch.cuda.synchronize()
+        hga_device_status()
+        return nu, nf, o, lse
+
+    nu, nf, o, lse = run(st.idx)
+    assert nu == nf == len(sets[0])
+    assert torch.equal(o, refs[0][0]) and torch.equal(lse, refs[0][1])
+    nu, nf, o, lse = run(st.idx)
+    assert nu == len(sets[0]) and nf == 0
+    assert torch.equal(o, refs[0][0]) and torch.equal(lse, refs[0][1])
+    resident = set(int(b) for b in cache.block_of_slot if b >= 0)
+    nu, nf, o, lse = run(idx2)
+    assert nu == len(sets[1]) and nf == len(sets[1] - resident)
+    # slots are no longer in block order, so the forward visits the history
+    # tiles in another order: equal up to fp32 summation order
+    assert (o.float() - refs[1][0].float()).abs().max().item() <= 2e-2
+    assert (lse - refs[1][1]).abs().max().item() <= 1e-4
+    # every resident block sits where the cache says
+    for slot, blk in enumerate(cache.block_of_slot.tolist()):
+        if blk >= 0:
+            assert torch.equal(pool_k[:, slot * 128:(slot + 1) * 128].cpu(), tier_k[:, blk * 128:(blk + 1) * 128])
