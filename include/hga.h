@@ -278,10 +278,10 @@ HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, co
 /*
  * Device block cache: history blocks stay in a layer's device pool across
  * calls, so a block selected again (by the next segment, or by the backward
- * of the same segment) is not copied over the host link again.  The pages'
- * Outlook names faster VRAM <-> RAM <-> NVMe transfer as the open problem;
- * the history tier's blocks never change once offloaded, so a resident copy
- * stays valid.
+ * of the same segment) is not copied over the host link again (article,
+ * Outlook; fr Perspectives: faster VRAM <-> RAM <-> NVMe transfer is the
+ * open problem).  The history tier's blocks never change once offloaded, so
+ * a resident copy stays valid.
  *
  * hga_block_cache is host memory owned by the caller and kept across calls:
  *   slot_of_block  [host_capacity_blocks] int32: pool slot holding block n, or -1
