@@ -332,6 +332,20 @@ HGA_API hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* hos
                                            hga_stream_t copy_stream, hga_event_t done, int timeout_ms);
 
 /*
+ * Keep a finished segment's blocks resident in a layer's device block cache
+ * as they enter the history: plans slots for history blocks [at_block,
+ * at_block + S/block) by the hga_block_cache_plan rules (they become the most
+ * recently used) and copies the segment's K/V (device, [B, S, Hkv, d]) into
+ * those slots of pool_k/pool_v (device-to-device, on `stream`; queue it after
+ * every kernel that may still read the pool).  With hga_offload_segment the
+ * blocks then exist in both tiers, and a later selection of them copies
+ * nothing over the host link.  Errors: HGA_ERR_INVALID_ARG (NULL pointers,
+ * blocks outside the cache's host capacity, a pool smaller than a segment).
+ */
+HGA_API hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* pool_k,
+                                     void* pool_v, hga_block_cache* cache, int at_block, hga_stream_t stream);
+
+/*
  * Segment-end offload (fr edition, Analyse approfondie: the KV of a finished
  * segment is offloaded right away).  Copies the segment's K and V (device,
  * [B, S, Hkv, d]) into the pinned host tier at history block `at_block`

@@ -98,6 +98,7 @@ _SIGNATURES = [
     ("hga_block_cache_plan", _I, [_C, _P, _I, _P, _P, ctypes.POINTER(ctypes.c_int)]),
     ("hga_fetch_blocks_cached", _I, [_D, _P, _P, _P, _P, _P, _P, _C, _P, ctypes.POINTER(ctypes.c_int),
                                      ctypes.POINTER(ctypes.c_int), _P, _P, _P, _I]),
+    ("hga_cache_segment", _I, [_D, _P, _P, _P, _P, _C, _I, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
     ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
 ]
@@ -374,6 +375,17 @@ def hga_fetch_blocks_cached(dims: Dims, host_k, host_v, idx_dev, host_idx_scratc
                                                   _stream(copy_stream), done.cuda_event, timeout_ms),
            "hga_fetch_blocks_cached")
     return n_unique.value, n_fetched.value
+
+
+def hga_cache_segment(dims: Dims, k_seg, v_seg, pool_k, pool_v, cache: BlockCache, at_block: int,
+                      stream=None) -> None:
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(v_seg, k_seg.shape, dims.torch_dtype, "v_seg")
+    _expect(pool_k, (dims.B, cache.pool_slots * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "pool_k")
+    _expect(pool_v, pool_k.shape, dims.torch_dtype, "pool_v")
+    _check(load_library().hga_cache_segment(ctypes.byref(dims.c()), _ptr(k_seg), _ptr(v_seg), _ptr(pool_k),
+                                            _ptr(pool_v), ctypes.byref(cache.c), at_block, _stream(stream)),
+           "hga_cache_segment")
 
 
 def hga_offload_segment(dims: Dims, k_seg, v_seg, host_k, host_v, capacity_blocks: int, at_block: int,

@@ -635,6 +635,42 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
   return HGA_OK;
 }
 
+hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* pool_k, void* pool_v,
+                             hga_block_cache* cache, int at_block, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(k_seg, v_seg, pool_k, pool_v, cache)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  const int nseg = s.nqb();
+  if (at_block < 0 || at_block + nseg > cache->host_capacity_blocks)
+    return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the cache's %d", at_block, at_block + nseg,
+                cache->host_capacity_blocks);
+  std::vector<int32_t> need(nseg), slot(nseg), miss(nseg);
+  for (int t = 0; t < nseg; ++t) need[t] = at_block + t;
+  int n_miss = 0;
+  if ((r = hga_block_cache_plan(cache, need.data(), nseg, slot.data(), miss.data(), &n_miss)) != HGA_OK) return r;
+  // every block is copied, resident or not: the caller states that these blocks now hold this segment
+  const size_t es = s.bf16 ? 2 : 4;
+  const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int t = 0; t < nseg;) {
+    int run = 1;
+    while (t + run < nseg && slot[t + run] == slot[t] + run) ++run;
+    for (int b = 0; b < s.B; ++b) {
+      const size_t src = ((size_t)b * nseg + t) * blk_bytes;
+      const size_t dst = ((size_t)b * cache->pool_slots + slot[t]) * blk_bytes;
+      cudaError_t e = cudaMemcpyAsync(static_cast<char*>(pool_k) + dst, static_cast<const char*>(k_seg) + src,
+                                      run * blk_bytes, cudaMemcpyDeviceToDevice, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(static_cast<char*>(pool_v) + dst, static_cast<const char*>(v_seg) + src,
+                            run * blk_bytes, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e, "segment cache copy");
+    }
+    t += run;
+  }
+  return HGA_OK;
+}
+
 hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
                                void* host_v, int capacity_blocks, int at_block, hga_stream_t stream) {
   hga::Shape s;

@@ -18,7 +18,8 @@ Per segment s (history = segments 0..s-1, 16 blocks each at 2,048 tokens):
                             forward; no second fetch)
   segment end, every layer: summaries of the segment's blocks appended to the
                             resident array; the segment's K/V copied to the
-                            host tier on a side stream
+                            host tier on a side stream and into the layer's
+                            device cache
 Every step is a libhga.so call; this module owns buffers, streams and order.
 Batch size 1 (one sequence): the resident summary array of a layer grows as a
 prefix, which is a valid summary array of the current history for B = 1.
@@ -28,14 +29,19 @@ from __future__ import annotations
 import torch
 
 from ._binding import (BlockCache, Dims, hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
-                       hga_fetch_blocks_cached, hga_offload_segment, hga_segment_summaries, hga_select_topk)
+                       hga_cache_segment, hga_fetch_blocks_cached, hga_offload_segment, hga_segment_summaries,
+                       hga_select_topk)
 
 
 class SegmentedPass:
     def __init__(self, seg: Dims, n_layers: int, n_segments: int, device="cuda", fetch_timeout_ms: int = 10000,
-                 pool_slots: int | None = None):
+                 pool_slots: int | None = None, keep_new_blocks: bool = True):
         """pool_slots: device pool (cache) size per layer in blocks; by default
-        the largest history, so no block is fetched twice in one sequence."""
+        the largest history, so no block is fetched twice in one sequence.
+        keep_new_blocks: a finished segment's blocks also enter the layer's
+        device cache (a device-to-device copy) as they are offloaded, so their
+        first selection needs no host transfer."""
+        self.keep_new_blocks = keep_new_blocks
         if seg.B != 1:
             raise ValueError("the segmented pass drives one sequence (B = 1)")
         self.seg, self.L, self.NS = seg, n_layers, n_segments
@@ -122,6 +128,8 @@ class SegmentedPass:
         host tier on the side stream (ordered after the work queued so far)."""
         st = torch.cuda.current_stream(self.device)
         hga_segment_summaries(self.seg.with_history(self.cap), k_seg, s * self.nqb, self.summ[l], st)
+        if self.keep_new_blocks and s + 1 < self.NS:
+            hga_cache_segment(self.seg, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.cache[l], s * self.nqb, st)
         self.offloaded.record(st)
         self.copy_stream.wait_event(self.offloaded)
         hga_offload_segment(self.seg, k_seg, v_seg, self.tier_k[l], self.tier_v[l], self.cap, s * self.nqb,

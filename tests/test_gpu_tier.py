@@ -7,8 +7,9 @@ import torch
 
 import synth
 from hga_testutil import dims_of, to_dev
-from segmented_fine_tuning_b200 import (BlockCache, HgaError, hga_attn_bwd, hga_attn_fwd, hga_device_status,
-                                        hga_fetch_blocks, hga_fetch_blocks_cached, hga_offload_segment)
+from segmented_fine_tuning_b200 import (BlockCache, HgaError, hga_attn_bwd, hga_attn_fwd, hga_cache_segment,
+                                        hga_device_status, hga_fetch_blocks, hga_fetch_blocks_cached,
+                                        hga_offload_segment)
 from segmented_fine_tuning_b200.step import AttentionStep
 
 pytestmark = pytest.mark.gpu
@@ -167,3 +168,39 @@ def test_cached_fetch_reuses_resident_blocks_and_evicts():
     for slot, blk in enumerate(cache.block_of_slot.tolist()):
         if blk >= 0:
             assert torch.equal(pool_k[:, slot * 128:(slot + 1) * 128].cpu(), tier_k[:, blk * 128:(blk + 1) * 128])
+
+
+def test_cache_segment_makes_new_blocks_resident():
+    """hga_cache_segment puts a segment's blocks into the device cache (with
+    hga_offload_segment they exist in both tiers); selecting them afterwards
+    copies nothing over the host link, and the pool holds exactly their K/V."""
+    w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 3, 2, "bf16", 45)
+    x = synth.draw(w)
+    D = dims_of(w)
+    ks, vs = to_dev(x.k_seg), to_dev(x.v_seg)
+    cap, slots = 8, 4
+    tk = torch.zeros((1, cap * 128, 2, 128), dtype=torch.bfloat16).pin_memory()
+    tv = torch.zeros_like(tk).pin_memory()
+    cache = BlockCache(cap, slots)
+    pool_k = torch.zeros((1, slots * 128, 2, 128), dtype=torch.bfloat16, device="cuda")
+    pool_v = torch.zeros_like(pool_k)
+    hga_offload_segment(D, ks, vs, tk, tv, cap, 5)
+    hga_cache_segment(D, ks, vs, pool_k, pool_v, cache, 5)
+    torch.cuda.synchronize()
+    assert cache.slot_of_block[5:7].tolist() == [0, 1]
+    assert torch.equal(pool_k[:, :256], ks) and torch.equal(pool_v[:, :256], vs)
+    Dh = D.with_history(7)
+    idx = torch.full((1, 2, 2, 2), -1, dtype=torch.int32, device="cuda")
+    idx[..., 0], idx[..., 1] = 5, 6
+    scratch = torch.empty((1, 2, 2, 2), dtype=torch.int32).pin_memory()
+    ip = torch.empty_like(idx)
+    cs = torch.cuda.Stream()
+    done = torch.cuda.Event()
+    done.record(cs)
+    nu, nf = hga_fetch_blocks_cached(Dh, tk, tv, idx, scratch, pool_k, pool_v, cache, ip,
+                                     torch.cuda.current_stream(), cs, done)
+    torch.cuda.synchronize()
+    assert (nu, nf) == (2, 0)
+    assert ip.cpu().unique().tolist() == [0, 1]
+    with pytest.raises(HgaError):
+        hga_cache_segment(D, ks, vs, pool_k, pool_v, cache, 7)  # blocks 7, 8 outside the capacity of 8
