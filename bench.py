@@ -436,7 +436,7 @@ def run_segmented(args, device):
     ms = float(np.mean(times))
     tokens = NS * w.S
     fetched = float(np.mean(sp.fetched_blocks))
-    selected = float(np.mean(sp.selected_blocks))
+    selected = float(np.mean(sp.selected_blocks)) if sp.selected_blocks else None
     blk_bytes = w.blk * w.Hkv * w.d * 2 * 2
     h2d_bytes = fetched * blk_bytes * L * (NS - 1)
     probe = h2d_probe(device)
@@ -447,12 +447,13 @@ def run_segmented(args, device):
             "config": {"workload": "segmented pass: 36 Qwen3-8B-shaped layers x 8 segments of 2,048 tokens, "
                                    "history +16 blocks of 128 per segment, K16, pinned host tier",
                        "layers": L, "segments": NS, "segment_tokens": w.S, "topk": w.topk},
-            "fetch": {"blocks_selected_per_layer_step": round(selected, 1),
+            "fetch": {"blocks_selected_per_host_fetch": None if selected is None else round(selected, 1),
                       "blocks_copied_per_layer_step": round(fetched, 1),
+                      "steps_remapped_on_device_per_pass": sp.device_remaps // (args.steps + args.warmup),
                       "device_block_cache_slots_per_layer": sp.pool_slots, "h2d_bytes_per_pass": int(h2d_bytes),
                       "h2d_probe_gbs": round(probe, 1),
                       "fetch_time_at_probe_ms": round(h2d_bytes / (probe * 1e9) * 1e3, 2)},
-            "gpu_launches": int(L * NS * 6 + L * NS), "clocks": clk.summary()}
+            "gpu_launches": int(L * NS * 6 + L * NS + L * (NS - 1)), "clocks": clk.summary()}
 
 
 # ---------------------------------------------------------------- oracle legs

@@ -346,6 +346,19 @@ HGA_API hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, co
                                      void* pool_v, hga_block_cache* cache, int at_block, hga_stream_t stream);
 
 /*
+ * idx -> pool slots on the device, for a cache that holds every selectable
+ * block (then no host round trip is needed):
+ *   idx_pool[k] = slot_of_block_dev[idx[k]]   (-1 kept)
+ * slot_of_block_dev: device int32 [n_hist_blocks], a copy of the cache's
+ * slot_of_block.  An idx entry outside [-1, n_hist_blocks) or a block that is
+ * not resident (slot -1) sets the device error flag (HGA_ERR_INDEX at the next
+ * hga_device_status) and gives -1, so the attention kernels skip it.
+ * Errors: HGA_ERR_INVALID_ARG (NULL pointers), HGA_ERR_SHAPE.
+ */
+HGA_API hga_status hga_remap_idx(const hga_dims* dims, const int32_t* idx_dev, const int32_t* slot_of_block_dev,
+                                 int32_t* idx_pool_dev, hga_stream_t stream);
+
+/*
  * Segment-end offload (fr edition, Analyse approfondie: the KV of a finished
  * segment is offloaded right away).  Copies the segment's K and V (device,
  * [B, S, Hkv, d]) into the pinned host tier at history block `at_block`

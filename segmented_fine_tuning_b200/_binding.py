@@ -99,6 +99,7 @@ _SIGNATURES = [
     ("hga_fetch_blocks_cached", _I, [_D, _P, _P, _P, _P, _P, _P, _C, _P, ctypes.POINTER(ctypes.c_int),
                                      ctypes.POINTER(ctypes.c_int), _P, _P, _P, _I]),
     ("hga_cache_segment", _I, [_D, _P, _P, _P, _P, _C, _I, _P]),
+    ("hga_remap_idx", _I, [_D, _P, _P, _P, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
     ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
 ]
@@ -386,6 +387,18 @@ def hga_cache_segment(dims: Dims, k_seg, v_seg, pool_k, pool_v, cache: BlockCach
     _check(load_library().hga_cache_segment(ctypes.byref(dims.c()), _ptr(k_seg), _ptr(v_seg), _ptr(pool_k),
                                             _ptr(pool_v), ctypes.byref(cache.c), at_block, _stream(stream)),
            "hga_cache_segment")
+
+
+def hga_remap_idx(dims: Dims, idx_dev, slot_of_block_dev, idx_pool_dev, stream=None) -> None:
+    _expect(idx_dev, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx_dev")
+    _expect(idx_pool_dev, idx_dev.shape, torch.int32, "idx_pool_dev")
+    if dims.n_hist_blocks > 0:
+        if (slot_of_block_dev.dtype != torch.int32 or not slot_of_block_dev.is_cuda or
+                slot_of_block_dev.numel() < dims.n_hist_blocks or not slot_of_block_dev.is_contiguous()):
+            raise ValueError("slot_of_block_dev: contiguous CUDA int32 with at least n_hist_blocks entries")
+    _check(load_library().hga_remap_idx(ctypes.byref(dims.c()), _ptr(idx_dev),
+                                        _ptr(slot_of_block_dev) if dims.n_hist_blocks > 0 else None,
+                                        _ptr(idx_pool_dev), _stream(stream)), "hga_remap_idx")
 
 
 def hga_offload_segment(dims: Dims, k_seg, v_seg, host_k, host_v, capacity_blocks: int, at_block: int,

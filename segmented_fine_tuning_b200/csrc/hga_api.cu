@@ -671,6 +671,20 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
   return HGA_OK;
 }
 
+hga_status hga_remap_idx(const hga_dims* dims, const int32_t* idx_dev, const int32_t* slot_of_block_dev,
+                         int32_t* idx_pool_dev, hga_stream_t stream) {
+  hga::Shape s;
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(idx_dev, idx_pool_dev) || (s.nblk > 0 && slot_of_block_dev == nullptr))
+    return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  int* err;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  cudaError_t e =
+      hga::launch_remap_idx(s, idx_dev, slot_of_block_dev, idx_pool_dev, err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "idx remap launch");
+}
+
 hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
                                void* host_v, int capacity_blocks, int at_block, hga_stream_t stream) {
   hga::Shape s;

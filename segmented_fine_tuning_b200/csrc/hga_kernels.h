@@ -30,6 +30,10 @@ cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src,
                                    float* summ, cudaStream_t st);
 cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
                                cudaStream_t st);
+// idx_pool = slot_of_block[idx] on the device (-1 kept; absent or out-of-range
+// blocks flag kDevErrIndex and give -1).
+cudaError_t launch_remap_idx(const Shape& s, const int32_t* idx, const int32_t* slot_of_block, int32_t* idx_pool,
+                             int* err, cudaStream_t st);
 // D[b,hq,p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k]  (fp32)
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st);
 

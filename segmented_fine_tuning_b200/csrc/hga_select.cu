@@ -310,6 +310,23 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const T* __restrict__ o
   }
 }
 
+// ------------------------------------------------------------ idx -> pool slots
+// idx_pool[k] = slot_of_block[idx[k]] (-1 kept).  A block outside
+// [0, nblk) or not resident (slot -1) flags the device error and yields -1.
+__global__ void __launch_bounds__(256) remap_kernel(const int32_t* __restrict__ idx,
+                                                    const int32_t* __restrict__ slot_of_block, int nblk, size_t n,
+                                                    int32_t* __restrict__ idx_pool, int* err) {
+  const size_t k = (size_t)blockIdx.x * 256 + threadIdx.x;
+  if (k >= n) return;
+  const int b = idx[k];
+  int slot = -1;
+  if (b >= 0) {
+    if (b < nblk) slot = slot_of_block[b];
+    if (slot < 0) flag_error(err, kDevErrIndex);
+  }
+  idx_pool[k] = slot;
+}
+
 }  // namespace
 
 cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src, int src_b0, int dst_b0, int nblocks,
@@ -366,4 +383,14 @@ cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o
   return cudaGetLastError();
 }
 
+}  // namespace hga
+
+namespace hga {
+cudaError_t launch_remap_idx(const Shape& s, const int32_t* idx, const int32_t* slot_of_block, int32_t* idx_pool,
+                             int* err, cudaStream_t st) {
+  const size_t n = (size_t)s.B * s.Hkv * s.nqb() * s.topk;
+  if (n == 0) return cudaSuccess;
+  remap_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(idx, slot_of_block, s.nblk, n, idx_pool, err);
+  return cudaGetLastError();
+}
 }  // namespace hga

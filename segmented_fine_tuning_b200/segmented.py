@@ -29,8 +29,8 @@ from __future__ import annotations
 import torch
 
 from ._binding import (BlockCache, Dims, hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
-                       hga_cache_segment, hga_fetch_blocks_cached, hga_offload_segment, hga_segment_summaries,
-                       hga_select_topk)
+                       hga_cache_segment, hga_fetch_blocks_cached, hga_offload_segment, hga_remap_idx,
+                       hga_segment_summaries, hga_select_topk)
 
 
 class SegmentedPass:
@@ -56,7 +56,7 @@ class SegmentedPass:
         self.pool_slots = pool_blocks
         self.tier_k, self.tier_v, self.summ, self.pool_k, self.pool_v = [], [], [], [], []
         self.idx, self.idx_pool, self.scratch, self.o, self.lse, self.done = [], [], [], [], [], []
-        self.cache = []
+        self.cache, self.slot_dev = [], []
         for _ in range(n_layers):
             self.tier_k.append(torch.empty((1, self.cap * blk, H, d), dtype=dt).pin_memory())
             self.tier_v.append(torch.empty((1, self.cap * blk, H, d), dtype=dt).pin_memory())
@@ -71,6 +71,7 @@ class SegmentedPass:
             ev = torch.cuda.Event()
             self.done.append(ev)
             self.cache.append(BlockCache(self.cap, pool_blocks))
+            self.slot_dev.append(torch.full((self.cap,), -1, dtype=torch.int32, device=self.device))
         self.dq = torch.empty((1, seg.S, seg.Hq, d), dtype=torch.float32, device=self.device)
         self.dk = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
         self.dv = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
@@ -79,14 +80,16 @@ class SegmentedPass:
         self.offloaded = torch.cuda.Event()
         for ev in self.done:
             ev.record(self.copy_stream)  # materialise the handles
-        self.fetched_blocks = []   # blocks copied per (layer, segment) fetch
-        self.selected_blocks = []  # distinct blocks selected per (layer, segment)
+        self.fetched_blocks = []   # blocks copied over the host link per (layer, segment) step
+        self.selected_blocks = []  # distinct blocks selected, per step that went through the host
+        self.device_remaps = 0     # steps whose whole history was resident: idx remapped on the device
 
     def new_sequence(self) -> None:
         """Start another sequence: its history tier replaces the previous one,
         so nothing resident in the pools is valid any more."""
-        for c in self.cache:
+        for c, d in zip(self.cache, self.slot_dev):
             c.reset()
+            d.fill_(-1)
 
     def dims(self, s: int) -> Dims:
         return self.seg.with_history(s * self.nqb)
@@ -100,12 +103,19 @@ class SegmentedPass:
         st = torch.cuda.current_stream(self.device)
         hga_select_topk(D, q, self.summ[l], self.idx[l], None, st)
         if s > 0:
-            nu, nf = hga_fetch_blocks_cached(D, self.tier_k[l], self.tier_v[l], self.idx[l], self.scratch[l],
-                                             self.pool_k[l], self.pool_v[l], self.cache[l], self.idx_pool[l], st,
-                                             self.copy_stream, self.done[l], self.timeout)
-            self.selected_blocks.append(nu)
-            self.fetched_blocks.append(nf)
-            st.wait_event(self.done[l])
+            if (self.cache[l].slot_of_block[: s * self.nqb] >= 0).all():
+                # every selectable block is resident: slots on the device, no host round trip
+                hga_remap_idx(D, self.idx[l], self.slot_dev[l], self.idx_pool[l], st)
+                self.fetched_blocks.append(0)
+                self.device_remaps += 1
+            else:
+                nu, nf = hga_fetch_blocks_cached(D, self.tier_k[l], self.tier_v[l], self.idx[l], self.scratch[l],
+                                                 self.pool_k[l], self.pool_v[l], self.cache[l], self.idx_pool[l],
+                                                 st, self.copy_stream, self.done[l], self.timeout)
+                self.selected_blocks.append(nu)
+                self.fetched_blocks.append(nf)
+                st.wait_event(self.done[l])
+                self._sync_slots(l, st)
             hga_attn_fwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.pool_slots, self.idx_pool[l],
                          self.o[l], self.lse[l], st)
         else:
@@ -130,6 +140,7 @@ class SegmentedPass:
         hga_segment_summaries(self.seg.with_history(self.cap), k_seg, s * self.nqb, self.summ[l], st)
         if self.keep_new_blocks and s + 1 < self.NS:
             hga_cache_segment(self.seg, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.cache[l], s * self.nqb, st)
+            self._sync_slots(l, st)
         self.offloaded.record(st)
         self.copy_stream.wait_event(self.offloaded)
         hga_offload_segment(self.seg, k_seg, v_seg, self.tier_k[l], self.tier_v[l], self.cap, s * self.nqb,
@@ -137,6 +148,13 @@ class SegmentedPass:
         # the caller may release k_seg/v_seg once the copy stream has passed here
         k_seg.record_stream(self.copy_stream)
         v_seg.record_stream(self.copy_stream)
+
+    def _sync_slots(self, l: int, st) -> None:
+        """Device copy of layer l's slot map, queued on st (a fresh pinned
+        staging buffer each time, so a pending copy is never overwritten)."""
+        staged = torch.from_numpy(self.cache[l].slot_of_block[: self.cap].copy()).pin_memory()
+        with torch.cuda.stream(st):
+            self.slot_dev[l].copy_(staged, non_blocking=True)
 
     def run_segment(self, s: int, inputs, on_step=None):
         """inputs[l] = (q, k_seg, v_seg, d_o) device tensors of layer l for

@@ -102,10 +102,10 @@ def test_segmented_pass_36_layers_8_segments():
                 want = torch.from_numpy(np.ascontiguousarray(t.store).view(np.int16)).view(torch.bfloat16)
                 assert torch.equal(tier[:, rows], want)
     print(f"selections: {L * (NS - 1)} steps with history, near-tie positions {n_near}, accepted {n_acc}; "
-          f"outputs checked for {n_checked} (layer, segment) steps; per step: distinct selected blocks "
-          f"mean {np.mean(sp.selected_blocks):.1f}, copied over the host link mean {np.mean(sp.fetched_blocks):.1f}")
+          f"outputs checked for {n_checked} (layer, segment) steps; blocks copied over the host link per step "
+          f"mean {np.mean(sp.fetched_blocks):.1f}; steps remapped on the device {sp.device_remaps}")
     assert n_checked == len(CHECK_LAYERS) * NS
-    # the device block cache holds a layer's whole history: no block crosses the host link twice
+    # finished segments enter each layer's device cache, which holds the whole
+    # history: nothing crosses the host link and every step remaps on the device
     copied = np.array(sp.fetched_blocks).reshape(NS - 1, L)
-    assert (copied <= np.array(sp.selected_blocks).reshape(NS - 1, L)).all()
-    assert (copied.sum(axis=0) <= sp.max_hist).all()
+    assert (copied == 0).all() and sp.device_remaps == L * (NS - 1)

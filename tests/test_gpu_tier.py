@@ -9,7 +9,7 @@ import synth
 from hga_testutil import dims_of, to_dev
 from segmented_fine_tuning_b200 import (BlockCache, HgaError, hga_attn_bwd, hga_attn_fwd, hga_cache_segment,
                                         hga_device_status, hga_fetch_blocks, hga_fetch_blocks_cached,
-                                        hga_offload_segment)
+                                        hga_offload_segment, hga_remap_idx)
 from segmented_fine_tuning_b200.step import AttentionStep
 
 pytestmark = pytest.mark.gpu
@@ -204,3 +204,24 @@ def test_cache_segment_makes_new_blocks_resident():
     assert ip.cpu().unique().tolist() == [0, 1]
     with pytest.raises(HgaError):
         hga_cache_segment(D, ks, vs, pool_k, pool_v, cache, 7)  # blocks 7, 8 outside the capacity of 8
+
+
+def test_remap_idx_on_device():
+    """hga_remap_idx: idx -> slots through a device copy of the slot map, -1
+    kept; a selected block that is not resident is flagged, never read."""
+    w = synth.Workload("t", 1, 4, 2, 128, 128, 256, 6, 3, "bf16", 46)
+    D = dims_of(w)
+    slot_of = torch.tensor([4, 0, 5, 1, 3, 2], dtype=torch.int32, device="cuda")
+    idx = torch.tensor([[0, 2, -1], [1, 3, 5], [4, -1, -1], [0, 1, 2]], dtype=torch.int32,
+                       device="cuda").reshape(1, 2, 2, 3)
+    ip = torch.empty_like(idx)
+    hga_remap_idx(D, idx, slot_of, ip)
+    hga_device_status()
+    want = torch.where(idx >= 0, slot_of[idx.clamp(min=0).long()], torch.full_like(idx, -1))
+    assert torch.equal(ip, want)
+    slot_of[3] = -1  # block 3 not resident
+    hga_remap_idx(D, idx, slot_of, ip)
+    with pytest.raises(HgaError) as e:
+        hga_device_status()
+    assert e.value.status == 4
+    assert ip[0, 0, 1, 1].item() == -1
