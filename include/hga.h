@@ -82,7 +82,7 @@ typedef enum {
   HGA_OK = 0,
   HGA_ERR_INVALID_ARG = 1, /* null pointer, bad enum, bad size */
   HGA_ERR_SHAPE = 2,       /* dimensions outside the supported set */
-  HGA_ERR_UNSUPPORTED = 3, /* valid request this build does not implement */
+  HGA_ERR_UNSUPPORTED = 3, /* valid request that the library does not implement */
   HGA_ERR_INDEX = 4,       /* a kernel met an out-of-range block index */
   HGA_ERR_TIMEOUT = 5,     /* a bounded wait expired (host or device) */
   HGA_ERR_CUDA = 6         /* a CUDA runtime call failed; see hga_last_error */
