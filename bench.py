@@ -488,7 +488,7 @@ def run_cpu_baseline(w, x_inputs, budget_s=12.0):
                       f"({done * w.G} of {w.Hq} query heads) in {el:.1f} s, scaled to the full layer"}
 
 
-def run_reference(args, rank):
+def run_reference(args, rank, world=1):
     if rank != 0:
         return None
     w = synth.QWEN3_8B_LAYER
@@ -505,7 +505,7 @@ def run_reference(args, rank):
     value = w.S * (1 / w.Hkv) / (ms / 1e3)
     sample = (f"each step: fp64 oracle selection for all heads + fwd and bwd for 1 of {w.Hkv} KV heads "
               f"(4 query heads), scaled to the full layer (x{w.Hkv})")
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 1,
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
             "config": workload_config(w, "n/a (CPU)"),
@@ -539,7 +539,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        out = run_reference(args, rank)
+        out = run_reference(args, rank, world)
         if out is not None:
             print(json.dumps(out), flush=True)
         return
