@@ -111,3 +111,25 @@ def test_oracle_and_library_share_nothing():
     for f in glob.glob(os.path.join(ROOT, "oracle", "*")):
         if f.endswith((".c", ".h", ".py")):
             assert "segmented_fine_tuning_b200" not in open(f).read(), f
+
+
+def test_headers_compile_as_c_and_cpp(tmp_path):
+    """The boundary is a C ABI: both public headers compile as C11 (no C++
+    in the signatures) and as C++17, warning-free, with only the CUDA runtime
+    headers on the include path."""
+    import shutil
+    import subprocess
+    cc, cxx = shutil.which("gcc"), shutil.which("g++")
+    if not cc or not cxx:
+        pytest.skip("no host compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "hga.h"\n#include "hga_selftest.h"\n'
+                   "int main(void) { hga_dims d; hga_block_cache c; (void)d; (void)c; return 0; }\n")
+    from torch.utils.cpp_extension import CUDA_HOME
+    if not CUDA_HOME:
+        pytest.skip("no CUDA toolkit headers")
+    inc = ["-I" + os.path.join(ROOT, "include"), "-I" + os.path.join(CUDA_HOME, "include")]
+    for tool, lang in ((cc, ["-std=c11"]), (cxx, ["-std=c++17", "-x", "c++"])):
+        r = subprocess.run([tool, *lang, "-Wall", "-Wextra", "-Werror", *inc, "-c", str(src), "-o",
+                            str(tmp_path / "use.o")], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
