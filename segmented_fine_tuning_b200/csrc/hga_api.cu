@@ -78,7 +78,7 @@ hga_status get_encoder(EncodeTiledFn* fn) {
 
 // bf16 tensor [B, T, H, 128] with a {64, 1, 128, 1} box, 128-byte swizzle.
 hga_status encode_tokens(CUtensorMap* m, const void* base, int B, int T, int H) {
-  EncodeTiledFn enc;
+  EncodeTiledFn enc = nullptr;
   hga_status s = get_encoder(&enc);
   if (s != HGA_OK) return s;
   const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -164,7 +164,7 @@ const char* hga_status_string(hga_status s) {
 const char* hga_last_error(void) { return g_last_error; }
 
 hga_status hga_device_status(hga_stream_t stream) {
-  int* flag;
+  int* flag = nullptr;
   hga_status s = device_err_ptr(&flag);
   if (s != HGA_OK) return s;
   int host = 0;
@@ -182,7 +182,7 @@ hga_status hga_device_status(hga_stream_t stream) {
 
 hga_status hga_block_summaries(const hga_dims* dims, const void* k_hist, int blk_begin, int blk_end, float* summ,
                                hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (blk_begin < 0 || blk_end > s.nblk || blk_begin > blk_end)
@@ -197,7 +197,7 @@ hga_status hga_block_summaries(const hga_dims* dims, const void* k_hist, int blk
 
 hga_status hga_segment_summaries(const hga_dims* dims, const void* k_seg, int at_block, float* summ,
                                  hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (at_block < 0 || at_block + s.nqb() > s.nblk)
@@ -212,7 +212,7 @@ hga_status hga_segment_summaries(const hga_dims* dims, const void* k_seg, int at
 
 hga_status hga_select_topk(const hga_dims* dims, const void* q_seg, const float* summ, int32_t* idx,
                            float* scores_or_null, hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (s.nblk > hga::kMaxSelectBlocks)
@@ -226,12 +226,12 @@ hga_status hga_select_topk(const hga_dims* dims, const void* q_seg, const float*
 hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
                         const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, void* o,
                         float* lse, hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if ((r = check_attn_ptrs(s, n_kv_blocks, q, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
   if (any_null(o, lse)) return fail(HGA_ERR_INVALID_ARG, "NULL output pointer");
-  int* err;
+  int* err = nullptr;
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
@@ -260,7 +260,7 @@ hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const
                    const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o, const float* lse,
                    const void* d_o, float* dq, float* dk_seg, float* dv_seg, const void* ws, size_t ws_bytes,
                    bool pre, int parts, hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(ws)) return fail(HGA_ERR_INVALID_ARG, "NULL workspace");
@@ -280,7 +280,7 @@ hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const
     if ((parts & hga::kBwdDkdv) && (any_null(dk_seg, dv_seg) || !aligned16(dk_seg) || !aligned16(dv_seg)))
       return fail(HGA_ERR_INVALID_ARG, "dk_seg/dv_seg must be non-NULL and 16-byte aligned");
   }
-  int* err;
+  int* err = nullptr;
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* Dr = static_cast<float*>(const_cast<void*>(ws));
@@ -395,7 +395,7 @@ hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void
                             int32_t* host_idx_scratch, void* pool_k, void* pool_v, int pool_slots,
                             int32_t* idx_pool_dev, int* n_unique_out, hga_stream_t compute_stream,
                             hga_stream_t copy_stream, hga_event_t done, int timeout_ms) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(host_k, host_v, idx_dev, host_idx_scratch, pool_k, pool_v, idx_pool_dev, done))
@@ -547,7 +547,7 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
                                    hga_block_cache* cache, int32_t* idx_pool_dev, int* n_unique_out,
                                    int* n_fetched_out, hga_stream_t compute_stream, hga_stream_t copy_stream,
                                    hga_event_t done, int timeout_ms) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(host_k, host_v, idx_dev, host_idx_scratch, pool_k, pool_v, cache, idx_pool_dev, done))
@@ -637,7 +637,7 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
 
 hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* pool_k, void* pool_v,
                              hga_block_cache* cache, int at_block, hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(k_seg, v_seg, pool_k, pool_v, cache)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
@@ -673,12 +673,12 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
 
 hga_status hga_remap_idx(const hga_dims* dims, const int32_t* idx_dev, const int32_t* slot_of_block_dev,
                          int32_t* idx_pool_dev, hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(idx_dev, idx_pool_dev) || (s.nblk > 0 && slot_of_block_dev == nullptr))
     return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
-  int* err;
+  int* err = nullptr;
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaError_t e =
       hga::launch_remap_idx(s, idx_dev, slot_of_block_dev, idx_pool_dev, err, reinterpret_cast<cudaStream_t>(stream));
@@ -687,7 +687,7 @@ hga_status hga_remap_idx(const hga_dims* dims, const int32_t* idx_dev, const int
 
 hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* host_k,
                                void* host_v, int capacity_blocks, int at_block, hga_stream_t stream) {
-  hga::Shape s;
+  hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(k_seg, v_seg, host_k, host_v)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
@@ -718,7 +718,7 @@ hga_status hga_selftest_umma(int form, const void* a, const void* b, float* d, h
   hga_status r;
   if ((r = encode_tokens(&ma, a, 1, 128, 1)) != HGA_OK) return r;
   if ((r = encode_tokens(&mb, b, 1, 128, 1)) != HGA_OK) return r;
-  int* err;
+  int* err = nullptr;
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaError_t e = hga::launch_selftest_umma(form, ma, mb, a, d, err, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "selftest launch");
