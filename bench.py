@@ -15,9 +15,11 @@ flushed (256 MiB write) between steps, outside the timed events.
 Extra keys: roofline of the dominant kernel, per-kernel breakdown, e2e
 (the same step through the public API with host buffers: pinned H2D of the
 segment's inputs, history blocks fetched from a pinned host tier by
-hga_fetch_blocks, D2H of the per-row log-sum-exp), cpu_baseline (the fp64
-oracle on a bounded sample, on this host's cores), and SM clocks sampled
-during the timed region.
+hga_fetch_blocks, D2H of every result: O, LSE, dQ, dK, dV), the 131K-token
+prefill's summaries, selection and forward timed the same way (where the
+HBM-bound kernels move enough bytes for their roofline fraction to mean
+something), cpu_baseline (the fp64 oracle on a bounded sample, on this
+host's cores), and SM clocks sampled during the timed region.
 
 --impl reference times the fp64 CPU oracle (the reference arm) on the same
 workload: each step is a bounded sample (selection for every head, forward
@@ -207,11 +209,12 @@ def committed_traffic(kernel: str):
 DEVICE_WORKLOADS = {"layer": synth.QWEN3_8B_LAYER, "dense": synth.DENSE_EQUIV, "prefill": synth.PREFILL_131K}
 
 
-def run_device(args, rank, world, device):
+def run_device(args, rank, world, device, w=None, steps=None):
     import segmented_fine_tuning_b200 as hga
     from segmented_fine_tuning_b200.step import AttentionStep
 
-    w = DEVICE_WORKLOADS[args.workload]
+    w = DEVICE_WORKLOADS[args.workload] if w is None else w
+    steps = args.steps if steps is None else steps
     D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
     x = synth.draw(w)
     dev = {n: to_dev(getattr(x, n), device) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
@@ -250,12 +253,12 @@ def run_device(args, rank, world, device):
     hga.hga_device_status(stream)
     keff_sum = float((st.idx >= 0).sum().item()) / (w.B * w.Hkv)  # sum over query blocks, per KV head
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(device.index if device.index is not None else 0) as clk:
-        for k in range(args.steps):
+        for k in range(steps):
             flush.zero_()
             step(evs[k])
         torch.cuda.synchronize(device)
@@ -270,7 +273,7 @@ def run_device(args, rank, world, device):
         for j, name in enumerate(KERNELS):
             per_kernel[name].append(e[j].elapsed_time(e[j + 1]))
     total_ms = max_over_ranks(float(sum(step_ms)), world, device)
-    ms_per_step = total_ms / args.steps
+    ms_per_step = total_ms / steps
     value = job_throughput(world, w.S, ms_per_step)
 
     peaks, peak_src = load_peaks()
@@ -301,7 +304,7 @@ def run_device(args, rank, world, device):
     fwd_bwd_flops = sum(flops[n] for n in attn)
     attn_ms = sum(kern[n]["ms"] for n in attn)
     out = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); block-structured keys)",
         "config": workload_config(w, "flushed between steps (256 MiB write, outside the timed events)"),
@@ -311,7 +314,7 @@ def run_device(args, rank, world, device):
                                                       peaks["bf16_tflops"], 3),
                               "algorithmic_gflop": round(fwd_bwd_flops / 1e9, 2)},
         "kernels": kern,
-        "gpu_launches": (3 if w.fwd_only else 6) * args.steps,
+        "gpu_launches": (3 if w.fwd_only else 6) * steps,
         "clocks": clk.summary(),
     }
     return out, (w, x, D, dev, st)
@@ -320,7 +323,8 @@ def run_device(args, rank, world, device):
 def run_e2e(args, ctx, device):
     """The same step through the public API with host buffers: the segment's
     Q, K, V, dO copied from pinned host memory, the selected history blocks
-    fetched from a pinned host tier, and the per-row log-sum-exp read back."""
+    fetched from a pinned host tier, and every result of the step (O, LSE,
+    dQ, dK, dV) copied back to pinned host memory."""
     import segmented_fine_tuning_b200 as hga
     w, x, D, dev, st = ctx
     stream = torch.cuda.current_stream(device)
@@ -328,7 +332,8 @@ def run_e2e(args, ctx, device):
     host = {n: to_pinned(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "d_o")}
     tier_k, tier_v = to_pinned(x.k_hist), to_pinned(x.v_hist)
     idx_scratch = torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory()
-    lse_host = torch.empty(tuple(st.lse.shape), dtype=torch.float32).pin_memory()
+    results = {"o": st.o, "lse": st.lse, "dq": st.dq, "dk": st.dk, "dv": st.dv}
+    out_host = {n: torch.empty(tuple(t.shape), dtype=t.dtype).pin_memory() for n, t in results.items()}
     pool_k = torch.empty_like(dev["k_hist"])
     pool_v = torch.empty_like(dev["v_hist"])
     idx_pool = torch.empty_like(st.idx)
@@ -353,7 +358,8 @@ def run_e2e(args, ctx, device):
                          st.lse, stream)
         hga.hga_attn_bwd(D, seg["q"], seg["k_seg"], seg["v_seg"], pool_k, pool_v, D.n_hist_blocks, idx_pool, st.o,
                          st.lse, seg["d_o"], st.dq, st.dk, st.dv, st.ws, stream)
-        lse_host.copy_(st.lse, non_blocking=True)
+        for n, t in results.items():
+            out_host[n].copy_(t, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         step()
@@ -370,10 +376,11 @@ def run_e2e(args, ctx, device):
     ms = e0.elapsed_time(e1) / n
     h2d = sum(t.numel() * t.element_size() for t in host.values()) + np.mean(fetched) * blk_bytes \
         + idx_pool.numel() * 4
-    d2h = idx_scratch.numel() * 4 + lse_host.numel() * 4
+    d2h = idx_scratch.numel() * 4 + sum(t.numel() * t.element_size() for t in out_host.values())
     return {"value": round(w.S / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "fetched_blocks_per_step": float(np.mean(fetched)), "path": "pinned host tier + hga_fetch_blocks"}
+            "fetched_blocks_per_step": float(np.mean(fetched)),
+            "path": "pinned host tier + hga_fetch_blocks; O, LSE, dQ, dK, dV copied back to pinned host memory"}
 
 
 # ---------------------------------------------------------------- segmented pass
@@ -524,6 +531,8 @@ def main():
     ap.add_argument("--impl", choices=("hga", "reference"), default="hga")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the 131K-token prefill sub-measurement of the default (layer) run")
     ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill"), default="layer",
                     help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
                          "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
@@ -564,6 +573,13 @@ def main():
             out["e2e"] = e2e
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = run_cpu_baseline(ctx[0], ctx[1])
+        if args.workload == "layer" and not args.no_prefill:
+            del ctx
+            torch.cuda.empty_cache()
+            pf, _ = run_device(args, rank, world, device, w=synth.PREFILL_131K, steps=min(args.steps, 20))
+            out["prefill_131k"] = {k: pf[k] for k in ("value", "unit", "ms_per_step", "steps", "config", "kernels",
+                                                      "attention_fwd", "gpu_launches", "clocks")}
+            out["prefill_131k"]["metric"] = "HGA attn fwd tokens/s per layer (131K-token prefill, forward only)"
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

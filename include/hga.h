@@ -268,6 +268,9 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
  * Errors: HGA_ERR_TIMEOUT (idx copy did not finish in time), HGA_ERR_INDEX
  * (an idx entry out of range), HGA_ERR_INVALID_ARG (more distinct blocks than
  * pool_slots, null pointers), HGA_ERR_CUDA.
+ * After HGA_ERR_TIMEOUT no pool copy has been queued, but the idx copy into
+ * host_idx_scratch is still pending on copy_stream: the caller must not reuse
+ * or free that buffer until copy_stream has drained (cudaStreamSynchronize).
  */
 HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,
                             const int32_t* idx_dev,
@@ -324,6 +327,11 @@ HGA_API hga_status hga_block_cache_plan(hga_block_cache* cache, const int32_t* n
  * copy_stream after the work already queued on compute_stream, so a slot is
  * never overwritten while earlier kernels may still read it.  host tier
  * capacity: cache->host_capacity_blocks.  Errors as hga_fetch_blocks.
+ * The cache is updated only once every copy of the call has been queued: on
+ * any error it is left exactly as it was, so no block is recorded as
+ * resident whose bytes were never sent.  After HGA_ERR_TIMEOUT the idx copy
+ * into host_idx_scratch is still pending on copy_stream, as for
+ * hga_fetch_blocks.
  */
 HGA_API hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, const void* host_v,
                                            const int32_t* idx_dev, int32_t* host_idx_scratch, void* pool_k,
@@ -340,7 +348,8 @@ HGA_API hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* hos
  * every kernel that may still read the pool).  With hga_offload_segment the
  * blocks then exist in both tiers, and a later selection of them copies
  * nothing over the host link.  Errors: HGA_ERR_INVALID_ARG (NULL pointers,
- * blocks outside the cache's host capacity, a pool smaller than a segment).
+ * blocks outside the cache's host capacity, a pool smaller than a segment),
+ * HGA_ERR_CUDA; on any error the cache is unchanged.
  */
 HGA_API hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* pool_k,
                                      void* pool_v, hga_block_cache* cache, int at_block, hga_stream_t stream);

@@ -27,6 +27,23 @@ extern "C" {
  */
 HGA_API hga_status hga_selftest_umma(int form, const void* a, const void* b, float* d, hga_stream_t stream);
 
+/*
+ * Self test of the device-side timeout path (the article has no counterpart).
+ * Runs the tensor-core forward of hga_attn_fwd (same arguments; bf16, d = 128,
+ * block = 128, even group size, else HGA_ERR_UNSUPPORTED) with its K/V tile
+ * loads withheld, so that a pipeline wait can never be satisfied.  Every
+ * wait in the kernels is bounded (1 s): the CTA that gives up raises its
+ * abort flag, every role leaves its loop, the CTA waits (bounded) for its own
+ * copies and tensor-core work in flight, frees its tensor memory and returns.
+ * The next hga_device_status() then reports HGA_ERR_TIMEOUT, and the CUDA
+ * context stays usable.  o and lse are left unwritten.  Expect about one
+ * second of device time per call.
+ */
+HGA_API hga_status hga_selftest_attn_fwd_stalled(const hga_dims* dims, const void* q, const void* k_seg,
+                                                 const void* v_seg, const void* k_hist, const void* v_hist,
+                                                 int n_kv_blocks, const int32_t* idx, void* o, float* lse,
+                                                 hga_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

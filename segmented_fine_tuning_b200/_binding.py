@@ -102,6 +102,7 @@ _SIGNATURES = [
     ("hga_remap_idx", _I, [_D, _P, _P, _P, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
     ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
+    ("hga_selftest_attn_fwd_stalled", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
 ]
 
 _lib = None
@@ -418,3 +419,15 @@ def hga_selftest_umma(form: int, a, b, d, stream=None) -> None:
     _expect(b, (128, 128), torch.bfloat16, "b")
     _expect(d, (128, 128), torch.float32, "d")
     _check(load_library().hga_selftest_umma(form, _ptr(a), _ptr(b), _ptr(d), _stream(stream)), "hga_selftest_umma")
+
+
+def hga_selftest_attn_fwd_stalled(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, o, lse,
+                                  stream=None) -> None:
+    """The tensor-core forward with its K/V loads withheld (timeout-path self test)."""
+    _attn_shapes(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx)
+    _expect(o, q.shape, dims.torch_dtype, "o")
+    _expect(lse, (dims.B, dims.Hq, dims.S), torch.float32, "lse")
+    _check(load_library().hga_selftest_attn_fwd_stalled(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg),
+                                                        _ptr(k_hist), _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o),
+                                                        _ptr(lse), _stream(stream)),
+           "hga_selftest_attn_fwd_stalled")

@@ -144,6 +144,40 @@ hga_status build_maps(const hga::Shape& s, int nkv, const void* q, const void* d
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// A working copy of a caller's block cache.  The fetch and segment-insert
+// calls plan on the copy and commit it only after every copy they depend on
+// has been queued, so a call that fails part-way leaves the caller's cache
+// as it was (no block is recorded as resident whose bytes were never sent).
+struct CacheDraft {
+  std::vector<int32_t> slot_of_block, block_of_slot;
+  std::vector<int64_t> last_use;
+  hga_block_cache view;
+  hga_block_cache* target;
+
+  explicit CacheDraft(hga_block_cache* c)
+      : slot_of_block(c->slot_of_block, c->slot_of_block + std::max(0, c->host_capacity_blocks)),
+        block_of_slot(c->block_of_slot, c->block_of_slot + std::max(0, c->pool_slots)),
+        last_use(c->last_use, c->last_use + std::max(0, c->pool_slots)),
+        target(c) {
+    view = *c;
+    view.slot_of_block = slot_of_block.data();
+    view.block_of_slot = block_of_slot.data();
+    view.last_use = last_use.data();
+  }
+  void commit() {
+    std::copy(slot_of_block.begin(), slot_of_block.end(), target->slot_of_block);
+    std::copy(block_of_slot.begin(), block_of_slot.end(), target->block_of_slot);
+    std::copy(last_use.begin(), last_use.end(), target->last_use);
+    target->tick = view.tick;
+  }
+};
+
+bool cache_arrays_ok(const hga_block_cache* c) {
+  return c->host_capacity_blocks >= 0 && c->pool_slots >= 0 &&
+         (c->host_capacity_blocks == 0 || c->slot_of_block != nullptr) &&
+         (c->pool_slots == 0 || (c->block_of_slot != nullptr && c->last_use != nullptr));
+}
+
 }  // namespace
 
 extern "C" {
@@ -552,6 +586,7 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
   if (r != HGA_OK) return r;
   if (any_null(host_k, host_v, idx_dev, host_idx_scratch, pool_k, pool_v, cache, idx_pool_dev, done))
     return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!cache_arrays_ok(cache)) return fail(HGA_ERR_INVALID_ARG, "block cache: NULL arrays or negative sizes");
   const int cap = cache->host_capacity_blocks, pool_slots = cache->pool_slots;
   if (cap < dims->n_hist_blocks)
     return fail(HGA_ERR_INVALID_ARG, "host tier holds %d blocks < n_hist_blocks %d", cap, dims->n_hist_blocks);
@@ -599,15 +634,18 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
     if (used[n]) need.push_back(n);
   std::vector<int32_t> slot(need.size() + 1), miss(need.size() + 1);
   int n_miss = 0;
-  if ((r = hga_block_cache_plan(cache, need.data(), (int)need.size(), slot.data(), miss.data(), &n_miss)) != HGA_OK)
+  CacheDraft draft(cache);
+  if ((r = hga_block_cache_plan(&draft.view, need.data(), (int)need.size(), slot.data(), miss.data(), &n_miss)) !=
+      HGA_OK)
     return r;
+  const int32_t* slot_of_block = draft.slot_of_block.data();
   // 3. host -> pool copies of the misses, merged where blocks and slots are both consecutive.
   const size_t es = s.bf16 ? 2 : 4;
   const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
   for (int k = 0; k < n_miss;) {
-    const int n0 = miss[k], s0 = cache->slot_of_block[n0];
+    const int n0 = miss[k], s0 = slot_of_block[n0];
     int run = 1;
-    while (k + run < n_miss && miss[k + run] == n0 + run && cache->slot_of_block[n0 + run] == s0 + run) ++run;
+    while (k + run < n_miss && miss[k + run] == n0 + run && slot_of_block[n0 + run] == s0 + run) ++run;
     for (int b = 0; b < s.B; ++b) {
       const size_t src = ((size_t)b * cap + n0) * blk_bytes;
       const size_t dst = ((size_t)b * pool_slots + s0) * blk_bytes;
@@ -623,13 +661,14 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
   // 4. idx rewritten to slots (in the pinned scratch), then uploaded.
   for (size_t k = 0; k < n_idx; ++k) {
     const int n = host_idx_scratch[k];
-    host_idx_scratch[k] = n < 0 ? -1 : cache->slot_of_block[n];
+    host_idx_scratch[k] = n < 0 ? -1 : slot_of_block[n];
   }
   if ((e = cudaMemcpyAsync(idx_pool_dev, host_idx_scratch, n_idx * sizeof(int32_t), cudaMemcpyHostToDevice, xst)) !=
       cudaSuccess)
     return cuda_fail(e, "pool idx upload");
   if ((e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(done), xst)) != cudaSuccess)
     return cuda_fail(e, "event record");
+  draft.commit();  // every copy is queued: the plan becomes the cache's state
   if (n_unique_out) *n_unique_out = (int)need.size();
   if (n_fetched_out) *n_fetched_out = n_miss;
   return HGA_OK;
@@ -641,6 +680,7 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(k_seg, v_seg, pool_k, pool_v, cache)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!cache_arrays_ok(cache)) return fail(HGA_ERR_INVALID_ARG, "block cache: NULL arrays or negative sizes");
   const int nseg = s.nqb();
   if (at_block < 0 || at_block + nseg > cache->host_capacity_blocks)
     return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the cache's %d", at_block, at_block + nseg,
@@ -648,7 +688,9 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
   std::vector<int32_t> need(nseg), slot(nseg), miss(nseg);
   for (int t = 0; t < nseg; ++t) need[t] = at_block + t;
   int n_miss = 0;
-  if ((r = hga_block_cache_plan(cache, need.data(), nseg, slot.data(), miss.data(), &n_miss)) != HGA_OK) return r;
+  CacheDraft draft(cache);
+  if ((r = hga_block_cache_plan(&draft.view, need.data(), nseg, slot.data(), miss.data(), &n_miss)) != HGA_OK)
+    return r;
   // every block is copied, resident or not: the caller states that these blocks now hold this segment
   const size_t es = s.bf16 ? 2 : 4;
   const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
@@ -668,6 +710,7 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
     }
     t += run;
   }
+  draft.commit();
   return HGA_OK;
 }
 
@@ -709,6 +752,24 @@ hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const vo
     if (e != cudaSuccess) return cuda_fail(e, "segment offload copy");
   }
   return HGA_OK;
+}
+
+hga_status hga_selftest_attn_fwd_stalled(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                                         const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx,
+                                         void* o, float* lse, hga_stream_t stream) {
+  hga::Shape s{};
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (!hga::tc_supported(s)) return fail(HGA_ERR_UNSUPPORTED, "the stall self test runs the tensor-core forward only");
+  if ((r = check_attn_ptrs(s, n_kv_blocks, q, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
+  if (any_null(o, lse)) return fail(HGA_ERR_INVALID_ARG, "NULL output pointer");
+  int* err = nullptr;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  hga::TcMaps m;
+  if ((r = build_maps(s, n_kv_blocks, q, nullptr, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
+  cudaError_t e =
+      hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, reinterpret_cast<cudaStream_t>(stream), true);
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "stalled forward launch");
 }
 
 hga_status hga_selftest_umma(int form, const void* a, const void* b, float* d, hga_stream_t stream) {

@@ -73,6 +73,7 @@ struct FwdArgs {
   __nv_bfloat16* o;
   float* lse;
   int* err;
+  int withhold_kv;  // self test of the timeout path: the producer issues no K/V loads
 };
 
 __global__ void __launch_bounds__(384, 1)
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int hh = 0; hh < 2; ++hh)
           tma_load_4d(&tm_q, &ctl->q_full, sQ + t * kTileBytes + hh * kHalf, hh * 64, hq0 + t, i * kBM, b);
       int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      for (int j = 0; j < (a.withhold_kv ? 0 : nt); ++j) {
         const int tile = ctl->tiles[j];
         const bool hist = tile >= 0;
         const int row0 = (hist ? tile : (-tile - 1)) * kBN;
@@ -362,13 +363,14 @@ bool tc_supported(const Shape& s) {
 }
 
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
-                               int* err, cudaStream_t st) {
+                               int* err, cudaStream_t st, bool withhold_kv) {
   cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
   a.sl2 = 1.4426950408889634f / sqrtf((float)kD);
   a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err;
+  a.withhold_kv = withhold_kv ? 1 : 0;
   const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
   fwd_tc_kernel<<<grid, 384, kSmemBytes, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
   return cudaGetLastError();

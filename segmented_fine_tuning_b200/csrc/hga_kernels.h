@@ -56,8 +56,10 @@ struct TcMaps {
   CUtensorMap q, d_o, ks, vs, kh, vh;
 };
 bool tc_supported(const Shape& s);
+// withhold_kv (self test only): the producer issues no K/V tile loads, so the
+// MMA warp's pipeline wait expires and the CTA takes its timeout path.
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
-                               int* err, cudaStream_t st);
+                               int* err, cudaStream_t st, bool withhold_kv = false);
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                                const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
                                cudaStream_t st);

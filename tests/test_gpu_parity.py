@@ -211,9 +211,11 @@ def test_dense_equivalence_full():
     assert_close("dV", to_host(st.dv), dv_ref, BF16_ABS, BF16_REL)
 
 
-def test_qwen3_8b_layer_sampled():
+def test_qwen3_8b_layer_all_heads():
     """Full-size Qwen3-8B-shaped layer (the benchmark launch): selection over
-    all heads; O/LSE/dQ/dK/dV for KV heads 0 and 7 (all their query heads)."""
+    all heads; O/LSE/dQ/dK/dV element by element for all 8 KV heads and
+    their 32 query heads (every head-dependent path of the kernels: the
+    forward's head pairs, the per-head partial sums of dK/dV)."""
     w = synth.QWEN3_8B_LAYER
     x = synth.draw(w)
     st, _ = _gpu_step(w, x)
@@ -222,15 +224,17 @@ def test_qwen3_8b_layer_sampled():
     idx = st.idx.cpu().numpy()
     check_selection(dims_of(w), idx, idx_ref, score_ref, oracle.near_tie_positions(od, score_ref))
     args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
-    for h in (0, 7):
-        o_ref, lse_ref = oracle.attn_fwd(od, *args, kv_heads=range(h, h + 1))
-        dq_ref, dk_ref, dv_ref = oracle.attn_bwd(od, *args, x.d_o.f64, kv_heads=range(h, h + 1))
-        hs = slice(4 * h, 4 * h + 4)
-        assert_close(f"O h{h}", to_host(st.o)[:, :, hs], o_ref[:, :, hs], BF16_ABS, BF16_REL)
-        assert_close(f"LSE h{h}", to_host(st.lse)[:, hs], lse_ref[:, hs], BF16_ABS, BF16_REL)
-        assert_close(f"dQ h{h}", to_host(st.dq)[:, :, hs], dq_ref[:, :, hs], BF16_ABS, BF16_REL)
-        assert_close(f"dK h{h}", to_host(st.dk)[:, :, h], dk_ref[:, :, h], BF16_ABS, BF16_REL)
-        assert_close(f"dV h{h}", to_host(st.dv)[:, :, h], dv_ref[:, :, h], BF16_ABS, BF16_REL)
+    o_ref, lse_ref = oracle.attn_fwd(od, *args)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(od, *args, x.d_o.f64)
+    got = {"O": to_host(st.o), "LSE": to_host(st.lse), "dQ": to_host(st.dq), "dK": to_host(st.dk),
+           "dV": to_host(st.dv)}
+    for h in range(w.Hkv):
+        hs = slice(w.G * h, w.G * h + w.G)
+        assert_close(f"O h{h}", got["O"][:, :, hs], o_ref[:, :, hs], BF16_ABS, BF16_REL)
+        assert_close(f"LSE h{h}", got["LSE"][:, hs], lse_ref[:, hs], BF16_ABS, BF16_REL)
+        assert_close(f"dQ h{h}", got["dQ"][:, :, hs], dq_ref[:, :, hs], BF16_ABS, BF16_REL)
+        assert_close(f"dK h{h}", got["dK"][:, :, h], dk_ref[:, :, h], BF16_ABS, BF16_REL)
+        assert_close(f"dV h{h}", got["dV"][:, :, h], dv_ref[:, :, h], BF16_ABS, BF16_REL)
 
 
 def test_prefill_131k_sampled():

@@ -5,8 +5,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
-from hga_testutil import dims_of, to_dev
+from hga_testutil import BF16_ABS, BF16_REL, assert_close, dims_of, to_dev, to_host
 from segmented_fine_tuning_b200 import (BlockCache, HgaError, hga_attn_bwd, hga_attn_fwd, hga_cache_segment,
                                         hga_device_status, hga_fetch_blocks, hga_fetch_blocks_cached,
                                         hga_offload_segment, hga_remap_idx)
@@ -19,8 +20,27 @@ def _pinned(t: synth.Tensor):
     return torch.from_numpy(np.ascontiguousarray(t.store).view(np.int16)).view(torch.bfloat16).pin_memory()
 
 
+def _oracle_check(tag, w, x, idx_blocks, o, lse, dq=None, dk=None, dv=None):
+    """Outputs computed over a fetched pool against the fp64 oracle run on
+    the resident history with the block numbers the pool slots stand for."""
+    od = oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk)
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx_blocks)
+    o_r, lse_r = oracle.attn_fwd(od, *args)
+    assert_close(f"{tag} O", to_host(o), o_r, BF16_ABS, BF16_REL)
+    assert_close(f"{tag} LSE", to_host(lse), lse_r, BF16_ABS, BF16_REL)
+    if dq is not None:
+        dq_r, dk_r, dv_r = oracle.attn_bwd(od, *args, x.d_o.f64)
+        assert_close(f"{tag} dQ", to_host(dq), dq_r, BF16_ABS, BF16_REL)
+        assert_close(f"{tag} dK", to_host(dk), dk_r, BF16_ABS, BF16_REL)
+        assert_close(f"{tag} dV", to_host(dv), dv_r, BF16_ABS, BF16_REL)
+
+
 @pytest.mark.parametrize("capacity_extra", [0, 3])
-def test_fetch_into_pool_matches_resident_history(capacity_extra):
+def test_fetch_into_pool_matches_oracle(capacity_extra):
+    """The selected blocks fetched from a pinned host tier into a compact pool
+    (slots in ascending block order), then forward and backward over the
+    pool: O, LSE, dQ, dK, dV against the fp64 oracle over the full history,
+    and equal to the same kernels run over the resident history."""
     w = synth.Workload("tier: Hq8/Hkv2 S512 hist20 K3", 1, 8, 2, 128, 128, 512, 20, 3, "bf16", 41,
                        structured_keys=True)
     x = synth.draw(w)
@@ -63,6 +83,7 @@ def test_fetch_into_pool_matches_resident_history(capacity_extra):
                  dev["d_o"], dq, dk, dv, st.ws)
     torch.cuda.synchronize()
     hga_device_status()
+    _oracle_check("pool", w, x, st.idx.cpu().numpy(), o, lse, dq, dk, dv)
     assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref) and torch.equal(dq, dq_ref)
     # dK/dV accumulate per-head partials with atomics: equal up to summation order
     assert torch.allclose(dk, dk_ref, rtol=0, atol=1e-5) and torch.allclose(dv, dv_ref, rtol=0, atol=1e-5)
@@ -154,12 +175,14 @@ def test_cached_fetch_reuses_resident_blocks_and_evicts():
     nu, nf, o, lse = run(st.idx)
     assert nu == nf == len(sets[0])
     assert torch.equal(o, refs[0][0]) and torch.equal(lse, refs[0][1])
+    _oracle_check("first fetch", w, x, st.idx.cpu().numpy(), o, lse)
     nu, nf, o, lse = run(st.idx)
     assert nu == len(sets[0]) and nf == 0
     assert torch.equal(o, refs[0][0]) and torch.equal(lse, refs[0][1])
     resident = set(int(b) for b in cache.block_of_slot if b >= 0)
     nu, nf, o, lse = run(idx2)
     assert nu == len(sets[1]) and nf == len(sets[1] - resident)
+    _oracle_check("after evictions", w, x, idx2.cpu().numpy(), o, lse)
     # slots are no longer in block order, so the forward visits the history
     # tiles in another order: equal up to fp32 summation order
     assert (o.float() - refs[1][0].float()).abs().max().item() <= 2e-2
