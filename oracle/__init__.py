@@ -66,6 +66,8 @@ def _lib():
         lib.ohga_attn_fwd.argtypes = [D, P, P, P, P, P, P, I, I, P, P, P]
         lib.ohga_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, I, I, P, P, P]
         lib.ohga_dense_causal_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P]
+        lib.ohga_decode_select.argtypes = [D, I, P, P, P, P]
+        lib.ohga_decode_attn.argtypes = [D, I, I, P, P, P, P, P, P, P, P]
         _LIB = lib
     return _LIB
 
@@ -181,6 +183,47 @@ def dense_causal_fwd(q, k, v):
     o = np.zeros_like(q)
     lse = np.zeros((B, Hq, T))
     _lib().ohga_dense_causal_fwd(B, T, Hq, Hkv, d, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def decode_select(D: Dims, q_new, summ):
+    """Decode-step selection: the nq = q_new.shape[1] new queries form one
+    query group.  summ [B,Hkv,nblk,d] (oracle layout).  Returns (idx
+    [B,Hkv,topk], score [B,Hkv,nblk])."""
+    q_new, summ = _f64(q_new), _f64(summ)
+    nq = q_new.shape[1]
+    _check(q_new, (D.B, nq, D.Hq, D.d), "q_new")
+    _check(summ, (D.B, D.Hkv, D.nblk, D.d), "summ")
+    score = np.zeros((D.B, D.Hkv, D.nblk))
+    idx = np.zeros((D.B, D.Hkv, D.topk), dtype=np.int32)
+    _lib().ohga_decode_select(ctypes.byref(D.c()), nq, _ptr(q_new), _ptr(summ), _ptr(score), _ptr(idx))
+    return idx, score
+
+
+def decode_attn(D: Dims, t0: int, q_new, k_seg, v_seg, k_hist, v_hist, idx):
+    """Decode-step attention: new query u (segment position t0+u) over the
+    selected history blocks idx [B,Hkv,topk] and segment tokens 0..t0+u.
+    k_seg/v_seg [B,S,Hkv,d] with S = D.S (the segment buffer's capacity).
+    Returns (O [B,nq,Hq,d], LSE [B,Hq,nq])."""
+    q_new, k_seg, v_seg, k_hist, v_hist = map(_f64, (q_new, k_seg, v_seg, k_hist, v_hist))
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    nq = q_new.shape[1]
+    _check(q_new, (D.B, nq, D.Hq, D.d), "q_new")
+    _check(k_seg, (D.B, D.S, D.Hkv, D.d), "k_seg")
+    _check(v_seg, k_seg.shape, "v_seg")
+    nb = k_hist.shape[1] // D.blk
+    _check(k_hist, (D.B, nb * D.blk, D.Hkv, D.d), "k_hist")
+    _check(v_hist, k_hist.shape, "v_hist")
+    _check(idx, (D.B, D.Hkv, D.topk), "idx")
+    if not (0 <= t0 and t0 + nq <= D.S):
+        raise ValueError("new tokens outside the segment buffer")
+    if idx.size and (idx.max() >= nb or idx.min() < -1):
+        raise ValueError("idx out of range")
+    Dc = Dims(D.B, D.Hq, D.Hkv, D.d, D.blk, D.S, nb, D.topk)
+    o = np.zeros((D.B, nq, D.Hq, D.d))
+    lse = np.zeros((D.B, D.Hq, nq))
+    _lib().ohga_decode_attn(ctypes.byref(Dc.c()), nq, t0, _ptr(q_new), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist),
+                            _ptr(v_hist), _ptr(idx), _ptr(o), _ptr(lse))
     return o, lse
 
 

@@ -319,6 +319,102 @@ void ohga_attn_bwd(const ohga_dims* D, const double* q, const double* k_seg, con
   free(o);
 }
 
+/* ---------------------------------------------------------------- decode
+ * Decode step (article, Industry impact / fr Impact: HGA also serves
+ * generation).  nq new query tokens (1 <= nq) at active-segment positions
+ * t0 .. t0+nq-1 form the step's query group, a partial query block:
+ *   qm[b,hq,:]  = (1/nq) * sum over the nq new queries of q_new[b,u,hq,:]
+ *   score[b,h,n] = max over hq in group(h) of qm[b,hq] . summ[b,h,n] / sqrt(d)
+ *   idx[b,h,:]  = the min(topk, nblk) best blocks (ties to the lower index),
+ *                 ascending, padded with -1
+ * and new query u attends to every token of the selected history blocks and
+ * to the segment tokens at positions 0 .. t0+u.  Layouts:
+ *   q_new, o     [B, nq, Hq, d]
+ *   k_seg, v_seg [B, S, Hkv, d]   (S = capacity of the segment's KV buffer;
+ *                                  positions >= t0+nq are never read)
+ *   summ         [B, Hkv, nblk, d];  score [B, Hkv, nblk];  idx [B, Hkv, topk]
+ *   lse          [B, Hq, nq]
+ */
+void ohga_decode_select(const ohga_dims* D, int nq, const double* q_new, const double* summ, double* score,
+                        int32_t* idx) {
+  const int G = D->Hq / D->Hkv;
+  const int keff = D->topk < D->nblk ? D->topk : D->nblk;
+  const double inv_sqrt_d = 1.0 / sqrt((double)D->d);
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < D->B; ++b)
+    for (int h = 0; h < D->Hkv; ++h) {
+      double* qm = (double*)malloc(sizeof(double) * (size_t)G * D->d);
+      for (int g = 0; g < G; ++g)
+        for (int k = 0; k < D->d; ++k) {
+          double s = 0.0;
+          for (int u = 0; u < nq; ++u) s += q_new[tok_off(b, u, nq, h * G + g, D->Hq, D->d) + k];
+          qm[(size_t)g * D->d + k] = s / nq;
+        }
+      double* row = score + ((size_t)b * D->Hkv + h) * D->nblk;
+      for (int n = 0; n < D->nblk; ++n) {
+        const double* sv = summ + (((size_t)b * D->Hkv + h) * D->nblk + n) * D->d;
+        double best = -INFINITY;
+        for (int g = 0; g < G; ++g) {
+          const double v = dot(qm + (size_t)g * D->d, sv, D->d) * inv_sqrt_d;
+          if (v > best) best = v;
+        }
+        row[n] = best;
+      }
+      ohga_cand* c = (ohga_cand*)malloc(sizeof(ohga_cand) * (D->nblk > 0 ? D->nblk : 1));
+      int* chosen = (int*)malloc(sizeof(int) * (keff > 0 ? keff : 1));
+      for (int n = 0; n < D->nblk; ++n) { c[n].s = row[n]; c[n].n = n; }
+      qsort(c, D->nblk, sizeof(ohga_cand), cand_cmp);
+      for (int r = 0; r < keff; ++r) chosen[r] = c[r].n;
+      qsort(chosen, keff, sizeof(int), int_cmp);
+      int32_t* out = idx + ((size_t)b * D->Hkv + h) * D->topk;
+      for (int r = 0; r < D->topk; ++r) out[r] = r < keff ? chosen[r] : -1;
+      free(chosen);
+      free(c);
+      free(qm);
+    }
+}
+
+void ohga_decode_attn(const ohga_dims* D, int nq, int t0, const double* q_new, const double* k_seg,
+                      const double* v_seg, const double* k_hist, const double* v_hist, const int32_t* idx, double* o,
+                      double* lse) {
+  const int G = D->Hq / D->Hkv;
+  const int T = D->nblk * D->blk;
+  const int maxk = D->topk * D->blk + t0 + nq;
+#pragma omp parallel
+  {
+    const double** keys = (const double**)malloc(sizeof(double*) * maxk);
+    const double** vals = (const double**)malloc(sizeof(double*) * maxk);
+    double* s_buf = (double*)malloc(sizeof(double) * maxk);
+#pragma omp for collapse(3) schedule(dynamic, 4)
+    for (int b = 0; b < D->B; ++b)
+      for (int hq = 0; hq < D->Hq; ++hq)
+        for (int u = 0; u < nq; ++u) {
+          const int h = hq / G;
+          const int32_t* sel = idx + ((size_t)b * D->Hkv + h) * D->topk;
+          int nk = 0;
+          for (int r = 0; r < D->topk; ++r) {
+            const int n = sel[r];
+            if (n < 0) continue;
+            for (int t = 0; t < D->blk; ++t) {
+              keys[nk] = k_hist + tok_off(b, n * D->blk + t, T, h, D->Hkv, D->d);
+              vals[nk] = v_hist + tok_off(b, n * D->blk + t, T, h, D->Hkv, D->d);
+              ++nk;
+            }
+          }
+          for (int t = 0; t <= t0 + u; ++t) {
+            keys[nk] = k_seg + tok_off(b, t, D->S, h, D->Hkv, D->d);
+            vals[nk] = v_seg + tok_off(b, t, D->S, h, D->Hkv, D->d);
+            ++nk;
+          }
+          row_attention(D->d, q_new + tok_off(b, u, nq, hq, D->Hq, D->d), nk, keys, vals,
+                        o + tok_off(b, u, nq, hq, D->Hq, D->d), &lse[((size_t)b * D->Hq + hq) * nq + u], s_buf, NULL);
+        }
+    free(keys);
+    free(vals);
+    free(s_buf);
+  }
+}
+
 /* Textbook dense causal attention over one whole sequence [B,T,H*,d] with
  * grouped KV heads: row t attends to keys 0..t.  Used only to check the
  * identity "every history block selected == dense causal attention". */

@@ -20,6 +20,11 @@ void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, con
 void ohga_attn_bwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
                    const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o, int h0, int h1,
                    double* dq, double* dk, double* dv);
+void ohga_decode_select(const ohga_dims* D, int nq, const double* q_new, const double* summ, double* score,
+                        int32_t* idx);
+void ohga_decode_attn(const ohga_dims* D, int nq, int t0, const double* q_new, const double* k_seg,
+                      const double* v_seg, const double* k_hist, const double* v_hist, const int32_t* idx, double* o,
+                      double* lse);
 void ohga_dense_causal_fwd(int B, int T, int Hq, int Hkv, int d, const double* q, const double* k, const double* v,
                            double* o, double* lse);
 #endif

@@ -363,3 +363,84 @@ def test_near_tie_flag():
     score = np.array([[[[3.0, 2.0, 1.9999, 0.0], [3.0, 2.0, 1.0, 0.0]]]])
     flags = oracle.near_tie_positions(D, score)
     assert flags.tolist() == [[[True, False]]]
+
+
+# ---------------------------------------------------------------- decode step
+
+def _summ_oracle_layout(D: Dims, kh):
+    return oracle.block_summaries(D, kh)
+
+
+@pytest.mark.parametrize("i", [0, 2, 3])
+def test_decode_whole_block_equals_prefill_block(i):
+    """nq = block new queries starting at a block boundary form a whole query
+    block: decode selection and attention equal the prefill oracle's for that
+    block (itself pinned by the tests above)."""
+    D = Dims(B=2, Hq=6, Hkv=2, d=8, blk=4, S=16, nblk=7, topk=3)
+    q, ks, vs, kh, vh, _ = _rand_inputs(D, 71 + i)
+    summ = oracle.block_summaries(D, kh)
+    idx_p, score_p = oracle.select(D, q, kh)
+    o_p, lse_p = oracle.attn_fwd(D, q, ks, vs, kh, vh, idx_p)
+    rows = slice(i * D.blk, (i + 1) * D.blk)
+    idx_d, score_d = oracle.decode_select(D, q[:, rows], summ)
+    np.testing.assert_array_equal(idx_d, idx_p[:, :, i])
+    np.testing.assert_allclose(score_d, score_p[:, :, i], rtol=0, atol=1e-14)
+    o_d, lse_d = oracle.decode_attn(D, i * D.blk, q[:, rows], ks, vs, kh, vh, idx_d)
+    np.testing.assert_allclose(o_d, o_p[:, rows], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse_d, lse_p[:, :, rows], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("nq,t0", [(1, 0), (1, 9), (3, 5), (5, 2)])
+def test_decode_bruteforce(nq, t0):
+    """Straight numpy restatement on a tiny case: mean of the new queries,
+    group-max scores, the best K-subset by enumeration, and a softmax over
+    the explicit key list of every new row."""
+    D = Dims(B=1, Hq=4, Hkv=2, d=4, blk=2, S=12, nblk=6, topk=2)
+    r = _rng(80 + nq + t0)
+    qn = r.standard_normal((1, nq, D.Hq, D.d))
+    ks = r.standard_normal((1, D.S, D.Hkv, D.d))
+    vs = r.standard_normal((1, D.S, D.Hkv, D.d))
+    kh = r.standard_normal((1, D.nblk * D.blk, D.Hkv, D.d))
+    vh = r.standard_normal((1, D.nblk * D.blk, D.Hkv, D.d))
+    summ = oracle.block_summaries(D, kh)
+    idx, score = oracle.decode_select(D, qn, summ)
+    G = D.Hq // D.Hkv
+    o, lse = oracle.decode_attn(D, t0, qn, ks, vs, kh, vh, idx)
+    for h in range(D.Hkv):
+        sm = kh[0, :, h].reshape(D.nblk, D.blk, D.d).mean(axis=1)
+        qm = qn[0, :, h * G:(h + 1) * G].mean(axis=0)                  # [G, d]
+        want = (qm @ sm.T).max(axis=0) / math.sqrt(D.d)
+        np.testing.assert_allclose(score[0, h], want, rtol=0, atol=1e-13)
+        assert idx[0, h].tolist() == list(_brute_topk(want.tolist(), D.topk))
+        for g in range(G):
+            hq = h * G + g
+            for u in range(nq):
+                keys = [kh[0, n * D.blk + t, h] for n in idx[0, h] for t in range(D.blk)]
+                vals = [vh[0, n * D.blk + t, h] for n in idx[0, h] for t in range(D.blk)]
+                keys += [ks[0, t, h] for t in range(t0 + u + 1)]
+                vals += [vs[0, t, h] for t in range(t0 + u + 1)]
+                s = np.array([qn[0, u, hq] @ k for k in keys]) / math.sqrt(D.d)
+                p = np.exp(s - s.max())
+                np.testing.assert_allclose(o[0, u, hq], (p / p.sum()) @ np.array(vals), rtol=0, atol=1e-13)
+                assert abs(lse[0, hq, u] - (s.max() + math.log(p.sum()))) < 1e-13
+
+
+def test_decode_q_zero_and_short_history():
+    """Q = 0: every score is 0, so blocks 0..K-1 are chosen (padding -1 when the
+    history is shorter than K) and each row is the plain mean of its values,
+    LSE = log(number of keys)."""
+    D = Dims(B=1, Hq=2, Hkv=1, d=4, blk=2, S=8, nblk=3, topk=5)
+    r = _rng(90)
+    qn = np.zeros((1, 2, 2, 4))
+    ks, vs = r.standard_normal((1, 8, 1, 4)), r.standard_normal((1, 8, 1, 4))
+    kh, vh = r.standard_normal((1, 6, 1, 4)), r.standard_normal((1, 6, 1, 4))
+    idx, score = oracle.decode_select(D, qn, oracle.block_summaries(D, kh))
+    assert idx.reshape(-1).tolist() == [0, 1, 2, -1, -1]
+    np.testing.assert_array_equal(score, 0.0)
+    t0 = 3
+    o, lse = oracle.decode_attn(D, t0, qn, ks, vs, kh, vh, idx)
+    for u in range(2):
+        vals = np.concatenate([vh[0, :, 0], vs[0, : t0 + u + 1, 0]])
+        for hq in range(2):
+            np.testing.assert_allclose(o[0, u, hq], vals.mean(axis=0), rtol=0, atol=1e-14)
+            assert abs(lse[0, hq, u] - math.log(len(vals))) < 1e-14
