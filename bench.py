@@ -401,6 +401,20 @@ def h2d_probe(device, nbytes=1 << 30, reps=5):
     return best
 
 
+SEGMENTED_MODES = {
+    # history served from the pinned host tier: finished segments are not
+    # inserted into the device pool, so every step copies its new blocks over
+    # the host link; selection and fetch of layer l+1 overlap layer l
+    "host_tier": dict(keep_new_blocks=False, prefetch=True),
+    # the same without the one-layer lookahead (the host waits for each
+    # layer's indices before its copies start)
+    "host_tier_no_prefetch": dict(keep_new_blocks=False, prefetch=False),
+    # finished segments also enter each layer's device block cache: no host
+    # transfer in the pass (the compute-only reference)
+    "resident": dict(keep_new_blocks=True, prefetch=True),
+}
+
+
 def run_segmented(args, device):
     """The full segmented pass: 36 Qwen3-8B-shaped layers over a 16,384-token
     sequence as 8 segments of 2,048 (history in a pinned host tier, selected
@@ -408,7 +422,8 @@ def run_segmented(args, device):
     layer's device block cache, summaries appended on the device).
     Inputs: the 8 segments of layer 0 drawn with the workload's recipe and
     reused for every layer (the kernels' speed does not depend on values;
-    selection, and so fetch volume, is representative).  One step = one pass."""
+    selection, and so fetch volume, is representative).  One step = one pass.
+    Every mode of --segmented-modes is timed; the first is the line's value."""
     import segmented_fine_tuning_b200 as hga
     from segmented_fine_tuning_b200.segmented import SegmentedPass
     w = synth.QWEN3_8B_LAYER
@@ -416,51 +431,165 @@ def run_segmented(args, device):
     seg = hga.Dims(1, w.Hq, w.Hkv, w.d, w.blk, w.S, 0, w.topk, "bf16")
     xs = [synth.draw_segment(w, 0, s) for s in range(NS)]
     dev = [tuple(to_dev(t, device) for t in (x.q, x.k_seg, x.v_seg, x.d_o)) for x in xs]
-    sp = SegmentedPass(seg, L, NS, device)
     stream = torch.cuda.current_stream(device)
+    blk_bytes = w.blk * w.Hkv * w.d * 2 * 2
+    probe = h2d_probe(device)
+    modes = [m for m in args.segmented_modes.split(",") if m]
+    results = {}
+    for mode in modes:
+        sp = SegmentedPass(seg, L, NS, device, pool_slots=args.pool_slots, **SEGMENTED_MODES[mode])
 
-    def one_pass():
-        sp.new_sequence()  # each pass is a new sequence: nothing resident carries over
-        for s in range(NS):
-            sp.run_segment(s, [dev[s]] * L)
+        def one_pass():
+            sp.new_sequence()  # each pass is a new sequence: nothing resident carries over
+            for s in range(NS):
+                sp.run_segment(s, [dev[s]] * L)
+
+        for _ in range(args.warmup):
+            one_pass()
+        torch.cuda.synchronize(device)
+        hga.hga_device_status(stream)
+        sp.fetched_blocks.clear()
+        sp.selected_blocks.clear()
+        sp.device_remaps = 0
+        times = []
+        with ClockSampler(device.index if device.index is not None else 0) as clk:
+            for _ in range(args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                one_pass()
+                e1.record(stream)
+                torch.cuda.synchronize(device)
+                times.append(e0.elapsed_time(e1))
+        hga.hga_device_status(stream)
+        ms = float(np.mean(times))
+        fetched = float(np.mean(sp.fetched_blocks))
+        h2d_bytes = float(np.sum(sp.fetched_blocks)) * blk_bytes / args.steps
+        remaps = sp.device_remaps // args.steps
+        results[mode] = {"ms_per_pass": round(ms, 3), "tokens_per_s": round(NS * w.S * L / (ms / 1e3), 1),
+                         "blocks_copied_per_layer_step": round(fetched, 1), "h2d_bytes_per_pass": int(h2d_bytes),
+                         "fetch_time_at_probe_ms": round(h2d_bytes / (probe * 1e9) * 1e3, 2),
+                         "steps_remapped_on_device_per_pass": remaps,
+                         "device_block_cache_slots_per_layer": sp.pool_slots,
+                         "gpu_launches_per_pass": int(L * NS * 6 + remaps), "clocks": clk.summary(),
+                         **SEGMENTED_MODES[mode]}
+        del sp
+        torch.cuda.empty_cache()
+    head = results[modes[0]]
+    out = {"metric": "HGA full segmented pass tokens/s per layer (fwd+bwd, history fetched from a pinned host tier)",
+           "value": head["tokens_per_s"], "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": head["ms_per_pass"], "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic (layer 0's 8 segments reused for all layers)",
+           "config": {"workload": "segmented pass: 36 Qwen3-8B-shaped layers x 8 segments of 2,048 tokens, "
+                                  "history +16 blocks of 128 per segment, K16, pinned host tier",
+                      "layers": L, "segments": NS, "segment_tokens": w.S, "topk": w.topk, "mode": modes[0]},
+           "h2d_probe_gbs": round(probe, 1), "modes": results,
+           "gpu_launches": head["gpu_launches_per_pass"] * args.steps, "clocks": head["clocks"]}
+    if "resident" in results and modes[0] != "resident":
+        compute = results["resident"]["ms_per_pass"]
+        bound = max(compute, head["fetch_time_at_probe_ms"])
+        out["overlap"] = {"compute_only_ms": compute, "h2d_at_probe_ms": head["fetch_time_at_probe_ms"],
+                          "pass_over_bound": round(head["ms_per_pass"] / bound, 3)}
+    return out
+
+
+def run_decode(args, device):
+    """Decode at 131K context: 992 history blocks with resident summaries, a
+    4,096-token segment buffer, one new token at its last position, K = 32.
+    One step = decode selection + decode attention (split over key chunks,
+    then the merge), L2 flushed between steps.  Each kernel's bytes are its
+    algorithmic HBM traffic: the summaries for the selection; the selected
+    history blocks, the segment prefix and the new queries for attention."""
+    import segmented_fine_tuning_b200 as hga
+    w = synth.DECODE_131K
+    nq, t0 = 1, w.S - 1
+    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
+    x = synth.draw_decode(w, nq, t0)
+    dev = {n: to_dev(getattr(x, n), device) for n in ("k_seg", "v_seg", "k_hist", "v_hist")}
+    qn = to_dev(x.extra["q_new"], device)
+    summ = torch.empty((w.B, w.nblk, w.Hkv, w.d), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    hga.hga_block_summaries(D, dev["k_hist"], 0, w.nblk, summ, stream)
+    idx = torch.empty((w.B, w.Hkv, w.topk), dtype=torch.int32, device=device)
+    o = torch.empty_like(qn)
+    lse = torch.empty((w.B, w.Hq, nq), dtype=torch.float32, device=device)
+    ws = torch.empty((hga.hga_decode_workspace_size(D, nq),), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        hga.hga_decode_select(D, qn, summ, idx, None, stream)
+        if evs:
+            evs[1].record(stream)
+        hga.hga_decode_attn(D, t0, qn, dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk, idx, o,
+                            lse, ws, stream)
+        if evs:
+            evs[2].record(stream)
 
     for _ in range(args.warmup):
-        one_pass()
+        flush.zero_()
+        step()
     torch.cuda.synchronize(device)
     hga.hga_device_status(stream)
-    sp.fetched_blocks.clear()
-    sp.selected_blocks.clear()
-    times = []
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     with ClockSampler(device.index if device.index is not None else 0) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            step(evs[k])
+        torch.cuda.synchronize(device)
+    hga.hga_device_status(stream)
+    t_sel = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms = t_sel + t_att
+    # whole step as one CUDA graph (three launches replayed without host launch cost)
+    graph = {}
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+                hga.hga_decode_select(D, qn, summ, idx, None, side)
+                hga.hga_decode_attn(D, t0, qn, dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk,
+                                    idx, o, lse, ws, side)
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize(device)
+        gt = []
         for _ in range(args.steps):
+            flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            one_pass()
+            g.replay()
             e1.record(stream)
             torch.cuda.synchronize(device)
-            times.append(e0.elapsed_time(e1))
-    hga.hga_device_status(stream)
-    ms = float(np.mean(times))
-    tokens = NS * w.S
-    fetched = float(np.mean(sp.fetched_blocks))
-    selected = float(np.mean(sp.selected_blocks)) if sp.selected_blocks else None
-    blk_bytes = w.blk * w.Hkv * w.d * 2 * 2
-    h2d_bytes = fetched * blk_bytes * L * (NS - 1)
-    probe = h2d_probe(device)
-    return {"metric": "HGA full segmented pass tokens/s per layer (fwd+bwd, history fetched from a pinned host tier)",
-            "value": round(tokens * L / (ms / 1e3), 1), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (layer 0's 8 segments reused for all layers)",
-            "config": {"workload": "segmented pass: 36 Qwen3-8B-shaped layers x 8 segments of 2,048 tokens, "
-                                   "history +16 blocks of 128 per segment, K16, pinned host tier",
-                       "layers": L, "segments": NS, "segment_tokens": w.S, "topk": w.topk},
-            "fetch": {"blocks_selected_per_host_fetch": None if selected is None else round(selected, 1),
-                      "blocks_copied_per_layer_step": round(fetched, 1),
-                      "steps_remapped_on_device_per_pass": sp.device_remaps // (args.steps + args.warmup),
-                      "device_block_cache_slots_per_layer": sp.pool_slots, "h2d_bytes_per_pass": int(h2d_bytes),
-                      "h2d_probe_gbs": round(probe, 1),
-                      "fetch_time_at_probe_ms": round(h2d_bytes / (probe * 1e9) * 1e3, 2)},
-            "gpu_launches": int(L * NS * 6 + L * NS + L * (NS - 1)), "clocks": clk.summary()}
+            gt.append(e0.elapsed_time(e1))
+        hga.hga_device_status(stream)
+        ms_graph = float(np.mean(gt))
+        graph = {"ms_per_step": round(ms_graph, 4), "tokens_per_s": round(nq / (ms_graph / 1e3), 1)}
+    except Exception as e:  # report, do not hide: the eager numbers above stand
+        graph = {"error": str(e)[:300]}
+    keff = min(w.topk, w.nblk)
+    kv_bytes = (keff * w.blk + t0 + nq) * w.Hkv * w.d * 2 * 2 + qn.numel() * 2
+    sel_bytes = w.nblk * w.Hkv * w.d * 4 + qn.numel() * 2
+    peaks, peak_src = load_peaks()
+    att_gbs = kv_bytes / (t_att / 1e3) / 1e9
+    return {"metric": "HGA decode tokens/s per layer (131K context, one new token per step)",
+            "value": round(nq / (ms / 1e3), 1), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); block-structured keys)",
+            "config": {"workload": w.name, "history_blocks": w.nblk, "segment_buffer": w.S, "t0": t0, "n_q": nq,
+                       "topk": w.topk, "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+            "kernels": {"decode_select": {"ms": round(t_sel, 4), "bytes": sel_bytes,
+                                          "gbs": round(sel_bytes / (t_sel / 1e3) / 1e9, 1)},
+                        "decode_attn": {"ms": round(t_att, 4), "bytes": kv_bytes, "gbs": round(att_gbs, 1),
+                                        "frac_hbm": round(att_gbs / peaks["hbm_gbs"], 3)}},
+            "roofline": {"kernel": "decode_attn (partial + merge)", "bound": "hbm", "achieved": round(att_gbs, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(att_gbs / peaks["hbm_gbs"], 4),
+                         "traffic": None, "peak_source": f"{peak_src} HBM copy bandwidth"},
+            "cuda_graph": graph,
+            "gpu_launches": 4 * args.steps, "clocks": clk.summary()}
 
 
 # ---------------------------------------------------------------- oracle legs
@@ -531,14 +660,18 @@ def main():
     ap.add_argument("--impl", choices=("hga", "reference"), default="hga")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--segmented-modes", default="host_tier,resident,host_tier_no_prefetch",
+                    help="comma list of " + ", ".join(SEGMENTED_MODES) + " for --workload segmented")
+    ap.add_argument("--pool-slots", type=int, default=None,
+                    help="device pool (cache) slots per layer for --workload segmented (default: the largest history)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the 131K-token prefill sub-measurement of the default (layer) run")
-    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill"), default="layer",
+    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode"), default="layer",
                     help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
                          "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
-                         "the 131K prefill forward, device-timed only")
+                         "the 131K prefill forward, device-timed only; decode: one new token at 131K context")
     args = ap.parse_args()
-    if args.workload in ("dense", "prefill"):
+    if args.workload in ("dense", "prefill", "decode"):
         args.no_e2e = args.no_cpu_baseline = True
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3
@@ -559,8 +692,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     try:
-        if args.workload == "segmented":
-            out = run_segmented(args, device)
+        if args.workload in ("segmented", "decode"):
+            out = run_segmented(args, device) if args.workload == "segmented" else run_decode(args, device)
             if rank == 0:
                 print(json.dumps(out), flush=True)
             return

@@ -247,6 +247,51 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
                                    hga_stream_t stream);
 
 /*
+ * Decode step (article, Industry impact; fr edition, Impact: HGA also serves
+ * generation and retrieval).  One step processes n_q new query tokens
+ * (1 <= n_q <= block) at active-segment positions t0 .. t0+n_q-1; they form
+ * one partial query block.  Here dims->S is the CAPACITY of the active
+ * segment's KV buffer (k_seg/v_seg [B, S, Hkv, d], positions 0 .. t0+n_q-1
+ * already written by the caller, the new tokens' K/V included), and
+ * dims->n_hist_blocks the history that selection ranks.
+ *
+ * hga_decode_select: for every (b, KV head h)
+ *   qm[g]     = mean over the n_q new rows of q_new[b, u, h*G+g, :]   (fp32)
+ *   score[n]  = max_g (qm[g] . summ[b,n,h,:]) / sqrt(d)
+ *   idx[b,h,:] = the K_eff = min(topk, n_hist_blocks) best n (ties to the
+ *                lower n), ascending, then -1 up to topk.
+ * q_new [B, n_q, Hq, d] dtype; summ as for hga_select_topk; idx [B, Hkv, topk]
+ * int32; scores_or_null fp32 [B, Hkv, topk] (the selected blocks' scores,
+ * -inf for padding).  With n_q = block and t0 a multiple of block this is
+ * exactly hga_select_topk's result for that query block.
+ *
+ * hga_decode_attn: new query u (position p = t0 + u) of head hq attends to the
+ * tokens of blocks idx[b, hq/G, :] (entries >= 0) of k_hist/v_hist (the
+ * history or a pool of n_kv_blocks blocks, as for hga_attn_fwd) and to
+ * segment positions 0 .. p; scale 1/sqrt(d), fp32 statistics.
+ *   o [B, n_q, Hq, d] dtype;  lse [B, Hq, n_q] fp32 (natural log)
+ * ws: device scratch of at least hga_decode_workspace_size(dims, n_q) bytes
+ * (16-byte aligned; contents need no initialisation), owned by the caller.
+ * With n_q = block and t0 a multiple of block the result equals hga_attn_fwd's
+ * rows of that query block.
+ * A finished segment joins the history as in the prefill: hga_segment_summaries
+ * appends its blocks' summaries, hga_offload_segment moves its K/V to the tier.
+ * Errors: HGA_ERR_SHAPE (n_q outside [1, block], new tokens outside the
+ * buffer, n_hist_blocks > 4096 for the selection), HGA_ERR_INVALID_ARG (null
+ * or misaligned pointers, short workspace); an idx entry outside
+ * [-1, n_kv_blocks) is skipped and flags HGA_ERR_INDEX on the device.
+ */
+HGA_API hga_status hga_decode_select(const hga_dims* dims, int n_q, const void* q_new, const float* summ,
+                                     int32_t* idx, float* scores_or_null, hga_stream_t stream);
+/* Bytes of device scratch hga_decode_attn needs for these dims and n_q (0 if
+ * they are invalid). */
+HGA_API size_t hga_decode_workspace_size(const hga_dims* dims, int n_q);
+HGA_API hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const void* q_new, const void* k_seg,
+                                   const void* v_seg, const void* k_hist, const void* v_hist, int n_kv_blocks,
+                                   const int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                                   hga_stream_t stream);
+
+/*
  * Targeted loading of the selected history (fr edition, Contexte: dynamic
  * loading of precise historical tokens per query block; Background: history
  * KV lives in system RAM).  host_k/host_v: pinned host memory (cudaHostAlloc)
@@ -277,6 +322,28 @@ HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, co
                             int32_t* host_idx_scratch, void* pool_k, void* pool_v, int pool_slots,
                             int32_t* idx_pool_dev, int* n_unique_out, hga_stream_t compute_stream,
                             hga_stream_t copy_stream, hga_event_t done, int timeout_ms);
+
+/*
+ * hga_fetch_blocks without the host: the distinct selected blocks are read by
+ * the GPU itself from the pinned host tier, mapped into the device's address
+ * space (zero copy), and the whole call is ordered on `stream` with no host
+ * wait (so it can be captured in a CUDA graph and queued ahead).  Same
+ * result as hga_fetch_blocks: pool slot k holds the k-th smallest selected
+ * block (K and V, all B and Hkv), idx_pool_dev = idx with block numbers
+ * replaced by slots (-1 kept).  host_k/host_v: pinned host memory
+ * (cudaHostAlloc, or registered as mapped) [B, host_capacity_blocks*block,
+ * Hkv, d], checked to be mapped over its whole extent; pool_k/pool_v device
+ * [B, pool_slots*block, Hkv, d].  A selected block ranked at or beyond
+ * pool_slots gets no slot: its idx_pool entries are -1 and the device error
+ * flag reports HGA_ERR_INDEX.  n_hist_blocks <= 32768.  The copies are made
+ * by the SMs over the host link (PCIe / C2C), not by the copy engines.
+ * Errors: HGA_ERR_INVALID_ARG (NULL or misaligned pointers, a tier that is not
+ * mapped pinned memory, tier smaller than the history), HGA_ERR_SHAPE.
+ */
+HGA_API hga_status hga_gather_blocks_mapped(const hga_dims* dims, const void* host_k, const void* host_v,
+                                            int host_capacity_blocks, const int32_t* idx_dev, void* pool_k,
+                                            void* pool_v, int pool_slots, int32_t* idx_pool_dev,
+                                            hga_stream_t stream);
 
 /*
  * Device block cache: history blocks stay in a layer's device pool across
@@ -353,6 +420,36 @@ HGA_API hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* hos
  */
 HGA_API hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, void* pool_k,
                                      void* pool_v, hga_block_cache* cache, int at_block, hga_stream_t stream);
+
+/*
+ * A finished segment enters the history in ONE pass over its K and V
+ * (article, Deep analysis: the summaries stay resident and grow with the
+ * context; fr edition, Analyse approfondie: a finished segment's KV is
+ * offloaded right away).  For the S/block blocks t of the segment
+ * (k_seg/v_seg [B, S, Hkv, d], device):
+ *   summ[b, at_block+t, h, :] = mean of the block's keys (fp32; as
+ *       hga_segment_summaries; dims->n_hist_blocks = the capacity of summ);
+ *   with a device block cache (cache != NULL): blocks at_block .. get slots
+ *       by the hga_block_cache_plan rules (as hga_cache_segment) and their K
+ *       and V are written into pool_k/pool_v [B, cache->pool_slots*block,
+ *       Hkv, d] by the same kernel that forms the summaries;
+ *   with a host tier (host_k/host_v != NULL, pinned, [B,
+ *       tier_capacity_blocks*block, Hkv, d]): the segment's K/V are copied
+ *       to the tier at block at_block on copy_stream (ordered after the work
+ *       already queued on `stream`; NULL copy_stream = `stream`), running
+ *       alongside the kernel; k_seg/v_seg must stay valid until copy_stream
+ *       has passed the copies.
+ * The kernel runs on `stream`; queue it after every kernel that may still read
+ * the pool slots it overwrites.  Replaces hga_segment_summaries +
+ * hga_cache_segment + hga_offload_segment (three passes over K) with one.
+ * S/block <= 128.  Errors: HGA_ERR_INVALID_ARG (NULL or misaligned pointers,
+ * blocks outside summ, the cache or the tier), HGA_ERR_SHAPE, HGA_ERR_CUDA; on
+ * any error the cache is unchanged.
+ */
+HGA_API hga_status hga_append_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, int at_block,
+                                      float* summ, void* pool_k, void* pool_v, hga_block_cache* cache, void* host_k,
+                                      void* host_v, int tier_capacity_blocks, hga_stream_t stream,
+                                      hga_stream_t copy_stream);
 
 /*
  * idx -> pool slots on the device, for a cache that holds every selectable

@@ -94,13 +94,18 @@ _SIGNATURES = [
     ("hga_attn_bwd_dq", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     ("hga_fetch_blocks", _I, [_D, _P, _P, _I, _P, _P, _P, _P, _I, _P, ctypes.POINTER(ctypes.c_int), _P, _P, _P,
                               _I]),
+    ("hga_gather_blocks_mapped", _I, [_D, _P, _P, _I, _P, _P, _P, _I, _P, _P]),
     ("hga_block_cache_reset", _I, [_C]),
     ("hga_block_cache_plan", _I, [_C, _P, _I, _P, _P, ctypes.POINTER(ctypes.c_int)]),
     ("hga_fetch_blocks_cached", _I, [_D, _P, _P, _P, _P, _P, _P, _C, _P, ctypes.POINTER(ctypes.c_int),
                                      ctypes.POINTER(ctypes.c_int), _P, _P, _P, _I]),
     ("hga_cache_segment", _I, [_D, _P, _P, _P, _P, _C, _I, _P]),
     ("hga_remap_idx", _I, [_D, _P, _P, _P, _P]),
+    ("hga_append_segment", _I, [_D, _P, _P, _I, _P, _P, _P, _C, _P, _P, _I, _P, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
+    ("hga_decode_select", _I, [_D, _I, _P, _P, _P, _P, _P]),
+    ("hga_decode_workspace_size", ctypes.c_size_t, [_D, _I]),
+    ("hga_decode_attn", _I, [_D, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
     ("hga_selftest_attn_fwd_stalled", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
 ]
@@ -431,3 +436,86 @@ def hga_selftest_attn_fwd_stalled(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n
                                                         _ptr(k_hist), _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o),
                                                         _ptr(lse), _stream(stream)),
            "hga_selftest_attn_fwd_stalled")
+
+
+def hga_decode_select(dims: Dims, q_new, summ, idx, scores=None, stream=None) -> None:
+    """Selection for the n_q = q_new.shape[1] new queries of a decode step."""
+    nq = q_new.shape[1]
+    _expect(q_new, (dims.B, nq, dims.Hq, dims.d), dims.torch_dtype, "q_new")
+    if dims.n_hist_blocks > 0:
+        if summ.dtype != torch.float32 or not summ.is_cuda or summ.numel() < dims.B * dims.n_hist_blocks * dims.Hkv * dims.d:
+            raise ValueError("summ: CUDA fp32 [B, n_hist_blocks, Hkv, d]")
+    _expect(idx, (dims.B, dims.Hkv, dims.topk), torch.int32, "idx")
+    if scores is not None:
+        _expect(scores, idx.shape, torch.float32, "scores")
+    _check(load_library().hga_decode_select(ctypes.byref(dims.c()), nq, _ptr(q_new), _ptr(summ), _ptr(idx),
+                                            _ptr(scores), _stream(stream)), "hga_decode_select")
+
+
+def hga_decode_workspace_size(dims: Dims, n_q: int) -> int:
+    return int(load_library().hga_decode_workspace_size(ctypes.byref(dims.c()), n_q))
+
+
+def hga_decode_attn(dims: Dims, t0: int, q_new, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, o, lse, ws,
+                    stream=None) -> None:
+    """Attention of the n_q new queries (segment positions t0..) over the
+    selected history blocks and the segment prefix; dims.S is the capacity of
+    the segment buffer k_seg/v_seg."""
+    nq = q_new.shape[1]
+    _expect(q_new, (dims.B, nq, dims.Hq, dims.d), dims.torch_dtype, "q_new")
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(v_seg, k_seg.shape, dims.torch_dtype, "v_seg")
+    if n_kv_blocks > 0:
+        _expect(k_hist, (dims.B, n_kv_blocks * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "k_hist")
+        _expect(v_hist, k_hist.shape, dims.torch_dtype, "v_hist")
+    _expect(idx, (dims.B, dims.Hkv, dims.topk), torch.int32, "idx")
+    _expect(o, q_new.shape, dims.torch_dtype, "o")
+    _expect(lse, (dims.B, dims.Hq, nq), torch.float32, "lse")
+    _check(load_library().hga_decode_attn(ctypes.byref(dims.c()), nq, t0, _ptr(q_new), _ptr(k_seg), _ptr(v_seg),
+                                          _ptr(k_hist), _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse),
+                                          _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hga_decode_attn")
+
+
+def hga_append_segment(dims: Dims, k_seg, v_seg, at_block: int, summ, pool_k=None, pool_v=None,
+                       cache: "BlockCache | None" = None, host_k=None, host_v=None, tier_capacity_blocks: int = 0,
+                       stream=None, copy_stream=None) -> None:
+    """A finished segment enters the history in one pass: summaries of its
+    blocks (dims.n_hist_blocks = summ's capacity), optionally its K/V into the
+    device block cache, optionally the copy to the pinned host tier."""
+    _expect(k_seg, (dims.B, dims.S, dims.Hkv, dims.d), dims.torch_dtype, "k_seg")
+    _expect(v_seg, k_seg.shape, dims.torch_dtype, "v_seg")
+    _expect(summ, (dims.B, dims.n_hist_blocks, dims.Hkv, dims.d), torch.float32, "summ")
+    if cache is not None:
+        _expect(pool_k, (dims.B, cache.pool_slots * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "pool_k")
+        _expect(pool_v, pool_k.shape, dims.torch_dtype, "pool_v")
+    if host_k is not None or host_v is not None:
+        shape = (dims.B, tier_capacity_blocks * dims.block, dims.Hkv, dims.d)
+        _expect(host_k, shape, dims.torch_dtype, "host_k", device=False)
+        _expect(host_v, shape, dims.torch_dtype, "host_v", device=False)
+        if not (host_k.is_pinned() and host_v.is_pinned()):
+            raise ValueError("host tier must be pinned host memory")
+    _check(load_library().hga_append_segment(
+        ctypes.byref(dims.c()), _ptr(k_seg), _ptr(v_seg), at_block, _ptr(summ),
+        _ptr(pool_k) if cache is not None else None, _ptr(pool_v) if cache is not None else None,
+        ctypes.byref(cache.c) if cache is not None else None, _ptr(host_k), _ptr(host_v), tier_capacity_blocks,
+        _stream(stream), _stream(copy_stream) if copy_stream is not None else None), "hga_append_segment")
+
+
+def hga_gather_blocks_mapped(dims: Dims, host_k, host_v, host_capacity_blocks: int, idx_dev, pool_k, pool_v,
+                             pool_slots: int, idx_pool_dev, stream=None) -> None:
+    """The distinct selected blocks copied by the GPU from the mapped pinned
+    host tier into a compact pool, idx rewritten to slots; no host wait."""
+    shape = (dims.B, host_capacity_blocks * dims.block, dims.Hkv, dims.d)
+    _expect(host_k, shape, dims.torch_dtype, "host_k", device=False)
+    _expect(host_v, shape, dims.torch_dtype, "host_v", device=False)
+    if not (host_k.is_pinned() and host_v.is_pinned()):
+        raise ValueError("host tier must be pinned host memory")
+    _expect(idx_dev, (dims.B, dims.Hkv, dims.nqb, dims.topk), torch.int32, "idx_dev")
+    _expect(pool_k, (dims.B, pool_slots * dims.block, dims.Hkv, dims.d), dims.torch_dtype, "pool_k")
+    _expect(pool_v, pool_k.shape, dims.torch_dtype, "pool_v")
+    _expect(idx_pool_dev, idx_dev.shape, torch.int32, "idx_pool_dev")
+    _check(load_library().hga_gather_blocks_mapped(ctypes.byref(dims.c()), _ptr(host_k), _ptr(host_v),
+                                                   host_capacity_blocks, _ptr(idx_dev), _ptr(pool_k), _ptr(pool_v),
+                                                   pool_slots, _ptr(idx_pool_dev), _stream(stream)),
+           "hga_gather_blocks_mapped")

@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <chrono>
+#include <memory>
 #include <mutex>
 #include <thread>
 #include <vector>
@@ -714,6 +715,128 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
   return HGA_OK;
 }
 
+namespace {
+
+// Device address of pinned, mapped host memory covering [p, p + bytes).
+hga_status mapped_device_ptr(const void* p, size_t bytes, const char* name, const void** out) {
+  cudaPointerAttributes a0, a1;
+  cudaError_t e = cudaPointerGetAttributes(&a0, p);
+  if (e == cudaSuccess && bytes > 0) e = cudaPointerGetAttributes(&a1, static_cast<const char*>(p) + bytes - 1);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HGA_ERR_INVALID_ARG, "%s: not pinned host memory (%s)", name, cudaGetErrorString(e));
+  }
+  if (a0.type != cudaMemoryTypeHost || (bytes > 0 && a1.type != cudaMemoryTypeHost) || a0.devicePointer == nullptr)
+    return fail(HGA_ERR_INVALID_ARG, "%s: the whole tier must be pinned host memory mapped into the device", name);
+  *out = a0.devicePointer;
+  return HGA_OK;
+}
+
+}  // namespace
+
+hga_status hga_gather_blocks_mapped(const hga_dims* dims, const void* host_k, const void* host_v,
+                                    int host_capacity_blocks, const int32_t* idx_dev, void* pool_k, void* pool_v,
+                                    int pool_slots, int32_t* idx_pool_dev, hga_stream_t stream) {
+  hga::Shape s{};
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (any_null(host_k, host_v, idx_dev, pool_k, pool_v, idx_pool_dev)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (pool_slots < 1) return fail(HGA_ERR_INVALID_ARG, "pool_slots < 1");
+  if (host_capacity_blocks < s.nblk)
+    return fail(HGA_ERR_INVALID_ARG, "host tier holds %d blocks < n_hist_blocks %d", host_capacity_blocks, s.nblk);
+  if (s.nblk > hga::gather_max_blocks())
+    return fail(HGA_ERR_SHAPE, "n_hist_blocks %d > %d", s.nblk, hga::gather_max_blocks());
+  if (!aligned16(host_k) || !aligned16(host_v) || !aligned16(pool_k) || !aligned16(pool_v))
+    return fail(HGA_ERR_INVALID_ARG, "tier and pool must be 16-byte aligned");
+  const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * (s.bf16 ? 2 : 4);
+  const size_t tier_bytes = (size_t)s.B * host_capacity_blocks * blk_bytes;
+  const void *dk = nullptr, *dv = nullptr;
+  if ((r = mapped_device_ptr(host_k, tier_bytes, "host_k", &dk)) != HGA_OK) return r;
+  if ((r = mapped_device_ptr(host_v, tier_bytes, "host_v", &dv)) != HGA_OK) return r;
+  int* err = nullptr;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  int dev = 0, n_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device attributes");
+  e = hga::launch_gather_mapped(s, idx_dev, dk, dv, host_capacity_blocks, pool_k, pool_v, pool_slots, idx_pool_dev,
+                                err, n_sm, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "mapped gather launch");
+}
+
+hga_status hga_append_segment(const hga_dims* dims, const void* k_seg, const void* v_seg, int at_block, float* summ,
+                              void* pool_k, void* pool_v, hga_block_cache* cache, void* host_k, void* host_v,
+                              int tier_capacity_blocks, hga_stream_t stream, hga_stream_t copy_stream) {
+  hga::Shape s{};
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  const int nseg = s.nqb();
+  if (nseg > hga::kMaxQueryBlocks) return fail(HGA_ERR_SHAPE, "segment of %d blocks > %d", nseg, hga::kMaxQueryBlocks);
+  if (any_null(k_seg, v_seg, summ)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k_seg) || !aligned16(v_seg)) return fail(HGA_ERR_INVALID_ARG, "k_seg/v_seg must be 16-byte aligned");
+  if (at_block < 0 || at_block + nseg > s.nblk)
+    return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the summary array's %d", at_block, at_block + nseg,
+                s.nblk);
+  if (cache) {
+    if (any_null(pool_k, pool_v)) return fail(HGA_ERR_INVALID_ARG, "NULL pool with a block cache");
+    if (!aligned16(pool_k) || !aligned16(pool_v)) return fail(HGA_ERR_INVALID_ARG, "pool must be 16-byte aligned");
+    if (!cache_arrays_ok(cache)) return fail(HGA_ERR_INVALID_ARG, "block cache: NULL arrays or negative sizes");
+    if (at_block + nseg > cache->host_capacity_blocks)
+      return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the cache's %d", at_block, at_block + nseg,
+                  cache->host_capacity_blocks);
+  }
+  const bool offload = host_k != nullptr || host_v != nullptr;
+  if (offload) {
+    if (any_null(host_k, host_v)) return fail(HGA_ERR_INVALID_ARG, "host_k and host_v go together");
+    if (at_block + nseg > tier_capacity_blocks)
+      return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the tier's %d", at_block, at_block + nseg,
+                  tier_capacity_blocks);
+  }
+  // 1. slots of the new blocks (planned on a draft of the cache)
+  std::vector<int32_t> need(nseg), slot(nseg), miss(nseg);
+  for (int t = 0; t < nseg; ++t) need[t] = at_block + t;
+  int n_miss = 0;
+  std::unique_ptr<CacheDraft> draft;
+  if (cache) {
+    draft.reset(new CacheDraft(cache));
+    if ((r = hga_block_cache_plan(&draft->view, need.data(), nseg, slot.data(), miss.data(), &n_miss)) != HGA_OK)
+      return r;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  // 2. the host-tier copy reads k_seg/v_seg on copy_stream, concurrently with the kernel
+  if (offload) {
+    cudaStream_t xst = copy_stream ? reinterpret_cast<cudaStream_t>(copy_stream) : st;
+    if (xst != st) {
+      cudaEvent_t ready = nullptr;
+      if ((e = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(e, "event create");
+      e = cudaEventRecord(ready, st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(xst, ready, 0);
+      cudaEventDestroy(ready);
+      if (e != cudaSuccess) return cuda_fail(e, "ordering the offload after the segment's producers");
+    }
+    const size_t es = s.bf16 ? 2 : 4;
+    const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * es;
+    for (int b = 0; b < s.B; ++b) {
+      const size_t dst = ((size_t)b * tier_capacity_blocks + at_block) * blk_bytes;
+      const size_t src = (size_t)b * nseg * blk_bytes;
+      e = cudaMemcpyAsync(static_cast<char*>(host_k) + dst, static_cast<const char*>(k_seg) + src, nseg * blk_bytes,
+                          cudaMemcpyDeviceToHost, xst);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(static_cast<char*>(host_v) + dst, static_cast<const char*>(v_seg) + src,
+                            nseg * blk_bytes, cudaMemcpyDeviceToHost, xst);
+      if (e != cudaSuccess) return cuda_fail(e, "segment offload copy");
+    }
+  }
+  // 3. one pass over K and V: summaries, and the pool copies when caching
+  e = hga::launch_append_segment(s, k_seg, v_seg, at_block, summ, cache ? pool_k : nullptr,
+                                 cache ? pool_v : nullptr, cache ? cache->pool_slots : 0, slot.data(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "segment append launch");
+  if (draft) draft->commit();
+  return HGA_OK;
+}
+
 hga_status hga_remap_idx(const hga_dims* dims, const int32_t* idx_dev, const int32_t* slot_of_block_dev,
                          int32_t* idx_pool_dev, hga_stream_t stream) {
   hga::Shape s{};
@@ -752,6 +875,52 @@ hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const vo
     if (e != cudaSuccess) return cuda_fail(e, "segment offload copy");
   }
   return HGA_OK;
+}
+
+hga_status hga_decode_select(const hga_dims* dims, int n_q, const void* q_new, const float* summ, int32_t* idx,
+                             float* scores_or_null, hga_stream_t stream) {
+  hga::Shape s{};
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (n_q < 1 || n_q > s.blk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, block = %d]", n_q, s.blk);
+  if (s.nblk > hga::kMaxSelectBlocks)
+    return fail(HGA_ERR_SHAPE, "n_hist_blocks %d > %d", s.nblk, hga::kMaxSelectBlocks);
+  if (any_null(q_new, idx) || (s.nblk > 0 && summ == nullptr)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q_new)) return fail(HGA_ERR_INVALID_ARG, "q_new must be 16-byte aligned");
+  // The new queries are one query block of n_q rows: the prefill selection
+  // kernel with S = block = n_q computes exactly the decode definition.
+  hga::Shape sq = s;
+  sq.S = n_q;
+  sq.blk = n_q;
+  cudaError_t e = hga::launch_select_topk(sq, q_new, summ, idx, scores_or_null, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "decode select launch");
+}
+
+size_t hga_decode_workspace_size(const hga_dims* dims, int n_q) {
+  hga::Shape s{};
+  if (check_dims(dims, &s) != HGA_OK || n_q < 1 || n_q > s.blk) return 0;
+  return round256(hga::decode_workspace_floats(s, n_q) * sizeof(float));
+}
+
+hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const void* q_new, const void* k_seg,
+                           const void* v_seg, const void* k_hist, const void* v_hist, int n_kv_blocks,
+                           const int32_t* idx, void* o, float* lse, void* ws, size_t ws_bytes, hga_stream_t stream) {
+  hga::Shape s{};
+  hga_status r = check_dims(dims, &s);
+  if (r != HGA_OK) return r;
+  if (n_q < 1 || n_q > s.blk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, block = %d]", n_q, s.blk);
+  if (t0 < 0 || t0 + n_q > s.S)
+    return fail(HGA_ERR_SHAPE, "new tokens [%d, %d) outside the segment buffer of %d", t0, t0 + n_q, s.S);
+  if ((r = check_attn_ptrs(s, n_kv_blocks, q_new, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
+  if (any_null(o, lse, ws)) return fail(HGA_ERR_INVALID_ARG, "NULL output or workspace pointer");
+  if (!aligned16(ws)) return fail(HGA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  const size_t need = hga_decode_workspace_size(dims, n_q);
+  if (ws_bytes < need) return fail(HGA_ERR_INVALID_ARG, "workspace %zu bytes < %zu", ws_bytes, need);
+  int* err = nullptr;
+  if ((r = device_err_ptr(&err)) != HGA_OK) return r;
+  cudaError_t e = hga::launch_decode_attn(s, n_q, t0, q_new, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse,
+                                          static_cast<float*>(ws), err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "decode attention launch");
 }
 
 hga_status hga_selftest_attn_fwd_stalled(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,

@@ -1,0 +1,292 @@
+// Decode step of HGA attention: a few new query tokens per step attend to the
+// top-K history blocks picked for them and to the active segment's prefix.
+//
+// Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention
+// and Segmented Backpropagation in Practice", Industry impact (fr edition,
+// Impact): the scheme also serves generation and retrieval.  The step's n_q
+// new queries (segment positions t0 .. t0+n_q-1) form one partial query
+// block: their mean is scored against the resident block summaries exactly as
+// a whole query block is in the prefill (hga_select_topk's kernel, run with a
+// query block of n_q rows), and new query u attends to the selected history
+// blocks plus segment positions 0 .. t0+u.
+//
+// Attention is split over the key axis (flash-decoding): one CTA per (chunk of
+// `block` keys, group of up to 16 query rows, batch x KV head).  The chunks are
+// the K selected history blocks and the segment prefix cut into blocks.  Each
+// CTA stages its K and V chunk in shared memory once (cp.async, 16-byte
+// vectors, rows padded by 16 bytes so that the per-key reads are conflict
+// free), forms the scores of its rows, and writes the chunk's partial softmax
+// state (running max m, sum l, unnormalised O) to the caller's workspace.  A
+// second kernel merges the chunks of every row: M = max m_c, L = sum l_c
+// 2^(m_c - M), O = sum O_c 2^(m_c - M) / L, LSE = (M + log2 L) ln 2.
+// The work is bound by HBM: the selected K/V blocks and the segment prefix
+// are read once.
+#include <float.h>
+
+#include "hga_kernels.h"
+#include "hga_ptx.cuh"
+
+namespace hga {
+namespace {
+
+constexpr int kDecThreads = 128;
+constexpr int kDecRows = 16;  // query rows per CTA
+
+template <typename T>
+struct DecElem;
+template <>
+struct DecElem<float> {
+  static constexpr int E = 4;  // elements per 16 bytes
+  __device__ static float at(const float* p) { return *p; }
+  __device__ static void unpack(uint4 v, float* out) {
+    out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+    out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+  }
+};
+template <>
+struct DecElem<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ static float at(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  __device__ static void unpack(uint4 v, float* out) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      out[2 * k] = __uint_as_float(w[k] << 16);
+      out[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+struct DecArgs {
+  int Hq, Hkv, S, d, blk, nq, t0, topk, nkv, n_chunks, G, R;
+  float sl2;             // log2(e) / sqrt(d)
+  const int32_t* idx;    // [B, Hkv, topk]
+  float* part_ml;        // [B, Hkv, n_chunks, R, 2]
+  float* part_o;         // [B, Hkv, n_chunks, R, d]
+  int* err;
+};
+
+// Shared memory: K and V chunk [blk][d + pad] of T, Q rows [16][d] fp32 (pre-
+// scaled to log2 units), scores / probabilities [16][blk] fp32, row max and sum.
+template <typename T>
+size_t dec_smem_bytes(int blk, int d) {
+  const size_t row = (size_t)d * sizeof(T) + 16;
+  return 2 * blk * row + (size_t)kDecRows * d * 4 + (size_t)kDecRows * blk * 4 + 2 * kDecRows * 4;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __restrict__ q_new,
+                                                                     const T* __restrict__ k_seg,
+                                                                     const T* __restrict__ v_seg,
+                                                                     const T* __restrict__ k_hist,
+                                                                     const T* __restrict__ v_hist, const DecArgs a) {
+  constexpr int E = DecElem<T>::E;
+  extern __shared__ __align__(16) uint8_t dec_smem[];
+  const int d = a.d, blk = a.blk;
+  const int row_bytes = d * (int)sizeof(T) + 16;
+  uint8_t* sK = dec_smem;
+  uint8_t* sV = sK + (size_t)blk * row_bytes;
+  float* sQ = reinterpret_cast<float*>(sV + (size_t)blk * row_bytes);  // [16][d]
+  float* sS = sQ + kDecRows * d;                                        // [16][blk]
+  float* sM = sS + kDecRows * blk;
+  float* sL = sM + kDecRows;
+
+  const int c = blockIdx.x, rg = blockIdx.y;
+  const int b = blockIdx.z / a.Hkv, h = blockIdx.z % a.Hkv;
+  const int tid = threadIdx.x;
+  const int r0 = rg * kDecRows;
+  const int nr = min(kDecRows, a.R - r0);
+
+  // The chunk: a selected history block, or a stretch of the segment prefix.
+  const bool hist = c < a.topk;
+  const T* kb;
+  const T* vb;
+  int nk, pos0 = 0;
+  if (hist) {
+    int n = __ldg(a.idx + ((size_t)b * a.Hkv + h) * a.topk + c);
+    if (n < -1 || n >= a.nkv) {
+      if (tid == 0) flag_error(a.err, kDevErrIndex);
+      n = -1;
+    }
+    nk = n >= 0 ? blk : 0;
+    const size_t off = (((size_t)b * a.nkv * blk + (size_t)(n >= 0 ? n : 0) * blk) * a.Hkv + h) * d;
+    kb = k_hist + off;
+    vb = v_hist + off;
+  } else {
+    pos0 = (c - a.topk) * blk;
+    nk = min(blk, a.t0 + a.nq - pos0);
+    const size_t off = (((size_t)b * a.S + pos0) * a.Hkv + h) * d;
+    kb = k_seg + off;
+    vb = v_seg + off;
+  }
+  const size_t key_stride = (size_t)a.Hkv * d;  // elements between consecutive tokens
+
+  // 1. stage K and V (16-byte vectors) and this CTA's query rows
+  const int vpr = d / E;  // vectors per row
+  for (int x = tid; x < nk * vpr; x += kDecThreads) {
+    const int j = x / vpr, v = x % vpr;
+    cp_async16(sK + (size_t)j * row_bytes + v * 16, kb + j * key_stride + v * E);
+    cp_async16(sV + (size_t)j * row_bytes + v * 16, vb + j * key_stride + v * E);
+  }
+  for (int x = tid; x < nr * d; x += kDecThreads) {
+    const int r = x / d, k = x % d;
+    const int rr = r0 + r, g = rr / a.nq, u = rr % a.nq;
+    const T* src = q_new + (((size_t)b * a.nq + u) * a.Hq + h * a.G + g) * d + k;
+    sQ[r * d + k] = DecElem<T>::at(src) * a.sl2;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // 2. scores (log2 units), one key per thread, all rows of the CTA
+  for (int j = tid; j < blk; j += kDecThreads) {
+    float acc[kDecRows];
+#pragma unroll
+    for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
+    if (j < nk) {
+      const uint8_t* krow = sK + (size_t)j * row_bytes;
+      for (int v = 0; v < vpr; ++v) {
+        float kv[E];
+        DecElem<T>::unpack(*reinterpret_cast<const uint4*>(krow + v * 16), kv);
+#pragma unroll
+        for (int r = 0; r < kDecRows; ++r) {
+          if (r < nr) {
+            const float* qr = sQ + r * d + v * E;
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[r] = fmaf(qr[e], kv[e], acc[r]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kDecRows; ++r) {
+      if (r < nr) {
+        const int u = (r0 + r) % a.nq;
+        const bool visible = j < nk && (hist || pos0 + j <= a.t0 + u);
+        sS[r * blk + j] = visible ? acc[r] : -INFINITY;
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. per row: max, probabilities 2^(s - m), sum (one warp per row)
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < nr; r += kDecThreads / 32) {
+    float m = -INFINITY;
+    for (int j = lane; j < blk; j += 32) m = fmaxf(m, sS[r * blk + j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int j = lane; j < blk; j += 32) {
+      const float p = (m == -INFINITY) ? 0.f : ex2_approx(sS[r * blk + j] - m);
+      sS[r * blk + j] = p;
+      l += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      sM[r] = m;
+      sL[r] = l;
+    }
+  }
+  __syncthreads();
+
+  // 4. unnormalised O of the chunk: thread = (column, row phase)
+  const int phases = kDecThreads / d;  // 1 (d = 128) or 2 (d = 64)
+  const int col = tid % d, ph = tid / d;
+  float acc[kDecRows];
+#pragma unroll
+  for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
+  for (int j = 0; j < nk; ++j) {
+    const float vj = DecElem<T>::at(reinterpret_cast<const T*>(sV + (size_t)j * row_bytes) + col);
+#pragma unroll
+    for (int r = 0; r < kDecRows; ++r)
+      if (r % phases == ph && r < nr) acc[r] = fmaf(sS[r * blk + j], vj, acc[r]);
+  }
+  const size_t base = (((size_t)b * a.Hkv + h) * a.n_chunks + c) * a.R + r0;
+#pragma unroll
+  for (int r = 0; r < kDecRows; ++r)
+    if (r % phases == ph && r < nr) a.part_o[(base + r) * d + col] = acc[r];
+  if (tid < nr) {
+    a.part_ml[(base + tid) * 2] = sM[tid];
+    a.part_ml[(base + tid) * 2 + 1] = sL[tid];
+  }
+}
+
+// One CTA per (batch x KV head, row); one thread per channel.
+template <typename T>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecArgs a, T* __restrict__ o,
+                                                             float* __restrict__ lse) {
+  const int rr = blockIdx.x % a.R;
+  const int bh = blockIdx.x / a.R;
+  const int b = bh / a.Hkv, h = bh % a.Hkv;
+  const int g = rr / a.nq, u = rr % a.nq;
+  const int hq = h * a.G + g;
+  const int col = threadIdx.x;
+  const float* ml = a.part_ml + ((size_t)bh * a.n_chunks * a.R + rr) * 2;
+  float M = -INFINITY;
+  for (int c = 0; c < a.n_chunks; ++c) M = fmaxf(M, ml[(size_t)c * a.R * 2]);
+  float L = 0.f, acc = 0.f;
+  for (int c = 0; c < a.n_chunks; ++c) {
+    const float mc = ml[(size_t)c * a.R * 2];
+    if (mc == -INFINITY) continue;
+    const float w = ex2_approx(mc - M);
+    L = fmaf(ml[(size_t)c * a.R * 2 + 1], w, L);
+    if (col < a.d) acc = fmaf(a.part_o[(((size_t)bh * a.n_chunks + c) * a.R + rr) * a.d + col], w, acc);
+  }
+  if (col < a.d) o[(((size_t)b * a.nq + u) * a.Hq + hq) * a.d + col] = (T)(acc / L);
+  if (col == 0) lse[((size_t)b * a.Hq + hq) * a.nq + u] = (M + log2f(L)) * 0.6931471805599453f;
+}
+
+}  // namespace
+
+size_t decode_workspace_floats(const Shape& s, int nq) {
+  const int n_chunks = s.topk + (s.S + s.blk - 1) / s.blk;
+  const size_t rows = (size_t)s.B * s.Hkv * n_chunks * s.G() * nq;
+  return rows * (2 + s.d);
+}
+
+cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new, const void* k_seg,
+                               const void* v_seg, const void* k_hist, const void* v_hist, int nkv,
+                               const int32_t* idx, void* o, float* lse, float* ws, int* err, cudaStream_t st) {
+  DecArgs a;
+  a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.d = s.d; a.blk = s.blk; a.nq = nq; a.t0 = t0; a.topk = s.topk;
+  a.nkv = nkv; a.G = s.G(); a.R = s.G() * nq;
+  a.n_chunks = s.topk + (t0 + nq + s.blk - 1) / s.blk;
+  a.sl2 = 1.4426950408889634f / sqrtf((float)s.d);
+  a.idx = idx; a.err = err;
+  a.part_ml = ws;
+  a.part_o = ws + (size_t)s.B * s.Hkv * a.n_chunks * a.R * 2;
+  const dim3 grid(a.n_chunks, (a.R + kDecRows - 1) / kDecRows, s.B * s.Hkv);
+  cudaError_t e;
+  if (s.bf16) {
+    const size_t smem = dec_smem_bytes<__nv_bfloat16>(s.blk, s.d);
+    auto kp = decode_partial_kernel<__nv_bfloat16>;
+    if ((e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    kp<<<grid, kDecThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q_new),
+                                        static_cast<const __nv_bfloat16*>(k_seg),
+                                        static_cast<const __nv_bfloat16*>(v_seg),
+                                        static_cast<const __nv_bfloat16*>(k_hist),
+                                        static_cast<const __nv_bfloat16*>(v_hist), a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    decode_combine_kernel<__nv_bfloat16><<<s.B * s.Hkv * a.R, 128, 0, st>>>(a, static_cast<__nv_bfloat16*>(o), lse);
+  } else {
+    const size_t smem = dec_smem_bytes<float>(s.blk, s.d);
+    auto kp = decode_partial_kernel<float>;
+    if ((e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    kp<<<grid, kDecThreads, smem, st>>>(static_cast<const float*>(q_new), static_cast<const float*>(k_seg),
+                                        static_cast<const float*>(v_seg), static_cast<const float*>(k_hist),
+                                        static_cast<const float*>(v_hist), a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    decode_combine_kernel<float><<<s.B * s.Hkv * a.R, 128, 0, st>>>(a, static_cast<float*>(o), lse);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hga

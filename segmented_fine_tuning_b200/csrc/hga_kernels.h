@@ -28,12 +28,27 @@ constexpr int kMaxQueryBlocks = 128;
 // per batch) -> destination blocks dst_b0.. of summ [B, s.nblk, Hkv, d].
 cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src, int src_b0, int dst_b0, int nblocks,
                                    float* summ, cudaStream_t st);
+// A finished segment enters the history in one pass over k_seg/v_seg [B,S,Hkv,d]:
+// summaries of its S/blk blocks -> summ blocks dst_b0.. of [B, s.nblk, Hkv, d],
+// and (pool_k != nullptr) block t of K and V -> pool slot slots[t] of
+// pool_k/pool_v [B, pool_slots*blk, Hkv, d].  S/blk <= kMaxQueryBlocks.
+cudaError_t launch_append_segment(const Shape& s, const void* k_seg, const void* v_seg, int dst_b0, float* summ,
+                                  void* pool_k, void* pool_v, int pool_slots, const int32_t* slots, cudaStream_t st);
 cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
                                cudaStream_t st);
 // idx_pool = slot_of_block[idx] on the device (-1 kept; absent or out-of-range
 // blocks flag kDevErrIndex and give -1).
 cudaError_t launch_remap_idx(const Shape& s, const int32_t* idx, const int32_t* slot_of_block, int32_t* idx_pool,
                              int* err, cudaStream_t st);
+// Zero-copy gather: the distinct blocks of idx from a mapped pinned host tier
+// (device addresses host_*_dev of [B, host_cap*blk, Hkv, d]) into a compact
+// pool (slot = rank among the selected blocks), idx_pool = idx rewritten to
+// slots; blocks without a slot (rank >= pool_slots) flag kDevErrIndex and give
+// -1.  s.nblk <= gather_max_blocks().
+int gather_max_blocks();
+cudaError_t launch_gather_mapped(const Shape& s, const int32_t* idx, const void* host_k_dev, const void* host_v_dev,
+                                 int host_cap, void* pool_k, void* pool_v, int pool_slots, int32_t* idx_pool,
+                                 int* err, int n_sm, cudaStream_t st);
 // D[b,hq,p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k]  (fp32)
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st);
 
@@ -63,6 +78,16 @@ cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const i
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                                const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
                                cudaStream_t st);
+
+// Decode step: split-key attention of nq new queries (segment positions
+// t0..t0+nq-1) over the selected history blocks idx [B,Hkv,topk] and the
+// segment prefix; partial softmax states go to ws (decode_workspace_floats
+// floats), then a merge kernel writes o [B,nq,Hq,d] and lse [B,Hq,nq].
+// s.S is the segment buffer's capacity.
+size_t decode_workspace_floats(const Shape& s, int nq);
+cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new, const void* k_seg,
+                               const void* v_seg, const void* k_hist, const void* v_hist, int nkv,
+                               const int32_t* idx, void* o, float* lse, float* ws, int* err, cudaStream_t st);
 
 // Tensor-core operand-layout self test (see hga_selftest.h).
 cudaError_t launch_selftest_umma(int form, const CUtensorMap& ma, const CUtensorMap& mb, const void* a_raw,

@@ -23,12 +23,18 @@ struct Vec<float> {
     const float4 v = __ldg(reinterpret_cast<const float4*>(p));
     out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
   }
+  __device__ static void unpack(uint4 v, float* out) {
+    out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+    out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+  }
 };
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int N = 8;
   __device__ static void load(const __nv_bfloat16* p, float* out) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), out);
+  }
+  __device__ static void unpack(uint4 v, float* out) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -79,6 +85,66 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T* __restrict__ k,
     for (int w = 0; w < 8; ++w) sacc += part[w][x];
     const int c = blockIdx.y * 32 * V + x;  // = h*d + channel: contiguous in the block-major layout
     if (c < cols) summ[((size_t)b * nblk_dst + dst_b0 + n) * cols + c] = sacc * (1.0f / blk);
+  }
+}
+
+// ------------------------------------------------------------ segment append
+// A finished segment entering the history, in one pass over its K and V:
+// summaries of its blocks (as summaries_kernel) and, when a device block
+// cache is given, the block copies of K and V into their pool slots.  CTA =
+// (segment block t, column chunk of 32 vectors, batch b); each thread moves
+// its column's 16-byte vector of every 8th row of the block.  Article: Deep
+// analysis (summaries resident and growing), fr edition Analyse approfondie
+// (finished segments leave the active window right away).
+struct AppendSlots {
+  int32_t slot[kMaxQueryBlocks];  // pool slot of segment block t
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ k_seg, const T* __restrict__ v_seg, int S,
+                                                     int Hkv, int d, int blk, int dst_b0, int nblk_dst,
+                                                     float* __restrict__ summ, T* __restrict__ pool_k,
+                                                     T* __restrict__ pool_v, int pool_slots, const AppendSlots slots) {
+  constexpr int V = Vec<T>::N;
+  const int t = blockIdx.x;
+  const int b = blockIdx.z;
+  const int cols = Hkv * d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int col = (blockIdx.y * 32 + lane) * V;
+  const bool copy = pool_k != nullptr;
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  if (col < cols) {
+    const size_t src0 = ((size_t)b * S + (size_t)t * blk) * cols + col;
+    const size_t dst0 = copy ? ((size_t)b * pool_slots * blk + (size_t)slots.slot[t] * blk) * cols + col : 0;
+    // K: every row is summed and, with a cache, stored to its slot
+#pragma unroll 16
+    for (int r = warp; r < blk; r += 8) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(k_seg + src0 + (size_t)r * cols));
+      float x[V];
+      Vec<T>::unpack(raw, x);
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] += x[e];
+      if (copy) *reinterpret_cast<uint4*>(pool_k + dst0 + (size_t)r * cols) = raw;
+    }
+    if (copy) {
+#pragma unroll 16
+      for (int r = warp; r < blk; r += 8)
+        *reinterpret_cast<uint4*>(pool_v + dst0 + (size_t)r * cols) =
+            __ldg(reinterpret_cast<const uint4*>(v_seg + src0 + (size_t)r * cols));
+    }
+  }
+  __shared__ float part[8][32 * 8];
+#pragma unroll
+  for (int e = 0; e < V; ++e) part[warp][lane * V + e] = acc[e];
+  __syncthreads();
+  for (int x = threadIdx.x; x < 32 * V; x += 256) {
+    float sacc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sacc += part[w][x];
+    const int c = blockIdx.y * 32 * V + x;
+    if (c < cols) summ[((size_t)b * nblk_dst + dst_b0 + t) * cols + c] = sacc * (1.0f / blk);
   }
 }
 
@@ -344,6 +410,26 @@ cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src,
   return cudaGetLastError();
 }
 
+cudaError_t launch_append_segment(const Shape& s, const void* k_seg, const void* v_seg, int dst_b0, float* summ,
+                                  void* pool_k, void* pool_v, int pool_slots, const int32_t* slots, cudaStream_t st) {
+  const int nqb = s.nqb();
+  if (nqb <= 0) return cudaSuccess;
+  AppendSlots sl;
+  for (int t = 0; t < kMaxQueryBlocks; ++t) sl.slot[t] = (pool_k && t < nqb) ? slots[t] : 0;
+  const int V = s.bf16 ? 8 : 4;
+  const int cols = s.Hkv * s.d;
+  dim3 grid(nqb, (cols + 32 * V - 1) / (32 * V), s.B);
+  if (s.bf16)
+    append_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k_seg), static_cast<const __nv_bfloat16*>(v_seg), s.S, s.Hkv, s.d, s.blk,
+        dst_b0, s.nblk, summ, static_cast<__nv_bfloat16*>(pool_k), static_cast<__nv_bfloat16*>(pool_v), pool_slots, sl);
+  else
+    append_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(k_seg), static_cast<const float*>(v_seg), s.S,
+                                               s.Hkv, s.d, s.blk, dst_b0, s.nblk, summ, static_cast<float*>(pool_k),
+                                               static_cast<float*>(pool_v), pool_slots, sl);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
                                cudaStream_t st) {
   int npow = 1;
@@ -393,4 +479,122 @@ cudaError_t launch_remap_idx(const Shape& s, const int32_t* idx, const int32_t* 
   remap_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(idx, slot_of_block, s.nblk, n, idx_pool, err);
   return cudaGetLastError();
 }
+}  // namespace hga
+
+// ------------------------------------------------------------ zero-copy gather
+// The distinct blocks selected in idx, copied from a pinned host tier mapped
+// into the device's address space straight into a compact pool (slot k = the
+// k-th smallest selected block), with idx rewritten to slots: the whole fetch
+// runs on the device, ordered on the stream, with no host round trip.  Every
+// CTA derives the same plan from idx (a bitmap of the selected blocks in
+// shared memory and its prefix counts), then copies its share of (slot,
+// 16 KB piece) work items with 16-byte loads from host memory; CTA 0 also
+// writes idx_pool.  Blocks ranked at or beyond pool_slots get no slot: their
+// entries become -1 and the device error flag is raised.
+namespace hga {
+namespace {
+
+constexpr int kGatherThreads = 512;
+constexpr int kGatherPiece = 16384;  // bytes per work item
+
+__global__ void __launch_bounds__(kGatherThreads) gather_mapped_kernel(
+    const int32_t* __restrict__ idx, size_t n_idx, int nblk, int B, size_t blk_bytes, int host_cap,
+    const uint8_t* __restrict__ host_k, const uint8_t* __restrict__ host_v, uint8_t* __restrict__ pool_k,
+    uint8_t* __restrict__ pool_v, int pool_slots, int32_t* __restrict__ idx_pool, int* err) {
+  extern __shared__ uint32_t gbits[];  // [W] bitmap, then [W] exclusive prefix counts
+  const int W = (nblk + 31) / 32;
+  uint32_t* pre = gbits + W;
+  __shared__ int s_total;
+  const int tid = threadIdx.x;
+  for (int w = tid; w < W; w += kGatherThreads) gbits[w] = 0u;
+  __syncthreads();
+  for (size_t k = tid; k < n_idx; k += kGatherThreads) {
+    const int n = idx[k];
+    if (n >= 0 && n < nblk) atomicOr(&gbits[n >> 5], 1u << (n & 31));
+  }
+  __syncthreads();
+  if (tid == 0) {  // W <= 1024 words: a plain scan by one thread
+    uint32_t run = 0;
+    for (int w = 0; w < W; ++w) {
+      pre[w] = run;
+      run += __popc(gbits[w]);
+    }
+    s_total = (int)run;
+  }
+  __syncthreads();
+  const int n_unique = s_total;
+  if (blockIdx.x == 0) {
+    for (size_t k = tid; k < n_idx; k += kGatherThreads) {
+      const int n = idx[k];
+      int slot = -1;
+      if (n >= 0) {
+        if (n < nblk) {
+          slot = (int)(pre[n >> 5] + __popc(gbits[n >> 5] & ((1u << (n & 31)) - 1u)));
+          if (slot >= pool_slots) slot = -1;
+        }
+        if (slot < 0) flag_error(err, kDevErrIndex);
+      }
+      idx_pool[k] = slot;
+    }
+  }
+  // work items: (slot, batch, tensor, piece)
+  const int pieces = (int)((blk_bytes + kGatherPiece - 1) / kGatherPiece);
+  const int n_copy = n_unique < pool_slots ? n_unique : pool_slots;
+  const long long items = (long long)n_copy * B * 2 * pieces;
+  for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+    const int piece = (int)(it % pieces);
+    const int tensor = (int)((it / pieces) % 2);
+    const int b = (int)((it / pieces / 2) % B);
+    const int slot = (int)(it / pieces / 2 / B);
+    // block of this slot: the slot-th set bit (binary search over the prefix counts)
+    int lo = 0, hi = W - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((int)pre[mid] <= slot) lo = mid; else hi = mid - 1;
+    }
+    uint32_t word = gbits[lo];
+    for (int r = slot - (int)pre[lo]; r > 0; --r) word &= word - 1u;  // drop the lower set bits
+    const int n = lo * 32 + (__ffs(word) - 1);
+    const size_t off = (size_t)piece * kGatherPiece;
+    const size_t len = blk_bytes - off < (size_t)kGatherPiece ? blk_bytes - off : (size_t)kGatherPiece;
+    const uint4* src = reinterpret_cast<const uint4*>((tensor ? host_v : host_k) +
+                                                      ((size_t)b * host_cap + n) * blk_bytes + off);
+    uint4* dst = reinterpret_cast<uint4*>((tensor ? pool_v : pool_k) + ((size_t)b * pool_slots + slot) * blk_bytes + off);
+    const int nv = (int)(len / 16);
+    // every load of the piece in flight before the stores
+    uint4 v[kGatherPiece / 16 / kGatherThreads];
+#pragma unroll
+    for (int x = 0; x < kGatherPiece / 16 / kGatherThreads; ++x) {
+      const int e = tid + x * kGatherThreads;
+      if (e < nv) v[x] = src[e];
+    }
+#pragma unroll
+    for (int x = 0; x < kGatherPiece / 16 / kGatherThreads; ++x) {
+      const int e = tid + x * kGatherThreads;
+      if (e < nv) dst[e] = v[x];
+    }
+  }
+}
+
+}  // namespace
+
+int gather_max_blocks() { return 1024 * 32; }
+
+cudaError_t launch_gather_mapped(const Shape& s, const int32_t* idx, const void* host_k_dev, const void* host_v_dev,
+                                 int host_cap, void* pool_k, void* pool_v, int pool_slots, int32_t* idx_pool,
+                                 int* err, int n_sm, cudaStream_t st) {
+  const size_t n_idx = (size_t)s.B * s.Hkv * s.nqb() * s.topk;
+  if (n_idx == 0) return cudaSuccess;
+  const int W = (s.nblk + 31) / 32;
+  const size_t smem = (size_t)2 * (W > 0 ? W : 1) * sizeof(uint32_t);
+  const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * (s.bf16 ? 2 : 4);
+  cudaError_t e = cudaFuncSetAttribute(gather_mapped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gather_mapped_kernel<<<2 * n_sm, kGatherThreads, smem, st>>>(
+      idx, n_idx, s.nblk, s.B, blk_bytes, host_cap, static_cast<const uint8_t*>(host_k_dev),
+      static_cast<const uint8_t*>(host_v_dev), static_cast<uint8_t*>(pool_k), static_cast<uint8_t*>(pool_v), pool_slots,
+      idx_pool, err);
+  return cudaGetLastError();
+}
+
 }  // namespace hga

@@ -16,10 +16,11 @@ Per segment s (history = segments 0..s-1, 16 blocks each at 2,048 tokens):
                             first) -> attention forward
   backward, layers L-1..0:  attention backward on the same pool (kept from the
                             forward; no second fetch)
-  segment end, every layer: summaries of the segment's blocks appended to the
-                            resident array; the segment's K/V copied to the
-                            host tier on a side stream and into the layer's
-                            device cache
+  segment end, every layer: one pass over the segment's K/V
+                            (hga_append_segment): summaries of its blocks
+                            appended to the resident array, the blocks copied
+                            into the layer's device cache, and K/V copied to
+                            the host tier on a side stream
 Every step is a libhga.so call; this module owns buffers, streams and order.
 Batch size 1 (one sequence): the resident summary array of a layer grows as a
 prefix, which is a valid summary array of the current history for B = 1.
@@ -28,20 +29,24 @@ from __future__ import annotations
 
 import torch
 
-from ._binding import (BlockCache, Dims, hga_attn_bwd, hga_attn_bwd_workspace_size, hga_attn_fwd,
-                       hga_cache_segment, hga_fetch_blocks_cached, hga_offload_segment, hga_remap_idx,
-                       hga_segment_summaries, hga_select_topk)
+from ._binding import (BlockCache, Dims, hga_append_segment, hga_attn_bwd, hga_attn_bwd_workspace_size,
+                       hga_attn_fwd, hga_fetch_blocks_cached, hga_remap_idx, hga_select_topk)
 
 
 class SegmentedPass:
     def __init__(self, seg: Dims, n_layers: int, n_segments: int, device="cuda", fetch_timeout_ms: int = 10000,
-                 pool_slots: int | None = None, keep_new_blocks: bool = True):
+                 pool_slots: int | None = None, keep_new_blocks: bool = True, prefetch: bool = True):
         """pool_slots: device pool (cache) size per layer in blocks; by default
         the largest history, so no block is fetched twice in one sequence.
         keep_new_blocks: a finished segment's blocks also enter the layer's
         device cache (a device-to-device copy) as they are offloaded, so their
-        first selection needs no host transfer."""
+        first selection needs no host transfer.
+        prefetch: the selection and fetch of layer l+1 are queued while the
+        forward of layer l runs (selection on a high-priority side stream,
+        block copies on the copy stream), so host-link transfers and the
+        host's wait for the selected indices overlap attention compute."""
         self.keep_new_blocks = keep_new_blocks
+        self.prefetch = prefetch
         if seg.B != 1:
             raise ValueError("the segmented pass drives one sequence (B = 1)")
         self.seg, self.L, self.NS = seg, n_layers, n_segments
@@ -77,7 +82,8 @@ class SegmentedPass:
         self.dv = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
         self.ws = torch.empty((max(256, hga_attn_bwd_workspace_size(seg)),), dtype=torch.uint8, device=self.device)
         self.copy_stream = torch.cuda.Stream(self.device)
-        self.offloaded = torch.cuda.Event()
+        self.sel_stream = torch.cuda.Stream(self.device, priority=-1)
+        self.ready = [torch.cuda.Event() for _ in range(n_layers)]
         for ev in self.done:
             ev.record(self.copy_stream)  # materialise the handles
         self.fetched_blocks = []   # blocks copied over the host link per (layer, segment) step
@@ -98,24 +104,38 @@ class SegmentedPass:
         return self.pool_slots if s > 0 else 0
 
     # ------------------------------------------------------------ steps
-    def forward(self, s: int, l: int, q, k_seg, v_seg):
+    def stage(self, s: int, l: int, q, stream) -> torch.cuda.Event:
+        """Selection of (segment s, layer l) and the history it needs in the
+        layer's pool: queued on `stream` (the block copies on the copy
+        stream).  Returns the event the forward must wait for."""
         D = self.dims(s)
-        st = torch.cuda.current_stream(self.device)
-        hga_select_topk(D, q, self.summ[l], self.idx[l], None, st)
+        hga_select_topk(D, q, self.summ[l], self.idx[l], None, stream)
         if s > 0:
             if (self.cache[l].slot_of_block[: s * self.nqb] >= 0).all():
                 # every selectable block is resident: slots on the device, no host round trip
-                hga_remap_idx(D, self.idx[l], self.slot_dev[l], self.idx_pool[l], st)
+                hga_remap_idx(D, self.idx[l], self.slot_dev[l], self.idx_pool[l], stream)
                 self.fetched_blocks.append(0)
                 self.device_remaps += 1
             else:
                 nu, nf = hga_fetch_blocks_cached(D, self.tier_k[l], self.tier_v[l], self.idx[l], self.scratch[l],
                                                  self.pool_k[l], self.pool_v[l], self.cache[l], self.idx_pool[l],
-                                                 st, self.copy_stream, self.done[l], self.timeout)
+                                                 stream, self.copy_stream, self.done[l], self.timeout)
                 self.selected_blocks.append(nu)
                 self.fetched_blocks.append(nf)
-                st.wait_event(self.done[l])
-                self._sync_slots(l, st)
+                self._sync_slots(l, stream)
+                stream.wait_event(self.done[l])
+        self.ready[l].record(stream)
+        return self.ready[l]
+
+    def forward(self, s: int, l: int, q, k_seg, v_seg, ready: torch.cuda.Event | None = None):
+        """Attention forward of (segment s, layer l); stages the selection
+        and fetch first unless `ready` says they are already queued."""
+        D = self.dims(s)
+        st = torch.cuda.current_stream(self.device)
+        if ready is None:
+            ready = self.stage(s, l, q, st)
+        st.wait_event(ready)
+        if s > 0:
             hga_attn_fwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.pool_slots, self.idx_pool[l],
                          self.o[l], self.lse[l], st)
         else:
@@ -134,17 +154,17 @@ class SegmentedPass:
         return self.dq, self.dk, self.dv
 
     def end_segment(self, s: int, l: int, k_seg, v_seg):
-        """Append the segment's blocks: summaries on the device, K/V to the
-        host tier on the side stream (ordered after the work queued so far)."""
+        """Append the segment's blocks in one pass over its K and V: summaries
+        on the device, the blocks into the layer's device cache (unless
+        keep_new_blocks is off), and K/V to the host tier on the side stream
+        (ordered after the work queued so far)."""
         st = torch.cuda.current_stream(self.device)
-        hga_segment_summaries(self.seg.with_history(self.cap), k_seg, s * self.nqb, self.summ[l], st)
-        if self.keep_new_blocks and s + 1 < self.NS:
-            hga_cache_segment(self.seg, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.cache[l], s * self.nqb, st)
+        cache = self.cache[l] if (self.keep_new_blocks and s + 1 < self.NS) else None
+        hga_append_segment(self.seg.with_history(self.cap), k_seg, v_seg, s * self.nqb, self.summ[l],
+                           self.pool_k[l], self.pool_v[l], cache, self.tier_k[l], self.tier_v[l], self.cap, st,
+                           self.copy_stream)
+        if cache is not None:
             self._sync_slots(l, st)
-        self.offloaded.record(st)
-        self.copy_stream.wait_event(self.offloaded)
-        hga_offload_segment(self.seg, k_seg, v_seg, self.tier_k[l], self.tier_v[l], self.cap, s * self.nqb,
-                            self.copy_stream)
         # the caller may release k_seg/v_seg once the copy stream has passed here
         k_seg.record_stream(self.copy_stream)
         v_seg.record_stream(self.copy_stream)
@@ -160,8 +180,17 @@ class SegmentedPass:
         """inputs[l] = (q, k_seg, v_seg, d_o) device tensors of layer l for
         segment s.  on_step(s, l, phase) is called after each layer's forward
         ("fwd") and backward ("bwd") calls are queued."""
+        st = torch.cuda.current_stream(self.device)
+        ahead = self.prefetch and s > 0
+        if ahead:
+            # the side stream starts after everything queued so far (earlier
+            # readers of the pools), then runs one layer ahead of the forward
+            self.sel_stream.wait_stream(st)
+            ready = self.stage(s, 0, inputs[0][0], self.sel_stream)
         for l in range(self.L):
-            self.forward(s, l, *inputs[l][:3])
+            self.forward(s, l, *inputs[l][:3], ready=ready if ahead else None)
+            if ahead and l + 1 < self.L:
+                ready = self.stage(s, l + 1, inputs[l + 1][0], self.sel_stream)
             if on_step:
                 on_step(s, l, "fwd")
         for l in reversed(range(self.L)):

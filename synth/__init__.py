@@ -164,6 +164,22 @@ def draw(w: Workload, seed: int | None = None, nblk: int | None = None) -> Input
                   _store(k[:, H:], w.dtype), _store(v[:, H:], w.dtype), _store(d_o, w.dtype))
 
 
+# Decode step at 131K context: the prefill's history (992 blocks) and a full
+# 4,096-token segment buffer, one new token at the last position.
+DECODE_131K = Workload("decode-131k: B1 Hq32/Hkv8 d128, hist 992x128, segment buffer 4096, K32, 1 new token", 1, 32,
+                       8, 128, 128, 4096, 992, 32, "bf16", 8, structured_keys=True, dominant_frac=0.01,
+                       fwd_only=True)
+
+
+def draw_decode(w: Workload, nq: int, t0: int, seed: int | None = None) -> Inputs:
+    """Inputs of a decode step: the workload's draw, whose segment tensors
+    serve as the segment KV buffer (capacity w.S); the new queries are the
+    segment's query rows t0 .. t0+nq-1 (in ``extra["q_new"]``)."""
+    x = draw(w, seed=seed)
+    x.extra["q_new"] = Tensor(np.ascontiguousarray(x.q.store[:, t0:t0 + nq]), x.q.dtype)
+    return x
+
+
 def draw_segment(w: Workload, layer: int, segment: int) -> Inputs:
     """Active-segment tensors of (layer, segment) for the segmented pass.  The
     history of that step is the concatenation of the earlier segments' K/V of

@@ -248,3 +248,124 @@ def test_remap_idx_on_device():
         hga_device_status()
     assert e.value.status == 4
     assert ip[0, 0, 1, 1].item() == -1
+
+
+@pytest.mark.parametrize("with_cache,with_tier", [(True, True), (False, True), (True, False), (False, False)])
+def test_append_segment_one_pass(with_cache, with_tier):
+    """hga_append_segment: the summaries of a finished segment's blocks (against
+    the oracle), its K/V in the device cache slots that the cache plan gives
+    them (byte-equal), and its K/V in the host tier (byte-equal), from one
+    pass over the segment; the rest of every buffer untouched."""
+    from segmented_fine_tuning_b200 import hga_append_segment
+    w = synth.Workload("append: B2 Hq4/Hkv2 S512", 2, 4, 2, 128, 128, 512, 0, 2, "bf16", 47)
+    x = synth.draw(w)
+    ks, vs = to_dev(x.k_seg), to_dev(x.v_seg)
+    cap, at = 10, 5
+    D = dims_of(w, nblk=cap)
+    summ = torch.full((2, cap, 2, 128), 7.0, device="cuda")
+    cache = BlockCache(cap, 6) if with_cache else None
+    if with_cache:
+        cache.plan(np.array([0, 1, 2], dtype=np.int32))  # slots 0..2 in use: the new blocks take 3..5
+    pool_k = torch.zeros((2, 6 * 128, 2, 128), dtype=torch.bfloat16, device="cuda")
+    pool_v = torch.zeros_like(pool_k)
+    tk = torch.zeros((2, cap * 128, 2, 128), dtype=torch.bfloat16).pin_memory() if with_tier else None
+    tv = torch.zeros_like(tk).pin_memory() if with_tier else None
+    cs = torch.cuda.Stream()
+    hga_append_segment(D, ks, vs, at, summ, pool_k, pool_v, cache, tk, tv, cap if with_tier else 0, None, cs)
+    torch.cuda.synchronize()
+    hga_device_status()
+    ref = oracle.block_summaries(oracle.Dims(2, 4, 2, 128, 128, 512, 4, 2), x.k_seg.f64)  # [B, Hkv, 4, d]
+    got = summ.cpu().numpy().transpose(0, 2, 1, 3)
+    assert np.abs(got[:, :, at:at + 4] - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+    assert np.all(got[:, :, :at] == 7.0) and np.all(got[:, :, at + 4:] == 7.0)
+    if with_cache:
+        slots = cache.slot_of_block[at:at + 4].tolist()
+        # empty slots 3, 4, 5 first, then the least recently used one (slot 0, block 0 evicted)
+        assert slots == [3, 4, 5, 0] and cache.slot_of_block[0] == -1
+        for t, sl in enumerate(slots):
+            assert torch.equal(pool_k[:, sl * 128:(sl + 1) * 128], ks[:, t * 128:(t + 1) * 128])
+            assert torch.equal(pool_v[:, sl * 128:(sl + 1) * 128], vs[:, t * 128:(t + 1) * 128])
+        assert cache.block_of_slot[slots].tolist() == list(range(at, at + 4))
+    else:
+        assert torch.count_nonzero(pool_k) == 0 and torch.count_nonzero(pool_v) == 0
+    if with_tier:
+        assert torch.equal(tk[:, at * 128:(at + 4) * 128], ks.cpu()) and torch.equal(tv[:, at * 128:(at + 4) * 128],
+                                                                                   vs.cpu())
+        assert torch.count_nonzero(tk[:, :at * 128]) == 0 and torch.count_nonzero(tk[:, (at + 4) * 128:]) == 0
+
+
+def test_gather_mapped_matches_fetch_and_oracle():
+    """hga_gather_blocks_mapped: the GPU reads the selected blocks from the
+    mapped pinned tier itself (no host wait).  Same pool and slot map as
+    hga_fetch_blocks, byte for byte; attention over the pool matches the
+    oracle; a pool too small for the selection is flagged, its unplaced
+    entries are -1; a tier that is not pinned is rejected before launch."""
+    from segmented_fine_tuning_b200 import hga_gather_blocks_mapped
+    w = synth.Workload("gather: B2 Hq8/Hkv2 S512 hist20 K3", 2, 8, 2, 128, 128, 512, 20, 3, "bf16", 48,
+                       structured_keys=True)
+    x = synth.draw(w)
+    D = dims_of(w)
+    dev = {n: to_dev(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
+    st = AttentionStep(D)
+    st.select(dev["q"], dev["k_hist"])
+    cap = w.nblk + 2
+    tier_k = torch.zeros((2, cap * 128, 2, 128), dtype=torch.bfloat16).pin_memory()
+    tier_v = torch.zeros_like(tier_k).pin_memory()
+    tier_k[:, : w.nblk * 128] = _pinned(x.k_hist)
+    tier_v[:, : w.nblk * 128] = _pinned(x.v_hist)
+    n_sel = len(set(st.idx.cpu().numpy().ravel().tolist()) - {-1})
+    slots = n_sel + 1
+    pools = {}
+    for how in ("fetch", "mapped"):
+        pk = torch.full((2, slots * 128, 2, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        pv = torch.full_like(pk, float("nan"))
+        ip = torch.full_like(st.idx, -7)
+        if how == "fetch":
+            cs = torch.cuda.Stream()
+            done = torch.cuda.Event()
+            done.record(cs)
+            scratch = torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory()
+            hga_fetch_blocks(D, tier_k, tier_v, cap, st.idx, scratch, pk, pv, slots, ip,
+                             torch.cuda.current_stream(), cs, done)
+            torch.cuda.current_stream().wait_event(done)
+        else:
+            hga_gather_blocks_mapped(D, tier_k, tier_v, cap, st.idx, pk, pv, slots, ip)
+        torch.cuda.synchronize()
+        hga_device_status()
+        pools[how] = (pk, pv, ip)
+    fk, fv, fi = pools["fetch"]
+    mk, mv, mi = pools["mapped"]
+    assert torch.equal(fi, mi)
+    # slots 0..n_sel-1 hold the same blocks; the spare slot stays untouched
+    assert torch.equal(fk[:, : n_sel * 128].cpu(), mk[:, : n_sel * 128].cpu())
+    assert torch.equal(fv[:, : n_sel * 128].cpu(), mv[:, : n_sel * 128].cpu())
+    assert torch.isnan(mk[:, n_sel * 128:].float()).all()
+    o, lse = torch.empty_like(st.o), torch.empty_like(st.lse)
+    hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], mk, mv, slots, mi, o, lse)
+    dq, dk, dv = torch.empty_like(st.dq), torch.empty_like(st.dk), torch.empty_like(st.dv)
+    hga_attn_bwd(D, dev["q"], dev["k_seg"], dev["v_seg"], mk, mv, slots, mi, o, lse, dev["d_o"], dq, dk, dv, st.ws)
+    torch.cuda.synchronize()
+    hga_device_status()
+    _oracle_check("mapped gather", w, x, st.idx.cpu().numpy(), o, lse, dq, dk, dv)
+    # too few slots: the last two selected blocks get none
+    small = n_sel - 2
+    pk = torch.zeros((2, small * 128, 2, 128), dtype=torch.bfloat16, device="cuda")
+    pv = torch.zeros_like(pk)
+    ip = torch.empty_like(st.idx)
+    hga_gather_blocks_mapped(D, tier_k, tier_v, cap, st.idx, pk, pv, small, ip)
+    with pytest.raises(HgaError) as e:
+        hga_device_status()
+    assert e.value.status == 4
+    ig, ipn = st.idx.cpu().numpy(), ip.cpu().numpy()
+    sel = sorted(set(ig.ravel().tolist()) - {-1})
+    assert np.all(ipn[np.isin(ig, sel[small:])] == -1)
+    assert np.array_equal(ipn[np.isin(ig, sel[:small])], fi.cpu().numpy()[np.isin(ig, sel[:small])])
+    # pageable (not pinned) host memory is refused before any launch
+    import ctypes
+    from segmented_fine_tuning_b200 import _binding
+    pageable = np.zeros(tier_k.numel(), dtype=np.uint16)
+    lib = _binding.load_library()
+    status = lib.hga_gather_blocks_mapped(ctypes.byref(D.c()), pageable.ctypes.data, pageable.ctypes.data, cap,
+                                          st.idx.data_ptr(), pk.data_ptr(), pv.data_ptr(), small, ip.data_ptr(),
+                                          None)
+    assert status == 1, lib.hga_last_error()
