@@ -619,9 +619,23 @@ def run_cpu_baseline(w, x_inputs, budget_s=12.0):
         oracle_sample(w, x, range(done, done + 1))
         done += 1
     el = time.perf_counter() - t0
-    return {"value": round(w.S * (done / w.Hkv) / el, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"fp64 oracle: selection for all heads + fwd and bwd for {done} of {w.Hkv} KV heads "
-                      f"({done * w.G} of {w.Hq} query heads) in {el:.1f} s, scaled to the full layer"}
+    out = {"value": round(w.S * (done / w.Hkv) / el, 2), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+           "sample": f"fp64 oracle: selection for all heads + fwd and bwd for {done} of {w.Hkv} KV heads "
+                     f"({done * w.G} of {w.Hq} query heads) in {el:.1f} s, scaled to the full layer"}
+    # the same oracle on one host core: selection for all heads + fwd and bwd of one KV head
+    import oracle
+    n0 = oracle.max_threads()
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle_sample(w, x, range(0, 1))
+        el1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(n0)
+    out["one_core"] = {"value": round(w.S * (1 / w.Hkv) / el1, 2), "unit": UNIT, "cores": 1,
+                       "sample": f"fp64 oracle on 1 thread: selection for all heads + fwd and bwd for 1 of "
+                                 f"{w.Hkv} KV heads in {el1:.1f} s, scaled to the full layer"}
+    return out
 
 
 def run_reference(args, rank, world=1):
@@ -665,7 +679,7 @@ def main():
     ap.add_argument("--pool-slots", type=int, default=None,
                     help="device pool (cache) slots per layer for --workload segmented (default: the largest history)")
     ap.add_argument("--no-prefill", action="store_true",
-                    help="skip the 131K-token prefill sub-measurement of the default (layer) run")
+                    help="skip the 131K-token prefill and dense-equivalence sub-measurements of the default (layer) run")
     ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode"), default="layer",
                     help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
                          "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
@@ -713,6 +727,9 @@ def main():
             out["prefill_131k"] = {k: pf[k] for k in ("value", "unit", "ms_per_step", "steps", "config", "kernels",
                                                       "attention_fwd", "gpu_launches", "clocks")}
             out["prefill_131k"]["metric"] = "HGA attn fwd tokens/s per layer (131K-token prefill, forward only)"
+            de, _ = run_device(args, rank, world, device, w=synth.DENSE_EQUIV, steps=min(args.steps, 20))
+            out["dense_equivalence"] = {k: de[k] for k in ("value", "unit", "ms_per_step", "steps", "config",
+                                                           "kernels", "attention_fwd_bwd", "gpu_launches")}
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -67,9 +67,20 @@ def _lib():
         lib.ohga_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, I, I, P, P, P]
         lib.ohga_dense_causal_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P]
         lib.ohga_decode_select.argtypes = [D, I, P, P, P, P]
+        lib.ohga_set_threads.argtypes = [I]
+        lib.ohga_max_threads.restype = I
         lib.ohga_decode_attn.argtypes = [D, I, I, P, P, P, P, P, P, P, P]
         _LIB = lib
     return _LIB
+
+
+def set_threads(n: int) -> None:
+    """Host threads of the oracle's parallel loops (results do not depend on it)."""
+    _lib().ohga_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(_lib().ohga_max_threads())
 
 
 def _f64(a) -> np.ndarray:

@@ -49,8 +49,14 @@
 #include "hga_oracle.h"
 
 #include <math.h>
+#include <omp.h>
 #include <stdlib.h>
 #include <string.h>
+
+/* Thread count of the OpenMP regions below (for timing the oracle on a given
+ * number of host cores); the arithmetic does not depend on it. */
+void ohga_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+int ohga_max_threads(void) { return omp_get_max_threads(); }
 
 static size_t tok_off(int b, int t, int T, int h, int H, int d) {
   return (((size_t)b * T + t) * H + h) * (size_t)d;

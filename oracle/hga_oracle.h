@@ -10,6 +10,8 @@ typedef struct {
   int B, Hq, Hkv, d, blk, S, nblk, topk;
 } ohga_dims;
 
+void ohga_set_threads(int n);
+int ohga_max_threads(void);
 void ohga_block_summaries(const ohga_dims* D, const double* k_hist, double* summ);
 void ohga_query_means(const ohga_dims* D, const double* q, double* qm);
 void ohga_block_scores(const ohga_dims* D, const double* qm, const double* summ, double* score);

@@ -12,7 +12,7 @@ LIB = os.path.join(HERE, "libhga.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
-         "-Xcompiler", "-fvisibility=hidden"]
+         "-Xcompiler", "-fvisibility=hidden"] + os.environ.get("HGA_NVCC_FLAGS", "").split()
 
 
 def _sources():
