@@ -67,6 +67,7 @@ def _lib():
         lib.ohga_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, I, I, P, P, P]
         lib.ohga_dense_causal_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P]
         lib.ohga_decode_select.argtypes = [D, I, P, P, P, P]
+        lib.ohga_attn_bwd_sparse.argtypes = [D, P, P, P, P, P, P, P, P, ctypes.c_double, I, I, P, P, P]
         lib.ohga_set_threads.argtypes = [I]
         lib.ohga_max_threads.restype = I
         lib.ohga_decode_attn.argtypes = [D, I, I, P, P, P, P, P, P, P, P]
@@ -182,6 +183,24 @@ def attn_bwd(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx, d_o, kv_heads=None):
     dv = np.full(v_seg.shape, np.nan)
     _lib().ohga_attn_bwd(ctypes.byref(Dc.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist), _ptr(v_hist),
                          _ptr(idx), _ptr(d_o), h0, h1, _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
+def attn_bwd_sparse(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx, d_o, qmask, scale: float, kv_heads=None):
+    """SpaCO-style sparse backward: only query blocks with qmask[b, i] != 0
+    propagate gradient, scaled by `scale` (qmask [B, S/blk]).  Returns
+    (dQ, dK_seg, dV_seg) like attn_bwd."""
+    Dc, q, k_seg, v_seg, k_hist, v_hist, idx = _attn_inputs(D, q, k_seg, v_seg, k_hist, v_hist, idx)
+    d_o = _f64(d_o)
+    _check(d_o, q.shape, "d_o")
+    qmask = np.ascontiguousarray(qmask, dtype=np.int8)
+    _check(qmask, (D.B, D.nqb), "qmask")
+    h0, h1 = (0, D.Hkv) if kv_heads is None else (kv_heads.start, kv_heads.stop)
+    dq = np.full(q.shape, np.nan)
+    dk = np.full(k_seg.shape, np.nan)
+    dv = np.full(v_seg.shape, np.nan)
+    _lib().ohga_attn_bwd_sparse(ctypes.byref(Dc.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist), _ptr(v_hist),
+                                _ptr(idx), _ptr(d_o), _ptr(qmask), float(scale), h0, h1, _ptr(dq), _ptr(dk), _ptr(dv))
     return dq, dk, dv
 
 

@@ -421,6 +421,35 @@ void ohga_decode_attn(const ohga_dims* D, int nq, int t0, const double* q_new, c
   }
 }
 
+/* ---------------------------------------------------------------- sparse backward
+ * Sparse segment backprop in the manner of SpaCO ("Training Long-Context
+ * LLMs Efficiently via Chunk-wise Optimization", proposed method): only a
+ * chosen subset of the segment's query blocks propagates gradient, and the
+ * chosen ones are scaled by a correction factor.  With the HGA history
+ * detached, a gradient path never leaves the segment, so the estimator is
+ * the backward of L = scale * sum over the chosen blocks' rows of <O, dO>:
+ * the plain backward (ohga_attn_bwd) with dO replaced by
+ *   dO_eff[b, p] = scale * dO[b, p]  if qmask[b, p / blk] != 0,  else 0.
+ * qmask: [B, S/blk] int8. */
+void ohga_attn_bwd_sparse(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
+                          const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o,
+                          const int8_t* qmask, double scale, int h0, int h1, double* dq, double* dk, double* dv) {
+  const size_t n = (size_t)D->B * D->S * D->Hq * D->d;
+  const int nqb = D->S / D->blk;
+  double* d_eff = (double*)malloc(sizeof(double) * (n > 0 ? n : 1));
+  for (int b = 0; b < D->B; ++b)
+    for (int p = 0; p < D->S; ++p) {
+      const double f = qmask[(size_t)b * nqb + p / D->blk] ? scale : 0.0;
+      for (int hq = 0; hq < D->Hq; ++hq)
+        for (int k = 0; k < D->d; ++k) {
+          const size_t off = tok_off(b, p, D->S, hq, D->Hq, D->d) + k;
+          d_eff[off] = f * d_o[off];
+        }
+    }
+  ohga_attn_bwd(D, q, k_seg, v_seg, k_hist, v_hist, idx, d_eff, h0, h1, dq, dk, dv);
+  free(d_eff);
+}
+
 /* Textbook dense causal attention over one whole sequence [B,T,H*,d] with
  * grouped KV heads: row t attends to keys 0..t.  Used only to check the
  * identity "every history block selected == dense causal attention". */

@@ -22,6 +22,9 @@ void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, con
 void ohga_attn_bwd(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
                    const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o, int h0, int h1,
                    double* dq, double* dk, double* dv);
+void ohga_attn_bwd_sparse(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
+                          const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o,
+                          const int8_t* qmask, double scale, int h0, int h1, double* dq, double* dk, double* dv);
 void ohga_decode_select(const ohga_dims* D, int nq, const double* q_new, const double* summ, double* score,
                         int32_t* idx);
 void ohga_decode_attn(const ohga_dims* D, int nq, int t0, const double* q_new, const double* k_seg,

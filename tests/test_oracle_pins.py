@@ -444,3 +444,65 @@ def test_decode_q_zero_and_short_history():
         for hq in range(2):
             np.testing.assert_allclose(o[0, u, hq], vals.mean(axis=0), rtol=0, atol=1e-14)
             assert abs(lse[0, hq, u] - math.log(len(vals))) < 1e-14
+
+
+# ---------------------------------------------------------------- sparse backward
+
+def test_sparse_backward_all_blocks_scale_one_is_the_backward():
+    D = Dims(B=2, Hq=4, Hkv=2, d=8, blk=4, S=12, nblk=5, topk=2)
+    q, ks, vs, kh, vh, do = _rand_inputs(D, 101)
+    idx, _ = oracle.select(D, q, kh)
+    ref = oracle.attn_bwd(D, q, ks, vs, kh, vh, idx, do)
+    got = oracle.attn_bwd_sparse(D, q, ks, vs, kh, vh, idx, do, np.ones((2, 3), dtype=np.int8), 1.0)
+    for a, b in zip(got, ref):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+
+
+def test_sparse_backward_matches_autograd_of_the_masked_loss():
+    """torch float64 autograd of L = c * sum over the chosen query blocks of
+    <O, dO>, with O from a dense masked softmax over the selected history
+    blocks and the causal segment (written out in torch, not the oracle)."""
+    D = Dims(B=1, Hq=4, Hkv=2, d=8, blk=4, S=16, nblk=6, topk=2)
+    q, ks, vs, kh, vh, do = _rand_inputs(D, 102)
+    idx, _ = oracle.select(D, q, kh)
+    mask = np.array([[1, 0, 0, 1]], dtype=np.int8)
+    c = 2.0
+    got = oracle.attn_bwd_sparse(D, q, ks, vs, kh, vh, idx, do, mask, c)
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(ks, requires_grad=True)
+    tv = torch.tensor(vs, requires_grad=True)
+    G = D.Hq // D.Hkv
+    T = D.nblk * D.blk
+    keys = torch.cat([torch.tensor(kh), tk], dim=1)       # [1, T+S, Hkv, d]
+    vals = torch.cat([torch.tensor(vh), tv], dim=1)
+    loss = 0
+    for hq in range(D.Hq):
+        h = hq // G
+        for p in range(D.S):
+            i = p // D.blk
+            if not mask[0, i]:
+                continue
+            cols = [n * D.blk + t for n in idx[0, h, i] if n >= 0 for t in range(D.blk)] + list(range(T, T + p + 1))
+            s = keys[0, cols, h] @ tq[0, p, hq] / math.sqrt(D.d)
+            o = torch.softmax(s, 0) @ vals[0, cols, h]
+            loss = loss + c * (o * torch.tensor(do[0, p, hq])).sum()
+    loss.backward()
+    np.testing.assert_allclose(got[0], tq.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[1], tk.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[2], tv.grad.numpy(), rtol=0, atol=1e-12)
+    # rows of unchosen blocks get exactly zero dQ
+    assert np.all(got[0][:, 4:12] == 0.0)
+
+
+def test_sparse_backward_ignores_unchosen_rows_of_d_o():
+    D = Dims(B=1, Hq=2, Hkv=1, d=4, blk=2, S=8, nblk=3, topk=2)
+    q, ks, vs, kh, vh, do = _rand_inputs(D, 103)
+    idx, _ = oracle.select(D, q, kh)
+    mask = np.array([[0, 1, 0, 1]], dtype=np.int8)
+    a = oracle.attn_bwd_sparse(D, q, ks, vs, kh, vh, idx, do, mask, 0.5)
+    do2 = do.copy()
+    do2[:, 0:2] = 1e3
+    do2[:, 4:6] = -7.0
+    b = oracle.attn_bwd_sparse(D, q, ks, vs, kh, vh, idx, do2, mask, 0.5)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
