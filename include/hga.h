@@ -226,6 +226,28 @@ HGA_API hga_status hga_attn_bwd_noalloc(const hga_dims* dims, const void* q, con
                                         float* dq, float* dk_seg, float* dv_seg, hga_stream_t stream);
 
 /*
+ * Sparse segment backward in the manner of SpaCO ("Training Long-Context LLMs
+ * Efficiently via Chunk-wise Optimization", proposed method: only a fixed
+ * number of chunks is backpropagated per step, each scaled by a correction
+ * factor that keeps the gradient estimate unbiased, with a cap for
+ * stability).  With the HGA history detached, a gradient path never leaves
+ * the active segment, so the estimator is the backward of
+ *   L = scale * sum over the rows of the chosen query blocks of <O, dO>:
+ * the hga_attn_bwd result with d_o replaced by scale * d_o on rows of query
+ * blocks i with qblock_mask[b*Nqb + i] != 0 and by 0 elsewhere.  dq rows of
+ * unchosen blocks are exactly 0.  qblock_mask: device uint8 [B, Nqb]; scale:
+ * finite (for k of t blocks sampled uniformly, t/k makes the estimate
+ * unbiased; the caller applies any cap).  Work for unchosen blocks is skipped
+ * (dQ CTAs of unchosen blocks only write zeros; dK/dV walk chosen blocks only).
+ * Other arguments, results and errors as hga_attn_bwd.
+ */
+HGA_API hga_status hga_attn_bwd_sparse(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                                       const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx,
+                                       const void* o, const float* lse, const void* d_o, const uint8_t* qblock_mask,
+                                       float scale, float* dq, float* dk_seg, float* dv_seg, void* ws,
+                                       size_t ws_bytes, hga_stream_t stream);
+
+/*
  * The three stages of hga_attn_bwd as separate calls (same arguments, same
  * results), for callers that schedule or time them individually.  ws is the
  * same caller-owned scratch; its first B*Hq*S floats hold Dr = rowsum(dO * O)

@@ -89,6 +89,8 @@ _SIGNATURES = [
     ("hga_attn_bwd_workspace_size", ctypes.c_size_t, [_D]),
     ("hga_attn_bwd", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("hga_attn_bwd_noalloc", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    ("hga_attn_bwd_sparse", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P,
+                                 ctypes.c_size_t, _P]),
     ("hga_attn_bwd_preprocess", _I, [_D, _P, _P, _P, ctypes.c_size_t, _P]),
     ("hga_attn_bwd_dkdv", _I, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _P]),
     ("hga_attn_bwd_dq", _I, [_D, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
@@ -519,3 +521,32 @@ def hga_gather_blocks_mapped(dims: Dims, host_k, host_v, host_capacity_blocks: i
                                                    host_capacity_blocks, _ptr(idx_dev), _ptr(pool_k), _ptr(pool_v),
                                                    pool_slots, _ptr(idx_pool_dev), _stream(stream)),
            "hga_gather_blocks_mapped")
+
+
+def hga_attn_bwd_sparse(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks: int, idx, o, lse, d_o,
+                        qblock_mask, scale: float, dq, dk_seg, dv_seg, ws, stream=None) -> None:
+    """SpaCO-style sparse backward: only query blocks with qblock_mask[b, i]
+    != 0 propagate gradient, every gradient multiplied by `scale`."""
+    _attn_shapes(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx)
+    _expect(qblock_mask, (dims.B, dims.nqb), torch.uint8, "qblock_mask")
+    for t, shp, nm in ((dq, q.shape, "dq"), (dk_seg, k_seg.shape, "dk_seg"), (dv_seg, v_seg.shape, "dv_seg")):
+        _expect(t, shp, torch.float32, nm)
+    _check(load_library().hga_attn_bwd_sparse(ctypes.byref(dims.c()), _ptr(q), _ptr(k_seg), _ptr(v_seg),
+                                              _ptr(k_hist), _ptr(v_hist), n_kv_blocks, _ptr(idx), _ptr(o), _ptr(lse),
+                                              _ptr(d_o), _ptr(qblock_mask), float(scale), _ptr(dq), _ptr(dk_seg),
+                                              _ptr(dv_seg), _ptr(ws), ws.numel() * ws.element_size(),
+                                              _stream(stream)), "hga_attn_bwd_sparse")
+
+
+def spaco_sample_blocks(B: int, n_qblocks: int, k: int, generator: torch.Generator, cap: float | None = None):
+    """Host helper for a sparse backward step: k of the n_qblocks query blocks
+    of each sequence chosen uniformly without replacement (seeded generator),
+    and the correction factor t/k (capped at `cap` when given).  Returns
+    (uint8 mask [B, n_qblocks] on the CPU, scale)."""
+    if not 1 <= k <= n_qblocks:
+        raise ValueError("need 1 <= k <= n_qblocks")
+    mask = torch.zeros((B, n_qblocks), dtype=torch.uint8)
+    for b in range(B):
+        mask[b, torch.randperm(n_qblocks, generator=generator)[:k]] = 1
+    scale = n_qblocks / k
+    return mask, (min(scale, cap) if cap is not None else scale)

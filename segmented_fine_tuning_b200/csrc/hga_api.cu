@@ -3,6 +3,7 @@
 // offload).  Declarations and the method's definition: include/hga.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -294,7 +295,7 @@ namespace {
 hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg, const void* k_hist,
                    const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o, const float* lse,
                    const void* d_o, float* dq, float* dk_seg, float* dv_seg, const void* ws, size_t ws_bytes,
-                   bool pre, int parts, hga_stream_t stream) {
+                   bool pre, int parts, hga_stream_t stream, const uint8_t* qmask = nullptr, float gscale = 1.0f) {
   hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
@@ -326,10 +327,10 @@ hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const
   if (hga::tc_supported(s)) {
     hga::TcMaps m;
     if ((r = build_maps(s, n_kv_blocks, q, d_o, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
-    e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, parts, err, st);
+    e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, parts, err, st, qmask, gscale);
   } else {
     e = hga::launch_attn_bwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, lse, Dr, d_o, dq, dk_seg,
-                                  dv_seg, parts, err, st);
+                                  dv_seg, parts, err, st, qmask, gscale);
   }
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "attention backward launch");
 }
@@ -344,6 +345,18 @@ hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, 
                         size_t ws_bytes, hga_stream_t stream) {
   return run_bwd(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse, d_o, dq, dk_seg, dv_seg, ws,
                  ws_bytes, true, hga::kBwdDq | hga::kBwdDkdv, stream);
+}
+
+hga_status hga_attn_bwd_sparse(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
+                               const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx,
+                               const void* o, const float* lse, const void* d_o, const uint8_t* qblock_mask,
+                               float scale, float* dq, float* dk_seg, float* dv_seg, void* ws, size_t ws_bytes,
+                               hga_stream_t stream) {
+  if (!qblock_mask) return fail(HGA_ERR_INVALID_ARG, "qblock_mask is NULL");
+  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
+    return fail(HGA_ERR_INVALID_ARG, "scale must be finite");
+  return run_bwd(dims, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse, d_o, dq, dk_seg, dv_seg, ws,
+                 ws_bytes, true, hga::kBwdDq | hga::kBwdDkdv, stream, qblock_mask, scale);
 }
 
 hga_status hga_attn_bwd_preprocess(const hga_dims* dims, const void* o, const void* d_o, void* ws, size_t ws_bytes,

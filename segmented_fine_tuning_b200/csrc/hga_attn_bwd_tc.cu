@@ -69,6 +69,11 @@ struct BwdArgs {
   float* dk;
   float* dv;
   int* err;
+  // Sparse backward (SpaCO-style): only query blocks i with qmask[b*nqb + i]
+  // != 0 propagate gradient, and every gradient is multiplied by gscale.
+  // qmask == nullptr and gscale == 1: the plain backward.
+  const uint8_t* qmask;
+  float gscale;
 };
 
 // ============================================================== dQ kernel
@@ -116,6 +121,15 @@ __global__ void __launch_bounds__(320, 1)
   const int rem = (int)(blockIdx.x % per_i);
   const int b = rem / a.Hq, hq = rem % a.Hq;
   const int kvh = hq / a.G;
+  if (a.qmask && !a.qmask[(size_t)b * a.nqb + i]) {
+    // a query block that propagates no gradient: its dQ rows are zero
+    for (int x = threadIdx.x; x < kB * kD / 4; x += blockDim.x) {
+      const int r = x / (kD / 4), c4 = x % (kD / 4);
+      reinterpret_cast<float4*>(a.dq + (((size_t)b * a.S + (size_t)i * kB + r) * a.Hq + hq) * kD)[c4] =
+          make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
 
   if (warp == 0) {
     const int32_t* row = a.idx + (((size_t)b * a.Hkv + kvh) * a.nqb + i) * a.topk;
@@ -307,6 +321,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dq_full, 0, abort, a.err))) {
       tc_fence_after();
+      const float osc = a.scale * a.gscale;
       float* out = a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + 64 * e;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -315,8 +330,8 @@ __global__ void __launch_bounds__(320, 1)
         float4* dst = reinterpret_cast<float4*>(out + 32 * cc);
 #pragma unroll
         for (int xx = 0; xx < 8; ++xx)
-          dst[xx] = make_float4(__uint_as_float(v[4 * xx]) * a.scale, __uint_as_float(v[4 * xx + 1]) * a.scale,
-                                __uint_as_float(v[4 * xx + 2]) * a.scale, __uint_as_float(v[4 * xx + 3]) * a.scale);
+          dst[xx] = make_float4(__uint_as_float(v[4 * xx]) * osc, __uint_as_float(v[4 * xx + 1]) * osc,
+                                __uint_as_float(v[4 * xx + 2]) * osc, __uint_as_float(v[4 * xx + 3]) * osc);
       }
     }
   }
@@ -339,6 +354,7 @@ struct DkvCtl {
   uint64_t dkv_full, mma_done;
   uint32_t tmem;
   int abort;
+  int qblocks[kMaxQueryBlocks];  // query blocks i >= jb that propagate gradient, ascending
 };
 struct __align__(16) RowStats {
   float lse[kB];
@@ -370,11 +386,17 @@ __global__ void __launch_bounds__(320, 1)
   const int rem = (int)(blockIdx.x % per_jb);
   const int b = rem / a.Hq, hq = rem % a.Hq;
   const int kvh = hq / a.G;
-  const int n = a.nqb - jb;  // query blocks jb..nqb-1
+  // query blocks jb..nqb-1 that propagate gradient (all of them unless sparse)
+  int n = 0;
+  for (int i = jb; i < a.nqb; ++i) n += (!a.qmask || a.qmask[(size_t)b * a.nqb + i]) ? 1 : 0;
+  if (n == 0) return;  // no gradient reaches this key block from head hq (outputs start at zero)
   const int nsub = 2 * n;
 
   if (warp == 0) {
     if (lane == 0) {
+      int c = 0;
+      for (int i = jb; i < a.nqb; ++i)
+        if (!a.qmask || a.qmask[(size_t)b * a.nqb + i]) ctl->qblocks[c++] = i;
       ctl->abort = 0;
       mbar_init(&ctl->kv_full, 1);
       for (int s = 0; s < kQStages; ++s) { mbar_init(&ctl->qd_full[s], 1); mbar_init(&ctl->qd_empty[s], 1); }
@@ -404,7 +426,7 @@ __global__ void __launch_bounds__(320, 1)
       int issued = 0;
       for (int it = 0; it < n; ++it) {
         const int s = it % kQStages;
-        const int i = jb + it;
+        const int i = ctl->qblocks[it];
         if (!mbar_wait(&ctl->qd_empty[s], ((it / kQStages) & 1) ^ 1, abort, a.err)) break;
         mbar_expect_tx(&ctl->qd_full[s], 2 * kTileBytes + sizeof(RowStats));
         for (int hh = 0; hh < 2; ++hh) {
@@ -501,7 +523,7 @@ __global__ void __launch_bounds__(320, 1)
         break;
       }
       tc_fence_after();
-      const bool diag = (it == 0);
+      const bool diag = (ctl->qblocks[it] == jb);
       const RowStats& rs = stats[s];
       tmem_ld32x2_wait(tmem + lane_off + kKvS + h * 64 + 32 * e, tmem + lane_off + kKvP + h * 64 + 32 * e, sd);
       const int q0 = 64 * h + 32 * e;  // query column of sd[0] within block i
@@ -531,6 +553,7 @@ __global__ void __launch_bounds__(320, 1)
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err))) {
       tc_fence_after();
       const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + 64 * e;
+      const float ks = a.scale * a.gscale, vsc = a.gscale;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t gk[32], gv[32];
@@ -540,10 +563,10 @@ __global__ void __launch_bounds__(320, 1)
         float* pv4 = a.dv + off + 32 * cc;
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          red_add_v4(pk4 + 4 * x, __uint_as_float(gk[4 * x]) * a.scale, __uint_as_float(gk[4 * x + 1]) * a.scale,
-                     __uint_as_float(gk[4 * x + 2]) * a.scale, __uint_as_float(gk[4 * x + 3]) * a.scale);
-          red_add_v4(pv4 + 4 * x, __uint_as_float(gv[4 * x]), __uint_as_float(gv[4 * x + 1]),
-                     __uint_as_float(gv[4 * x + 2]), __uint_as_float(gv[4 * x + 3]));
+          red_add_v4(pk4 + 4 * x, __uint_as_float(gk[4 * x]) * ks, __uint_as_float(gk[4 * x + 1]) * ks,
+                     __uint_as_float(gk[4 * x + 2]) * ks, __uint_as_float(gk[4 * x + 3]) * ks);
+          red_add_v4(pv4 + 4 * x, __uint_as_float(gv[4 * x]) * vsc, __uint_as_float(gv[4 * x + 1]) * vsc,
+                     __uint_as_float(gv[4 * x + 2]) * vsc, __uint_as_float(gv[4 * x + 3]) * vsc);
         }
       }
     }
@@ -561,7 +584,7 @@ __global__ void __launch_bounds__(320, 1)
 
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                                const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
-                               cudaStream_t st) {
+                               cudaStream_t st, const uint8_t* qmask, float gscale) {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDqSmem)) !=
       cudaSuccess)
@@ -574,6 +597,7 @@ cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const i
   a.scale = 1.0f / sqrtf((float)kD);
   a.sl2 = kLog2e * a.scale;
   a.idx = idx; a.lse = lse; a.Dr = Dr; a.dq = dq; a.dk = dk; a.dv = dv; a.err = err;
+  a.qmask = qmask; a.gscale = gscale;
   if (parts & kBwdDkdv) {
     // Per-head partials are added into the outputs: start from zero.
     const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * kD * sizeof(float);

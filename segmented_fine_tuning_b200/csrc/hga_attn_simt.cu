@@ -53,7 +53,13 @@ struct SimtArgs {
   float scale;  // 1/sqrt(d)
   const int32_t* idx;
   int* err;
+  const uint8_t* qmask;  // sparse backward: query blocks that propagate gradient (nullptr: all)
+  float gscale;          // sparse backward: factor on every gradient (1: plain backward)
 };
+
+__device__ __forceinline__ bool block_on(const SimtArgs& a, int b, int p) {
+  return !a.qmask || a.qmask[(size_t)b * a.nqb + p / a.blk];
+}
 
 // Key j of query block i: either history token (block idx, offset) or a
 // segment token.  Enumerates history tokens of valid selected blocks first,
@@ -132,6 +138,11 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(SimtArgs a, const T* __res
   const int p = row % a.S, hq = (row / a.S) % a.Hq, b = row / (a.S * a.Hq);
   const int h = hq / a.G;
   const size_t qoff = (((size_t)b * a.S + p) * a.Hq + hq) * a.d;
+  if (!block_on(a, b, p)) {
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) dq[qoff + lane + 32 * e] = 0.f;
+    return;
+  }
   const size_t r = ((size_t)b * a.Hq + hq) * a.S + p;
   const float L = lse[r], Dv = Dr[r];
   float qv[DPL], dov[DPL], acc[DPL];
@@ -161,7 +172,7 @@ __global__ void __launch_bounds__(256) dq_simt_kernel(SimtArgs a, const T* __res
     for (int e = 0; e < DPL; ++e) acc[e] += ds * kv[e];
   });
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) dq[qoff + lane + 32 * e] = acc[e] * a.scale;
+  for (int e = 0; e < DPL; ++e) dq[qoff + lane + 32 * e] = acc[e] * (a.scale * a.gscale);
 }
 
 // dK/dV: warp = (b, h, segment key j); sums over the G heads and rows p >= j.
@@ -187,6 +198,7 @@ __global__ void __launch_bounds__(256) dkdv_simt_kernel(SimtArgs a, const T* __r
   for (int g = 0; g < a.G; ++g) {
     const int hq = h * a.G + g;
     for (int p = j; p < a.S; ++p) {
+      if (!block_on(a, b, p)) continue;
       const size_t qoff = (((size_t)b * a.S + p) * a.Hq + hq) * a.d;
       const size_t r = ((size_t)b * a.Hq + hq) * a.S + p;
       float qv[DPL], dov[DPL];
@@ -211,8 +223,8 @@ __global__ void __launch_bounds__(256) dkdv_simt_kernel(SimtArgs a, const T* __r
   }
 #pragma unroll
   for (int e = 0; e < DPL; ++e) {
-    dk[koff + lane + 32 * e] = gk[e] * a.scale;
-    dv[koff + lane + 32 * e] = gv[e];
+    dk[koff + lane + 32 * e] = gk[e] * (a.scale * a.gscale);
+    dv[koff + lane + 32 * e] = gv[e] * a.gscale;
   }
 }
 
@@ -220,6 +232,7 @@ SimtArgs make_args(const Shape& s, int nkv, const int32_t* idx, int* err) {
   SimtArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.d = s.d; a.blk = s.blk; a.S = s.S; a.nkv = nkv; a.topk = s.topk;
   a.nqb = s.nqb(); a.G = s.G(); a.scale = 1.0f / sqrtf((float)s.d); a.idx = idx; a.err = err;
+  a.qmask = nullptr; a.gscale = 1.0f;
   return a;
 }
 
@@ -266,8 +279,11 @@ cudaError_t launch_attn_fwd_simt(const Shape& s, const void* q, const void* k_se
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
                                  const void* k_hist, const void* v_hist, int nkv, const int32_t* idx,
                                  const float* lse, const float* Dr, const void* d_o, float* dq, float* dk,
-                                 float* dv, int parts, int* err, cudaStream_t st) {
-  const SimtArgs a = make_args(s, nkv, idx, err);
+                                 float* dv, int parts, int* err, cudaStream_t st, const uint8_t* qmask,
+                                 float gscale) {
+  SimtArgs a = make_args(s, nkv, idx, err);
+  a.qmask = qmask;
+  a.gscale = gscale;
   if (s.d == 64) {
     if (s.bf16) bwd_simt<2, __nv_bfloat16>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, parts, st);
     else bwd_simt<2, float>(a, q, k_seg, v_seg, k_hist, v_hist, lse, Dr, d_o, dq, dk, dv, parts, st);

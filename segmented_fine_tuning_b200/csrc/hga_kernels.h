@@ -62,7 +62,8 @@ cudaError_t launch_attn_fwd_simt(const Shape& s, const void* q, const void* k_se
 cudaError_t launch_attn_bwd_simt(const Shape& s, const void* q, const void* k_seg, const void* v_seg,
                                  const void* k_hist, const void* v_hist, int nkv, const int32_t* idx,
                                  const float* lse, const float* Dr, const void* d_o, float* dq, float* dk,
-                                 float* dv, int parts, int* err, cudaStream_t st);
+                                 float* dv, int parts, int* err, cudaStream_t st, const uint8_t* qmask = nullptr,
+                                 float gscale = 1.0f);
 
 // Tensor-core attention (bf16, d = 128, block = 128, even G).  Tensor maps:
 // q/d_o [B,S,Hq,128], k/v seg [B,S,Hkv,128], k/v hist [B,nkv*128,Hkv,128],
@@ -75,9 +76,12 @@ bool tc_supported(const Shape& s);
 // MMA warp's pipeline wait expires and the CTA takes its timeout path.
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
                                int* err, cudaStream_t st, bool withhold_kv = false);
+// qmask/gscale (sparse backward): only query blocks i with qmask[b*nqb + i] != 0
+// propagate gradient, and every gradient is multiplied by gscale; nullptr / 1
+// give the plain backward.
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                                const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
-                               cudaStream_t st);
+                               cudaStream_t st, const uint8_t* qmask = nullptr, float gscale = 1.0f);
 
 // Decode step: split-key attention of nq new queries (segment positions
 // t0..t0+nq-1) over the selected history blocks idx [B,Hkv,topk] and the
