@@ -51,7 +51,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 // (exp2_poly2) instead of the ex2 unit.  Measured on B200 with this
 // kernel's two warps per scheduler: every split tried (4, 6 or 8 of 16
 // pairs) was slower than none, so all pairs use the ex2 unit.
-constexpr uint32_t kBwdPolyPairs = 0x0u;
+#ifndef HGA_BWD_POLY
+#define HGA_BWD_POLY 0x0u
+#endif
+constexpr uint32_t kBwdPolyPairs = HGA_BWD_POLY;
 
 // A bf16 chunk of 32 elements packed as 16 columns sits at the first 16 of
 // the 32 fp32 columns it was computed from; k-step kk (16 elements) of a

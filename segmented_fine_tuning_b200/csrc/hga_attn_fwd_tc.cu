@@ -1,5 +1,5 @@
 // Tensor-core (tcgen05) forward of the HGA attention step, bf16 in, fp32
-// accumulate, for d = 128 and 128-token blocks.
+// accumulate, for d in {64, 128} and 128-token blocks.
 //
 // Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention
 // and Segmented Backpropagation in Practice", Background: each query block
@@ -37,9 +37,7 @@ namespace {
 
 constexpr int kBM = 128;                      // query rows per tile
 constexpr int kBN = 128;                      // keys per tile
-constexpr int kD = 128;                       // head dim
-constexpr int kTileBytes = kBM * kD * 2;      // 32 KB bf16 tile
-constexpr int kHalf = kTileBytes / 2;         // one 64-column TMA box
+constexpr int kHalf = kBM * 128;              // one 64-column TMA box: 128 rows x 128 bytes
 constexpr int kStages = 5;                    // K/V ring slots
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -47,7 +45,10 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units
 // (exp2_poly2) instead of the ex2 unit.  Measured on B200 with this
 // kernel's two warps per scheduler: every split tried (4, 6 or 8 of 16
 // pairs) was slower than none, so all pairs use the ex2 unit.
-constexpr uint32_t kFwdPolyPairs = 0x0u;
+#ifndef HGA_FWD_POLY
+#define HGA_FWD_POLY 0x0u
+#endif
+constexpr uint32_t kFwdPolyPairs = HGA_FWD_POLY;
 
 struct FwdCtl {
   uint64_t q_full;
@@ -63,8 +64,9 @@ struct FwdCtl {
   int tiles[kMaxTiles];  // >= 0: history block; < 0: segment block -(t+1)
 };
 
-constexpr size_t kSmemBytes = 1024 + 2 * kTileBytes + kStages * kTileBytes + sizeof(FwdCtl);
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Head dim d in {64, 128}: a Q, K or V tile is 128 rows x d bf16 (d/64 boxes).
+constexpr size_t fwd_smem_bytes(int d) { return 1024 + 2 * (kBM * d * 2) + kStages * (kBM * d * 2) + sizeof(FwdCtl); }
+static_assert(fwd_smem_bytes(128) <= 232448, "shared memory budget");
 
 struct FwdArgs {
   int B, Hq, Hkv, S, nkv, topk, nqb, G;
@@ -76,10 +78,14 @@ struct FwdArgs {
   int withhold_kv;  // self test of the timeout path: the producer issues no K/V loads
 };
 
+template <int KD>
 __global__ void __launch_bounds__(384, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                   const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kh,
                   const __grid_constant__ CUtensorMap tm_vh, const FwdArgs a) {
+  constexpr int kD = KD;                      // head dim
+  constexpr int kTileBytes = kBM * kD * 2;    // bf16 tile: 32 KB at d = 128
+  constexpr int kBoxes = kD / 64;             // 64-column TMA boxes per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sQ = sm;                                // 2 Q tiles
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(&tm_vs);
       mbar_expect_tx(&ctl->q_full, 2 * kTileBytes);
       for (int t = 0; t < 2; ++t)
-        for (int hh = 0; hh < 2; ++hh)
+        for (int hh = 0; hh < kBoxes; ++hh)
           tma_load_4d(&tm_q, &ctl->q_full, sQ + t * kTileBytes + hh * kHalf, hh * 64, hq0 + t, i * kBM, b);
       int issued = 0;
       for (int j = 0; j < (a.withhold_kv ? 0 : nt); ++j) {
@@ -163,8 +169,8 @@ __global__ void __launch_bounds__(384, 1)
           }
           const CUtensorMap* m = hist ? (w ? &tm_vh : &tm_kh) : (w ? &tm_vs : &tm_ks);
           mbar_expect_tx(&ctl->kv_full[s], kTileBytes);
-          tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes, 0, kvh, row0, b);
-          tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes + kHalf, 64, kvh, row0, b);
+          for (int hh = 0; hh < kBoxes; ++hh)
+            tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes + hh * kHalf, hh * 64, kvh, row0, b);
           issued = pos + 1;
         }
         if (!ok) break;
@@ -310,7 +316,7 @@ __global__ void __launch_bounds__(384, 1)
         // O_t holds the sum up to tile j-1 (PV_t(j-1) completed before S_t(j)
         // was announced): bring it to the new reference.
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kD / 32; ++c) {
           uint32_t ov[32];
           HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
 #pragma unroll
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(384, 1)
       const int hq = hq0 + t;
       __nv_bfloat16* orow = a.o + (((size_t)b * a.S + p) * a.Hq + hq) * kD;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kD / 32; ++c) {
         uint32_t ov[32];
         HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -358,22 +364,30 @@ __global__ void __launch_bounds__(384, 1)
 }  // namespace
 
 bool tc_supported(const Shape& s) {
-  return s.bf16 && s.d == kD && s.blk == kBM && (s.G() % 2) == 0 && s.topk <= kMaxTopk &&
+  return s.bf16 && (s.d == 128 || s.d == 64) && s.blk == kBM && (s.G() % 2) == 0 && s.topk <= kMaxTopk &&
          s.nqb() <= kMaxQueryBlocks;
+}
+
+template <int KD>
+cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse, int* err,
+                       cudaStream_t st, bool withhold_kv) {
+  constexpr size_t smem = fwd_smem_bytes(KD);
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  FwdArgs a;
+  a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
+  a.sl2 = 1.4426950408889634f / sqrtf((float)KD);
+  a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err;
+  a.withhold_kv = withhold_kv ? 1 : 0;
+  const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
+  fwd_tc_kernel<KD><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
                                int* err, cudaStream_t st, bool withhold_kv) {
-  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  FwdArgs a;
-  a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
-  a.sl2 = 1.4426950408889634f / sqrtf((float)kD);
-  a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err;
-  a.withhold_kv = withhold_kv ? 1 : 0;
-  const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
-  fwd_tc_kernel<<<grid, 384, kSmemBytes, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
-  return cudaGetLastError();
+  return s.d == 64 ? launch_fwd<64>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
+                   : launch_fwd<128>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
 }
 
 }  // namespace hga

@@ -77,8 +77,8 @@ def _check_against_oracle(w, nq, t0, x, idx, scores, o, lse):
         kth = np.sort(score_ref[b, h])[::-1][keff - 1]
         assert len(set(v.tolist())) == keff and np.all(score_ref[b, h][v] >= kth - 1e-3 * max(abs(kth), 1e-6))
     ok = idx >= 0
-    ref_sel = np.take_along_axis(score_ref, np.maximum(idx, 0), axis=-1)
     if ok.any():
+        ref_sel = np.take_along_axis(score_ref, np.maximum(idx, 0), axis=-1)
         assert np.abs(scores[ok] - ref_sel[ok]).max() <= 1e-4 * max(1.0, np.abs(score_ref).max())
     assert np.all(idx[~ok] == -1) and np.all(np.isneginf(scores[~ok]))
     o_ref, lse_ref = oracle.decode_attn(od, t0, qn, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
