@@ -320,13 +320,14 @@ HGA_API hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const 
  * of one layer's history tier [B, host_capacity_blocks*block, Hkv, d] in
  * dtype, of which the first n_hist_blocks blocks are valid.  idx_dev:
  * device idx from hga_select_topk.  The call
- *   1. copies idx to the host on copy_stream (after the work already queued on
- *      compute_stream) and waits for it, at most timeout_ms;
+ *   1. copies idx to the host on compute_stream (after the work already
+ *      queued there) and waits for it, at most timeout_ms;
  *   2. forms the sorted set of distinct selected blocks (at most pool_slots);
- *   3. on copy_stream, copies each of those blocks' K and V (all B and Hkv)
- *      from host to the device pool (pool_k/pool_v [B, pool_slots*block, Hkv,
- *      d]), and writes idx_pool_dev = idx with each block number replaced by its
- *      pool slot (-1 kept);
+ *   3. on copy_stream, ordered after that idx copy (so after every kernel
+ *      queued on compute_stream before the call), copies each of those
+ *      blocks' K and V (all B and Hkv) from host to the device pool (pool_k/
+ *      pool_v [B, pool_slots*block, Hkv, d]), and writes idx_pool_dev = idx
+ *      with each block number replaced by its pool slot (-1 kept);
  *   4. records `done` on copy_stream; compute work that reads the pool must
  *      wait on it (cudaStreamWaitEvent).
  * host_idx_scratch: pinned host buffer of B*Hkv*Nqb*topk int32 owned by the
@@ -336,8 +337,9 @@ HGA_API hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const 
  * (an idx entry out of range), HGA_ERR_INVALID_ARG (more distinct blocks than
  * pool_slots, null pointers), HGA_ERR_CUDA.
  * After HGA_ERR_TIMEOUT no pool copy has been queued, but the idx copy into
- * host_idx_scratch is still pending on copy_stream: the caller must not reuse
- * or free that buffer until copy_stream has drained (cudaStreamSynchronize).
+ * host_idx_scratch is still pending on compute_stream: the caller must not
+ * reuse or free that buffer until compute_stream has drained
+ * (cudaStreamSynchronize).
  */
 HGA_API hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,
                             const int32_t* idx_dev,
@@ -419,7 +421,7 @@ HGA_API hga_status hga_block_cache_plan(hga_block_cache* cache, const int32_t* n
  * The cache is updated only once every copy of the call has been queued: on
  * any error it is left exactly as it was, so no block is recorded as
  * resident whose bytes were never sent.  After HGA_ERR_TIMEOUT the idx copy
- * into host_idx_scratch is still pending on copy_stream, as for
+ * into host_idx_scratch is still pending on compute_stream, as for
  * hga_fetch_blocks.
  */
 HGA_API hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, const void* host_v,

@@ -455,24 +455,22 @@ hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void
   cudaStream_t cst = reinterpret_cast<cudaStream_t>(compute_stream);
   cudaStream_t xst = reinterpret_cast<cudaStream_t>(copy_stream);
   const size_t n_idx = (size_t)s.B * s.Hkv * s.nqb() * s.topk;
-  cudaEvent_t ready = nullptr, landed = nullptr;
-  cudaError_t e = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&landed, cudaEventDisableTiming);
-  if (e != cudaSuccess) {
-    if (ready) cudaEventDestroy(ready);
-    return cuda_fail(e, "event create");
-  }
+  cudaEvent_t landed = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&landed, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(e, "event create");
   struct Guard {
-    cudaEvent_t a, b;
-    ~Guard() { cudaEventDestroy(a); cudaEventDestroy(b); }
-  } guard{ready, landed};
-  // 1. idx -> host, after the selection queued on the compute stream.
-  if ((e = cudaEventRecord(ready, cst)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = cudaStreamWaitEvent(xst, ready, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
-  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, xst)) !=
+    cudaEvent_t a;
+    ~Guard() { cudaEventDestroy(a); }
+  } guard{landed};
+  // 1. idx -> host on the compute stream, after the selection queued there (so
+  //    the wait does not queue behind earlier block copies on copy_stream);
+  //    the copies below are ordered after it, hence after every kernel queued
+  //    on the compute stream so far.
+  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, cst)) !=
       cudaSuccess)
     return cuda_fail(e, "idx copy to host");
-  if ((e = cudaEventRecord(landed, xst)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaEventRecord(landed, cst)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaStreamWaitEvent(xst, landed, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
   const auto t0 = std::chrono::steady_clock::now();
   while (true) {
     e = cudaEventQuery(landed);
@@ -607,25 +605,21 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
   cudaStream_t cst = reinterpret_cast<cudaStream_t>(compute_stream);
   cudaStream_t xst = reinterpret_cast<cudaStream_t>(copy_stream);
   const size_t n_idx = (size_t)s.B * s.Hkv * s.nqb() * s.topk;
-  cudaEvent_t ready = nullptr, landed = nullptr;
-  cudaError_t e = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&landed, cudaEventDisableTiming);
-  if (e != cudaSuccess) {
-    if (ready) cudaEventDestroy(ready);
-    return cuda_fail(e, "event create");
-  }
+  cudaEvent_t landed = nullptr;
+  cudaError_t e = cudaEventCreateWithFlags(&landed, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(e, "event create");
   struct Guard {
-    cudaEvent_t a, b;
-    ~Guard() { cudaEventDestroy(a); cudaEventDestroy(b); }
-  } guard{ready, landed};
-  // 1. idx -> host, after the work queued on the compute stream (which also
-  //    orders every later pool write after the kernels that read the pool).
-  if ((e = cudaEventRecord(ready, cst)) != cudaSuccess) return cuda_fail(e, "event record");
-  if ((e = cudaStreamWaitEvent(xst, ready, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
-  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, xst)) !=
+    cudaEvent_t a;
+    ~Guard() { cudaEventDestroy(a); }
+  } guard{landed};
+  // 1. idx -> host on the compute stream, after the work queued there; the
+  //    pool copies on copy_stream are ordered after it, hence after every
+  //    kernel that may still read the pool slots they overwrite.
+  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, cst)) !=
       cudaSuccess)
     return cuda_fail(e, "idx copy to host");
-  if ((e = cudaEventRecord(landed, xst)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaEventRecord(landed, cst)) != cudaSuccess) return cuda_fail(e, "event record");
+  if ((e = cudaStreamWaitEvent(xst, landed, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
   const auto t0 = std::chrono::steady_clock::now();
   while (true) {
     e = cudaEventQuery(landed);

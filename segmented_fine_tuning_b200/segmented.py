@@ -81,9 +81,13 @@ class SegmentedPass:
         self.dk = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
         self.dv = torch.empty((1, seg.S, H, d), dtype=torch.float32, device=self.device)
         self.ws = torch.empty((max(256, hga_attn_bwd_workspace_size(seg)),), dtype=torch.uint8, device=self.device)
+        # host -> device block copies and device -> host segment offloads on
+        # separate streams, so the two directions of the host link overlap
         self.copy_stream = torch.cuda.Stream(self.device)
+        self.offload_stream = torch.cuda.Stream(self.device)
         self.sel_stream = torch.cuda.Stream(self.device, priority=-1)
         self.ready = [torch.cuda.Event() for _ in range(n_layers)]
+        self.offloaded = [torch.cuda.Event() for _ in range(n_layers)]
         for ev in self.done:
             ev.record(self.copy_stream)  # materialise the handles
         self.fetched_blocks = []   # blocks copied over the host link per (layer, segment) step
@@ -117,6 +121,8 @@ class SegmentedPass:
                 self.fetched_blocks.append(0)
                 self.device_remaps += 1
             else:
+                # the tier's newest blocks come from this layer's last offload
+                self.copy_stream.wait_event(self.offloaded[l])
                 nu, nf = hga_fetch_blocks_cached(D, self.tier_k[l], self.tier_v[l], self.idx[l], self.scratch[l],
                                                  self.pool_k[l], self.pool_v[l], self.cache[l], self.idx_pool[l],
                                                  stream, self.copy_stream, self.done[l], self.timeout)
@@ -162,12 +168,13 @@ class SegmentedPass:
         cache = self.cache[l] if (self.keep_new_blocks and s + 1 < self.NS) else None
         hga_append_segment(self.seg.with_history(self.cap), k_seg, v_seg, s * self.nqb, self.summ[l],
                            self.pool_k[l], self.pool_v[l], cache, self.tier_k[l], self.tier_v[l], self.cap, st,
-                           self.copy_stream)
+                           self.offload_stream)
+        self.offloaded[l].record(self.offload_stream)
         if cache is not None:
             self._sync_slots(l, st)
-        # the caller may release k_seg/v_seg once the copy stream has passed here
-        k_seg.record_stream(self.copy_stream)
-        v_seg.record_stream(self.copy_stream)
+        # the caller may release k_seg/v_seg once the offload stream has passed here
+        k_seg.record_stream(self.offload_stream)
+        v_seg.record_stream(self.offload_stream)
 
     def _sync_slots(self, l: int, st) -> None:
         """Device copy of layer l's slot map, queued on st (a fresh pinned
