@@ -78,13 +78,15 @@ hga_status get_encoder(EncodeTiledFn* fn) {
   return HGA_OK;
 }
 
-// bf16 tensor [B, T, H, 128] with a {64, 1, 128, 1} box, 128-byte swizzle.
-hga_status encode_tokens(CUtensorMap* m, const void* base, int B, int T, int H) {
+// bf16 tensor [B, T, H, d] (d in {64, 128}) with a {64, 1, 128, 1} box (128
+// tokens x 64 channels = 128-byte rows), 128-byte swizzle.
+hga_status encode_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
   EncodeTiledFn enc = nullptr;
   hga_status s = get_encoder(&enc);
   if (s != HGA_OK) return s;
-  const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)H * 128 * 2, (cuuint64_t)T * H * 128 * 2};
+  const cuuint64_t D = (cuuint64_t)d;
+  const cuuint64_t dims[4] = {D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -134,13 +136,13 @@ hga_status check_attn_ptrs(const hga::Shape& s, int n_kv_blocks, const void* q, 
 hga_status build_maps(const hga::Shape& s, int nkv, const void* q, const void* d_o, const void* ks, const void* vs,
                       const void* kh, const void* vh, hga::TcMaps* m) {
   hga_status r;
-  if ((r = encode_tokens(&m->q, q, s.B, s.S, s.Hq)) != HGA_OK) return r;
-  if ((r = encode_tokens(&m->d_o, d_o ? d_o : q, s.B, s.S, s.Hq)) != HGA_OK) return r;
-  if ((r = encode_tokens(&m->ks, ks, s.B, s.S, s.Hkv)) != HGA_OK) return r;
-  if ((r = encode_tokens(&m->vs, vs, s.B, s.S, s.Hkv)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->q, q, s.B, s.S, s.Hq, s.d)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->d_o, d_o ? d_o : q, s.B, s.S, s.Hq, s.d)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->ks, ks, s.B, s.S, s.Hkv, s.d)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->vs, vs, s.B, s.S, s.Hkv, s.d)) != HGA_OK) return r;
   // With no history the history maps are never read; point them at the segment.
-  if ((r = encode_tokens(&m->kh, nkv > 0 ? kh : ks, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv)) != HGA_OK) return r;
-  if ((r = encode_tokens(&m->vh, nkv > 0 ? vh : vs, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->kh, nkv > 0 ? kh : ks, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv, s.d)) != HGA_OK) return r;
+  if ((r = encode_tokens(&m->vh, nkv > 0 ? vh : vs, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv, s.d)) != HGA_OK) return r;
   return HGA_OK;
 }
 
@@ -953,8 +955,8 @@ hga_status hga_selftest_umma(int form, const void* a, const void* b, float* d, h
   if (any_null(a, b, d) || !aligned16(a) || !aligned16(b)) return fail(HGA_ERR_INVALID_ARG, "bad pointer");
   CUtensorMap ma, mb;
   hga_status r;
-  if ((r = encode_tokens(&ma, a, 1, 128, 1)) != HGA_OK) return r;
-  if ((r = encode_tokens(&mb, b, 1, 128, 1)) != HGA_OK) return r;
+  if ((r = encode_tokens(&ma, a, 1, 128, 1, 128)) != HGA_OK) return r;
+  if ((r = encode_tokens(&mb, b, 1, 128, 1, 128)) != HGA_OK) return r;
   int* err = nullptr;
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaError_t e = hga::launch_selftest_umma(form, ma, mb, a, d, err, reinterpret_cast<cudaStream_t>(stream));

@@ -1,5 +1,5 @@
 // Tensor-core (tcgen05) backward of the HGA attention step for the active
-// segment, bf16 in, fp32 accumulate, d = 128, 128-token blocks.
+// segment, bf16 in, fp32 accumulate, d in {64, 128}, 128-token blocks.
 //
 // Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention
 // and Segmented Backpropagation in Practice", Background and (fr edition)
@@ -40,9 +40,7 @@ namespace hga {
 namespace {
 
 constexpr int kB = 128;  // rows / keys per tile
-constexpr int kD = 128;
-constexpr int kTileBytes = kB * kD * 2;
-constexpr int kHalf = kTileBytes / 2;        // one 64-channel TMA box: 128 rows x 128 B
+constexpr int kHalf = kB * 128;              // one 64-channel TMA box: 128 rows x 128 B
 constexpr int kSubRows = 64;                 // rows of a sub-tile
 constexpr int kSubOff = kSubRows * 128;      // byte offset of the second 64-row half inside a box
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
@@ -94,8 +92,9 @@ struct DqCtl {
   int nt;
   int tiles[kMaxTiles];
 };
-constexpr size_t kDqSmem = 1024 + (2 + kKStages + kVStages) * kTileBytes + sizeof(DqCtl);
-static_assert(kDqSmem <= 232448, "shared memory budget");
+// Head dim d in {64, 128}: a tile is 128 rows x d bf16 (d/64 TMA boxes).
+constexpr size_t dq_smem_bytes(int d) { return 1024 + (2 + kKStages + kVStages) * (kB * d * 2) + sizeof(DqCtl); }
+static_assert(dq_smem_bytes(128) <= 232448, "shared memory budget");
 
 // Tensor-memory columns of the dQ kernel: S double buffer, dP, dQ.
 constexpr uint32_t kDqS = 0, kDqP = 256, kDqAcc = 384;
@@ -105,11 +104,15 @@ constexpr uint32_t kDqS = 0, kDqP = 256, kDqAcc = 384;
 // and runs two tiles ahead.  dP has one buffer, but the dS pass releases it as
 // soon as it has loaded its columns (dp_free), so dP(j+1) is computed while
 // dS(j) is being formed; dQ(j) follows dS(j).
+template <int KD>
 __global__ void __launch_bounds__(320, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                  const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
                  const BwdArgs a) {
+  constexpr int kD = KD;
+  constexpr int kTileBytes = kB * kD * 2;
+  constexpr int kBoxes = kD / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sQ = sm;
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_expect_tx(&ctl->qdo_full, 2 * kTileBytes);
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < kBoxes; ++hh) {
         tma_load_4d(&tm_q, &ctl->qdo_full, sQ + hh * kHalf, hh * 64, hq, i * kB, b);
         tma_load_4d(&tm_do, &ctl->qdo_full, sDO + hh * kHalf, hh * 64, hq, i * kB, b);
       }
@@ -186,13 +189,13 @@ __global__ void __launch_bounds__(320, 1)
         const int ks = j % kKStages, vs = j % kVStages;
         if (!mbar_wait(&ctl->k_empty[ks], ((j / kKStages) & 1) ^ 1, abort, a.err)) break;
         mbar_expect_tx(&ctl->k_full[ks], kTileBytes);
-        for (int hh = 0; hh < 2; ++hh)
+        for (int hh = 0; hh < kBoxes; ++hh)
           tma_load_4d(hist ? &tm_kh : &tm_ks, &ctl->k_full[ks], sK + ks * kTileBytes + hh * kHalf, hh * 64, kvh,
                       row0, b);
         k_issued = j + 1;
         if (!mbar_wait(&ctl->v_empty[vs], ((j / kVStages) & 1) ^ 1, abort, a.err)) break;
         mbar_expect_tx(&ctl->v_full[vs], kTileBytes);
-        for (int hh = 0; hh < 2; ++hh)
+        for (int hh = 0; hh < kBoxes; ++hh)
           tma_load_4d(hist ? &tm_vh : &tm_vs, &ctl->v_full[vs], sV + vs * kTileBytes + hh * kHalf, hh * 64, kvh,
                       row0, b);
         v_issued = j + 1;
@@ -325,11 +328,12 @@ __global__ void __launch_bounds__(320, 1)
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dq_full, 0, abort, a.err))) {
       tc_fence_after();
       const float osc = a.scale * a.gscale;
-      float* out = a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + 64 * e;
+      // warpgroup e writes head-dim columns [e*d/2, (e+1)*d/2) of the row
+      float* out = a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + (kD / 2) * e;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < kD / 64; ++cc) {
         uint32_t v[32];
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + kDqAcc + 64 * e + 32 * cc, v);
+        HGA_TMEM_LD32_WAIT(tmem + lane_off + kDqAcc + (kD / 2) * e + 32 * cc, v);
         float4* dst = reinterpret_cast<float4*>(out + 32 * cc);
 #pragma unroll
         for (int xx = 0; xx < 8; ++xx)
@@ -363,16 +367,22 @@ struct __align__(16) RowStats {
   float lse[kB];
   float D[kB];
 };
-constexpr size_t kDkvSmem = 1024 + (2 + 2 * kQStages) * kTileBytes + kQStages * sizeof(RowStats) + sizeof(DkvCtl);
-static_assert(kDkvSmem <= 232448, "shared memory budget");
+constexpr size_t dkdv_smem_bytes(int d) {
+  return 1024 + (2 + 2 * kQStages) * (kB * d * 2) + kQStages * sizeof(RowStats) + sizeof(DkvCtl);
+}
+static_assert(dkdv_smem_bytes(128) <= 232448, "shared memory budget");
 
 // Tensor-memory columns of the dK/dV kernel.
 constexpr uint32_t kKvS = 0, kKvP = 128, kKvDK = 256, kKvDV = 384;
 
+template <int KD>
 __global__ void __launch_bounds__(320, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                    const BwdArgs a) {
+  constexpr int kD = KD;
+  constexpr int kTileBytes = kB * kD * 2;
+  constexpr int kBoxes = kD / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sK = sm;
@@ -422,7 +432,7 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_expect_tx(&ctl->kv_full, 2 * kTileBytes);
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < kBoxes; ++hh) {
         tma_load_4d(&tm_ks, &ctl->kv_full, sK + hh * kHalf, hh * 64, kvh, jb * kB, b);
         tma_load_4d(&tm_vs, &ctl->kv_full, sV + hh * kHalf, hh * 64, kvh, jb * kB, b);
       }
@@ -432,7 +442,7 @@ __global__ void __launch_bounds__(320, 1)
         const int i = ctl->qblocks[it];
         if (!mbar_wait(&ctl->qd_empty[s], ((it / kQStages) & 1) ^ 1, abort, a.err)) break;
         mbar_expect_tx(&ctl->qd_full[s], 2 * kTileBytes + sizeof(RowStats));
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < kBoxes; ++hh) {
           tma_load_4d(&tm_q, &ctl->qd_full[s], sQ + s * kTileBytes + hh * kHalf, hh * 64, hq, i * kB, b);
           tma_load_4d(&tm_do, &ctl->qd_full[s], sDO + s * kTileBytes + hh * kHalf, hh * 64, hq, i * kB, b);
         }
@@ -555,13 +565,14 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err))) {
       tc_fence_after();
-      const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + 64 * e;
+      // warpgroup e adds head-dim columns [e*d/2, (e+1)*d/2) of the key row
+      const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + (kD / 2) * e;
       const float ks = a.scale * a.gscale, vsc = a.gscale;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < kD / 64; ++cc) {
         uint32_t gk[32], gv[32];
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDK + 64 * e + 32 * cc, gk);
-        HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDV + 64 * e + 32 * cc, gv);
+        HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDK + (kD / 2) * e + 32 * cc, gk);
+        HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDV + (kD / 2) * e + 32 * cc, gv);
         float* pk4 = a.dk + off + 32 * cc;
         float* pv4 = a.dv + off + 32 * cc;
 #pragma unroll
@@ -585,35 +596,44 @@ __global__ void __launch_bounds__(320, 1)
 
 }  // namespace
 
-cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
-                               const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
-                               cudaStream_t st, const uint8_t* qmask, float gscale) {
+template <int KD>
+cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
+                       const float* Dr, float* dq, float* dk, float* dv, int parts, int* err, cudaStream_t st,
+                       const uint8_t* qmask, float gscale) {
+  constexpr size_t dq_smem = dq_smem_bytes(KD), kv_smem = dkdv_smem_bytes(KD);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDqSmem)) !=
+  if ((e = cudaFuncSetAttribute(dq_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem)) !=
       cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDkvSmem)) !=
+  if ((e = cudaFuncSetAttribute(dkdv_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem)) !=
       cudaSuccess)
     return e;
   BwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
-  a.scale = 1.0f / sqrtf((float)kD);
+  a.scale = 1.0f / sqrtf((float)KD);
   a.sl2 = kLog2e * a.scale;
   a.idx = idx; a.lse = lse; a.Dr = Dr; a.dq = dq; a.dk = dk; a.dv = dv; a.err = err;
   a.qmask = qmask; a.gscale = gscale;
   if (parts & kBwdDkdv) {
     // Per-head partials are added into the outputs: start from zero.
-    const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * kD * sizeof(float);
+    const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * KD * sizeof(float);
     if ((e = cudaMemsetAsync(dk, 0, kv_bytes, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dv, 0, kv_bytes, st)) != cudaSuccess) return e;
-    dkdv_tc_kernel<<<s.B * s.Hq * s.nqb(), 320, kDkvSmem, st>>>(m.q, m.d_o, m.ks, m.vs, a);
+    dkdv_tc_kernel<KD><<<s.B * s.Hq * s.nqb(), 320, kv_smem, st>>>(m.q, m.d_o, m.ks, m.vs, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (parts & kBwdDq) {
-    dq_tc_kernel<<<s.B * s.Hq * s.nqb(), 320, kDqSmem, st>>>(m.q, m.d_o, m.ks, m.vs, m.kh, m.vh, a);
+    dq_tc_kernel<KD><<<s.B * s.Hq * s.nqb(), 320, dq_smem, st>>>(m.q, m.d_o, m.ks, m.vs, m.kh, m.vh, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
+                               const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
+                               cudaStream_t st, const uint8_t* qmask, float gscale) {
+  return s.d == 64 ? launch_bwd<64>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale)
+                   : launch_bwd<128>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale);
 }
 
 }  // namespace hga

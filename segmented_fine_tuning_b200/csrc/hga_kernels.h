@@ -65,8 +65,8 @@ cudaError_t launch_attn_bwd_simt(const Shape& s, const void* q, const void* k_se
                                  float* dv, int parts, int* err, cudaStream_t st, const uint8_t* qmask = nullptr,
                                  float gscale = 1.0f);
 
-// Tensor-core attention (bf16, d = 128, block = 128, even G).  Tensor maps:
-// q/d_o [B,S,Hq,128], k/v seg [B,S,Hkv,128], k/v hist [B,nkv*128,Hkv,128],
+// Tensor-core attention (bf16, d in {64, 128}, block = 128, even G).  Tensor
+// maps: q/d_o [B,S,Hq,d], k/v seg [B,S,Hkv,d], k/v hist [B,nkv*128,Hkv,d],
 // all with a 64 x 1 x 128 x 1 box and 128-byte swizzle.
 struct TcMaps {
   CUtensorMap q, d_o, ks, vs, kh, vh;

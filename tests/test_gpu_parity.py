@@ -135,6 +135,10 @@ ATTN_CASES = [
     synth.Workload("tc-K>hist: hist2 K5", 1, 8, 2, 128, 128, 256, 2, 5, "bf16", 34),
     synth.Workload("tc-K1: hist6 K1", 1, 4, 2, 128, 128, 256, 6, 1, "bf16", 35),
     synth.Workload("simt-bf16-d64-blk64-G3", 1, 6, 2, 64, 64, 192, 5, 2, "bf16", 36),
+    # head dim 64 on the tensor-core path (one 64-column TMA box per tile)
+    synth.Workload("tc-d64: Hq8/Hkv2 d64 S384 hist6 K3", 1, 8, 2, 64, 128, 384, 6, 3, "bf16", 41,
+                   structured_keys=True),
+    synth.Workload("tc-d64-B2-G2: B2 Hq4/Hkv2 d64 S256 hist3 K2", 2, 4, 2, 64, 128, 256, 3, 2, "bf16", 42),
     synth.Workload("simt-f32-d128-blk32", 1, 2, 2, 128, 32, 96, 6, 3, "f32", 37),
 ]
 
