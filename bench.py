@@ -321,66 +321,101 @@ def run_device(args, rank, world, device, w=None, steps=None):
 
 
 def run_e2e(args, ctx, device):
-    """The same step through the public API with host buffers: the segment's
-    Q, K, V, dO copied from pinned host memory, the selected history blocks
-    fetched from a pinned host tier, and every result of the step (O, LSE,
-    dQ, dK, dV) copied back to pinned host memory."""
+    """The same step through the public API with host buffers: every step
+    copies the segment's Q, K, V, dO from pinned host memory, fetches its
+    selected history blocks from a pinned host tier (hga_fetch_blocks), runs
+    selection, forward and backward, and copies every result (O, LSE, dQ,
+    dK, dV) back to pinned host memory.  Steps are pipelined two deep, as a
+    training loop with a prefetching data loader runs them: step k+1's
+    inputs travel host -> device and step k-1's results device -> host while
+    step k computes (separate copy streams, double-buffered device sets).
+    The timed region spans the first input copy to the last result copy."""
     import segmented_fine_tuning_b200 as hga
-    w, x, D, dev, st = ctx
+    w, x, D, dev, st0 = ctx
     stream = torch.cuda.current_stream(device)
-    copy_stream = torch.cuda.Stream(device)
+    h2d, d2h, fetch_stream = (torch.cuda.Stream(device) for _ in range(3))
     host = {n: to_pinned(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "d_o")}
     tier_k, tier_v = to_pinned(x.k_hist), to_pinned(x.v_hist)
-    idx_scratch = torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory()
-    results = {"o": st.o, "lse": st.lse, "dq": st.dq, "dk": st.dk, "dv": st.dv}
-    out_host = {n: torch.empty(tuple(t.shape), dtype=t.dtype).pin_memory() for n, t in results.items()}
-    pool_k = torch.empty_like(dev["k_hist"])
-    pool_v = torch.empty_like(dev["v_hist"])
-    idx_pool = torch.empty_like(st.idx)
     # the history's summaries are resident on the device (computed once, when
     # the blocks entered the history)
-    hga.hga_block_summaries(D, dev["k_hist"], 0, D.n_hist_blocks, st.summ, stream)
-    seg = {n: torch.empty_like(dev[n]) for n in host}
-    done = torch.cuda.Event()
-    done.record(copy_stream)  # materialise the event handle
+    hga.hga_block_summaries(D, dev["k_hist"], 0, D.n_hist_blocks, st0.summ, stream)
+    from segmented_fine_tuning_b200.step import AttentionStep
+    sets = []
+    for _ in range(2):
+        st = AttentionStep(D, device)
+        r = {"st": st, "seg": {n: torch.empty_like(dev[n]) for n in host},
+             "pool_k": torch.empty_like(dev["k_hist"]), "pool_v": torch.empty_like(dev["v_hist"]),
+             "idx_pool": torch.empty_like(st.idx),
+             "scratch": torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory(),
+             "results": {"o": st.o, "lse": st.lse, "dq": st.dq, "dk": st.dk, "dv": st.dv}}
+        r["out"] = {n: torch.empty(tuple(t.shape), dtype=t.dtype).pin_memory() for n, t in r["results"].items()}
+        r["ev"] = {e: torch.cuda.Event() for e in ("h2d", "comp", "d2h", "fetch")}
+        r["ev"]["fetch"].record(fetch_stream)  # materialise the handle the C call records into
+        sets.append(r)
     blk_bytes = w.blk * w.Hkv * w.d * 2 * 2  # K and V of one block
     fetched = []
 
-    def step():
-        for n in host:
-            seg[n].copy_(host[n], non_blocking=True)
-        hga.hga_select_topk(D, seg["q"], st.summ, st.idx, None, stream)
-        nu = hga.hga_fetch_blocks(D, tier_k, tier_v, D.n_hist_blocks, st.idx, idx_scratch, pool_k, pool_v,
-                                  D.n_hist_blocks, idx_pool, stream, copy_stream, done)
-        fetched.append(nu)
-        stream.wait_event(done)
-        hga.hga_attn_fwd(D, seg["q"], seg["k_seg"], seg["v_seg"], pool_k, pool_v, D.n_hist_blocks, idx_pool, st.o,
-                         st.lse, stream)
-        hga.hga_attn_bwd(D, seg["q"], seg["k_seg"], seg["v_seg"], pool_k, pool_v, D.n_hist_blocks, idx_pool, st.o,
-                         st.lse, seg["d_o"], st.dq, st.dk, st.dv, st.ws, stream)
-        for n, t in results.items():
-            out_host[n].copy_(t, non_blocking=True)
+    def inputs_in(k):
+        r = sets[k % 2]
+        h2d.wait_event(r["ev"]["comp"])  # step k-2 has consumed this set's inputs
+        with torch.cuda.stream(h2d):
+            for n in host:
+                r["seg"][n].copy_(host[n], non_blocking=True)
+        r["ev"]["h2d"].record(h2d)
 
-    for _ in range(max(1, args.warmup)):
-        step()
+    def compute_and_out(k):
+        r = sets[k % 2]
+        st, seg = r["st"], r["seg"]
+        stream.wait_event(r["ev"]["h2d"])
+        stream.wait_event(r["ev"]["d2h"])  # step k-2's results have left this set's outputs
+        hga.hga_select_topk(D, seg["q"], st0.summ, st.idx, None, stream)
+        nu = hga.hga_fetch_blocks(D, tier_k, tier_v, D.n_hist_blocks, st.idx, r["scratch"], r["pool_k"],
+                                  r["pool_v"], D.n_hist_blocks, r["idx_pool"], stream, fetch_stream,
+                                  r["ev"]["fetch"])
+        fetched.append(nu)
+        stream.wait_event(r["ev"]["fetch"])
+        hga.hga_attn_fwd(D, seg["q"], seg["k_seg"], seg["v_seg"], r["pool_k"], r["pool_v"], D.n_hist_blocks,
+                         r["idx_pool"], st.o, st.lse, stream)
+        hga.hga_attn_bwd(D, seg["q"], seg["k_seg"], seg["v_seg"], r["pool_k"], r["pool_v"], D.n_hist_blocks,
+                         r["idx_pool"], st.o, st.lse, seg["d_o"], st.dq, st.dk, st.dv, st.ws, stream)
+        r["ev"]["comp"].record(stream)
+        d2h.wait_event(r["ev"]["comp"])
+        with torch.cuda.stream(d2h):
+            for n, t in r["results"].items():
+                r["out"][n].copy_(t, non_blocking=True)
+        r["ev"]["d2h"].record(d2h)
+
+    def run(n):
+        inputs_in(0)
+        for k in range(n):
+            if k + 1 < n:
+                inputs_in(k + 1)
+            compute_and_out(k)
+        for s_ in (h2d, d2h, fetch_stream):
+            stream.wait_stream(s_)
+
+    run(max(2, args.warmup))
     torch.cuda.synchronize(device)
     fetched.clear()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n = args.steps
     e0.record(stream)
-    for _ in range(n):
-        step()
+    for s_ in (h2d, d2h, fetch_stream):
+        s_.wait_event(e0)
+    run(n)
     e1.record(stream)
     torch.cuda.synchronize(device)
     hga.hga_device_status(stream)
     ms = e0.elapsed_time(e1) / n
-    h2d = sum(t.numel() * t.element_size() for t in host.values()) + np.mean(fetched) * blk_bytes \
-        + idx_pool.numel() * 4
-    d2h = idx_scratch.numel() * 4 + sum(t.numel() * t.element_size() for t in out_host.values())
+    r0 = sets[0]
+    h2d_bytes = sum(t.numel() * t.element_size() for t in host.values()) + np.mean(fetched) * blk_bytes \
+        + r0["idx_pool"].numel() * 4
+    d2h_bytes = r0["scratch"].numel() * 4 + sum(t.numel() * t.element_size() for t in r0["out"].values())
     return {"value": round(w.S / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
             "fetched_blocks_per_step": float(np.mean(fetched)),
-            "path": "pinned host tier + hga_fetch_blocks; O, LSE, dQ, dK, dV copied back to pinned host memory"}
+            "path": "pinned host tier + hga_fetch_blocks; O, LSE, dQ, dK, dV copied back to pinned host memory; "
+                    "steps pipelined two deep (inputs of k+1 and results of k-1 in flight during k)"}
 
 
 # ---------------------------------------------------------------- segmented pass
