@@ -299,7 +299,8 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
  * A finished segment joins the history as in the prefill: hga_segment_summaries
  * appends its blocks' summaries, hga_offload_segment moves its K/V to the tier.
  * Errors: HGA_ERR_SHAPE (n_q outside [1, block], new tokens outside the
- * buffer, n_hist_blocks > 4096 for the selection), HGA_ERR_INVALID_ARG (null
+ * buffer, n_hist_blocks > 4096 for the selection, topk + S/block > 512 for the
+ * attention), HGA_ERR_INVALID_ARG (null
  * or misaligned pointers, short workspace); an idx entry outside
  * [-1, n_kv_blocks) is skipped and flags HGA_ERR_INDEX on the device.
  */

@@ -920,6 +920,8 @@ hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const void* q_
   if (n_q < 1 || n_q > s.blk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, block = %d]", n_q, s.blk);
   if (t0 < 0 || t0 + n_q > s.S)
     return fail(HGA_ERR_SHAPE, "new tokens [%d, %d) outside the segment buffer of %d", t0, t0 + n_q, s.S);
+  if (s.topk + (s.S + s.blk - 1) / s.blk > 512)
+    return fail(HGA_ERR_SHAPE, "topk + S/block = %d key chunks > 512", s.topk + (s.S + s.blk - 1) / s.blk);
   if ((r = check_attn_ptrs(s, n_kv_blocks, q_new, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
   if (any_null(o, lse, ws)) return fail(HGA_ERR_INVALID_ARG, "NULL output or workspace pointer");
   if (!aligned16(ws)) return fail(HGA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");

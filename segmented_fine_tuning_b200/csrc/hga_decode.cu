@@ -217,29 +217,61 @@ __global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __
   }
 }
 
-// One CTA per (batch x KV head, row); one thread per channel.
+// One CTA per (batch x KV head, row); one thread per channel.  The chunks
+// (m, l) pairs are staged in shared memory by all threads at once, the merge
+// weights computed once per chunk, and the unnormalised O partials summed
+// with every load of a group in flight (the loop is latency bound otherwise).
+constexpr int kMaxChunks = 512;
 template <typename T>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecArgs a, T* __restrict__ o,
                                                              float* __restrict__ lse) {
+  __shared__ float w_s[kMaxChunks];
+  __shared__ float l_s[kMaxChunks];
+  __shared__ float red[4];
   const int rr = blockIdx.x % a.R;
   const int bh = blockIdx.x / a.R;
   const int b = bh / a.Hkv, h = bh % a.Hkv;
   const int g = rr / a.nq, u = rr % a.nq;
   const int hq = h * a.G + g;
-  const int col = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* ml = a.part_ml + ((size_t)bh * a.n_chunks * a.R + rr) * 2;
-  float M = -INFINITY;
-  for (int c = 0; c < a.n_chunks; ++c) M = fmaxf(M, ml[(size_t)c * a.R * 2]);
-  float L = 0.f, acc = 0.f;
-  for (int c = 0; c < a.n_chunks; ++c) {
+  float mloc = -INFINITY;
+  for (int c = tid; c < a.n_chunks; c += 128) {
     const float mc = ml[(size_t)c * a.R * 2];
-    if (mc == -INFINITY) continue;
-    const float w = ex2_approx(mc - M);
-    L = fmaf(ml[(size_t)c * a.R * 2 + 1], w, L);
-    if (col < a.d) acc = fmaf(a.part_o[(((size_t)bh * a.n_chunks + c) * a.R + rr) * a.d + col], w, acc);
+    w_s[c] = mc;
+    l_s[c] = ml[(size_t)c * a.R * 2 + 1];
+    mloc = fmaxf(mloc, mc);
   }
-  if (col < a.d) o[(((size_t)b * a.nq + u) * a.Hq + hq) * a.d + col] = (T)(acc / L);
-  if (col == 0) lse[((size_t)b * a.Hq + hq) * a.nq + u] = (M + log2f(L)) * 0.6931471805599453f;
+#pragma unroll
+  for (int k = 16; k > 0; k >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, k));
+  if (lane == 0) red[warp] = mloc;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  for (int c = tid; c < a.n_chunks; c += 128) {
+    const float mc = w_s[c];
+    w_s[c] = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
+  }
+  __syncthreads();
+  float L = 0.f;
+  for (int c = 0; c < a.n_chunks; ++c) L = fmaf(l_s[c], w_s[c], L);
+  if (tid < a.d) {
+    const float* po = a.part_o + ((size_t)bh * a.n_chunks * a.R + rr) * a.d + tid;
+    const size_t cstride = (size_t)a.R * a.d;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    int c = 0;
+    for (; c + 8 <= a.n_chunks; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = po[(size_t)(c + k) * cstride];
+      acc0 = fmaf(v[0], w_s[c], acc0); acc1 = fmaf(v[1], w_s[c + 1], acc1);
+      acc2 = fmaf(v[2], w_s[c + 2], acc2); acc3 = fmaf(v[3], w_s[c + 3], acc3);
+      acc0 = fmaf(v[4], w_s[c + 4], acc0); acc1 = fmaf(v[5], w_s[c + 5], acc1);
+      acc2 = fmaf(v[6], w_s[c + 6], acc2); acc3 = fmaf(v[7], w_s[c + 7], acc3);
+    }
+    for (; c < a.n_chunks; ++c) acc0 = fmaf(po[(size_t)c * cstride], w_s[c], acc0);
+    o[(((size_t)b * a.nq + u) * a.Hq + hq) * a.d + tid] = (T)(((acc0 + acc1) + (acc2 + acc3)) / L);
+  }
+  if (tid == 0) lse[((size_t)b * a.Hq + hq) * a.nq + u] = (M + log2f(L)) * 0.6931471805599453f;
 }
 
 }  // namespace
@@ -257,6 +289,7 @@ cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new
   a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.d = s.d; a.blk = s.blk; a.nq = nq; a.t0 = t0; a.topk = s.topk;
   a.nkv = nkv; a.G = s.G(); a.R = s.G() * nq;
   a.n_chunks = s.topk + (t0 + nq + s.blk - 1) / s.blk;
+  if (a.n_chunks > kMaxChunks) return cudaErrorInvalidValue;
   a.sl2 = 1.4426950408889634f / sqrtf((float)s.d);
   a.idx = idx; a.err = err;
   a.part_ml = ws;

@@ -193,17 +193,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
   const int cpl = d >> 5;  // summary channels per lane (d is 64 or 128)
 
   // first scoring round's summary channels, in flight during step 1
-  float sv[kSelU][4];
-  auto load_round = [&](int n0) {
+  float sv[kSelU][4], sn[kSelU][4];
+  auto load_round = [&](float (&dst)[kSelU][4], int n0) {
 #pragma unroll
     for (int u = 0; u < kSelU; ++u) {
       const int n = n0 + u;
       const float* src = summ + (((size_t)b * nblk + (n < nblk ? n : 0)) * Hkv + h) * d + lane;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) sv[u][m] = (n < nblk && m < cpl) ? __ldg(src + 32 * m) : 0.f;
+      for (int m = 0; m < 4; ++m) dst[u][m] = (n < nblk && m < cpl) ? __ldg(src + 32 * m) : 0.f;
     }
   };
-  load_round(warp * kSelU);
+  load_round(sv, warp * kSelU);
 
   // 1. query means: thread = (row phase r0, vector vt); rows r0, r0+rpp, ...
   //    are summed per thread, the rpp partials are then combined.
@@ -237,9 +237,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
     __syncthreads();
   }
 
-  // 2. scores -> keys
+  // 2. scores -> keys; the next round's summary channels are loaded before
+  //    this round's arithmetic, so a load latency is paid once, not per round
   for (int n0 = warp * kSelU; n0 < npow; n0 += kSelWarps * kSelU) {
-    if (n0 != warp * kSelU) load_round(n0);
+    const int n1 = n0 + kSelWarps * kSelU;
+    if (n1 < npow) load_round(sn, n1);
     float best[kSelU];
 #pragma unroll
     for (int u = 0; u < kSelU; ++u) best[u] = -FLT_MAX;
@@ -264,6 +266,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
       const int n = n0 + u;
       if (lane == u && n < npow) keys[n] = n < nblk ? sel_key(best[u] * inv_sqrt_d, n) : 0ull;
     }
+#pragma unroll
+    for (int u = 0; u < kSelU; ++u)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sv[u][m] = sn[u][m];
   }
   __syncthreads();
 
