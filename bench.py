@@ -553,7 +553,7 @@ def run_decode(args, device):
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        hga.hga_decode_select(D, qn, summ, idx, None, stream)
+        hga.hga_decode_select(D, qn, summ, idx, None, ws, stream)
         if evs:
             evs[1].record(stream)
         hga.hga_decode_attn(D, t0, qn, dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk, idx, o,
@@ -584,7 +584,7 @@ def run_decode(args, device):
         side.wait_stream(stream)
         with torch.cuda.stream(side):
             with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
-                hga.hga_decode_select(D, qn, summ, idx, None, side)
+                hga.hga_decode_select(D, qn, summ, idx, None, ws, side)
                 hga.hga_decode_attn(D, t0, qn, dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk,
                                     idx, o, lse, ws, side)
         stream.wait_stream(side)

@@ -285,7 +285,10 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
  * q_new [B, n_q, Hq, d] dtype; summ as for hga_select_topk; idx [B, Hkv, topk]
  * int32; scores_or_null fp32 [B, Hkv, topk] (the selected blocks' scores,
  * -inf for padding).  With n_q = block and t0 a multiple of block this is
- * exactly hga_select_topk's result for that query block.
+ * exactly hga_select_topk's result for that query block (up to fp32 rounding
+ * of the mean near ties).  The blocks are scored in parallel into ws, then
+ * selected per (b, KV head); ws as for hga_decode_attn (the same buffer may
+ * serve both calls when they run in order on one stream).
  *
  * hga_decode_attn: new query u (position p = t0 + u) of head hq attends to the
  * tokens of blocks idx[b, hq/G, :] (entries >= 0) of k_hist/v_hist (the
@@ -305,9 +308,10 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
  * [-1, n_kv_blocks) is skipped and flags HGA_ERR_INDEX on the device.
  */
 HGA_API hga_status hga_decode_select(const hga_dims* dims, int n_q, const void* q_new, const float* summ,
-                                     int32_t* idx, float* scores_or_null, hga_stream_t stream);
-/* Bytes of device scratch hga_decode_attn needs for these dims and n_q (0 if
- * they are invalid). */
+                                     int32_t* idx, float* scores_or_null, void* ws, size_t ws_bytes,
+                                     hga_stream_t stream);
+/* Bytes of device scratch hga_decode_select and hga_decode_attn need for these
+ * dims and n_q (0 if they are invalid). */
 HGA_API size_t hga_decode_workspace_size(const hga_dims* dims, int n_q);
 HGA_API hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const void* q_new, const void* k_seg,
                                    const void* v_seg, const void* k_hist, const void* v_hist, int n_kv_blocks,

@@ -105,7 +105,7 @@ _SIGNATURES = [
     ("hga_remap_idx", _I, [_D, _P, _P, _P, _P]),
     ("hga_append_segment", _I, [_D, _P, _P, _I, _P, _P, _P, _C, _P, _P, _I, _P, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
-    ("hga_decode_select", _I, [_D, _I, _P, _P, _P, _P, _P]),
+    ("hga_decode_select", _I, [_D, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("hga_decode_workspace_size", ctypes.c_size_t, [_D, _I]),
     ("hga_decode_attn", _I, [_D, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("hga_selftest_umma", _I, [_I, _P, _P, _P, _P]),
@@ -440,8 +440,9 @@ def hga_selftest_attn_fwd_stalled(dims: Dims, q, k_seg, v_seg, k_hist, v_hist, n
            "hga_selftest_attn_fwd_stalled")
 
 
-def hga_decode_select(dims: Dims, q_new, summ, idx, scores=None, stream=None) -> None:
-    """Selection for the n_q = q_new.shape[1] new queries of a decode step."""
+def hga_decode_select(dims: Dims, q_new, summ, idx, scores, ws, stream=None) -> None:
+    """Selection for the n_q = q_new.shape[1] new queries of a decode step
+    (scores may be None; ws of hga_decode_workspace_size bytes)."""
     nq = q_new.shape[1]
     _expect(q_new, (dims.B, nq, dims.Hq, dims.d), dims.torch_dtype, "q_new")
     if dims.n_hist_blocks > 0:
@@ -451,7 +452,8 @@ def hga_decode_select(dims: Dims, q_new, summ, idx, scores=None, stream=None) ->
     if scores is not None:
         _expect(scores, idx.shape, torch.float32, "scores")
     _check(load_library().hga_decode_select(ctypes.byref(dims.c()), nq, _ptr(q_new), _ptr(summ), _ptr(idx),
-                                            _ptr(scores), _stream(stream)), "hga_decode_select")
+                                            _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)), "hga_decode_select")
 
 
 def hga_decode_workspace_size(dims: Dims, n_q: int) -> int:

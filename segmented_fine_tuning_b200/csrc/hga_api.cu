@@ -887,28 +887,28 @@ hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const vo
 }
 
 hga_status hga_decode_select(const hga_dims* dims, int n_q, const void* q_new, const float* summ, int32_t* idx,
-                             float* scores_or_null, hga_stream_t stream) {
+                             float* scores_or_null, void* ws, size_t ws_bytes, hga_stream_t stream) {
   hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (n_q < 1 || n_q > s.blk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, block = %d]", n_q, s.blk);
   if (s.nblk > hga::kMaxSelectBlocks)
     return fail(HGA_ERR_SHAPE, "n_hist_blocks %d > %d", s.nblk, hga::kMaxSelectBlocks);
-  if (any_null(q_new, idx) || (s.nblk > 0 && summ == nullptr)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
-  if (!aligned16(q_new)) return fail(HGA_ERR_INVALID_ARG, "q_new must be 16-byte aligned");
-  // The new queries are one query block of n_q rows: the prefill selection
-  // kernel with S = block = n_q computes exactly the decode definition.
-  hga::Shape sq = s;
-  sq.S = n_q;
-  sq.blk = n_q;
-  cudaError_t e = hga::launch_select_topk(sq, q_new, summ, idx, scores_or_null, reinterpret_cast<cudaStream_t>(stream));
+  if (any_null(q_new, idx, ws) || (s.nblk > 0 && summ == nullptr)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q_new) || !aligned16(ws)) return fail(HGA_ERR_INVALID_ARG, "q_new and ws must be 16-byte aligned");
+  const size_t need = hga_decode_workspace_size(dims, n_q);
+  if (ws_bytes < need) return fail(HGA_ERR_INVALID_ARG, "workspace %zu bytes < %zu", ws_bytes, need);
+  cudaError_t e = hga::launch_decode_select(s, n_q, q_new, summ, idx, scores_or_null, ws,
+                                            reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "decode select launch");
 }
 
 size_t hga_decode_workspace_size(const hga_dims* dims, int n_q) {
   hga::Shape s{};
   if (check_dims(dims, &s) != HGA_OK || n_q < 1 || n_q > s.blk) return 0;
-  return round256(hga::decode_workspace_floats(s, n_q) * sizeof(float));
+  const size_t attn = hga::decode_workspace_floats(s, n_q) * sizeof(float);
+  const size_t select = (size_t)s.B * s.Hkv * (s.nblk > 0 ? s.nblk : 1) * sizeof(unsigned long long);
+  return round256(attn > select ? attn : select);
 }
 
 hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const void* q_new, const void* k_seg,

@@ -40,6 +40,11 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
 // blocks flag kDevErrIndex and give -1).
 cudaError_t launch_remap_idx(const Shape& s, const int32_t* idx, const int32_t* slot_of_block, int32_t* idx_pool,
                              int* err, cudaStream_t st);
+// Decode selection: keys of every history block (scored in parallel over the
+// blocks) into ws (B*Hkv*nblk 64-bit keys), then top-K per (b, KV head) into
+// idx [B, Hkv, topk] (and optional scores).
+cudaError_t launch_decode_select(const Shape& s, int nq, const void* q_new, const float* summ, int32_t* idx,
+                                 float* scores, void* ws, cudaStream_t st);
 // Zero-copy gather: the distinct blocks of idx from a mapped pinned host tier
 // (device addresses host_*_dev of [B, host_cap*blk, Hkv, d]) into a compact
 // pool (slot = rank among the selected blocks), idx_pool = idx rewritten to

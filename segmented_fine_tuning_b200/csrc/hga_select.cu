@@ -156,6 +156,102 @@ __device__ __forceinline__ unsigned long long sel_key(float s, int n) {
   return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)n);
 }
 
+// The keff largest of keys[0..n) (distinct 64-bit keys, n >= keff >= 1) into
+// chosen (block index) / chosen_key, in no particular order.  The keff-th
+// largest key is found one byte at a time from the most significant end: per
+// pass, a histogram of the next byte of the keys that still match the prefix
+// found so far, and one warp walks it from the top to the byte where the count
+// reaches the number of keys still to take.  Then every key at or above that
+// threshold is taken.  Eight passes of three barriers each, for any n.
+__device__ void topk_radix(const unsigned long long* keys, int n, int keff, int* chosen,
+                           unsigned long long* chosen_key) {
+  __shared__ unsigned int hist[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_need;
+  __shared__ int s_count;
+  const int tid = threadIdx.x;
+  unsigned long long prefix = 0ull, mask = 0ull;
+  int need = keff;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int x = tid; x < 256; x += blockDim.x) hist[x] = 0u;
+    __syncthreads();
+    for (int x = tid; x < n; x += blockDim.x) {
+      const unsigned long long k = keys[x];
+      if ((k & mask) == prefix) atomicAdd(&hist[(unsigned)(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l holds the counts of bytes 255-8l down to 248-8l
+      unsigned int c[8], sum = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        c[k] = hist[255 - 8 * tid - k];
+        sum += c[k];
+      }
+      unsigned int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const unsigned int excl = incl - sum;
+      if (excl < (unsigned)need && incl >= (unsigned)need) {  // exactly one lane
+        unsigned int cum = excl;
+        int digit = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (cum + c[k] >= (unsigned)need) {
+            digit = 255 - 8 * tid - k;
+            break;
+          }
+          cum += c[k];
+        }
+        s_prefix = prefix | ((unsigned long long)digit << shift);
+        s_need = need - (int)cum;
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    mask |= 0xFFull << shift;
+  }
+  // prefix is now the keff-th largest key
+  if (tid == 0) s_count = 0;
+  __syncthreads();
+  for (int x = tid; x < n; x += blockDim.x) {
+    const unsigned long long k = keys[x];
+    if (k >= prefix) {
+      const int slot = atomicAdd(&s_count, 1);
+      chosen[slot] = x;
+      chosen_key[slot] = k;
+    }
+  }
+  __syncthreads();
+}
+
+// Writes one selection row: the chosen blocks in ascending order, then -1
+// padding; scores (optional) recovered from the keys.  Threads 0..topk-1.
+__device__ void write_selection(const int* chosen, const unsigned long long* chosen_key, int keff, int topk,
+                                int32_t* idx_row, float* scores_row) {
+  const int tid = threadIdx.x;
+  if (tid >= topk) return;
+  if (tid < keff) {
+    const int n = chosen[tid];
+    int rank = 0;
+    for (int u = 0; u < keff; ++u) rank += chosen[u] < n;
+    idx_row[rank] = n;
+    if (scores_row) {
+      // recover the score from the key (inverse of the ordering map)
+      uint32_t u = (uint32_t)(chosen_key[tid] >> 32);
+      u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+      scores_row[rank] = __uint_as_float(u);
+    }
+  } else {
+    idx_row[tid] = -1;
+    if (scores_row) scores_row[tid] = -INFINITY;
+  }
+}
+
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelU = 4;  // blocks per warp per scoring round
@@ -168,8 +264,8 @@ constexpr int kSelRankMax = 256;  // largest padded block count ranked by counti
 //     blocks per round: their summary channels are loaded before any
 //     arithmetic (the first round's before step 1), and the G * kSelU dot
 //     products are reduced across the warp together.
-//  3. top K_eff of the (score, index) keys by rank counting or a bitonic
-//     sort, then listed in ascending block order.
+//  3. top K_eff of the (score, index) keys by rank counting (up to 256
+//     blocks) or a byte-wise radix select, then listed in ascending order.
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict__ q, const float* __restrict__ summ,
                                                              int S, int Hq, int Hkv, int d, int blk, int nblk, int topk,
@@ -181,11 +277,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
   const int G = Hq / Hkv;
   const int nqb = S / blk;
   const int cols = G * d;
-  int npow = 1;
-  while (npow < nblk) npow <<= 1;
   float* qm = reinterpret_cast<float*>(sel_smem);                                        // [G*d]
   float* part = qm + cols + (cols & 1);                                                  // [kSelThreads*V]
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part + kSelThreads * V);  // [npow]
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(part + kSelThreads * V);  // [nblk]
   __shared__ int chosen[kMaxTopk];
   __shared__ unsigned long long chosen_key[kMaxTopk];
   const int tid = threadIdx.x;
@@ -239,9 +333,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
 
   // 2. scores -> keys; the next round's summary channels are loaded before
   //    this round's arithmetic, so a load latency is paid once, not per round
-  for (int n0 = warp * kSelU; n0 < npow; n0 += kSelWarps * kSelU) {
+  for (int n0 = warp * kSelU; n0 < nblk; n0 += kSelWarps * kSelU) {
     const int n1 = n0 + kSelWarps * kSelU;
-    if (n1 < npow) load_round(sn, n1);
+    if (n1 < nblk) load_round(sn, n1);
     float best[kSelU];
 #pragma unroll
     for (int u = 0; u < kSelU; ++u) best[u] = -FLT_MAX;
@@ -264,7 +358,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
 #pragma unroll
     for (int u = 0; u < kSelU; ++u) {
       const int n = n0 + u;
-      if (lane == u && n < npow) keys[n] = n < nblk ? sel_key(best[u] * inv_sqrt_d, n) : 0ull;
+      if (lane == u && n < nblk) keys[n] = sel_key(best[u] * inv_sqrt_d, n);
     }
 #pragma unroll
     for (int u = 0; u < kSelU; ++u)
@@ -274,10 +368,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
   __syncthreads();
 
   // 3. top K_eff.  Up to kSelRankMax blocks: every block counts the keys
-  //    above its own (keys are distinct), no sort needed; beyond that a
-  //    bitonic sort, descending.
+  //    above its own (keys are distinct), no sort needed; beyond that the
+  //    radix select above.
   const int keff = topk < nblk ? topk : nblk;
-  if (npow <= kSelRankMax) {
+  if (nblk <= kSelRankMax) {
     for (int n = tid; n < nblk; n += kSelThreads) {
       const unsigned long long kn = keys[n];
       int rank = 0;
@@ -287,47 +381,106 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
         chosen_key[rank] = kn;
       }
     }
-  } else {
-    for (int size = 2; size <= npow; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int x = tid; x < npow; x += kSelThreads) {
-          const int y = x ^ stride;
-          if (y > x) {
-            const bool desc = ((x & size) == 0);
-            const unsigned long long a = keys[x], c = keys[y];
-            if (desc ? (a < c) : (a > c)) {
-              keys[x] = c;
-              keys[y] = a;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-    if (tid < keff) {
-      chosen[tid] = (int)(0xFFFFFFFFu - (uint32_t)(keys[tid] & 0xFFFFFFFFull));
-      chosen_key[tid] = keys[tid];
-    }
+  } else if (keff > 0) {
+    topk_radix(keys, nblk, keff, chosen, chosen_key);
   }
   __syncthreads();
   const size_t row = (((size_t)b * Hkv + h) * nqb + i) * topk;
-  if (tid < topk) {
-    if (tid < keff) {
-      const int n = chosen[tid];
-      int rank = 0;
-      for (int u = 0; u < keff; ++u) rank += chosen[u] < n;
-      idx[row + rank] = n;
-      if (scores) {
-        // recover the score from the key (inverse of the ordering map)
-        uint32_t u = (uint32_t)(chosen_key[tid] >> 32);
-        u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
-        scores[row + rank] = __uint_as_float(u);
-      }
-    } else {
-      idx[row + tid] = -1;
-      if (scores) scores[row + tid] = -INFINITY;
-    }
+  write_selection(chosen, chosen_key, keff, topk, idx + row, scores ? scores + row : nullptr);
+}
+
+// ------------------------------------------------------------ decode selection
+// A decode step has one (partial) query block per (b, KV head), so one CTA per
+// selection would leave the GPU nearly idle while it walks a long history.
+// The scoring is therefore spread over the blocks: decode_score_kernel, CTA =
+// (64 history blocks, KV head, batch), forms the mean of the n_q new queries
+// of the G heads and writes each block's (score, index) key to the
+// workspace; decode_topk_kernel, one CTA per (b, KV head), selects from them.
+constexpr int kDecBlocksPerWarp = 8;
+constexpr int kDecScoreWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kDecScoreWarps * 32)
+    decode_score_kernel(const T* __restrict__ q_new, const float* __restrict__ summ, int nq, int Hq, int Hkv, int d,
+                        int nblk, float inv_sqrt_d, unsigned long long* __restrict__ keys_out) {
+  extern __shared__ __align__(16) float dsc_qm[];  // [G*d]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int G = Hq / Hkv, cols = G * d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cpl = d >> 5;
+  const int n_base = blockIdx.x * kDecScoreWarps * kDecBlocksPerWarp + warp * kDecBlocksPerWarp;
+  // this warp's summary channels, in flight while the query mean is formed
+  float sv[kDecBlocksPerWarp][4];
+#pragma unroll
+  for (int u = 0; u < kDecBlocksPerWarp; ++u) {
+    const int n = n_base + u;
+    const float* src = summ + (((size_t)b * nblk + (n < nblk ? n : 0)) * Hkv + h) * d + lane;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) sv[u][m] = (n < nblk && m < cpl) ? __ldg(src + 32 * m) : 0.f;
   }
+  // mean of the new queries of the G heads of KV head h (contiguous in a token row)
+  const float inv_nq = 1.0f / nq;
+  for (int c = tid; c < cols; c += blockDim.x) {
+    const T* src = q_new + ((size_t)b * nq * Hq + (size_t)h * G) * d + c;
+    float acc = 0.f;
+    for (int u = 0; u < nq; ++u) acc += (float)src[(size_t)u * Hq * d];
+    dsc_qm[c] = acc * inv_nq;
+  }
+  __syncthreads();
+  float best[kDecBlocksPerWarp];
+#pragma unroll
+  for (int u = 0; u < kDecBlocksPerWarp; ++u) best[u] = -FLT_MAX;
+  for (int g = 0; g < G; ++g) {
+    float qv[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) qv[m] = m < cpl ? dsc_qm[g * d + lane + 32 * m] : 0.f;
+    float dot[kDecBlocksPerWarp];
+#pragma unroll
+    for (int u = 0; u < kDecBlocksPerWarp; ++u)
+      dot[u] = (qv[0] * sv[u][0] + qv[1] * sv[u][1]) + (qv[2] * sv[u][2] + qv[3] * sv[u][3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int u = 0; u < kDecBlocksPerWarp; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+    }
+#pragma unroll
+    for (int u = 0; u < kDecBlocksPerWarp; ++u) best[u] = fmaxf(best[u], dot[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < kDecBlocksPerWarp; ++u) {
+    const int n = n_base + u;
+    if (lane == u && n < nblk) keys_out[((size_t)b * Hkv + h) * nblk + n] = sel_key(best[u] * inv_sqrt_d, n);
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads) decode_topk_kernel(const unsigned long long* __restrict__ keys_in,
+                                                                  int Hkv, int nblk, int topk,
+                                                                  int32_t* __restrict__ idx, float* __restrict__ scores) {
+  extern __shared__ __align__(16) unsigned long long dtk_keys[];  // [nblk]
+  __shared__ int chosen[kMaxTopk];
+  __shared__ unsigned long long chosen_key[kMaxTopk];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x;
+  const unsigned long long* src = keys_in + ((size_t)b * Hkv + h) * nblk;
+  for (int n = tid; n < nblk; n += kSelThreads) dtk_keys[n] = src[n];
+  __syncthreads();
+  const int keff = topk < nblk ? topk : nblk;
+  if (nblk <= kSelRankMax) {
+    for (int n = tid; n < nblk; n += kSelThreads) {
+      const unsigned long long kn = dtk_keys[n];
+      int rank = 0;
+      for (int m = 0; m < nblk; ++m) rank += dtk_keys[m] > kn;
+      if (rank < keff) {
+        chosen[rank] = n;
+        chosen_key[rank] = kn;
+      }
+    }
+  } else if (keff > 0) {
+    topk_radix(dtk_keys, nblk, keff, chosen, chosen_key);
+  }
+  __syncthreads();
+  const size_t row = ((size_t)b * Hkv + h) * topk;
+  write_selection(chosen, chosen_key, keff, topk, idx + row, scores ? scores + row : nullptr);
 }
 
 // ------------------------------------------------------------ bwd preprocess
@@ -438,10 +591,9 @@ cudaError_t launch_append_segment(const Shape& s, const void* k_seg, const void*
 
 cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ, int32_t* idx, float* scores,
                                cudaStream_t st) {
-  int npow = 1;
-  while (npow < s.nblk) npow <<= 1;
   const int cols = s.G() * s.d;
-  const size_t smem = (size_t)(cols + (cols & 1) + kSelThreads * (s.bf16 ? 8 : 4)) * sizeof(float) + (size_t)npow * 8;
+  const size_t smem = (size_t)(cols + (cols & 1) + kSelThreads * (s.bf16 ? 8 : 4)) * sizeof(float) +
+                      (size_t)(s.nblk > 0 ? s.nblk : 1) * 8;
   dim3 grid(s.nqb(), s.Hkv, s.B);
   const float isd = 1.0f / sqrtf((float)s.d);
   cudaError_t e;
@@ -458,6 +610,38 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
     kern<<<grid, kSelThreads, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk, s.topk,
                                   isd, idx, scores);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_select(const Shape& s, int nq, const void* q_new, const float* summ, int32_t* idx,
+                                 float* scores, void* ws, cudaStream_t st) {
+  unsigned long long* keys = static_cast<unsigned long long*>(ws);
+  const float isd = 1.0f / sqrtf((float)s.d);
+  cudaError_t e;
+  if (s.nblk > 0) {
+    const int per_cta = kDecScoreWarps * kDecBlocksPerWarp;
+    const dim3 grid((s.nblk + per_cta - 1) / per_cta, s.Hkv, s.B);
+    const size_t smem = (size_t)s.G() * s.d * sizeof(float);
+    if (s.bf16) {
+      if ((e = cudaFuncSetAttribute(decode_score_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem)) != cudaSuccess)
+        return e;
+      decode_score_kernel<__nv_bfloat16><<<grid, kDecScoreWarps * 32, smem, st>>>(
+          static_cast<const __nv_bfloat16*>(q_new), summ, nq, s.Hq, s.Hkv, s.d, s.nblk, isd, keys);
+    } else {
+      if ((e = cudaFuncSetAttribute(decode_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem)) != cudaSuccess)
+        return e;
+      decode_score_kernel<float><<<grid, kDecScoreWarps * 32, smem, st>>>(static_cast<const float*>(q_new), summ,
+                                                                          nq, s.Hq, s.Hkv, s.d, s.nblk, isd, keys);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t smem = (size_t)(s.nblk > 0 ? s.nblk : 1) * 8;
+  if ((e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+      cudaSuccess)
+    return e;
+  decode_topk_kernel<<<dim3(s.Hkv, s.B), kSelThreads, smem, st>>>(keys, s.Hkv, s.nblk, s.topk, idx, scores);
   return cudaGetLastError();
 }
 

@@ -51,10 +51,10 @@ def _decode(w, nq, t0, x):
         hga_block_summaries(D, dev["k_hist"], 0, w.nblk, summ)
     idx = torch.empty((w.B, w.Hkv, w.topk), dtype=torch.int32, device="cuda")
     scores = torch.empty(idx.shape, dtype=torch.float32, device="cuda")
-    hga_decode_select(D, qn, summ, idx, scores)
+    ws = torch.empty((hga_decode_workspace_size(D, nq),), dtype=torch.uint8, device="cuda")
+    hga_decode_select(D, qn, summ, idx, scores, ws)
     o = torch.empty_like(qn)
     lse = torch.empty((w.B, w.Hq, nq), dtype=torch.float32, device="cuda")
-    ws = torch.empty((hga_decode_workspace_size(D, nq),), dtype=torch.uint8, device="cuda")
     hga_decode_attn(D, t0, qn, dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk, idx, o, lse, ws)
     torch.cuda.synchronize()
     hga_device_status()
@@ -111,7 +111,13 @@ def test_decode_whole_block_equals_prefill_kernels():
     lse_p = torch.empty((1, w.Hq, w.S), device="cuda")
     hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], w.nblk, idx_p, o_p, lse_p)
     torch.cuda.synchronize()
-    assert np.array_equal(idx, idx_p.cpu().numpy()[:, :, i])
+    # the two kernels sum the query mean in different fp32 orders: equal
+    # selections wherever the oracle's K-th and (K+1)-th scores are not a near-tie
+    od = oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk)
+    _, score_ref = oracle.select(od, x.q.f64, x.k_hist.f64)
+    near = oracle.near_tie_positions(od, score_ref)[:, :, i]
+    same = np.all(idx == idx_p.cpu().numpy()[:, :, i], axis=-1)
+    assert np.all(same | near)
     rows = slice(t0, t0 + nq)
     assert (o.float() - o_p[:, rows].float()).abs().max().item() <= 2e-2
     assert (lse - lse_p[:, :, rows]).abs().max().item() <= 1e-4
