@@ -375,12 +375,7 @@ static_assert(dkdv_smem_bytes(128) <= 232448, "shared memory budget");
 // Tensor-memory columns of the dK/dV kernel.
 constexpr uint32_t kKvS = 0, kKvP = 128, kKvDK = 256, kKvDV = 384;
 
-// kFull = false: 64-query sub-tiles, two in flight (S^T/dP^T double-buffered).
-// kFull = true: whole 128-query blocks (N = 128 products, no shared-memory
-// re-read of K and V per half), one in flight: S^T | dP^T | dK | dV fill the
-// tensor memory; the next block's S^T/dP^T follow its dV/dK products in issue
-// order (in-order completion makes the overwrite of the P^T/dS^T columns safe).
-template <int KD, bool kFull>
+template <int KD>
 __global__ void __launch_bounds__(320, 1)
     dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
@@ -408,9 +403,7 @@ __global__ void __launch_bounds__(320, 1)
   int n = 0;
   for (int i = jb; i < a.nqb; ++i) n += (!a.qmask || a.qmask[(size_t)b * a.nqb + i]) ? 1 : 0;
   if (n == 0) return;  // no gradient reaches this key block from head hq (outputs start at zero)
-  constexpr int kSub = kFull ? kB : kSubRows;  // queries per MMA sub-tile
-  constexpr int kPer = kB / kSub;              // sub-tiles per query block
-  const int nsub = kPer * n;
+  const int nsub = 2 * n;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -466,15 +459,15 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdT = idesc_bf16(kB, kSub, false, false);  // [128 keys x kSub queries]
+      constexpr uint32_t kIdT = idesc_bf16(kB, kSubRows, false, false);  // [128 keys x 64 queries]
       constexpr uint32_t kIdG = idesc_bf16(kB, kD, false, true);         // dV += P^T dO_half, dK += dS^T Q_half
       // Descriptors built once; k-steps, query halves and stages are constant adds.
       const uint64_t dKd = sdesc_sw128(smem_u32(sK), 16, 1024), dVd = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024), dOk = sdesc_sw128(smem_u32(sDO), 16, 1024);
       const uint64_t dQmn = sdesc_sw128(smem_u32(sQ), kHalf, 1024), dOmn = sdesc_sw128(smem_u32(sDO), kHalf, 1024);
-      // S^T and dP^T of sub-tile u (query block qblocks[u / kPer], part u % kPer) into buffer u % kPer.
+      // S^T and dP^T of sub-tile u (query block jb + u/2, query half u%2) into buffer u%2.
       auto issue_sdp = [=](int u) -> bool {
-        const int it = u / kPer, h = u % kPer, s = it % kQStages;
+        const int it = u >> 1, h = u & 1, s = it % kQStages;
         if (h == 0) {
           if (!mbar_wait(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err)) return false;
           tc_fence_after();
@@ -495,30 +488,29 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(&ctl->sdp_full[h]);
         return true;
       };
-      constexpr int kAhead = kFull ? 1 : 2;  // sub-tiles whose S^T/dP^T are in flight
       bool ok = mbar_wait(&ctl->kv_full, 0, abort, a.err);
       if (ok) {
         tc_fence_after();
-        for (int u = 0; ok && u < kAhead && u < nsub; ++u) ok = issue_sdp(u);
+        ok = issue_sdp(0) && issue_sdp(1);
       }
       for (int u = 0; ok && u < nsub; ++u) {
-        const int it = u / kPer, h = u % kPer, s = it % kQStages;
-        if (!mbar_wait(&ctl->pds_full[h], (u / kPer) & 1, abort, a.err)) break;
+        const int it = u >> 1, h = u & 1, s = it % kQStages;
+        if (!mbar_wait(&ctl->pds_full[h], (u >> 1) & 1, abort, a.err)) break;
         tc_fence_after();
         const uint32_t so = sdesc_units(s * kTileBytes + h * kSubOff);
         const uint64_t qb = dQmn + so, ob = dOmn + so;
         const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kSub / 16; ++kk)  // dV += P^T dO (this sub-tile's queries)
+        for (int kk = 0; kk < kSubRows / 16; ++kk)  // dV += P^T dO_half
           umma_ts(tmem + kKvDV, tmem + kKvS + h * 64 + packed_col(kk), ob + sdesc_units(kk * 2048), kIdG,
                   kk > 0 ? 1u : acc0);
 #pragma unroll
-        for (int kk = 0; kk < kSub / 16; ++kk)  // dK += dS^T Q
+        for (int kk = 0; kk < kSubRows / 16; ++kk)  // dK += dS^T Q_half
           umma_ts(tmem + kKvDK, tmem + kKvP + h * 64 + packed_col(kk), qb + sdesc_units(kk * 2048), kIdG,
                   kk > 0 ? 1u : acc0);
-        if (h == kPer - 1) umma_commit(&ctl->qd_empty[s]);
-        if (u + kAhead < nsub) {
-          if (!issue_sdp(u + kAhead)) break;
+        if (h == 1) umma_commit(&ctl->qd_empty[s]);
+        if (u + 2 < nsub) {
+          if (!issue_sdp(u + 2)) break;
         }
         if (u == nsub - 1) umma_commit(&ctl->dkv_full);
       }
@@ -533,15 +525,12 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const float2 s2 = make_float2(a.sl2, a.sl2), nlog2e = make_float2(-kLog2e, -kLog2e);
     bool ok = true;
-    // Each warpgroup takes half of a sub-tile's queries: kCols columns of S^T
-    // then kCols columns of dP^T of this thread's key row.
-    constexpr int kCols = kSub / 2;
-    uint32_t sd[2 * kCols];
+    uint32_t sd[64];  // 32 S^T columns then 32 dP^T columns of this thread's key row
     for (int u = 0; u < nsub; ++u) {
-      const int it = u / kPer, h = u % kPer, s = it % kQStages;
+      const int it = u >> 1, h = u & 1, s = it % kQStages;
       // The row statistics arrive with the Q/dO stage: observe that stage's
       // barrier directly (its phase is complete by now) before reading them.
-      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full[h], (u / kPer) & 1, abort, a.err) &&
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl->sdp_full[h], (u >> 1) & 1, abort, a.err) &&
                                        mbar_wait(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err))) {
         ok = false;
         break;
@@ -549,37 +538,27 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const bool diag = (ctl->qblocks[it] == jb);
       const RowStats& rs = stats[s];
-      if constexpr (kFull)
-        tmem_ld64x2_wait(tmem + lane_off + kKvS + kCols * e, tmem + lane_off + kKvP + kCols * e, sd);
-      else
-        tmem_ld32x2_wait(tmem + lane_off + kKvS + h * 64 + kCols * e, tmem + lane_off + kKvP + h * 64 + kCols * e,
-                         sd);
-      const int q0 = kSub * h + kCols * e;  // query column of sd[0] within block i
+      tmem_ld32x2_wait(tmem + lane_off + kKvS + h * 64 + 32 * e, tmem + lane_off + kKvP + h * 64 + 32 * e, sd);
+      const int q0 = 64 * h + 32 * e;  // query column of sd[0] within block i
+      uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int cc = 0; cc < kCols / 32; ++cc) {
-        uint32_t pp[16], pd[16];
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const int c = 32 * cc + x;  // column within this thread's share
-          const int q = q0 + c;
-          const float2 lq = *reinterpret_cast<const float2*>(&rs.lse[q]);  // same for every key row: broadcast
-          const float2 dq2 = *reinterpret_cast<const float2*>(&rs.D[q]);
-          const float2 arg = fma2(make_float2(__uint_as_float(sd[c]), __uint_as_float(sd[c + 1])), s2,
-                                  mul2(lq, nlog2e));
-          float2 pr = exp2_pair(arg, (kBwdPolyPairs >> (x >> 1)) & 1u);
-          if (diag) {
-            pr.x = q >= r ? pr.x : 0.f;
-            pr.y = q + 1 >= r ? pr.y : 0.f;
-          }
-          pp[x >> 1] = pack_bf16x2_softmax(pr.x, pr.y);
-          const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[kCols + c]),
-                                                      __uint_as_float(sd[kCols + c + 1])), dq2));
-          pd[x >> 1] = pack_bf16x2_softmax(ds.x, ds.y);
+      for (int x = 0; x < 32; x += 2) {
+        const int q = q0 + x;
+        const float2 lq = *reinterpret_cast<const float2*>(&rs.lse[q]);  // same for every key row: broadcast
+        const float2 dq2 = *reinterpret_cast<const float2*>(&rs.D[q]);
+        const float2 arg = fma2(make_float2(__uint_as_float(sd[x]), __uint_as_float(sd[x + 1])), s2,
+                                mul2(lq, nlog2e));
+        float2 pr = exp2_pair(arg, (kBwdPolyPairs >> (x >> 1)) & 1u);
+        if (diag) {
+          pr.x = q >= r ? pr.x : 0.f;
+          pr.y = q + 1 >= r ? pr.y : 0.f;
         }
-        // packed bf16 of query chunk (32 queries) -> the first 16 of its 32 columns
-        HGA_TMEM_ST16(tmem + lane_off + kKvS + h * 64 + kCols * e + 32 * cc, pp);
-        HGA_TMEM_ST16(tmem + lane_off + kKvP + h * 64 + kCols * e + 32 * cc, pd);
+        pp[x >> 1] = pack_bf16x2_softmax(pr.x, pr.y);
+        const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[32 + x]), __uint_as_float(sd[33 + x])), dq2));
+        pd[x >> 1] = pack_bf16x2_softmax(ds.x, ds.y);
       }
+      HGA_TMEM_ST16(tmem + lane_off + kKvS + h * 64 + 32 * e, pp);
+      HGA_TMEM_ST16(tmem + lane_off + kKvP + h * 64 + 32 * e, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ctl->pds_full[h]);
@@ -617,12 +596,6 @@ __global__ void __launch_bounds__(320, 1)
 
 }  // namespace
 
-// Which dK/dV schedule runs: whole 128-query blocks (1) or 64-query halves (0).
-#ifndef HGA_DKDV_FULL
-#define HGA_DKDV_FULL 0
-#endif
-constexpr bool kDkvFull = HGA_DKDV_FULL != 0;
-
 template <int KD>
 cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                        const float* Dr, float* dq, float* dk, float* dv, int parts, int* err, cudaStream_t st,
@@ -632,8 +605,8 @@ cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
   if ((e = cudaFuncSetAttribute(dq_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem)) !=
       cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(dkdv_tc_kernel<KD, kDkvFull>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kv_smem)) != cudaSuccess)
+  if ((e = cudaFuncSetAttribute(dkdv_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem)) !=
+      cudaSuccess)
     return e;
   BwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
@@ -646,7 +619,7 @@ cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
     const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * KD * sizeof(float);
     if ((e = cudaMemsetAsync(dk, 0, kv_bytes, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dv, 0, kv_bytes, st)) != cudaSuccess) return e;
-    dkdv_tc_kernel<KD, kDkvFull><<<s.B * s.Hq * s.nqb(), 320, kv_smem, st>>>(m.q, m.d_o, m.ks, m.vs, a);
+    dkdv_tc_kernel<KD><<<s.B * s.Hq * s.nqb(), 320, kv_smem, st>>>(m.q, m.d_o, m.ks, m.vs, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (parts & kBwdDq) {

@@ -142,32 +142,38 @@ __global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __
   cp_async_wait_all();
   __syncthreads();
 
-  // 2. scores (log2 units), one key per thread, all rows of the CTA
+  // 2. scores (log2 units), one key per thread, rows in groups of four (a
+  //    group's products are only formed for rows that exist)
   for (int j = tid; j < blk; j += kDecThreads) {
-    float acc[kDecRows];
+    const uint8_t* krow = sK + (size_t)j * row_bytes;
+    for (int rq = 0; rq < nr; rq += 4) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j < nk) {
+        for (int v = 0; v < vpr; ++v) {
+          float kv[E];
+          DecElem<T>::unpack(*reinterpret_cast<const uint4*>(krow + v * 16), kv);
 #pragma unroll
-    for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
-    if (j < nk) {
-      const uint8_t* krow = sK + (size_t)j * row_bytes;
-      for (int v = 0; v < vpr; ++v) {
-        float kv[E];
-        DecElem<T>::unpack(*reinterpret_cast<const uint4*>(krow + v * 16), kv);
+          for (int r4 = 0; r4 < 4; ++r4) {
+            const float4* qr = reinterpret_cast<const float4*>(sQ + (rq + r4) * d + v * E);
 #pragma unroll
-        for (int r = 0; r < kDecRows; ++r) {
-          if (r < nr) {
-            const float* qr = sQ + r * d + v * E;
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[r] = fmaf(qr[e], kv[e], acc[r]);
+            for (int e4 = 0; e4 < E / 4; ++e4) {
+              const float4 q4 = qr[e4];  // same address in every lane: broadcast
+              acc[r4] = fmaf(q4.x, kv[4 * e4], acc[r4]);
+              acc[r4] = fmaf(q4.y, kv[4 * e4 + 1], acc[r4]);
+              acc[r4] = fmaf(q4.z, kv[4 * e4 + 2], acc[r4]);
+              acc[r4] = fmaf(q4.w, kv[4 * e4 + 3], acc[r4]);
+            }
           }
         }
       }
-    }
 #pragma unroll
-    for (int r = 0; r < kDecRows; ++r) {
-      if (r < nr) {
-        const int u = (r0 + r) % a.nq;
-        const bool visible = j < nk && (hist || pos0 + j <= a.t0 + u);
-        sS[r * blk + j] = visible ? acc[r] : -INFINITY;
+      for (int r4 = 0; r4 < 4; ++r4) {
+        const int r = rq + r4;
+        if (r < nr) {
+          const int u = (r0 + r) % a.nq;
+          const bool visible = j < nk && (hist || pos0 + j <= a.t0 + u);
+          sS[r * blk + j] = visible ? acc[r4] : -INFINITY;
+        }
       }
     }
   }
@@ -195,22 +201,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __
   }
   __syncthreads();
 
-  // 4. unnormalised O of the chunk: thread = (column, row phase)
+  // 4. unnormalised O of the chunk: thread = (column, row phase), rows in
+  //    groups of four
   const int phases = kDecThreads / d;  // 1 (d = 128) or 2 (d = 64)
   const int col = tid % d, ph = tid / d;
-  float acc[kDecRows];
-#pragma unroll
-  for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
-  for (int j = 0; j < nk; ++j) {
-    const float vj = DecElem<T>::at(reinterpret_cast<const T*>(sV + (size_t)j * row_bytes) + col);
-#pragma unroll
-    for (int r = 0; r < kDecRows; ++r)
-      if (r % phases == ph && r < nr) acc[r] = fmaf(sS[r * blk + j], vj, acc[r]);
-  }
   const size_t base = (((size_t)b * a.Hkv + h) * a.n_chunks + c) * a.R + r0;
+  for (int rq = 4 * ph; rq < nr; rq += 4 * phases) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < nk; ++j) {
+      const float vj = DecElem<T>::at(reinterpret_cast<const T*>(sV + (size_t)j * row_bytes) + col);
 #pragma unroll
-  for (int r = 0; r < kDecRows; ++r)
-    if (r % phases == ph && r < nr) a.part_o[(base + r) * d + col] = acc[r];
+      for (int r4 = 0; r4 < 4; ++r4) acc[r4] = fmaf(sS[(rq + r4) * blk + j], vj, acc[r4]);
+    }
+#pragma unroll
+    for (int r4 = 0; r4 < 4; ++r4)
+      if (rq + r4 < nr) a.part_o[(base + rq + r4) * d + col] = acc[r4];
+  }
   if (tid < nr) {
     a.part_ml[(base + tid) * 2] = sM[tid];
     a.part_ml[(base + tid) * 2 + 1] = sL[tid];

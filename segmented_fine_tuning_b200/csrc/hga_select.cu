@@ -257,13 +257,63 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelU = 4;  // blocks per warp per scoring round
 constexpr int kSelRankMax = 256;  // largest padded block count ranked by counting
 
+// Scores of all nblk blocks for one selection, when the group size G divides
+// 32: a warp takes U = 32/G blocks per round, every lane forms the partial dot
+// products of its channels for all U*G (block, head) pairs, and one transposing
+// butterfly (31 shuffles) leaves lane L with the full product of pair L --
+// instead of 5 shuffles per product.  The group maximum is then log2(G) more
+// shuffles, and lanes L with L % G == 0 write the keys.
+template <int G>
+__device__ void score_blocks_transposed(const float* qm, const float* __restrict__ summ, int b, int h, int Hkv, int d,
+                                        int nblk, float inv_sqrt_d, unsigned long long* keys) {
+  constexpr int U = 32 / G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cpl = d >> 5;  // channels per lane: 2 or 4
+  for (int n0 = warp * U; n0 < nblk; n0 += kSelWarps * U) {
+    float sv[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int n = n0 + u;
+      const float* src = summ + (((size_t)b * nblk + (n < nblk ? n : 0)) * Hkv + h) * d + lane;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sv[u][m] = (n < nblk && m < cpl) ? __ldg(src + 32 * m) : 0.f;
+    }
+    float v[32];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float qv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) qv[m] = m < cpl ? qm[g * d + lane + 32 * m] : 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        v[u * G + g] = (qv[0] * sv[u][0] + qv[1] * sv[u][1]) + (qv[2] * sv[u][2] + qv[3] * sv[u][3]);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int k = 0; k < off; ++k) {
+        const float send = upper ? v[k] : v[k + off];
+        const float keep = upper ? v[k + off] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+    }
+    float best = v[0];  // pair index = lane = u * G + g
+#pragma unroll
+    for (int off = 1; off < G; off <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+    const int n = n0 + lane / G;
+    if ((lane % G) == 0 && n < nblk) keys[n] = sel_key(best * inv_sqrt_d, n);
+  }
+}
+
 // CTA = (query block i, KV head h, batch b).  512 threads.
 //  1. qm[g][:] = mean of the block's rows of Q for the G query heads of h
 //     (the G heads of a KV head are contiguous in a token row).
-//  2. score[n] = max_g qm[g] . summ[b,n,h] / sqrt(d).  A warp scores kSelU
-//     blocks per round: their summary channels are loaded before any
-//     arithmetic (the first round's before step 1), and the G * kSelU dot
-//     products are reduced across the warp together.
+//  2. score[n] = max_g qm[g] . summ[b,n,h] / sqrt(d): for G = 4 (the GQA
+//     group of the Qwen3-8B shapes) with one transposing warp reduction per
+//     32 (block, head) products;
+//     otherwise a warp scores kSelU blocks per round, their summary channels
+//     loaded before any arithmetic, the G * kSelU products reduced together.
 //  3. top K_eff of the (score, index) keys by rank counting (up to 256
 //     blocks) or a byte-wise radix select, then listed in ascending order.
 template <typename T>
@@ -297,7 +347,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
       for (int m = 0; m < 4; ++m) dst[u][m] = (n < nblk && m < cpl) ? __ldg(src + 32 * m) : 0.f;
     }
   };
-  load_round(sv, warp * kSelU);
+  const bool transposed = (G == 4);
+  if (!transposed) load_round(sv, warp * kSelU);
 
   // 1. query means: thread = (row phase r0, vector vt); rows r0, r0+rpp, ...
   //    are summed per thread, the rpp partials are then combined.
@@ -331,9 +382,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
     __syncthreads();
   }
 
-  // 2. scores -> keys; the next round's summary channels are loaded before
-  //    this round's arithmetic, so a load latency is paid once, not per round
-  for (int n0 = warp * kSelU; n0 < nblk; n0 += kSelWarps * kSelU) {
+  // 2. scores -> keys.  G = 4: transposed reduction (above).
+  //    Otherwise a warp scores kSelU blocks per round, the next round's
+  //    summary channels loaded before this round's arithmetic.
+  if (G == 4) score_blocks_transposed<4>(qm, summ, b, h, Hkv, d, nblk, inv_sqrt_d, keys);
+  for (int n0 = warp * kSelU; !transposed && n0 < nblk; n0 += kSelWarps * kSelU) {
     const int n1 = n0 + kSelWarps * kSelU;
     if (n1 < nblk) load_round(sn, n1);
     float best[kSelU];
