@@ -627,6 +627,118 @@ def run_decode(args, device):
             "gpu_launches": 4 * args.steps, "clocks": clk.summary()}
 
 
+def run_tier(args, device):
+    """The history-tier paths on the Qwen3-8B-shaped layer: fetching the
+    selected blocks (every one of the 112 history blocks is selected by some
+    query block) from a pinned host tier by the copy engines
+    (hga_fetch_blocks) and by the SMs over mapped memory
+    (hga_gather_blocks_mapped), the device idx remap, and a finished segment's
+    append in one pass (hga_append_segment) against the three separate calls
+    it replaces.  Each timed on the stream with CUDA events (mean of --steps,
+    L2 flushed between steps); bytes are the algorithmic bytes moved."""
+    import segmented_fine_tuning_b200 as hga
+    w = synth.QWEN3_8B_LAYER
+    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
+    x = synth.draw(w)
+    stream = torch.cuda.current_stream(device)
+    copy_stream = torch.cuda.Stream(device)
+    q, ks, vs, kh = (to_dev(t, device) for t in (x.q, x.k_seg, x.v_seg, x.k_hist))
+    tier_k, tier_v = to_pinned(x.k_hist), to_pinned(x.v_hist)
+    summ = torch.empty((1, w.nblk, w.Hkv, w.d), dtype=torch.float32, device=device)
+    idx = torch.empty((1, w.Hkv, w.nqb, w.topk), dtype=torch.int32, device=device)
+    hga.hga_block_summaries(D, kh, 0, w.nblk, summ, stream)
+    hga.hga_select_topk(D, q, summ, idx, None, stream)
+    torch.cuda.synchronize(device)
+    n_sel = len(set(idx.cpu().numpy().ravel().tolist()) - {-1})
+    pool_k = torch.empty((1, w.nblk * w.blk, w.Hkv, w.d), dtype=torch.bfloat16, device=device)
+    pool_v = torch.empty_like(pool_k)
+    idx_pool = torch.empty_like(idx)
+    scratch = torch.empty(tuple(idx.shape), dtype=torch.int32).pin_memory()
+    done = torch.cuda.Event()
+    done.record(copy_stream)
+    slot_of = torch.arange(w.nblk, dtype=torch.int32, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    blk_bytes = w.blk * w.Hkv * w.d * 2
+    # append: a segment entering a history of capacity nblk + nqb blocks
+    cap = w.nblk + w.nqb
+    Da = hga.Dims(1, w.Hq, w.Hkv, w.d, w.blk, w.S, cap, w.topk, "bf16")
+    summ_a = torch.zeros((1, cap, w.Hkv, w.d), dtype=torch.float32, device=device)
+    cache = hga.BlockCache(cap, w.nblk + w.nqb)
+    pk = torch.empty((1, cache.pool_slots * w.blk, w.Hkv, w.d), dtype=torch.bfloat16, device=device)
+    pv = torch.empty_like(pk)
+    tk = torch.empty((1, cap * w.blk, w.Hkv, w.d), dtype=torch.bfloat16).pin_memory()
+    tv = torch.empty_like(tk).pin_memory()
+
+    def fetch():
+        hga.hga_fetch_blocks(D, tier_k, tier_v, w.nblk, idx, scratch, pool_k, pool_v, w.nblk, idx_pool, stream,
+                             copy_stream, done)
+        stream.wait_event(done)
+
+    def gather():
+        hga.hga_gather_blocks_mapped(D, tier_k, tier_v, w.nblk, idx, pool_k, pool_v, w.nblk, idx_pool, stream)
+
+    def remap():
+        hga.hga_remap_idx(D, idx, slot_of, idx_pool, stream)
+
+    def append_fused():
+        cache.reset()
+        hga.hga_append_segment(Da, ks, vs, w.nblk, summ_a, pk, pv, cache, None, None, 0, stream)
+
+    def append_separate():
+        cache.reset()
+        hga.hga_segment_summaries(Da, ks, w.nblk, summ_a, stream)
+        hga.hga_cache_segment(hga.Dims(1, w.Hq, w.Hkv, w.d, w.blk, w.S, 0, w.topk, "bf16"), ks, vs, pk, pv, cache,
+                              w.nblk, stream)
+
+    def append_with_offload():
+        cache.reset()
+        hga.hga_append_segment(Da, ks, vs, w.nblk, summ_a, pk, pv, cache, tk, tv, cap, stream, copy_stream)
+        stream.wait_stream(copy_stream)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize(device)
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            ts.append(e0.elapsed_time(e1))
+        hga.hga_device_status(stream)
+        return float(np.mean(ts))
+
+    probe = h2d_probe(device)
+    peaks, peak_src = load_peaks()
+    fetch_bytes = n_sel * blk_bytes * 2
+    seg_bytes = w.S * w.Hkv * w.d * 2
+    res = {}
+    for name, fn, nbytes, ref in (
+            ("fetch_copy_engines", fetch, fetch_bytes, "h2d"), ("gather_mapped_sms", gather, fetch_bytes, "h2d"),
+            ("remap_idx", remap, idx.numel() * 8, "hbm"),
+            ("append_fused", append_fused, 4 * seg_bytes + w.nqb * w.Hkv * w.d * 4, "hbm"),
+            ("append_separate", append_separate, 5 * seg_bytes + w.nqb * w.Hkv * w.d * 4, "hbm"),
+            ("append_fused_with_tier_offload", append_with_offload, 2 * seg_bytes, "d2h")):
+        ms = timed(fn)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        e = {"ms": round(ms, 4), "bytes": int(nbytes), "gbs": round(gbs, 1)}
+        if ref == "h2d":
+            e["frac_of_h2d_probe"] = round(gbs / probe, 3)
+        elif ref == "hbm":
+            e["frac_hbm"] = round(gbs / peaks["hbm_gbs"], 3)
+        res[name] = e
+    return {"metric": "HGA history-tier paths on the Qwen3-8B-shaped layer (fetch, gather, remap, segment append)",
+            "value": res["fetch_copy_engines"]["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "selected_blocks": n_sel, "l2": "flushed between steps"},
+            "h2d_probe_gbs": round(probe, 1), "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
+            "paths": res}
+
+
 # ---------------------------------------------------------------- oracle legs
 
 def oracle_sample(w: synth.Workload, x, kv_heads):
@@ -715,12 +827,13 @@ def main():
                     help="device pool (cache) slots per layer for --workload segmented (default: the largest history)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the 131K-token prefill and dense-equivalence sub-measurements of the default (layer) run")
-    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode"), default="layer",
+    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode", "tier"), default="layer",
                     help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
                          "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
-                         "the 131K prefill forward, device-timed only; decode: one new token at 131K context")
+                         "the 131K prefill forward, device-timed only; decode: one new token at 131K context; "
+                         "tier: the history-tier fetch, gather, remap and segment-append paths")
     args = ap.parse_args()
-    if args.workload in ("dense", "prefill", "decode"):
+    if args.workload in ("dense", "prefill", "decode", "tier"):
         args.no_e2e = args.no_cpu_baseline = True
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3
@@ -741,8 +854,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     try:
-        if args.workload in ("segmented", "decode"):
-            out = run_segmented(args, device) if args.workload == "segmented" else run_decode(args, device)
+        if args.workload in ("segmented", "decode", "tier"):
+            out = {"segmented": run_segmented, "decode": run_decode, "tier": run_tier}[args.workload](args, device)
             if rank == 0:
                 print(json.dumps(out), flush=True)
             return
