@@ -93,6 +93,38 @@ def test_null_and_invalid_arguments(lib):
     assert lib.hga_offload_segment(ctypes.byref(d), p, p, p, p, 4, 3, None) == 1  # 2 blocks at 3 > capacity 4
 
 
+def test_new_entry_points_validate_on_host(lib):
+    """Decode, sparse backward, segment append and zero-copy gather reject bad
+    arguments before touching a device."""
+    d = _dims()
+    p = ctypes.c_void_p(16)
+    ws = lib.hga_decode_workspace_size(ctypes.byref(d), 1)
+    assert ws > 0 and ws % 256 == 0
+    assert lib.hga_decode_workspace_size(ctypes.byref(d), 0) == 0       # n_q < 1
+    assert lib.hga_decode_workspace_size(ctypes.byref(d), 129) == 0     # n_q > block
+    # n_q outside [1, block]
+    assert lib.hga_decode_select(ctypes.byref(d), 0, p, p, p, None, p, ws, None) == 2
+    assert lib.hga_decode_attn(ctypes.byref(d), 200, 0, p, p, p, p, p, 4, p, p, p, p, ws, None) == 2
+    # new tokens past the segment buffer (S = 256)
+    assert lib.hga_decode_attn(ctypes.byref(d), 2, 255, p, p, p, p, p, 4, p, p, p, p, ws, None) == 2
+    # short workspace
+    assert lib.hga_decode_select(ctypes.byref(d), 1, p, p, p, None, p, 8, None) == 1
+    assert lib.hga_decode_attn(ctypes.byref(d), 1, 0, p, p, p, p, p, 4, p, p, p, p, 8, None) == 1
+    # sparse backward: mask required, scale finite
+    wsb = lib.hga_attn_bwd_workspace_size(ctypes.byref(d))
+    w256 = ctypes.c_void_p(256)
+    assert lib.hga_attn_bwd_sparse(ctypes.byref(d), p, p, p, p, p, 4, p, p, p, p, None, 1.0, p, p, p, w256, wsb,
+                                   None) == 1
+    assert lib.hga_attn_bwd_sparse(ctypes.byref(d), p, p, p, p, p, 4, p, p, p, p, p, float("inf"), p, p, p, w256,
+                                   wsb, None) == 1
+    # append: blocks outside the summary array, host tier halves must come together
+    assert lib.hga_append_segment(ctypes.byref(d), p, p, 3, p, None, None, None, None, None, 0, None, None) == 1
+    assert lib.hga_append_segment(ctypes.byref(d), p, p, 0, p, None, None, None, p, None, 8, None, None) == 1
+    # gather: a pool of no slots, a tier shorter than the history
+    assert lib.hga_gather_blocks_mapped(ctypes.byref(d), p, p, 4, p, p, p, 0, p, None) == 1
+    assert lib.hga_gather_blocks_mapped(ctypes.byref(d), p, p, 3, p, p, p, 4, p, None) == 1
+
+
 def test_binding_rejects_wrong_shapes():
     import torch
     D = _binding.Dims(1, 4, 2, 128, 128, 256, 4, 2, "bf16")

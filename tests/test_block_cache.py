@@ -93,3 +93,28 @@ def test_reset_empties():
     c.reset()
     assert (c.slot_of_block == -1).all() and (c.block_of_slot == -1).all() and c.c.tick == 0
     assert c.plan([4])[1].tolist() == [4]
+
+
+def test_spaco_sampler_picks_k_blocks_per_sequence_and_caps_the_factor():
+    """Host sampler of the sparse backward: exactly k of the t query blocks
+    of every sequence, reproducible from the generator's seed, factor t/k
+    (the inverse of the inclusion probability), capped when asked."""
+    import torch
+    from segmented_fine_tuning_b200 import spaco_sample_blocks
+    g = torch.Generator().manual_seed(3)
+    mask, scale = spaco_sample_blocks(4, 16, 4, g)
+    assert mask.dtype == torch.uint8 and tuple(mask.shape) == (4, 16)
+    assert (mask.sum(dim=1) == 4).all() and scale == 4.0
+    again, _ = spaco_sample_blocks(4, 16, 4, torch.Generator().manual_seed(3))
+    assert torch.equal(mask, again)
+    _, capped = spaco_sample_blocks(1, 16, 1, torch.Generator().manual_seed(0), cap=8.0)
+    assert capped == 8.0
+    # over many draws every block is chosen with probability k/t
+    counts = torch.zeros(16)
+    gen = torch.Generator().manual_seed(11)
+    for _ in range(2000):
+        m, _ = spaco_sample_blocks(1, 16, 4, gen)
+        counts += m[0].float()
+    assert ((counts / 2000 - 0.25).abs() < 0.04).all()
+    with pytest.raises(ValueError):
+        spaco_sample_blocks(1, 16, 0, gen)
