@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(320, 1)
           const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[64 + 32 * cc + xx]),
                                                       __uint_as_float(sd[64 + 32 * cc + xx + 1])),
                                           D2));
-          pk[xx >> 1] = pack_bf16x2_softmax(ds.x, ds.y);
+          pk[xx >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         HGA_TMEM_ST16(tmem + lane_off + kDqS + x * 128 + 64 * e + 32 * cc, pk);
       }
@@ -553,9 +553,9 @@ __global__ void __launch_bounds__(320, 1)
           pr.x = q >= r ? pr.x : 0.f;
           pr.y = q + 1 >= r ? pr.y : 0.f;
         }
-        pp[x >> 1] = pack_bf16x2_softmax(pr.x, pr.y);
+        pp[x >> 1] = pack_bf16x2(pr.x, pr.y);
         const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[32 + x]), __uint_as_float(sd[33 + x])), dq2));
-        pd[x >> 1] = pack_bf16x2_softmax(ds.x, ds.y);
+        pd[x >> 1] = pack_bf16x2(ds.x, ds.y);
       }
       HGA_TMEM_ST16(tmem + lane_off + kKvS + h * 64 + 32 * e, pp);
       HGA_TMEM_ST16(tmem + lane_off + kKvP + h * 64 + 32 * e, pd);

@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const float2 x = fma2(make_float2(__uint_as_float(v[c * 32 + e]), __uint_as_float(v[c * 32 + e + 1])), s2, nm);
           const float2 p = exp2_pair(x, (kFwdPolyPairs >> (e >> 1)) & 1u);
           l2[(e >> 1) & 1] = add2(l2[(e >> 1) & 1], p);
-          pk[e >> 1] = pack_bf16x2_softmax(p.x, p.y);
+          pk[e >> 1] = pack_bf16x2(p.x, p.y);
         }
         HGA_TMEM_ST16(tS + c * 32, pk);
       }
@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const float2 x = fma2(make_float2(__uint_as_float(v[c * 32 + e]), __uint_as_float(v[c * 32 + e + 1])), s2, nm);
           const float2 p = exp2_pair(x, (kFwdPolyPairs >> (e >> 1)) & 1u);
           l2[(e >> 1) & 1] = add2(l2[(e >> 1) & 1], p);
-          pk[e >> 1] = pack_bf16x2_softmax(p.x, p.y);
+          pk[e >> 1] = pack_bf16x2(p.x, p.y);
         }
         HGA_TMEM_ST16(tS + c * 32, pk);
       }

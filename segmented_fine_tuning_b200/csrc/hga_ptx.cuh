@@ -354,24 +354,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The same packing with integer instructions only, for the softmax passes:
-// adding half a bf16 unit in the last place (0x8000) to the fp32 bit pattern
-// and keeping the upper 16 bits rounds to nearest, ties away from zero (the
-// sign is separate in the encoding, so both signs round symmetrically); it
-// differs from round-to-nearest-even only on exact ties.  Two integer adds
-// and one byte permute, which keeps the conversion off the pipe that also
-// evaluates 2^x.  Finite inputs only (a NaN may come out as inf).
-#ifndef HGA_PACK_ALU
-#define HGA_PACK_ALU 0
-#endif
-__device__ __forceinline__ uint32_t pack_bf16x2_softmax(float lo, float hi) {
-#if HGA_PACK_ALU
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-#else
-  return pack_bf16x2(lo, hi);
-#endif
-}
-
 // Fire-and-forget vector float add to global memory (no value returned, so
 // consecutive reductions from one thread do not wait on each other).
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
