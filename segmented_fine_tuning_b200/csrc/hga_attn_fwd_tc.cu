@@ -38,18 +38,7 @@ namespace {
 constexpr int kBM = 128;                      // query rows per tile
 constexpr int kBN = 128;                      // keys per tile
 constexpr int kHalf = kBM * 128;              // one 64-column TMA box: 128 rows x 128 bytes
-// Softmax layout: one thread per query row and 128 key columns (8 softmax
-// warps), or -- with HGA_FWD_SPLIT -- two threads per row, 64 columns each (16
-// softmax warps, four per scheduler), exchanging the row maximum per tile
-// through shared memory.
-#ifndef HGA_FWD_SPLIT
-#define HGA_FWD_SPLIT 0
-#endif
-constexpr bool kFwdSplit = HGA_FWD_SPLIT != 0;
-constexpr int kSoftWarps = kFwdSplit ? 16 : 8;
-constexpr int kFwdThreads = (kSoftWarps + 2) * 32;
-constexpr int kProducerWarp = kSoftWarps, kMmaWarp = kSoftWarps + 1;
-constexpr int kStages = kFwdSplit ? 4 : 5;    // K/V ring slots
+constexpr int kStages = 5;                    // K/V ring slots
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 // Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
@@ -60,7 +49,6 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units
 #define HGA_FWD_POLY 0x0u
 #endif
 constexpr uint32_t kFwdPolyPairs = HGA_FWD_POLY;
-
 
 struct FwdCtl {
   uint64_t q_full;
@@ -74,9 +62,6 @@ struct FwdCtl {
   int abort;
   int nt;
   int tiles[kMaxTiles];  // >= 0: history block; < 0: segment block -(t+1)
-  // split softmax only: row maxima [tile parity][head][half][row], row sums [head][half][row]
-  float red_max[2][2][2][kFwdSplit ? 128 : 1];
-  float red_l[2][2][kFwdSplit ? 128 : 1];
 };
 
 // Head dim d in {64, 128}: a Q, K or V tile is 128 rows x d bf16 (d/64 boxes).
@@ -94,7 +79,7 @@ struct FwdArgs {
 };
 
 template <int KD>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                   const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kh,
                   const __grid_constant__ CUtensorMap tm_vh, const FwdArgs a) {
@@ -140,7 +125,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       for (int t = 0; t < 2; ++t) {
         mbar_init(&ctl->s_full[t], 1);
-        mbar_init(&ctl->p_full[t], kSoftWarps / 2 * 32);
+        mbar_init(&ctl->p_full[t], 128);
         mbar_init(&ctl->o_full[t], 1);
       }
       mbar_init(&ctl->mma_done, 1);
@@ -157,7 +142,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int nt = ctl->nt;
   volatile int* abort = &ctl->abort;
 
-  if (warp == kProducerWarp) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -197,7 +182,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int pos = issued - kStages > 0 ? issued - kStages : 0; pos < issued; ++pos)
         mbar_wait(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, &no_abort, a.err);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);  // Q, K both K-major
@@ -271,119 +256,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       umma_commit(&ctl->mma_done);
       volatile int no_abort = 0;
       mbar_wait(&ctl->mma_done, 0, &no_abort, a.err);
-    }
-  } else if (kFwdSplit) {
-    // ------------------------------------------------------------ softmax, two threads per row
-    const int t = warp >> 3, half = (warp >> 2) & 1, wq = warp & 3;
-    const int r = wq * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128 + 64 * half;
-    const uint32_t tO = tmem + lane_off + 256 + t * 128 + (kD / 2) * half;
-    const int bar_id = 1 + t * 4 + wq;  // the two warps that share these rows
-    const float sl2 = a.sl2;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    uint32_t v[64];
-    for (int j = 0; j < nt; ++j) {
-      // Both warps of a row pair take the same branch: each contributes its
-      // wait's outcome to one barrier-with-AND (which also publishes the
-      // row-max halves), so neither can wait at a barrier the other has left.
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&ctl->s_full[t], j & 1, abort, a.err));
-      if (got) {
-        tc_fence_after();
-        tmem_ld32x2_wait(tS, tS + 32, v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) v[e] = 0xFF800000u;
-      }
-      if (j == nt - 1) {
-#pragma unroll
-        for (int e = 0; e < 64; ++e)
-          if (64 * half + e > r) v[e] = 0xFF800000u;  // -inf
-      }
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int e = 0; e < 64; e += 2)
-        m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-      const float mh = max3f(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
-      ctl->red_max[j & 1][t][half][r] = mh;
-      uint32_t both;
-      asm volatile(
-          "{\n\t.reg .pred pin, pout;\n\t"
-          "setp.ne.u32 pin, %1, 0;\n\t"
-          "bar.red.and.pred pout, %2, 64, pin;\n\t"
-          "selp.u32 %0, 1, 0, pout;\n\t}\n"
-          : "=r"(both)
-          : "r"(got ? 1u : 0u), "r"(bar_id)
-          : "memory");
-      if (!both) {
-        ok = false;
-        break;
-      }
-      const float mx = fmaxf(mh, ctl->red_max[j & 1][t][half ^ 1][r]);
-      const bool need = mx > m_ref + kRescaleThreshold;
-      const bool any_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.0f;
-      if (need) {
-        alpha = ex2_approx(m_ref - mx);
-        l *= alpha;
-        m_ref = mx;
-      }
-      const float2 s2 = make_float2(sl2, sl2), nm = make_float2(-m_ref, -m_ref);
-      float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 x = fma2(make_float2(__uint_as_float(v[c * 32 + e]), __uint_as_float(v[c * 32 + e + 1])), s2, nm);
-          const float2 p = exp2_pair(x, (kFwdPolyPairs >> (e >> 1)) & 1u);
-          l2[(e >> 1) & 1] = add2(l2[(e >> 1) & 1], p);
-          pk[e >> 1] = pack_bf16x2(p.x, p.y);
-        }
-        HGA_TMEM_ST16(tS + c * 32, pk);
-      }
-      l += (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
-      if (any_need && j > 0) {
-#pragma unroll
-        for (int c = 0; c < kD / 64; ++c) {
-          uint32_t ov[32];
-          HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          HGA_TMEM_ST32(tO + c * 32, ov);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&ctl->p_full[t]);
-    }
-    // the row's sum: the two halves' partial sums (same reference maximum)
-    ctl->red_l[t][half][r] = l;
-    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-    l += ctl->red_l[t][half ^ 1][r];
-    if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->o_full[t], 0, abort, a.err))) {
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const int p = i * kBM + r;
-      const int hq = hq0 + t;
-      __nv_bfloat16* orow = a.o + (((size_t)b * a.S + p) * a.Hq + hq) * kD + (kD / 2) * half;
-#pragma unroll
-      for (int c = 0; c < kD / 64; ++c) {
-        uint32_t ov[32];
-        HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(ov[8 * qd + 0]) * inv_l, __uint_as_float(ov[8 * qd + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(ov[8 * qd + 2]) * inv_l, __uint_as_float(ov[8 * qd + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(ov[8 * qd + 4]) * inv_l, __uint_as_float(ov[8 * qd + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(ov[8 * qd + 6]) * inv_l, __uint_as_float(ov[8 * qd + 7]) * inv_l);
-          dst[qd] = w;
-        }
-      }
-      if (half == 0) a.lse[((size_t)b * a.Hq + hq) * a.S + p] = (m_ref + log2f(l)) * 0.6931471805599453f;
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
@@ -508,7 +380,7 @@ cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
   a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err;
   a.withhold_kv = withhold_kv ? 1 : 0;
   const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
-  fwd_tc_kernel<KD><<<grid, kFwdThreads, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
+  fwd_tc_kernel<KD><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
   return cudaGetLastError();
 }
 
