@@ -209,21 +209,21 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp: one elected lane issues
       constexpr uint32_t kIdS = idesc_bf16(kB, kB, false, false);  // [128 q x 128 keys] = Q K^T, dO V^T
       constexpr uint32_t kIdQ = idesc_bf16(kB, kD, false, true);   // dQ += dS (tmem) K (MN-major)
       // Descriptors built once; k-steps and ring slots are constant adds.
       const uint64_t dQd = sdesc_sw128(smem_u32(sQ), 16, 1024), dOd = sdesc_sw128(smem_u32(sDO), 16, 1024);
       const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024), dVk = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dKmn = sdesc_sw128(smem_u32(sK), kHalf, 1024);  // K as the MN-major B of dQ += dS K
-      auto wait_k = [=](int j) { return mbar_wait(&ctl->k_full[j % kKStages], (j / kKStages) & 1, abort, a.err); };
-      auto wait_v = [=](int j) { return mbar_wait(&ctl->v_full[j % kVStages], (j / kVStages) & 1, abort, a.err); };
+      auto wait_k = [=](int j) { return mbar_wait_w(&ctl->k_full[j % kKStages], (j / kKStages) & 1, abort, a.err); };
+      auto wait_v = [=](int j) { return mbar_wait_w(&ctl->v_full[j % kVStages], (j / kVStages) & 1, abort, a.err); };
       auto issue_s = [=](int j) {  // S(j) = Q K_j^T into buffer j % 2
         const uint64_t kb = dKk + sdesc_units((j % kKStages) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
-          umma_ss(tmem + kDqS + (j & 1) * 128, dQd + off, kb + off, kIdS, kk > 0);
+          umma_ss_w(tmem + kDqS + (j & 1) * 128, dQd + off, kb + off, kIdS, kk > 0);
         }
       };
       auto issue_dp = [=](int j) {  // dP(j) = dO V_j^T
@@ -231,12 +231,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
-          umma_ss(tmem + kDqP, dOd + off, vb + off, kIdS, kk > 0);
+          umma_ss_w(tmem + kDqP, dOd + off, vb + off, kIdS, kk > 0);
         }
-        umma_commit(&ctl->sdp_full[j & 1]);           // S(j) was issued earlier: both ready
-        umma_commit(&ctl->v_empty[j % kVStages]);     // V_j's only reader
+        umma_commit_w(&ctl->sdp_full[j & 1]);           // S(j) was issued earlier: both ready
+        umma_commit_w(&ctl->v_empty[j % kVStages]);     // V_j's only reader
       };
-      bool ok = mbar_wait(&ctl->qdo_full, 0, abort, a.err) && wait_k(0) && wait_v(0);
+      bool ok = mbar_wait_w(&ctl->qdo_full, 0, abort, a.err) && wait_k(0) && wait_v(0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -252,30 +252,30 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; ok && j < nt; ++j) {
         if (j + 1 < nt) {
           // dP(j+1) as soon as the dS pass has read dP(j)
-          if (!mbar_wait(&ctl->dp_free, j & 1, abort, a.err) || !wait_v(j + 1)) break;
+          if (!mbar_wait_w(&ctl->dp_free, j & 1, abort, a.err) || !wait_v(j + 1)) break;
           tc_fence_after();
           issue_dp(j + 1);
         }
-        if (!mbar_wait(&ctl->ds_full[j & 1], (j >> 1) & 1, abort, a.err)) break;
+        if (!mbar_wait_w(&ctl->ds_full[j & 1], (j >> 1) & 1, abort, a.err)) break;
         tc_fence_after();
         const uint64_t kb = dKmn + sdesc_units((j % kKStages) * kTileBytes);
         const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kB / 16; ++kk)
-          umma_ts(tmem + kDqAcc, tmem + kDqS + (j & 1) * 128 + packed_col(kk), kb + sdesc_units(kk * 2048), kIdQ,
+          umma_ts_w(tmem + kDqAcc, tmem + kDqS + (j & 1) * 128 + packed_col(kk), kb + sdesc_units(kk * 2048), kIdQ,
                   kk > 0 ? 1u : acc0);
-        umma_commit(&ctl->k_empty[j % kKStages]);  // K_j's last reader
+        umma_commit_w(&ctl->k_empty[j % kKStages]);  // K_j's last reader
         if (j + 2 < nt) {
           if (!wait_k(j + 2)) break;
           tc_fence_after();
           issue_s(j + 2);  // into buffer j % 2, after dQ(j) read dS(j) from it
         }
-        if (j == nt - 1) umma_commit(&ctl->dq_full);
+        if (j == nt - 1) umma_commit_w(&ctl->dq_full);
       }
       // All issued MMAs must finish before tensor memory is released.
-      umma_commit(&ctl->mma_done);
+      umma_commit_w(&ctl->mma_done);
       volatile int no_abort = 0;
-      mbar_wait(&ctl->mma_done, 0, &no_abort, a.err);
+      mbar_wait_w(&ctl->mma_done, 0, &no_abort, a.err);
     }
   } else {
     // ------------------------------------------------------------ dS pass
@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp: one elected lane issues
       constexpr uint32_t kIdT = idesc_bf16(kB, kSubRows, false, false);  // [128 keys x 64 queries]
       constexpr uint32_t kIdG = idesc_bf16(kB, kD, false, true);         // dV += P^T dO_half, dK += dS^T Q_half
       // Descriptors built once; k-steps, query halves and stages are constant adds.
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(320, 1)
       auto issue_sdp = [=](int u) -> bool {
         const int it = u >> 1, h = u & 1, s = it % kQStages;
         if (h == 0) {
-          if (!mbar_wait(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err)) return false;
+          if (!mbar_wait_w(&ctl->qd_full[s], (it / kQStages) & 1, abort, a.err)) return false;
           tc_fence_after();
         }
         const uint32_t so = sdesc_units(s * kTileBytes + h * kSubOff);
@@ -478,45 +478,45 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
-          umma_ss(ts, dKd + off, qb + off, kIdT, kk > 0);
+          umma_ss_w(ts, dKd + off, qb + off, kIdT, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
-          umma_ss(tp, dVd + off, ob + off, kIdT, kk > 0);
+          umma_ss_w(tp, dVd + off, ob + off, kIdT, kk > 0);
         }
-        umma_commit(&ctl->sdp_full[h]);
+        umma_commit_w(&ctl->sdp_full[h]);
         return true;
       };
-      bool ok = mbar_wait(&ctl->kv_full, 0, abort, a.err);
+      bool ok = mbar_wait_w(&ctl->kv_full, 0, abort, a.err);
       if (ok) {
         tc_fence_after();
         ok = issue_sdp(0) && issue_sdp(1);
       }
       for (int u = 0; ok && u < nsub; ++u) {
         const int it = u >> 1, h = u & 1, s = it % kQStages;
-        if (!mbar_wait(&ctl->pds_full[h], (u >> 1) & 1, abort, a.err)) break;
+        if (!mbar_wait_w(&ctl->pds_full[h], (u >> 1) & 1, abort, a.err)) break;
         tc_fence_after();
         const uint32_t so = sdesc_units(s * kTileBytes + h * kSubOff);
         const uint64_t qb = dQmn + so, ob = dOmn + so;
         const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kSubRows / 16; ++kk)  // dV += P^T dO_half
-          umma_ts(tmem + kKvDV, tmem + kKvS + h * 64 + packed_col(kk), ob + sdesc_units(kk * 2048), kIdG,
+          umma_ts_w(tmem + kKvDV, tmem + kKvS + h * 64 + packed_col(kk), ob + sdesc_units(kk * 2048), kIdG,
                   kk > 0 ? 1u : acc0);
 #pragma unroll
         for (int kk = 0; kk < kSubRows / 16; ++kk)  // dK += dS^T Q_half
-          umma_ts(tmem + kKvDK, tmem + kKvP + h * 64 + packed_col(kk), qb + sdesc_units(kk * 2048), kIdG,
+          umma_ts_w(tmem + kKvDK, tmem + kKvP + h * 64 + packed_col(kk), qb + sdesc_units(kk * 2048), kIdG,
                   kk > 0 ? 1u : acc0);
-        if (h == 1) umma_commit(&ctl->qd_empty[s]);
+        if (h == 1) umma_commit_w(&ctl->qd_empty[s]);
         if (u + 2 < nsub) {
           if (!issue_sdp(u + 2)) break;
         }
-        if (u == nsub - 1) umma_commit(&ctl->dkv_full);
+        if (u == nsub - 1) umma_commit_w(&ctl->dkv_full);
       }
-      umma_commit(&ctl->mma_done);
+      umma_commit_w(&ctl->mma_done);
       volatile int no_abort = 0;
-      mbar_wait(&ctl->mma_done, 0, &no_abort, a.err);
+      mbar_wait_w(&ctl->mma_done, 0, &no_abort, a.err);
     }
   } else {
     // ------------------------------------------------------------ P^T / dS^T pass

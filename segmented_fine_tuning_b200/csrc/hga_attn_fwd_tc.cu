@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp: one elected lane issues
       constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);  // Q, K both K-major
       constexpr uint32_t kIdO = idesc_bf16(kBM, kD, false, true);    // P (tmem) x V (MN-major)
       // Descriptors are built once; every k-step and ring slot is a constant
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
-          umma_ss(tmem + t * 128, a0 + off, b0 + off, kIdS, kk > 0);
+          umma_ss_w(tmem + t * 128, a0 + off, b0 + off, kIdS, kk > 0);
         }
       };
       auto issue_PV = [=](int t, int s, bool acc) {
@@ -208,54 +208,54 @@ __global__ void __launch_bounds__(384, 1)
         for (int kk = 0; kk < kBN / 16; ++kk) {
           // P chunk c (keys 32c..32c+31) sits at S columns [32c, 32c+16).
           const uint32_t pcol = (kk >> 1) * 32 + (kk & 1) * 8;
-          umma_ts(tmem + 256 + t * 128, tmem + t * 128 + pcol, b0 + sdesc_units(kk * 2048), kIdO,
+          umma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + pcol, b0 + sdesc_units(kk * 2048), kIdO,
                   kk > 0 ? 1u : acc0);
         }
       };
       auto wait_full = [=](int pos) {
-        return mbar_wait(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, abort, a.err);
+        return mbar_wait_w(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, abort, a.err);
       };
-      bool ok = mbar_wait(&ctl->q_full, 0, abort, a.err) && wait_full(0);
+      bool ok = mbar_wait_w(&ctl->q_full, 0, abort, a.err) && wait_full(0);
       if (ok) {
         tc_fence_after();
         issue_S(0, 0);
-        umma_commit(&ctl->s_full[0]);
+        umma_commit_w(&ctl->s_full[0]);
         issue_S(1, 0);
-        umma_commit(&ctl->s_full[1]);
-        umma_commit(&ctl->kv_empty[0]);
+        umma_commit_w(&ctl->s_full[1]);
+        umma_commit_w(&ctl->kv_empty[0]);
         for (int j = 0; j < nt; ++j) {
           const int sV = (2 * j + 1) % kStages;
           const int sK = (2 * j + 2) % kStages;
           const bool more = j + 1 < nt;
           if (!wait_full(2 * j + 1)) break;
-          if (!mbar_wait(&ctl->p_full[0], j & 1, abort, a.err)) break;
+          if (!mbar_wait_w(&ctl->p_full[0], j & 1, abort, a.err)) break;
           tc_fence_after();
           issue_PV(0, sV, j > 0);
           if (more) {
             if (!wait_full(2 * j + 2)) break;
             tc_fence_after();
             issue_S(0, sK);
-            umma_commit(&ctl->s_full[0]);
+            umma_commit_w(&ctl->s_full[0]);
           } else {
-            umma_commit(&ctl->o_full[0]);
+            umma_commit_w(&ctl->o_full[0]);
           }
-          if (!mbar_wait(&ctl->p_full[1], j & 1, abort, a.err)) break;
+          if (!mbar_wait_w(&ctl->p_full[1], j & 1, abort, a.err)) break;
           tc_fence_after();
           issue_PV(1, sV, j > 0);
-          umma_commit(&ctl->kv_empty[sV]);
+          umma_commit_w(&ctl->kv_empty[sV]);
           if (more) {
             issue_S(1, sK);
-            umma_commit(&ctl->s_full[1]);
-            umma_commit(&ctl->kv_empty[sK]);
+            umma_commit_w(&ctl->s_full[1]);
+            umma_commit_w(&ctl->kv_empty[sK]);
           } else {
-            umma_commit(&ctl->o_full[1]);
+            umma_commit_w(&ctl->o_full[1]);
           }
         }
       }
       // All issued MMAs must finish before tensor memory is released.
-      umma_commit(&ctl->mma_done);
+      umma_commit_w(&ctl->mma_done);
       volatile int no_abort = 0;
-      mbar_wait(&ctl->mma_done, 0, &no_abort, a.err);
+      mbar_wait_w(&ctl->mma_done, 0, &no_abort, a.err);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
