@@ -326,7 +326,11 @@ HGA_API hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const 
  * dtype, of which the first n_hist_blocks blocks are valid.  idx_dev:
  * device idx from hga_select_topk.  The call
  *   1. copies idx to the host on compute_stream (after the work already
- *      queued there) and waits for it, at most timeout_ms;
+ *      queued there) and waits for it, at most timeout_ms.  Pinned scratch
+ *      mapped into the device (any cudaHostAlloc / cudaHostRegister memory
+ *      with unified addressing) is written by a small kernel through that
+ *      mapping, so the copy does not wait behind large device-to-host copies
+ *      queued on other streams; other host memory takes cudaMemcpyAsync;
  *   2. forms the sorted set of distinct selected blocks (at most pool_slots);
  *   3. on copy_stream, ordered after that idx copy (so after every kernel
  *      queued on compute_stream before the call), copies each of those

@@ -440,6 +440,25 @@ hga_status hga_attn_bwd_noalloc(const hga_dims* dims, const void* q, const void*
                  kNoAllocScratchFloats * sizeof(float), true, hga::kBwdDq | hga::kBwdDkdv, stream);
 }
 
+namespace {
+// The selection's idx into the caller's host scratch, queued on `st`.  Pinned
+// scratch mapped into the device is written by a small kernel (SM stores over
+// the host link), so this transfer does not wait in the device-to-host copy
+// queue behind large copies queued earlier on other streams (the offload of a
+// finished segment to the host tier); other host memory takes a copy.
+hga_status idx_to_host(const int32_t* idx_dev, int32_t* host_scratch, size_t n, cudaStream_t st) {
+  cudaPointerAttributes at;
+  cudaError_t e = cudaPointerGetAttributes(&at, host_scratch);
+  if (e != cudaSuccess) cudaGetLastError();  // memory CUDA does not know: plain pageable host memory
+  if (e == cudaSuccess && at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
+    e = hga::launch_store_mapped_i32(idx_dev, static_cast<int32_t*>(at.devicePointer), n, st);
+    return e == cudaSuccess ? HGA_OK : cuda_fail(e, "idx store to host");
+  }
+  e = cudaMemcpyAsync(host_scratch, idx_dev, n * sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+  return e == cudaSuccess ? HGA_OK : cuda_fail(e, "idx copy to host");
+}
+}  // namespace
+
 hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void* host_v, int host_capacity_blocks,
                             const int32_t* idx_dev,
                             int32_t* host_idx_scratch, void* pool_k, void* pool_v, int pool_slots,
@@ -468,9 +487,7 @@ hga_status hga_fetch_blocks(const hga_dims* dims, const void* host_k, const void
   //    the wait does not queue behind earlier block copies on copy_stream);
   //    the copies below are ordered after it, hence after every kernel queued
   //    on the compute stream so far.
-  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, cst)) !=
-      cudaSuccess)
-    return cuda_fail(e, "idx copy to host");
+  if ((r = idx_to_host(idx_dev, host_idx_scratch, n_idx, cst)) != HGA_OK) return r;
   if ((e = cudaEventRecord(landed, cst)) != cudaSuccess) return cuda_fail(e, "event record");
   if ((e = cudaStreamWaitEvent(xst, landed, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
   const auto t0 = std::chrono::steady_clock::now();
@@ -617,9 +634,7 @@ hga_status hga_fetch_blocks_cached(const hga_dims* dims, const void* host_k, con
   // 1. idx -> host on the compute stream, after the work queued there; the
   //    pool copies on copy_stream are ordered after it, hence after every
   //    kernel that may still read the pool slots they overwrite.
-  if ((e = cudaMemcpyAsync(host_idx_scratch, idx_dev, n_idx * sizeof(int32_t), cudaMemcpyDeviceToHost, cst)) !=
-      cudaSuccess)
-    return cuda_fail(e, "idx copy to host");
+  if ((r = idx_to_host(idx_dev, host_idx_scratch, n_idx, cst)) != HGA_OK) return r;
   if ((e = cudaEventRecord(landed, cst)) != cudaSuccess) return cuda_fail(e, "event record");
   if ((e = cudaStreamWaitEvent(xst, landed, 0)) != cudaSuccess) return cuda_fail(e, "stream wait");
   const auto t0 = std::chrono::steady_clock::now();

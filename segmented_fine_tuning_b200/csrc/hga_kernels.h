@@ -54,6 +54,9 @@ int gather_max_blocks();
 cudaError_t launch_gather_mapped(const Shape& s, const int32_t* idx, const void* host_k_dev, const void* host_v_dev,
                                  int host_cap, void* pool_k, void* pool_v, int pool_slots, int32_t* idx_pool,
                                  int* err, int n_sm, cudaStream_t st);
+// dst_dev_view[0..n) = src[0..n) (int32), dst being pinned host memory seen
+// through its device mapping: a device-to-host transfer by SM stores.
+cudaError_t launch_store_mapped_i32(const int32_t* src, int32_t* dst_dev_view, size_t n, cudaStream_t st);
 // D[b,hq,p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k]  (fp32)
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st);
 

@@ -840,4 +840,25 @@ cudaError_t launch_gather_mapped(const Shape& s, const int32_t* idx, const void*
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- idx to host
+// n int32 words from device memory into pinned host memory mapped into the
+// device (dst is the device view), by SM stores.  A transfer this small then
+// never waits in a copy engine's queue behind large copies of the same
+// direction (a finished segment's K/V going to the host tier).  Each thread
+// fences at system scope before it exits, so the words are visible to the host
+// once the stream has passed the kernel.
+__global__ void __launch_bounds__(256) store_mapped_i32_kernel(const int32_t* __restrict__ src, int32_t* dst,
+                                                               size_t n) {
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (size_t)gridDim.x * blockDim.x)
+    dst[k] = __ldg(src + k);
+  __threadfence_system();
+}
+
+cudaError_t launch_store_mapped_i32(const int32_t* src, int32_t* dst_dev_view, size_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, 32);
+  store_mapped_i32_kernel<<<blocks, 256, 0, st>>>(src, dst_dev_view, n);
+  return cudaGetLastError();
+}
+
 }  // namespace hga

@@ -16,11 +16,14 @@ Per segment s (history = segments 0..s-1, 16 blocks each at 2,048 tokens):
                             first) -> attention forward
   backward, layers L-1..0:  attention backward on the same pool (kept from the
                             forward; no second fetch)
+  after the forward, every layer: the segment's K/V (final once the layer's
+                            forward has run) copied to the host tier on a
+                            side stream, so the copies cross the host link
+                            during the backward, when it carries nothing else
   segment end, every layer: one pass over the segment's K/V
                             (hga_append_segment): summaries of its blocks
-                            appended to the resident array, the blocks copied
-                            into the layer's device cache, and K/V copied to
-                            the host tier on a side stream
+                            appended to the resident array and the blocks
+                            copied into the layer's device cache
 Every step is a libhga.so call; this module owns buffers, streams and order.
 Batch size 1 (one sequence): the resident summary array of a layer grows as a
 prefix, which is a valid summary array of the current history for B = 1.
@@ -30,7 +33,7 @@ from __future__ import annotations
 import torch
 
 from ._binding import (BlockCache, Dims, hga_append_segment, hga_attn_bwd, hga_attn_bwd_workspace_size,
-                       hga_attn_fwd, hga_fetch_blocks_cached, hga_remap_idx, hga_select_topk)
+                       hga_attn_fwd, hga_fetch_blocks_cached, hga_offload_segment, hga_remap_idx, hga_select_topk)
 
 
 class SegmentedPass:
@@ -86,6 +89,7 @@ class SegmentedPass:
         self.copy_stream = torch.cuda.Stream(self.device)
         self.offload_stream = torch.cuda.Stream(self.device)
         self.sel_stream = torch.cuda.Stream(self.device, priority=-1)
+        self.slots_stale = [False] * n_layers  # slot_dev[l] lags the host cache state
         self.ready = [torch.cuda.Event() for _ in range(n_layers)]
         self.offloaded = [torch.cuda.Event() for _ in range(n_layers)]
         for ev in self.done:
@@ -100,6 +104,7 @@ class SegmentedPass:
         for c, d in zip(self.cache, self.slot_dev):
             c.reset()
             d.fill_(-1)
+        self.slots_stale = [False] * self.L
 
     def dims(self, s: int) -> Dims:
         return self.seg.with_history(s * self.nqb)
@@ -108,15 +113,24 @@ class SegmentedPass:
         return self.pool_slots if s > 0 else 0
 
     # ------------------------------------------------------------ steps
-    def stage(self, s: int, l: int, q, stream) -> torch.cuda.Event:
+    def stage(self, s: int, l: int, q, stream) -> list[torch.cuda.Event]:
         """Selection of (segment s, layer l) and the history it needs in the
         layer's pool: queued on `stream` (the block copies on the copy
-        stream).  Returns the event the forward must wait for."""
+        stream).  Returns the events the forward must wait for: the end of
+        the selection on `stream`, and the end of the copies on the copy
+        stream when blocks crossed the host link.  `stream` itself never
+        waits for the copies, so the selection of the next layer (and with
+        it the host's plan of the next copies) runs while they are in
+        flight, and the copy stream goes from one layer's blocks to the
+        next without a gap."""
         D = self.dims(s)
         hga_select_topk(D, q, self.summ[l], self.idx[l], None, stream)
+        waits = []
         if s > 0:
             if (self.cache[l].slot_of_block[: s * self.nqb] >= 0).all():
                 # every selectable block is resident: slots on the device, no host round trip
+                if self.slots_stale[l]:
+                    self._sync_slots(l, stream)
                 hga_remap_idx(D, self.idx[l], self.slot_dev[l], self.idx_pool[l], stream)
                 self.fetched_blocks.append(0)
                 self.device_remaps += 1
@@ -128,19 +142,21 @@ class SegmentedPass:
                                                  stream, self.copy_stream, self.done[l], self.timeout)
                 self.selected_blocks.append(nu)
                 self.fetched_blocks.append(nf)
-                self._sync_slots(l, stream)
-                stream.wait_event(self.done[l])
+                self.slots_stale[l] = True
+                waits.append(self.done[l])
         self.ready[l].record(stream)
-        return self.ready[l]
+        return [self.ready[l]] + waits
 
-    def forward(self, s: int, l: int, q, k_seg, v_seg, ready: torch.cuda.Event | None = None):
+    def forward(self, s: int, l: int, q, k_seg, v_seg, ready: list[torch.cuda.Event] | None = None):
         """Attention forward of (segment s, layer l); stages the selection
-        and fetch first unless `ready` says they are already queued."""
+        and fetch first unless `ready` (the events stage() returned) says
+        they are already queued."""
         D = self.dims(s)
         st = torch.cuda.current_stream(self.device)
         if ready is None:
             ready = self.stage(s, l, q, st)
-        st.wait_event(ready)
+        for ev in ready:
+            st.wait_event(ev)
         if s > 0:
             hga_attn_fwd(D, q, k_seg, v_seg, self.pool_k[l], self.pool_v[l], self.pool_slots, self.idx_pool[l],
                          self.o[l], self.lse[l], st)
@@ -159,29 +175,48 @@ class SegmentedPass:
                          self.dk, self.dv, self.ws, st)
         return self.dq, self.dk, self.dv
 
-    def end_segment(self, s: int, l: int, k_seg, v_seg):
-        """Append the segment's blocks in one pass over its K and V: summaries
-        on the device, the blocks into the layer's device cache (unless
-        keep_new_blocks is off), and K/V to the host tier on the side stream
-        (ordered after the work queued so far)."""
+    def offload(self, s: int, l: int, k_seg, v_seg):
+        """Copy the segment's K/V of layer l to the host tier on the offload
+        stream, ordered after the work queued so far (they are final once the
+        layer's forward has been queued)."""
         st = torch.cuda.current_stream(self.device)
-        cache = self.cache[l] if (self.keep_new_blocks and s + 1 < self.NS) else None
-        hga_append_segment(self.seg.with_history(self.cap), k_seg, v_seg, s * self.nqb, self.summ[l],
-                           self.pool_k[l], self.pool_v[l], cache, self.tier_k[l], self.tier_v[l], self.cap, st,
-                           self.offload_stream)
+        self.offload_stream.wait_stream(st)
+        hga_offload_segment(self.seg, k_seg, v_seg, self.tier_k[l], self.tier_v[l], self.cap, s * self.nqb,
+                            self.offload_stream)
         self.offloaded[l].record(self.offload_stream)
-        if cache is not None:
-            self._sync_slots(l, st)
         # the caller may release k_seg/v_seg once the offload stream has passed here
         k_seg.record_stream(self.offload_stream)
         v_seg.record_stream(self.offload_stream)
 
+    def end_segment(self, s: int, l: int, k_seg, v_seg, offloaded: bool = False):
+        """Append the segment's blocks in one pass over its K and V: summaries
+        on the device, the blocks into the layer's device cache (unless
+        keep_new_blocks is off), and -- unless `offloaded` says offload() has
+        queued it already -- K/V to the host tier on the side stream (ordered
+        after the work queued so far)."""
+        st = torch.cuda.current_stream(self.device)
+        cache = self.cache[l] if (self.keep_new_blocks and s + 1 < self.NS) else None
+        tier = (None, None) if offloaded else (self.tier_k[l], self.tier_v[l])
+        hga_append_segment(self.seg.with_history(self.cap), k_seg, v_seg, s * self.nqb, self.summ[l],
+                           self.pool_k[l], self.pool_v[l], cache, tier[0], tier[1], self.cap, st,
+                           self.offload_stream)
+        if not offloaded:
+            self.offloaded[l].record(self.offload_stream)
+            k_seg.record_stream(self.offload_stream)
+            v_seg.record_stream(self.offload_stream)
+        if cache is not None:
+            self.slots_stale[l] = True
+
     def _sync_slots(self, l: int, st) -> None:
         """Device copy of layer l's slot map, queued on st (a fresh pinned
-        staging buffer each time, so a pending copy is never overwritten)."""
+        staging buffer each time, so a pending copy is never overwritten).
+        Done only when a device remap is about to read it, so steps that
+        take the host path queue no extra transfer behind their block
+        copies."""
         staged = torch.from_numpy(self.cache[l].slot_of_block[: self.cap].copy()).pin_memory()
         with torch.cuda.stream(st):
             self.slot_dev[l].copy_(staged, non_blocking=True)
+        self.slots_stale[l] = False
 
     def run_segment(self, s: int, inputs, on_step=None):
         """inputs[l] = (q, k_seg, v_seg, d_o) device tensors of layer l for
@@ -200,10 +235,13 @@ class SegmentedPass:
                 ready = self.stage(s, l + 1, inputs[l + 1][0], self.sel_stream)
             if on_step:
                 on_step(s, l, "fwd")
+        # every layer's K/V is final: the tier copies run during the backward
+        for l in range(self.L):
+            self.offload(s, l, inputs[l][1], inputs[l][2])
         for l in reversed(range(self.L)):
             q, k, v, do = inputs[l]
             self.backward(s, l, q, k, v, do)
             if on_step:
                 on_step(s, l, "bwd")
         for l in range(self.L):
-            self.end_segment(s, l, inputs[l][1], inputs[l][2])
+            self.end_segment(s, l, inputs[l][1], inputs[l][2], offloaded=True)
