@@ -222,28 +222,28 @@ def run_device(args, rank, world, device, w=None, steps=None):
     stream = torch.cuda.current_stream(device)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
 
-    def step(evs=None):
+    def step(evs=None, s=stream):
         def mark(k):
             if evs is not None:
-                evs[k].record(stream)
+                evs[k].record(s)
         mark(0)
-        hga.hga_block_summaries(D, dev["k_hist"], 0, D.n_hist_blocks, st.summ, stream)
+        hga.hga_block_summaries(D, dev["k_hist"], 0, D.n_hist_blocks, st.summ, s)
         mark(1)
-        hga.hga_select_topk(D, dev["q"], st.summ, st.idx, None, stream)
+        hga.hga_select_topk(D, dev["q"], st.summ, st.idx, None, s)
         mark(2)
         hga.hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], D.n_hist_blocks,
-                         st.idx, st.o, st.lse, stream)
+                         st.idx, st.o, st.lse, s)
         mark(3)
         if not w.fwd_only:
-            hga.hga_attn_bwd_preprocess(D, st.o, dev["d_o"], st.ws, stream)
+            hga.hga_attn_bwd_preprocess(D, st.o, dev["d_o"], st.ws, s)
         mark(4)
         if not w.fwd_only:
             hga.hga_attn_bwd_dkdv(D, dev["q"], dev["k_seg"], dev["v_seg"], st.lse, dev["d_o"], st.ws, st.dk, st.dv,
-                                  stream)
+                                  s)
         mark(5)
         if not w.fwd_only:
             hga.hga_attn_bwd_dq(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"],
-                                D.n_hist_blocks, st.idx, st.lse, dev["d_o"], st.ws, st.dq, stream)
+                                D.n_hist_blocks, st.idx, st.lse, dev["d_o"], st.ws, st.dq, s)
         mark(6)
 
     for _ in range(args.warmup):
@@ -272,7 +272,36 @@ def run_device(args, rank, world, device, w=None, steps=None):
         step_ms.append(e[0].elapsed_time(e[6]))
         for j, name in enumerate(KERNELS):
             per_kernel[name].append(e[j].elapsed_time(e[j + 1]))
-    total_ms = max_over_ranks(float(sum(step_ms)), world, device)
+    eager_ms = max_over_ranks(float(sum(step_ms)), world, device) / steps
+
+    # The same step captured once as a CUDA graph and replayed: the kernels
+    # and their arguments are identical, but no host work (argument checks,
+    # tensor-map encoding, launch calls) sits between them on the timeline.
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(graph, stream=cap, capture_error_mode="relaxed"):
+        step(s=cap)
+    stream.wait_stream(cap)
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as gclk:
+        for e0, e1 in gev:
+            flush.zero_()
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    hga.hga_device_status(stream)
+    del graph
+    total_ms = max_over_ranks(float(sum(e0.elapsed_time(e1) for e0, e1 in gev)), world, device)
     ms_per_step = total_ms / steps
     value = job_throughput(world, w.S, ms_per_step)
 
@@ -314,8 +343,12 @@ def run_device(args, rank, world, device, w=None, steps=None):
                                                       peaks["bf16_tflops"], 3),
                               "algorithmic_gflop": round(fwd_bwd_flops / 1e9, 2)},
         "kernels": kern,
+        "launch": "the step replayed as one CUDA graph; per-kernel times from the same step launched eagerly "
+                  "with an event between kernels (small kernels' spans include their launch latency)",
+        "eager": {"ms_per_step": round(eager_ms, 4), "tokens_per_s": round(job_throughput(world, w.S, eager_ms), 1),
+                  "clocks": clk.summary()},
         "gpu_launches": (3 if w.fwd_only else 6) * steps,
-        "clocks": clk.summary(),
+        "clocks": gclk.summary(),
     }
     return out, (w, x, D, dev, st)
 

@@ -19,6 +19,36 @@
 #include "../../include/hga_selftest.h"
 #include "hga_kernels.h"
 
+namespace hga {
+cudaError_t smem_limit(const void* kernel, size_t bytes) {
+  struct Set {
+    const void* kernel;
+    int device;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Set> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Set& x : done)
+      if (x.kernel == kernel && x.device == dev && x.bytes >= bytes) return cudaSuccess;
+  }
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
+    return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Set& x : done)
+    if (x.kernel == kernel && x.device == dev) {
+      x.bytes = std::max(x.bytes, bytes);
+      return cudaSuccess;
+    }
+  done.push_back({kernel, dev, bytes});
+  return cudaSuccess;
+}
+}  // namespace hga
+
 namespace {
 
 thread_local char g_last_error[512] = "";

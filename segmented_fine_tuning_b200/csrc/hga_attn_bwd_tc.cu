@@ -602,10 +602,10 @@ cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
                        const uint8_t* qmask, float gscale) {
   constexpr size_t dq_smem = dq_smem_bytes(KD), kv_smem = dkdv_smem_bytes(KD);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(dq_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem)) !=
+  if ((e = smem_limit(reinterpret_cast<const void*>(dq_tc_kernel<KD>), dq_smem)) !=
       cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(dkdv_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem)) !=
+  if ((e = smem_limit(reinterpret_cast<const void*>(dkdv_tc_kernel<KD>), kv_smem)) !=
       cudaSuccess)
     return e;
   BwdArgs a;

@@ -372,7 +372,7 @@ template <int KD>
 cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse, int* err,
                        cudaStream_t st, bool withhold_kv) {
   constexpr size_t smem = fwd_smem_bytes(KD);
-  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<KD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_limit(reinterpret_cast<const void*>(fwd_tc_kernel<KD>), smem);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();

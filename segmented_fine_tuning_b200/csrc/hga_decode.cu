@@ -305,7 +305,7 @@ cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new
   if (s.bf16) {
     const size_t smem = dec_smem_bytes<__nv_bfloat16>(s.blk, s.d);
     auto kp = decode_partial_kernel<__nv_bfloat16>;
-    if ((e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    if ((e = smem_limit(reinterpret_cast<const void*>(kp), smem)) != cudaSuccess)
       return e;
     kp<<<grid, kDecThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q_new),
                                         static_cast<const __nv_bfloat16*>(k_seg),
@@ -317,7 +317,7 @@ cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new
   } else {
     const size_t smem = dec_smem_bytes<float>(s.blk, s.d);
     auto kp = decode_partial_kernel<float>;
-    if ((e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    if ((e = smem_limit(reinterpret_cast<const void*>(kp), smem)) != cudaSuccess)
       return e;
     kp<<<grid, kDecThreads, smem, st>>>(static_cast<const float*>(q_new), static_cast<const float*>(k_seg),
                                         static_cast<const float*>(v_seg), static_cast<const float*>(k_hist),

@@ -24,6 +24,12 @@ constexpr int kMaxSelectBlocks = 4096;
 // Longest segment (in query blocks) the tensor-core kernels handle.
 constexpr int kMaxQueryBlocks = 128;
 
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes), called
+// for a (kernel, device) pair only when `bytes` exceeds what was already set
+// there: the attribute persists, and setting it on every launch costs host
+// time that small kernels cannot hide.
+cudaError_t smem_limit(const void* kernel, size_t bytes);
+
 // Summaries of `nblocks` blocks: source blocks src_b0.. of k_src (T_src tokens
 // per batch) -> destination blocks dst_b0.. of summ [B, s.nblk, Hkv, d].
 cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src, int src_b0, int dst_b0, int nblocks,

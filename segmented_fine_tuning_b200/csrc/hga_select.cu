@@ -652,13 +652,13 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
   cudaError_t e;
   if (s.bf16) {
     auto kern = select_kernel<__nv_bfloat16>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    if ((e = smem_limit(reinterpret_cast<const void*>(kern), smem)) != cudaSuccess)
       return e;
     kern<<<grid, kSelThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk,
                                   s.topk, isd, idx, scores);
   } else {
     auto kern = select_kernel<float>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    if ((e = smem_limit(reinterpret_cast<const void*>(kern), smem)) != cudaSuccess)
       return e;
     kern<<<grid, kSelThreads, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk, s.topk,
                                   isd, idx, scores);
@@ -676,14 +676,12 @@ cudaError_t launch_decode_select(const Shape& s, int nq, const void* q_new, cons
     const dim3 grid((s.nblk + per_cta - 1) / per_cta, s.Hkv, s.B);
     const size_t smem = (size_t)s.G() * s.d * sizeof(float);
     if (s.bf16) {
-      if ((e = cudaFuncSetAttribute(decode_score_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem)) != cudaSuccess)
+      if ((e = smem_limit(reinterpret_cast<const void*>(decode_score_kernel<__nv_bfloat16>), smem)) != cudaSuccess)
         return e;
       decode_score_kernel<__nv_bfloat16><<<grid, kDecScoreWarps * 32, smem, st>>>(
           static_cast<const __nv_bfloat16*>(q_new), summ, nq, s.Hq, s.Hkv, s.d, s.nblk, isd, keys);
     } else {
-      if ((e = cudaFuncSetAttribute(decode_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem)) != cudaSuccess)
+      if ((e = smem_limit(reinterpret_cast<const void*>(decode_score_kernel<float>), smem)) != cudaSuccess)
         return e;
       decode_score_kernel<float><<<grid, kDecScoreWarps * 32, smem, st>>>(static_cast<const float*>(q_new), summ,
                                                                           nq, s.Hq, s.Hkv, s.d, s.nblk, isd, keys);
@@ -691,7 +689,7 @@ cudaError_t launch_decode_select(const Shape& s, int nq, const void* q_new, cons
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const size_t smem = (size_t)(s.nblk > 0 ? s.nblk : 1) * 8;
-  if ((e = cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+  if ((e = smem_limit(reinterpret_cast<const void*>(decode_topk_kernel), smem)) !=
       cudaSuccess)
     return e;
   decode_topk_kernel<<<dim3(s.Hkv, s.B), kSelThreads, smem, st>>>(keys, s.Hkv, s.nblk, s.topk, idx, scores);
@@ -831,7 +829,7 @@ cudaError_t launch_gather_mapped(const Shape& s, const int32_t* idx, const void*
   const int W = (s.nblk + 31) / 32;
   const size_t smem = (size_t)2 * (W > 0 ? W : 1) * sizeof(uint32_t);
   const size_t blk_bytes = (size_t)s.blk * s.Hkv * s.d * (s.bf16 ? 2 : 4);
-  cudaError_t e = cudaFuncSetAttribute(gather_mapped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_limit(reinterpret_cast<const void*>(gather_mapped_kernel), smem);
   if (e != cudaSuccess) return e;
   gather_mapped_kernel<<<2 * n_sm, kGatherThreads, smem, st>>>(
       idx, n_idx, s.nblk, s.B, blk_bytes, host_cap, static_cast<const uint8_t*>(host_k_dev),
