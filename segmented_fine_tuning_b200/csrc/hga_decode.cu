@@ -60,7 +60,12 @@ struct DecElem<__nv_bfloat16> {
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N committed groups of this thread are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 struct DecArgs {
   int Hq, Hkv, S, d, blk, nq, t0, topk, nkv, n_chunks, G, R;
@@ -126,20 +131,26 @@ __global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __
   }
   const size_t key_stride = (size_t)a.Hkv * d;  // elements between consecutive tokens
 
-  // 1. stage K and V (16-byte vectors) and this CTA's query rows
+  // 1. stage K, then V (16-byte vectors, two copy groups: the scores only
+  //    wait for K), and this CTA's query rows
   const int vpr = d / E;  // vectors per row
   for (int x = tid; x < nk * vpr; x += kDecThreads) {
     const int j = x / vpr, v = x % vpr;
     cp_async16(sK + (size_t)j * row_bytes + v * 16, kb + j * key_stride + v * E);
+  }
+  cp_async_commit();
+  for (int x = tid; x < nk * vpr; x += kDecThreads) {
+    const int j = x / vpr, v = x % vpr;
     cp_async16(sV + (size_t)j * row_bytes + v * 16, vb + j * key_stride + v * E);
   }
+  cp_async_commit();
   for (int x = tid; x < nr * d; x += kDecThreads) {
     const int r = x / d, k = x % d;
     const int rr = r0 + r, g = rr / a.nq, u = rr % a.nq;
     const T* src = q_new + (((size_t)b * a.nq + u) * a.Hq + h * a.G + g) * d + k;
     sQ[r * d + k] = DecElem<T>::at(src) * a.sl2;
   }
-  cp_async_wait_all();
+  cp_async_wait_group<1>();  // this thread's K copies have landed
   __syncthreads();
 
   // 2. scores (log2 units), one key per thread, rows in groups of four (a
@@ -199,6 +210,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __
       sL[r] = l;
     }
   }
+  cp_async_wait_group<0>();  // this thread's V copies have landed
   __syncthreads();
 
   // 4. unnormalised O of the chunk: thread = (column, row phase), rows in
@@ -223,23 +235,28 @@ __global__ void __launch_bounds__(kDecThreads) decode_partial_kernel(const T* __
   }
 }
 
-// One CTA per (batch x KV head, row); one thread per channel.  The chunks
-// (m, l) pairs are staged in shared memory by all threads at once, the merge
-// weights computed once per chunk, and the unnormalised O partials summed
-// with every load of a group in flight (the loop is latency bound otherwise).
+// One CTA per (batch x KV head, row), four warps.  The chunks' (m, l) pairs
+// are staged in shared memory and turned into merge weights 2^(m_c - M) once;
+// warp w then sums the unnormalised O partials of chunks w, w+4, ... with lane
+// L owning channels L, L+32, ... (each chunk's row is one coalesced read per
+// warp, and a warp's loads for four chunks are in flight together), and the
+// four warp sums meet in shared memory.
 constexpr int kMaxChunks = 512;
+constexpr int kMaxHeadDim = 128;
 template <typename T>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecArgs a, T* __restrict__ o,
                                                              float* __restrict__ lse) {
   __shared__ float w_s[kMaxChunks];
   __shared__ float l_s[kMaxChunks];
   __shared__ float red[4];
+  __shared__ float osum[4][kMaxHeadDim];
   const int rr = blockIdx.x % a.R;
   const int bh = blockIdx.x / a.R;
   const int b = bh / a.Hkv, h = bh % a.Hkv;
   const int g = rr / a.nq, u = rr % a.nq;
   const int hq = h * a.G + g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d = a.d, cpl = d >> 5;  // channels per lane: 2 or 4
   const float* ml = a.part_ml + ((size_t)bh * a.n_chunks * a.R + rr) * 2;
   float mloc = -INFINITY;
   for (int c = tid; c < a.n_chunks; c += 128) {
@@ -258,24 +275,45 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecArgs a, T*
     w_s[c] = (mc == -INFINITY) ? 0.f : ex2_approx(mc - M);
   }
   __syncthreads();
-  float L = 0.f;
-  for (int c = 0; c < a.n_chunks; ++c) L = fmaf(l_s[c], w_s[c], L);
-  if (tid < a.d) {
-    const float* po = a.part_o + ((size_t)bh * a.n_chunks * a.R + rr) * a.d + tid;
-    const size_t cstride = (size_t)a.R * a.d;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-    int c = 0;
-    for (; c + 8 <= a.n_chunks; c += 8) {
-      float v[8];
+  const float* po = a.part_o + ((size_t)bh * a.n_chunks * a.R + rr) * d + lane;
+  const size_t cstride = (size_t)a.R * d;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int c = warp;
+  for (; c + 12 < a.n_chunks; c += 16) {
+    float v[4][4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = po[(size_t)(c + k) * cstride];
-      acc0 = fmaf(v[0], w_s[c], acc0); acc1 = fmaf(v[1], w_s[c + 1], acc1);
-      acc2 = fmaf(v[2], w_s[c + 2], acc2); acc3 = fmaf(v[3], w_s[c + 3], acc3);
-      acc0 = fmaf(v[4], w_s[c + 4], acc0); acc1 = fmaf(v[5], w_s[c + 5], acc1);
-      acc2 = fmaf(v[6], w_s[c + 6], acc2); acc3 = fmaf(v[7], w_s[c + 7], acc3);
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) v[k][m] = m < cpl ? po[(size_t)(c + 4 * k) * cstride + 32 * m] : 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float wk = w_s[c + 4 * k];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m] = fmaf(v[k][m], wk, acc[m]);
     }
-    for (; c < a.n_chunks; ++c) acc0 = fmaf(po[(size_t)c * cstride], w_s[c], acc0);
-    o[(((size_t)b * a.nq + u) * a.Hq + hq) * a.d + tid] = (T)(((acc0 + acc1) + (acc2 + acc3)) / L);
+  }
+  for (; c < a.n_chunks; c += 4) {
+    const float wk = w_s[c];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      if (m < cpl) acc[m] = fmaf(po[(size_t)c * cstride + 32 * m], wk, acc[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    if (m < cpl) osum[warp][lane + 32 * m] = acc[m];
+  // L = sum_c l_c w_c, by warp 0 while the sums land
+  float L = 0.f;
+  if (warp == 0) {
+    for (int k = lane; k < a.n_chunks; k += 32) L = fmaf(l_s[k], w_s[k], L);
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) L += __shfl_xor_sync(0xffffffffu, L, k);
+    if (lane == 0) red[0] = L;
+  }
+  __syncthreads();
+  L = red[0];
+  if (tid < d) {
+    const float sum = (osum[0][tid] + osum[1][tid]) + (osum[2][tid] + osum[3][tid]);
+    o[(((size_t)b * a.nq + u) * a.Hq + hq) * d + tid] = (T)(sum / L);
   }
   if (tid == 0) lse[((size_t)b * a.Hq + hq) * a.nq + u] = (M + log2f(L)) * 0.6931471805599453f;
 }
@@ -295,7 +333,7 @@ cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new
   a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.d = s.d; a.blk = s.blk; a.nq = nq; a.t0 = t0; a.topk = s.topk;
   a.nkv = nkv; a.G = s.G(); a.R = s.G() * nq;
   a.n_chunks = s.topk + (t0 + nq + s.blk - 1) / s.blk;
-  if (a.n_chunks > kMaxChunks) return cudaErrorInvalidValue;
+  if (a.n_chunks > kMaxChunks || s.d > kMaxHeadDim || s.d % 32 != 0) return cudaErrorInvalidValue;
   a.sl2 = 1.4426950408889634f / sqrtf((float)s.d);
   a.idx = idx; a.err = err;
   a.part_ml = ws;

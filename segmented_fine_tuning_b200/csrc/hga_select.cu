@@ -162,7 +162,10 @@ __device__ __forceinline__ unsigned long long sel_key(float s, int n) {
 // pass, a histogram of the next byte of the keys that still match the prefix
 // found so far, and one warp walks it from the top to the byte where the count
 // reaches the number of keys still to take.  Then every key at or above that
-// threshold is taken.  Eight passes of three barriers each, for any n.
+// threshold is taken.  Eight passes of three barriers each, for any n.  The
+// scores of one selection tend to share their leading bytes, so a warp whose
+// counted keys all fall in one bin adds them with one atomic (the per-key
+// atomics on a single address would serialise the warp).
 __device__ void topk_radix(const unsigned long long* keys, int n, int keff, int* chosen,
                            unsigned long long* chosen_key) {
   __shared__ unsigned int hist[256];
@@ -175,9 +178,20 @@ __device__ void topk_radix(const unsigned long long* keys, int n, int keff, int*
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int x = tid; x < 256; x += blockDim.x) hist[x] = 0u;
     __syncthreads();
-    for (int x = tid; x < n; x += blockDim.x) {
-      const unsigned long long k = keys[x];
-      if ((k & mask) == prefix) atomicAdd(&hist[(unsigned)(k >> shift) & 255u], 1u);
+    const int nw = (n + 31) & ~31;  // whole warps take part in every iteration (blockDim.x % 32 == 0)
+    for (int x = tid; x < nw; x += blockDim.x) {
+      const unsigned long long k = x < n ? keys[x] : 0ull;
+      const bool in = x < n && (k & mask) == prefix;
+      const unsigned bin = (unsigned)(k >> shift) & 255u;
+      const unsigned ins = __ballot_sync(0xffffffffu, in);
+      if (ins == 0u) continue;
+      const unsigned b0 = __shfl_sync(0xffffffffu, bin, __ffs(ins) - 1);
+      const unsigned same = __ballot_sync(0xffffffffu, in && bin == b0);
+      if (same == ins) {
+        if ((tid & 31) == __ffs(ins) - 1) atomicAdd(&hist[b0], (unsigned)__popc(ins));
+      } else if (in) {
+        atomicAdd(&hist[bin], 1u);
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -446,10 +460,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const T* __restrict
 // A decode step has one (partial) query block per (b, KV head), so one CTA per
 // selection would leave the GPU nearly idle while it walks a long history.
 // The scoring is therefore spread over the blocks: decode_score_kernel, CTA =
-// (64 history blocks, KV head, batch), forms the mean of the n_q new queries
+// (32 history blocks, KV head, batch), forms the mean of the n_q new queries
 // of the G heads and writes each block's (score, index) key to the
 // workspace; decode_topk_kernel, one CTA per (b, KV head), selects from them.
-constexpr int kDecBlocksPerWarp = 8;
+constexpr int kDecBlocksPerWarp = 4;
 constexpr int kDecScoreWarps = 8;
 
 template <typename T>
