@@ -184,8 +184,12 @@ def to_pinned(t: synth.Tensor):
 
 
 def source_sha(fname: str) -> str:
-    with open(os.path.join(ROOT, "segmented_fine_tuning_b200", "csrc", fname), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of a kernel's source file and the headers every kernel includes."""
+    h = hashlib.sha256()
+    for name in (fname, "hga_ptx.cuh", "hga_kernels.h"):
+        with open(os.path.join(ROOT, "segmented_fine_tuning_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def committed_traffic(kernel: str):
