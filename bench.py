@@ -910,11 +910,12 @@ def main():
             torch.cuda.empty_cache()
             pf, _ = run_device(args, rank, world, device, w=synth.PREFILL_131K, steps=min(args.steps, 20))
             out["prefill_131k"] = {k: pf[k] for k in ("value", "unit", "ms_per_step", "steps", "config", "kernels",
-                                                      "attention_fwd", "gpu_launches", "clocks")}
+                                                      "attention_fwd", "launch", "eager", "gpu_launches", "clocks")}
             out["prefill_131k"]["metric"] = "HGA attn fwd tokens/s per layer (131K-token prefill, forward only)"
             de, _ = run_device(args, rank, world, device, w=synth.DENSE_EQUIV, steps=min(args.steps, 20))
             out["dense_equivalence"] = {k: de[k] for k in ("value", "unit", "ms_per_step", "steps", "config",
-                                                           "kernels", "attention_fwd_bwd", "gpu_launches")}
+                                                           "kernels", "attention_fwd_bwd", "launch", "eager",
+                                                           "gpu_launches")}
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
