@@ -162,10 +162,7 @@ __device__ __forceinline__ unsigned long long sel_key(float s, int n) {
 // pass, a histogram of the next byte of the keys that still match the prefix
 // found so far, and one warp walks it from the top to the byte where the count
 // reaches the number of keys still to take.  Then every key at or above that
-// threshold is taken.  Eight passes of three barriers each, for any n.  The
-// scores of one selection tend to share their leading bytes, so a warp whose
-// counted keys all fall in one bin adds them with one atomic (the per-key
-// atomics on a single address would serialise the warp).
+// threshold is taken.  Eight passes of three barriers each, for any n.
 __device__ void topk_radix(const unsigned long long* keys, int n, int keff, int* chosen,
                            unsigned long long* chosen_key) {
   __shared__ unsigned int hist[256];
@@ -178,20 +175,9 @@ __device__ void topk_radix(const unsigned long long* keys, int n, int keff, int*
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int x = tid; x < 256; x += blockDim.x) hist[x] = 0u;
     __syncthreads();
-    const int nw = (n + 31) & ~31;  // whole warps take part in every iteration (blockDim.x % 32 == 0)
-    for (int x = tid; x < nw; x += blockDim.x) {
-      const unsigned long long k = x < n ? keys[x] : 0ull;
-      const bool in = x < n && (k & mask) == prefix;
-      const unsigned bin = (unsigned)(k >> shift) & 255u;
-      const unsigned ins = __ballot_sync(0xffffffffu, in);
-      if (ins == 0u) continue;
-      const unsigned b0 = __shfl_sync(0xffffffffu, bin, __ffs(ins) - 1);
-      const unsigned same = __ballot_sync(0xffffffffu, in && bin == b0);
-      if (same == ins) {
-        if ((tid & 31) == __ffs(ins) - 1) atomicAdd(&hist[b0], (unsigned)__popc(ins));
-      } else if (in) {
-        atomicAdd(&hist[bin], 1u);
-      }
+    for (int x = tid; x < n; x += blockDim.x) {
+      const unsigned long long k = keys[x];
+      if ((k & mask) == prefix) atomicAdd(&hist[(unsigned)(k >> shift) & 255u], 1u);
     }
     __syncthreads();
     if (tid < 32) {

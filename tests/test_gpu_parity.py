@@ -66,6 +66,13 @@ SEL_CASES = [
     synth.Workload("k-exceeds-history", 1, 4, 2, 128, 128, 256, 3, 8, "bf16", 23),
     synth.QWEN3_8B_LAYER,
     synth.PREFILL_131K,
+    # histories above 256 blocks take the staged scoring path: G = 1, 2, 8, d = 64, fp32, B = 2, and
+    # block counts that leave a partial last chunk of 64
+    synth.Workload("long-hist-G1-d64: Hq2/Hkv2 d64 blk64 S256 hist300 K8", 1, 2, 2, 64, 64, 256, 300, 8, "bf16", 26),
+    synth.Workload("long-hist-G2-f32-B2: B2 Hq4/Hkv2 blk32 S128 hist277 K5", 2, 4, 2, 128, 32, 128, 277, 5, "f32",
+                   27),
+    synth.Workload("long-hist-G8: Hq16/Hkv2 S256 hist400 K16", 1, 16, 2, 128, 128, 256, 400, 16, "bf16", 28,
+                   structured_keys=True),
 ]
 
 
