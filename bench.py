@@ -226,7 +226,10 @@ def run_device(args, rank, world, device, w=None, steps=None):
     stream = torch.cuda.current_stream(device)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
 
-    def step(evs=None, s=stream):
+    def step(evs=None, s=stream, combined=False):
+        """combined: the backward through hga_attn_bwd (preprocess, then dQ and
+        dK/dV on two streams); otherwise one entry point per kernel, so that
+        events can sit between them."""
         def mark(k):
             if evs is not None:
                 evs[k].record(s)
@@ -238,6 +241,11 @@ def run_device(args, rank, world, device, w=None, steps=None):
         hga.hga_attn_fwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"], D.n_hist_blocks,
                          st.idx, st.o, st.lse, s)
         mark(3)
+        if combined:
+            if not w.fwd_only:
+                hga.hga_attn_bwd(D, dev["q"], dev["k_seg"], dev["v_seg"], dev["k_hist"], dev["v_hist"],
+                                 D.n_hist_blocks, st.idx, st.o, st.lse, dev["d_o"], st.dq, st.dk, st.dv, st.ws, s)
+            return
         if not w.fwd_only:
             hga.hga_attn_bwd_preprocess(D, st.o, dev["d_o"], st.ws, s)
         mark(4)
@@ -285,7 +293,7 @@ def run_device(args, rank, world, device, w=None, steps=None):
     cap = torch.cuda.Stream(device)
     cap.wait_stream(stream)
     with torch.cuda.graph(graph, stream=cap, capture_error_mode="relaxed"):
-        step(s=cap)
+        step(s=cap, combined=True)
     stream.wait_stream(cap)
     for _ in range(args.warmup):
         flush.zero_()
@@ -347,8 +355,10 @@ def run_device(args, rank, world, device, w=None, steps=None):
                                                       peaks["bf16_tflops"], 3),
                               "algorithmic_gflop": round(fwd_bwd_flops / 1e9, 2)},
         "kernels": kern,
-        "launch": "the step replayed as one CUDA graph; per-kernel times from the same step launched eagerly "
-                  "with an event between kernels (small kernels' spans include their launch latency)",
+        "launch": "the step (summaries, selection, forward, hga_attn_bwd: preprocess, then dQ and dK/dV on two "
+                  "streams) replayed as one CUDA graph; per-kernel times from the same kernels launched eagerly one "
+                  "entry point at a time with an event between them (small kernels' spans include their launch "
+                  "latency)",
         "eager": {"ms_per_step": round(eager_ms, 4), "tokens_per_s": round(job_throughput(world, w.S, eager_ms), 1),
                   "clocks": clk.summary()},
         "gpu_launches": (3 if w.fwd_only else 6) * steps,

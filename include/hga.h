@@ -188,6 +188,12 @@ HGA_API size_t hga_attn_bwd_workspace_size(const hga_dims* dims);
  * dv_seg are fp32 and fully overwritten.  ws: device scratch of at least
  * hga_attn_bwd_workspace_size(dims) bytes, owned by the caller; its contents
  * need no initialisation and are undefined afterwards.
+ * On the tensor-core path the dQ kernel runs on `stream` and the dK/dV kernel
+ * on a side stream the library creates once per device, forked from `stream`
+ * after the preprocess and joined back into it with events: work queued on
+ * `stream` after the call sees all three outputs, and the call records into
+ * a CUDA graph under stream capture (as two branches).  The same holds for
+ * hga_attn_bwd_sparse and hga_attn_bwd_noalloc.
  * Errors: as hga_attn_fwd, plus HGA_ERR_INVALID_ARG for a short workspace.
  */
 HGA_API hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,

@@ -324,6 +324,37 @@ namespace {
 
 // Shared checks and dispatch of the backward stages (parts: hga::kBwdDq |
 // hga::kBwdDkdv; preprocess when `pre` is set).
+// A library-owned side stream per device, with a fork and a join event: the
+// dQ and dK/dV kernels of one backward run concurrently (each kernel's last
+// partial wave is filled by the other's CTAs).  The mutex is held from the
+// fork's record to the join's wait, so concurrent callers never see each
+// other's events.  Stream capture follows the fork into the side stream and
+// back, so the pair also records into a CUDA graph as two branches.
+struct SideStream {
+  std::mutex mu;
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool tried = false;
+};
+SideStream* side_stream(int dev) {
+  static SideStream pool[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  SideStream* x = &pool[dev];
+  return x;
+}
+bool side_ready(SideStream* x) {  // called with x->mu held
+  if (!x->tried) {
+    x->tried = true;
+    if (cudaStreamCreateWithFlags(&x->side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x->fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x->join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      x->side = nullptr;
+    }
+  }
+  return x->side != nullptr;
+}
+
 hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg, const void* k_hist,
                    const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o, const float* lse,
                    const void* d_o, float* dq, float* dk_seg, float* dv_seg, const void* ws, size_t ws_bytes,
@@ -359,6 +390,28 @@ hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const
   if (hga::tc_supported(s)) {
     hga::TcMaps m;
     if ((r = build_maps(s, n_kv_blocks, q, d_o, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
+    int dev = 0;
+    SideStream* x = (parts == (hga::kBwdDq | hga::kBwdDkdv) && cudaGetDevice(&dev) == cudaSuccess) ? side_stream(dev)
+                                                                                                   : nullptr;
+    if (x) {
+      std::lock_guard<std::mutex> lock(x->mu);
+      if (side_ready(x)) {
+        // dQ (the longer kernel) first on the caller's stream, dK/dV on the side stream, joined back
+        if ((e = cudaEventRecord(x->fork, st)) != cudaSuccess || (e = cudaStreamWaitEvent(x->side, x->fork, 0)) !=
+                                                                       cudaSuccess)
+          return cuda_fail(e, "backward fork");
+        if ((e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, hga::kBwdDq, err, st,
+                                         qmask, gscale)) != cudaSuccess)
+          return cuda_fail(e, "attention backward launch (dQ)");
+        if ((e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, hga::kBwdDkdv, err,
+                                         x->side, qmask, gscale)) != cudaSuccess)
+          return cuda_fail(e, "attention backward launch (dK/dV)");
+        if ((e = cudaEventRecord(x->join, x->side)) != cudaSuccess || (e = cudaStreamWaitEvent(st, x->join, 0)) !=
+                                                                          cudaSuccess)
+          return cuda_fail(e, "backward join");
+        return HGA_OK;
+      }
+    }
     e = hga::launch_attn_bwd_tc(s, m, n_kv_blocks, idx, lse, Dr, dq, dk_seg, dv_seg, parts, err, st, qmask, gscale);
   } else {
     e = hga::launch_attn_bwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, lse, Dr, d_o, dq, dk_seg,
