@@ -374,13 +374,15 @@ def run_e2e(args, ctx, device):
     selection, forward and backward, and copies every result (O, LSE, dQ,
     dK, dV) back to pinned host memory.  Steps are pipelined two deep, as a
     training loop with a prefetching data loader runs them: step k+1's
-    inputs travel host -> device and step k-1's results device -> host while
-    step k computes (separate copy streams, double-buffered device sets).
+    inputs travel host -> device, its selection runs and its history blocks
+    are fetched, and step k-1's results travel device -> host, while step k
+    computes (separate copy and selection streams, double-buffered device
+    sets).
     The timed region spans the first input copy to the last result copy."""
     import segmented_fine_tuning_b200 as hga
     w, x, D, dev, st0 = ctx
     stream = torch.cuda.current_stream(device)
-    h2d, d2h, fetch_stream = (torch.cuda.Stream(device) for _ in range(3))
+    h2d, d2h, fetch_stream, sel_stream = (torch.cuda.Stream(device) for _ in range(4))
     host = {n: to_pinned(getattr(x, n)) for n in ("q", "k_seg", "v_seg", "d_o")}
     tier_k, tier_v = to_pinned(x.k_hist), to_pinned(x.v_hist)
     # the history's summaries are resident on the device (computed once, when
@@ -410,16 +412,24 @@ def run_e2e(args, ctx, device):
                 r["seg"][n].copy_(host[n], non_blocking=True)
         r["ev"]["h2d"].record(h2d)
 
+    def select_and_fetch(k):
+        # selection needs only this step's queries and the resident summaries, so it (and the history
+        # fetch it drives) runs as soon as the inputs land, while the previous step computes
+        r = sets[k % 2]
+        st, seg = r["st"], r["seg"]
+        sel_stream.wait_event(r["ev"]["h2d"])
+        sel_stream.wait_event(r["ev"]["comp"])  # step k-2 has finished with this set's idx and pool
+        hga.hga_select_topk(D, seg["q"], st0.summ, st.idx, None, sel_stream)
+        nu = hga.hga_fetch_blocks(D, tier_k, tier_v, D.n_hist_blocks, st.idx, r["scratch"], r["pool_k"],
+                                  r["pool_v"], D.n_hist_blocks, r["idx_pool"], sel_stream, fetch_stream,
+                                  r["ev"]["fetch"])
+        fetched.append(nu)
+
     def compute_and_out(k):
         r = sets[k % 2]
         st, seg = r["st"], r["seg"]
         stream.wait_event(r["ev"]["h2d"])
         stream.wait_event(r["ev"]["d2h"])  # step k-2's results have left this set's outputs
-        hga.hga_select_topk(D, seg["q"], st0.summ, st.idx, None, stream)
-        nu = hga.hga_fetch_blocks(D, tier_k, tier_v, D.n_hist_blocks, st.idx, r["scratch"], r["pool_k"],
-                                  r["pool_v"], D.n_hist_blocks, r["idx_pool"], stream, fetch_stream,
-                                  r["ev"]["fetch"])
-        fetched.append(nu)
         stream.wait_event(r["ev"]["fetch"])
         hga.hga_attn_fwd(D, seg["q"], seg["k_seg"], seg["v_seg"], r["pool_k"], r["pool_v"], D.n_hist_blocks,
                          r["idx_pool"], st.o, st.lse, stream)
@@ -434,11 +444,14 @@ def run_e2e(args, ctx, device):
 
     def run(n):
         inputs_in(0)
+        select_and_fetch(0)
         for k in range(n):
             if k + 1 < n:
                 inputs_in(k + 1)
             compute_and_out(k)
-        for s_ in (h2d, d2h, fetch_stream):
+            if k + 1 < n:
+                select_and_fetch(k + 1)  # the host waits here for step k+1's indices, step k already queued
+        for s_ in (h2d, d2h, fetch_stream, sel_stream):
             stream.wait_stream(s_)
 
     run(max(2, args.warmup))
@@ -447,7 +460,7 @@ def run_e2e(args, ctx, device):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n = args.steps
     e0.record(stream)
-    for s_ in (h2d, d2h, fetch_stream):
+    for s_ in (h2d, d2h, fetch_stream, sel_stream):
         s_.wait_event(e0)
     run(n)
     e1.record(stream)
@@ -462,7 +475,8 @@ def run_e2e(args, ctx, device):
             "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
             "fetched_blocks_per_step": float(np.mean(fetched)),
             "path": "pinned host tier + hga_fetch_blocks; O, LSE, dQ, dK, dV copied back to pinned host memory; "
-                    "steps pipelined two deep (inputs of k+1 and results of k-1 in flight during k)"}
+                    "steps pipelined two deep (inputs, selection and history fetch of k+1 and results of k-1 in "
+                    "flight during k)"}
 
 
 # ---------------------------------------------------------------- segmented pass
