@@ -165,3 +165,20 @@ def test_headers_compile_as_c_and_cpp(tmp_path):
         r = subprocess.run([tool, *lang, "-Wall", "-Wextra", "-Werror", *inc, "-c", str(src), "-o",
                             str(tmp_path / "use.o")], capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_size_limits_rejected_on_host(lib):
+    """One past each documented maximum is rejected with HGA_ERR_SHAPE before
+    any device work: 4,096 history blocks for a selection (prefill and
+    decode), 128 blocks for an appended segment."""
+    p = ctypes.c_void_p(16)
+    d = _dims(n_hist_blocks=4097, block=32, S=128)
+    assert lib.hga_select_topk(ctypes.byref(d), p, p, p, None, None) == 2
+    assert "4096" in lib.hga_last_error().decode()
+    ws = ctypes.c_size_t(1 << 30)
+    assert lib.hga_decode_select(ctypes.byref(d), 1, p, p, p, None, p, ws, None) == 2
+    d = _dims(n_hist_blocks=4096, block=32, S=128)
+    assert lib.hga_decode_workspace_size(ctypes.byref(d), 1) > 0
+    d = _dims(S=129 * 128, n_hist_blocks=129 * 128 // 128 + 1)
+    assert lib.hga_append_segment(ctypes.byref(d), p, p, 0, p, None, None, None, None, None, 0, None, None) == 2
+    assert "128" in lib.hga_last_error().decode()
