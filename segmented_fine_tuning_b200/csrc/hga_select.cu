@@ -162,17 +162,51 @@ __device__ __forceinline__ unsigned long long sel_key(float s, int n) {
 // pass, a histogram of the next byte of the keys that still match the prefix
 // found so far, and one warp walks it from the top to the byte where the count
 // reaches the number of keys still to take.  Then every key at or above that
-// threshold is taken.  Eight passes of three barriers each, for any n.
+// threshold is taken.  Up to eight passes of three barriers each.  One pass
+// first forms the bitwise AND and OR of all keys: the leading bytes on which
+// every key agrees (one selection's scores often share their sign and
+// exponent byte, and the index bytes above the largest index are constant)
+// are taken as they are, without a histogram pass whose counts would all fall
+// in one bin.
 __device__ void topk_radix(const unsigned long long* keys, int n, int keff, int* chosen,
                            unsigned long long* chosen_key) {
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
   __shared__ int s_need;
   __shared__ int s_count;
-  const int tid = threadIdx.x;
+  __shared__ unsigned long long red_and[32], red_or[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned long long k_and = ~0ull, k_or = 0ull;
+  for (int x = tid; x < n; x += blockDim.x) {
+    const unsigned long long k = keys[x];
+    k_and &= k;
+    k_or |= k;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
+    k_or |= __shfl_xor_sync(0xffffffffu, k_or, o);
+  }
+  if (lane == 0) {
+    red_and[warp] = k_and;
+    red_or[warp] = k_or;
+  }
+  __syncthreads();
+  k_and = ~0ull;
+  k_or = 0ull;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    k_and &= red_and[w];
+    k_or |= red_or[w];
+  }
   unsigned long long prefix = 0ull, mask = 0ull;
   int need = keff;
   for (int shift = 56; shift >= 0; shift -= 8) {
+    if ((((k_and ^ k_or) >> shift) & 0xFFull) == 0ull) {
+      // every key has this byte: so has the keff-th largest
+      prefix |= k_and & (0xFFull << shift);
+      mask |= 0xFFull << shift;
+      continue;
+    }
     for (int x = tid; x < 256; x += blockDim.x) hist[x] = 0u;
     __syncthreads();
     for (int x = tid; x < n; x += blockDim.x) {
