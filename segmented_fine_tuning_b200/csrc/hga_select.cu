@@ -8,6 +8,8 @@
 // query-block-mean . summary / sqrt(d), ties to the lower block index.
 #include <float.h>
 
+#include <algorithm>
+
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
 
@@ -574,49 +576,58 @@ __global__ void __launch_bounds__(kSelThreads) decode_topk_kernel(const unsigned
 // D = sum_k dO * O in fp32 per (b, p, hq) row.  A row is read by d/V lanes
 // (16-byte vectors), so a warp covers 32V/d rows per pass; kPreRows passes are
 // loaded before any arithmetic to keep enough bytes in flight.
-constexpr int kPreRows = 4;
+// Dr[b, hq, p] = sum_k dO[b,p,hq,k] * O[b,p,hq,k].  Rows (token, head) are
+// taken by the warps in a grid-stride loop, kPreRows rows per thread and pass
+// with all their 16-byte loads in flight (kept as raw vectors, widened only
+// at the multiply), lpr = d / V lanes per row, combined by shuffles.
+constexpr int kPreRows = 8;
 template <typename T>
 __global__ void __launch_bounds__(256) preprocess_kernel(const T* __restrict__ o, const T* __restrict__ d_o, int S,
                                                          int Hq, int d, int rows, float* __restrict__ Dr) {
   constexpr int V = Vec<T>::N;
   const int lpr = d / V;    // lanes per row
   const int rpw = 32 / lpr;  // rows per warp per pass
-  const int gw = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   const int sub = lane / lpr, cl = lane % lpr;
-  const int row0 = gw * rpw * kPreRows + sub;
-  float x[kPreRows][V], y[kPreRows][V];
-#pragma unroll
-  for (int r = 0; r < kPreRows; ++r) {
-    const int row = row0 + r * rpw;
-    if (row < rows) {
-      // rows are enumerated token-major: row = (b*S + p)*Hq + hq
-      Vec<T>::load(o + (size_t)row * d + cl * V, x[r]);
-      Vec<T>::load(d_o + (size_t)row * d + cl * V, y[r]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < V; ++e) x[r][e] = y[r][e] = 0.f;
-    }
-  }
-  float acc[kPreRows];
-#pragma unroll
-  for (int r = 0; r < kPreRows; ++r) {
-    acc[r] = 0.f;
-#pragma unroll
-    for (int e = 0; e < V; ++e) acc[r] = fmaf(x[r][e], y[r][e], acc[r]);
-  }
-  for (int k = lpr >> 1; k > 0; k >>= 1) {
-#pragma unroll
-    for (int r = 0; r < kPreRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], k);
-  }
-  if (cl == 0) {
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  for (int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; gw * rpw * kPreRows < rows; gw += warps) {
+    const int row0 = gw * rpw * kPreRows + sub;
+    uint4 xr[kPreRows], yr[kPreRows];
 #pragma unroll
     for (int r = 0; r < kPreRows; ++r) {
       const int row = row0 + r * rpw;
       if (row < rows) {
-        const int hq = row % Hq;
-        const int bp = row / Hq;
-        const int b = bp / S, p = bp % S;
-        Dr[((size_t)b * Hq + hq) * S + p] = acc[r];
+        // rows are enumerated token-major: row = (b*S + p)*Hq + hq
+        xr[r] = __ldg(reinterpret_cast<const uint4*>(o + (size_t)row * d + cl * V));
+        yr[r] = __ldg(reinterpret_cast<const uint4*>(d_o + (size_t)row * d + cl * V));
+      } else {
+        xr[r] = yr[r] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float acc[kPreRows];
+#pragma unroll
+    for (int r = 0; r < kPreRows; ++r) {
+      float x[V], y[V];
+      Vec<T>::unpack(xr[r], x);
+      Vec<T>::unpack(yr[r], y);
+      acc[r] = 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[r] = fmaf(x[e], y[e], acc[r]);
+    }
+    for (int k = lpr >> 1; k > 0; k >>= 1) {
+#pragma unroll
+      for (int r = 0; r < kPreRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], k);
+    }
+    if (cl == 0) {
+#pragma unroll
+      for (int r = 0; r < kPreRows; ++r) {
+        const int row = row0 + r * rpw;
+        if (row < rows) {
+          const int hq = row % Hq;
+          const int bp = row / Hq;
+          const int b = bp / S, p = bp % S;
+          Dr[((size_t)b * Hq + hq) * S + p] = acc[r];
+        }
       }
     }
   }
@@ -733,7 +744,10 @@ cudaError_t launch_decode_select(const Shape& s, int nq, const void* q_new, cons
 cudaError_t launch_bwd_preprocess(const Shape& s, const void* o, const void* d_o, float* Dr, cudaStream_t st) {
   const int rows = s.B * s.S * s.Hq;
   const int rows_per_cta = 8 * (32 * (s.bf16 ? 8 : 4) / s.d) * kPreRows;
-  const int grid = (rows + rows_per_cta - 1) / rows_per_cta;
+  int dev = 0, n_sm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  // at most the CTAs that are resident at once (4 per SM); the warps then stride over the rows
+  const int grid = std::max(1, std::min((rows + rows_per_cta - 1) / rows_per_cta, 4 * n_sm));
   if (s.bf16)
     preprocess_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
                                                            static_cast<const __nv_bfloat16*>(d_o), s.S, s.Hq, s.d,
