@@ -49,10 +49,12 @@
  * Conventions:
  *   - Ownership: the caller owns every buffer (device memory unless stated).
  *     The library allocates no device or pinned memory; scratch space is
- *     passed in by the caller (hga_attn_bwd_workspace_size).
+ *     passed in by the caller (hga_attn_bwd_workspace_size).  It creates one
+ *     side stream and two events per device, once, for the two-stream
+ *     backward (hga_attn_bwd).
  *   - Asynchrony: every call enqueues work on `stream` and returns; errors in
- *     arguments are reported before anything is enqueued.  hga_fetch_blocks is
- *     the exception: it waits (bounded by timeout_ms) for a small index copy.
+ *     arguments are reported before anything is enqueued.  The fetch calls are
+ *     the exception: they wait (bounded by timeout_ms) for a small index copy.
  *   - Device-side faults that a kernel can detect (an out-of-range idx entry,
  *     an expired pipeline wait) set a per-device flag instead of trapping;
  *     hga_device_status() synchronizes the stream and reports and clears it.
