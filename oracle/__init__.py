@@ -29,7 +29,7 @@ _LIB = None
 
 
 class _Dims(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in ("B", "Hq", "Hkv", "d", "blk", "S", "nblk", "topk")]
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "Hq", "Hkv", "d", "blk", "S", "nblk", "topk", "qblk")]
 
 
 @dataclass(frozen=True)
@@ -42,13 +42,18 @@ class Dims:
     S: int
     nblk: int
     topk: int
+    qblk: int = 0  # query-block size; 0 = blk (history blocks and query blocks of one size)
+
+    @property
+    def qb(self) -> int:
+        return self.qblk or self.blk
 
     @property
     def nqb(self) -> int:
-        return self.S // self.blk
+        return self.S // self.qb
 
     def c(self) -> _Dims:
-        return _Dims(self.B, self.Hq, self.Hkv, self.d, self.blk, self.S, self.nblk, self.topk)
+        return _Dims(self.B, self.Hq, self.Hkv, self.d, self.blk, self.S, self.nblk, self.topk, self.qblk)
 
 
 def _lib():
@@ -150,7 +155,7 @@ def _attn_inputs(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx):
     if idx.size and (idx.max() >= nb or idx.min() < -1):
         raise ValueError("idx out of range")
     # the C code indexes history with nblk rows of blocks
-    Dc = Dims(D.B, D.Hq, D.Hkv, D.d, D.blk, D.S, nb, D.topk)
+    Dc = Dims(D.B, D.Hq, D.Hkv, D.d, D.blk, D.S, nb, D.topk, D.qblk)
     return Dc, q, k_seg, v_seg, k_hist, v_hist, idx
 
 
@@ -188,7 +193,7 @@ def attn_bwd(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx, d_o, kv_heads=None):
 
 def attn_bwd_sparse(D: Dims, q, k_seg, v_seg, k_hist, v_hist, idx, d_o, qmask, scale: float, kv_heads=None):
     """SpaCO-style sparse backward: only query blocks with qmask[b, i] != 0
-    propagate gradient, scaled by `scale` (qmask [B, S/blk]).  Returns
+    propagate gradient, scaled by `scale` (qmask [B, S/qblk]).  Returns
     (dQ, dK_seg, dV_seg) like attn_bwd."""
     Dc, q, k_seg, v_seg, k_hist, v_hist, idx = _attn_inputs(D, q, k_seg, v_seg, k_hist, v_hist, idx)
     d_o = _f64(d_o)
@@ -249,7 +254,7 @@ def decode_attn(D: Dims, t0: int, q_new, k_seg, v_seg, k_hist, v_hist, idx):
         raise ValueError("new tokens outside the segment buffer")
     if idx.size and (idx.max() >= nb or idx.min() < -1):
         raise ValueError("idx out of range")
-    Dc = Dims(D.B, D.Hq, D.Hkv, D.d, D.blk, D.S, nb, D.topk)
+    Dc = Dims(D.B, D.Hq, D.Hkv, D.d, D.blk, D.S, nb, D.topk, D.qblk)
     o = np.zeros((D.B, nq, D.Hq, D.d))
     lse = np.zeros((D.B, D.Hq, nq))
     _lib().ohga_decode_attn(ctypes.byref(Dc.c()), nq, t0, _ptr(q_new), _ptr(k_seg), _ptr(v_seg), _ptr(k_hist),

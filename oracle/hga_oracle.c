@@ -30,6 +30,11 @@
  *              at positions <= the query's own], scale 1/sqrt(d);
  *   backward = gradients of <O, dO> with respect to Q, K_seg, V_seg only;
  *              the selection and the history are constants.
+ * Block sizes: history blocks hold blk tokens (summaries, selection units);
+ * query blocks hold qblk tokens (the rows that share one selection), qblk = blk
+ * unless the dims say otherwise.  With qblk != blk nothing else changes: a
+ * query block's mean is over its qblk rows, and a row attends to the blk
+ * tokens of each block selected for its query block.
  *
  * Every function is a direct transcription of those definitions in double
  * precision: no blocking, no fusion, no reordering of sums.  OpenMP only
@@ -40,9 +45,9 @@
  *   k_seg, v_seg, dk, dv [B, S, Hkv, d]
  *   k_hist, v_hist       [B, nblk*blk, Hkv, d]
  *   summ                 [B, Hkv, nblk, d]
- *   qm                   [B, Hq, S/blk, d]
- *   score                [B, Hkv, S/blk, nblk]
- *   idx                  [B, Hkv, S/blk, topk]  (int32)
+ *   qm                   [B, Hq, S/qblk, d]
+ *   score                [B, Hkv, S/qblk, nblk]
+ *   idx                  [B, Hkv, S/qblk, topk]  (int32)
  *   lse                  [B, Hq, S]
  * Query head hq belongs to KV head hq / (Hq/Hkv).
  */
@@ -61,6 +66,9 @@ int ohga_max_threads(void) { return omp_get_max_threads(); }
 static size_t tok_off(int b, int t, int T, int h, int H, int d) {
   return (((size_t)b * T + t) * H + h) * (size_t)d;
 }
+
+/* Query-block size: qblk, or blk when the dims leave it 0. */
+static int qb(const ohga_dims* D) { return D->qblk > 0 ? D->qblk : D->blk; }
 
 static double dot(const double* a, const double* b, int d) {
   double s = 0.0;
@@ -84,9 +92,10 @@ void ohga_block_summaries(const ohga_dims* D, const double* k_hist, double* summ
       }
 }
 
-/* qm[b,hq,i,:] = (1/blk) * sum over the blk queries of segment query block i. */
+/* qm[b,hq,i,:] = (1/qblk) * sum over the qblk queries of segment query block i. */
 void ohga_query_means(const ohga_dims* D, const double* q, double* qm) {
-  const int nqb = D->S / D->blk;
+  const int Q = qb(D);
+  const int nqb = D->S / Q;
 #pragma omp parallel for collapse(3) schedule(static)
   for (int b = 0; b < D->B; ++b)
     for (int hq = 0; hq < D->Hq; ++hq)
@@ -94,15 +103,15 @@ void ohga_query_means(const ohga_dims* D, const double* q, double* qm) {
         double* out = qm + (((size_t)b * D->Hq + hq) * nqb + i) * D->d;
         for (int k = 0; k < D->d; ++k) {
           double s = 0.0;
-          for (int t = 0; t < D->blk; ++t) s += q[tok_off(b, i * D->blk + t, D->S, hq, D->Hq, D->d) + k];
-          out[k] = s / D->blk;
+          for (int t = 0; t < Q; ++t) s += q[tok_off(b, i * Q + t, D->S, hq, D->Hq, D->d) + k];
+          out[k] = s / Q;
         }
       }
 }
 
 /* score[b,h,i,n] = max over hq in group(h) of qm[b,hq,i] . summ[b,h,n] / sqrt(d). */
 void ohga_block_scores(const ohga_dims* D, const double* qm, const double* summ, double* score) {
-  const int nqb = D->S / D->blk;
+  const int nqb = D->S / qb(D);
   const int G = D->Hq / D->Hkv;
   const double inv_sqrt_d = 1.0 / sqrt((double)D->d);
 #pragma omp parallel for collapse(3) schedule(static)
@@ -142,7 +151,7 @@ static int int_cmp(const void* pa, const void* pb) {
 /* idx[b,h,i,:]: the min(topk, nblk) best blocks by the order above, listed in
  * ascending block index, padded with -1. */
 void ohga_select_topk(const ohga_dims* D, const double* score, int32_t* idx) {
-  const int nqb = D->S / D->blk;
+  const int nqb = D->S / qb(D);
   const int keff = D->topk < D->nblk ? D->topk : D->nblk;
 #pragma omp parallel for collapse(3) schedule(static)
   for (int b = 0; b < D->B; ++b)
@@ -167,7 +176,7 @@ void ohga_select_topk(const ohga_dims* D, const double* score, int32_t* idx) {
 static int gather_keys(const ohga_dims* D, int b, int h, int i, int p, const double* k_seg, const double* v_seg,
                        const double* k_hist, const double* v_hist, const int32_t* idx, const double** keys,
                        const double** vals) {
-  const int nqb = D->S / D->blk;
+  const int nqb = D->S / qb(D);
   const int T = D->nblk * D->blk;
   int nk = 0;
   const int32_t* sel = idx + (((size_t)b * D->Hkv + h) * nqb + i) * D->topk;
@@ -231,7 +240,7 @@ void ohga_attn_fwd(const ohga_dims* D, const double* q, const double* k_seg, con
           const int h = hq / G;
           if (!in_range(h, h0, h1)) continue;
           if (row_mask && !row_mask[p]) continue;
-          const int nk = gather_keys(D, b, h, p / D->blk, p, k_seg, v_seg, k_hist, v_hist, idx, keys, vals);
+          const int nk = gather_keys(D, b, h, p / qb(D), p, k_seg, v_seg, k_hist, v_hist, idx, keys, vals);
           row_attention(D->d, q + tok_off(b, p, D->S, hq, D->Hq, D->d), nk, keys, vals,
                         o + tok_off(b, p, D->S, hq, D->Hq, D->d), &lse[((size_t)b * D->Hq + hq) * D->S + p], s_buf,
                         NULL);
@@ -277,7 +286,7 @@ void ohga_attn_bwd(const ohga_dims* D, const double* q, const double* k_seg, con
           if (!in_range(h, h0, h1)) continue;
           const size_t r = ((size_t)b * D->Hq + hq) * D->S + p;
           const size_t off = tok_off(b, p, D->S, hq, D->Hq, d);
-          const int nk = gather_keys(D, b, h, p / D->blk, p, k_seg, v_seg, k_hist, v_hist, idx, keys, vals);
+          const int nk = gather_keys(D, b, h, p / qb(D), p, k_seg, v_seg, k_hist, v_hist, idx, keys, vals);
           row_attention(d, q + off, nk, keys, vals, o + r * d, &lse[r], s_buf, p_buf);
           Dr[r] = dot(d_o + off, o + r * d, d);
           for (int k = 0; k < d; ++k) dq[off + k] = 0.0;
@@ -429,17 +438,17 @@ void ohga_decode_attn(const ohga_dims* D, int nq, int t0, const double* q_new, c
  * detached, a gradient path never leaves the segment, so the estimator is
  * the backward of L = scale * sum over the chosen blocks' rows of <O, dO>:
  * the plain backward (ohga_attn_bwd) with dO replaced by
- *   dO_eff[b, p] = scale * dO[b, p]  if qmask[b, p / blk] != 0,  else 0.
- * qmask: [B, S/blk] int8. */
+ *   dO_eff[b, p] = scale * dO[b, p]  if qmask[b, p / qblk] != 0,  else 0.
+ * qmask: [B, S/qblk] int8. */
 void ohga_attn_bwd_sparse(const ohga_dims* D, const double* q, const double* k_seg, const double* v_seg,
                           const double* k_hist, const double* v_hist, const int32_t* idx, const double* d_o,
                           const int8_t* qmask, double scale, int h0, int h1, double* dq, double* dk, double* dv) {
   const size_t n = (size_t)D->B * D->S * D->Hq * D->d;
-  const int nqb = D->S / D->blk;
+  const int nqb = D->S / qb(D);
   double* d_eff = (double*)malloc(sizeof(double) * (n > 0 ? n : 1));
   for (int b = 0; b < D->B; ++b)
     for (int p = 0; p < D->S; ++p) {
-      const double f = qmask[(size_t)b * nqb + p / D->blk] ? scale : 0.0;
+      const double f = qmask[(size_t)b * nqb + p / qb(D)] ? scale : 0.0;
       for (int hq = 0; hq < D->Hq; ++hq)
         for (int k = 0; k < D->d; ++k) {
           const size_t off = tok_off(b, p, D->S, hq, D->Hq, D->d) + k;

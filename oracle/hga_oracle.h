@@ -8,6 +8,7 @@
 
 typedef struct {
   int B, Hq, Hkv, d, blk, S, nblk, topk;
+  int qblk; /* query-block size; 0 = blk (the history block size) */
 } ohga_dims;
 
 void ohga_set_threads(int n);

@@ -506,3 +506,81 @@ def test_sparse_backward_ignores_unchosen_rows_of_d_o():
     b = oracle.attn_bwd_sparse(D, q, ks, vs, kh, vh, idx, do2, mask, 0.5)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# ---------------------------------------------------------------- query blocks of another size than history blocks
+
+def test_query_means_over_query_blocks_of_two_history_blocks():
+    """qblk = 2*blk: a query block's mean is the average of the means of its
+    two halves (computed with qblk = blk), exactly for integer inputs."""
+    D2 = Dims(B=2, Hq=3, Hkv=1, d=4, blk=2, S=12, nblk=1, topk=1, qblk=4)
+    D1 = Dims(B=2, Hq=3, Hkv=1, d=4, blk=2, S=12, nblk=1, topk=1)
+    q = _rng(31).integers(-8, 8, size=(D2.B, D2.S, D2.Hq, D2.d)).astype(np.float64)
+    qm2, qm1 = oracle.query_means(D2, q), oracle.query_means(D1, q)
+    assert qm2.shape[2] == 3 and qm1.shape[2] == 6
+    np.testing.assert_array_equal(qm2, 0.5 * (qm1[:, :, 0::2] + qm1[:, :, 1::2]))
+
+
+def test_scores_over_query_blocks_of_two_history_blocks_g1():
+    """G = 1, qblk = 2*blk: the score is linear in the query mean, so a query
+    block's scores are the average of its halves' scores."""
+    D2 = Dims(B=1, Hq=2, Hkv=2, d=8, blk=4, S=16, nblk=5, topk=2, qblk=8)
+    D1 = Dims(B=1, Hq=2, Hkv=2, d=8, blk=4, S=16, nblk=5, topk=2)
+    q, _, _, kh, _, _ = _rand_inputs(D2, 32)
+    _, s2 = oracle.select(D2, q, kh)
+    _, s1 = oracle.select(D1, q, kh)
+    np.testing.assert_allclose(s2, 0.5 * (s1[:, :, 0::2] + s1[:, :, 1::2]), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("blk,qblk", [(2, 4), (4, 2), (3, 6)])
+def test_query_zero_k1_closed_form_with_other_query_block_size(blk, qblk):
+    """Q = 0, K = 1, history block n holding the value n+1, segment values 0:
+    row p attends to the blk tokens of the block chosen for query block
+    p // qblk and to the p+1 segment keys, all with equal weight, so
+    O[p] = blk * (n + 1) / (blk + p + 1).  A row mapped to the wrong query
+    block, or a block of the wrong length, fails it."""
+    nblk, S = 5, 12
+    D = Dims(B=1, Hq=2, Hkv=1, d=3, blk=blk, S=S, nblk=nblk, topk=1, qblk=qblk)
+    nqb = S // qblk
+    chosen = (np.arange(nqb) * 2 + 1) % nblk  # a different block for neighbouring query blocks
+    idx = chosen.astype(np.int32).reshape(1, 1, nqb, 1)
+    vh = np.repeat((np.arange(nblk, dtype=np.float64) + 1.0), blk)[None, :, None, None] * np.ones((1, 1, 1, D.d))
+    kh = _rng(33).standard_normal((1, nblk * blk, 1, D.d))
+    ks = _rng(34).standard_normal((1, S, 1, D.d))
+    o, lse = oracle.attn_fwd(D, np.zeros((1, S, D.Hq, D.d)), ks, np.zeros_like(ks), kh, vh, idx)
+    for p in range(S):
+        n = chosen[p // qblk]
+        want = blk * (n + 1.0) / (blk + p + 1.0)
+        np.testing.assert_allclose(o[0, p], want, rtol=0, atol=1e-14)
+        assert abs(lse[0, 0, p] - math.log(blk + p + 1.0)) < 1e-14
+
+
+def test_all_blocks_selected_equals_dense_with_other_query_block_size():
+    """K = every history block makes the query-block size irrelevant: HGA
+    equals dense causal attention over history + segment for qblk != blk."""
+    Hkv, G, blk, nblk, S = 2, 2, 4, 3, 16
+    D = Dims(B=1, Hq=Hkv * G, Hkv=Hkv, d=8, blk=blk, S=S, nblk=nblk, topk=nblk, qblk=8)
+    q, ks, vs, kh, vh, _ = _rand_inputs(D, 35)
+    idx, _ = oracle.select(D, q, kh)
+    assert idx.shape == (1, Hkv, 2, nblk) and np.all(idx == np.arange(nblk))
+    o, lse = oracle.attn_fwd(D, q, ks, vs, kh, vh, idx)
+    H = nblk * blk
+    qf = np.concatenate([_rng(36).standard_normal((1, H, D.Hq, D.d)), q], axis=1)
+    o2, lse2 = oracle.dense_causal_fwd(qf, np.concatenate([kh, ks], axis=1), np.concatenate([vh, vs], axis=1))
+    np.testing.assert_allclose(o, o2[:, H:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2[:, :, H:], rtol=0, atol=1e-12)
+
+
+def test_sparse_backward_mask_counts_query_blocks_of_qblk_rows():
+    """qmask has one entry per query block of qblk rows: with only query block
+    1 chosen, dQ is zero outside rows [qblk, 2*qblk) and non-zero inside."""
+    D = Dims(B=1, Hq=2, Hkv=1, d=4, blk=2, S=12, nblk=4, topk=2, qblk=4)
+    q, ks, vs, kh, vh, do = _rand_inputs(D, 37)
+    idx, _ = oracle.select(D, q, kh)
+    mask = np.zeros((1, D.nqb), np.int8)
+    mask[0, 1] = 1
+    dq, dk, dv = oracle.attn_bwd_sparse(D, q, ks, vs, kh, vh, idx, do, mask, 1.0)
+    rows = np.abs(dq[0]).sum(axis=(1, 2))
+    assert np.all(rows[:4] == 0) and np.all(rows[8:] == 0) and np.all(rows[4:8] > 0)
+    # keys after the chosen rows get no gradient
+    assert np.all(dk[0, 8:] == 0) and np.all(dv[0, 8:] == 0)
