@@ -97,6 +97,13 @@ typedef enum { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype;
 typedef struct {
   int B, Hq, Hkv, d, block, S, n_hist_blocks, topk;
   hga_dtype dtype;
+  /* Query-block size: the segment rows that share one selection.  0 = block
+   * (one size for history blocks and query blocks).  Otherwise in
+   * {16, 32, 64, 128}, S % q_block == 0; a query block's mean is over its
+   * q_block rows, and each of its rows attends to the `block` tokens of every
+   * block selected for it.  idx and qblock_mask have S / q_block query
+   * blocks; a finished segment still becomes S / block history blocks. */
+  int q_block;
 } hga_dims;
 
 /* A CUDA stream (cudaStream_t); NULL = legacy default stream. */

@@ -34,7 +34,7 @@ class HgaError(RuntimeError):
 class hga_dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
                 ("block", ctypes.c_int), ("S", ctypes.c_int), ("n_hist_blocks", ctypes.c_int),
-                ("topk", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("topk", ctypes.c_int), ("dtype", ctypes.c_int), ("q_block", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -48,10 +48,15 @@ class Dims:
     n_hist_blocks: int
     topk: int
     dtype: str = "bf16"  # "bf16" or "f32"
+    q_block: int = 0     # query-block size; 0 = block (one size for history and query blocks)
+
+    @property
+    def qb(self) -> int:
+        return self.q_block or self.block
 
     @property
     def nqb(self) -> int:
-        return self.S // self.block
+        return self.S // self.qb
 
     @property
     def torch_dtype(self):
@@ -59,10 +64,11 @@ class Dims:
 
     def c(self) -> hga_dims:
         return hga_dims(self.B, self.Hq, self.Hkv, self.d, self.block, self.S, self.n_hist_blocks, self.topk,
-                        HGA_BF16 if self.dtype == "bf16" else HGA_F32)
+                        HGA_BF16 if self.dtype == "bf16" else HGA_F32, self.q_block)
 
     def with_history(self, n_hist_blocks: int) -> "Dims":
-        return Dims(self.B, self.Hq, self.Hkv, self.d, self.block, self.S, n_hist_blocks, self.topk, self.dtype)
+        return Dims(self.B, self.Hq, self.Hkv, self.d, self.block, self.S, n_hist_blocks, self.topk, self.dtype,
+                    self.q_block)
 
 
 class hga_block_cache(ctypes.Structure):

@@ -139,11 +139,15 @@ hga_status check_dims(const hga_dims* d, hga::Shape* out) {
   if (d->block != 16 && d->block != 32 && d->block != 64 && d->block != 128)
     return fail(HGA_ERR_SHAPE, "block %d not in {16,32,64,128}", d->block);
   if (d->S % d->block) return fail(HGA_ERR_SHAPE, "S (%d) not a multiple of block (%d)", d->S, d->block);
+  if (d->q_block != 0 && d->q_block != 16 && d->q_block != 32 && d->q_block != 64 && d->q_block != 128)
+    return fail(HGA_ERR_SHAPE, "q_block %d not in {0,16,32,64,128}", d->q_block);
+  const int qblk = d->q_block ? d->q_block : d->block;
+  if (d->S % qblk) return fail(HGA_ERR_SHAPE, "S (%d) not a multiple of q_block (%d)", d->S, qblk);
   if (d->topk > hga::kMaxTopk) return fail(HGA_ERR_SHAPE, "topk %d > %d", d->topk, hga::kMaxTopk);
   const double tokens = (double)d->B * ((double)d->n_hist_blocks * d->block + d->S) * d->Hq * d->d;
   if (tokens > 4.0e12) return fail(HGA_ERR_SHAPE, "problem too large");
   out->B = d->B; out->Hq = d->Hq; out->Hkv = d->Hkv; out->d = d->d; out->blk = d->block; out->S = d->S;
-  out->nblk = d->n_hist_blocks; out->topk = d->topk; out->bf16 = (d->dtype == HGA_BF16);
+  out->nblk = d->n_hist_blocks; out->topk = d->topk; out->bf16 = (d->dtype == HGA_BF16); out->qblk = qblk;
   return HGA_OK;
 }
 
@@ -268,12 +272,12 @@ hga_status hga_segment_summaries(const hga_dims* dims, const void* k_seg, int at
   hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
-  if (at_block < 0 || at_block + s.nqb() > s.nblk)
-    return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the summary array's %d", at_block, at_block + s.nqb(),
+  if (at_block < 0 || at_block + s.nsb() > s.nblk)
+    return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the summary array's %d", at_block, at_block + s.nsb(),
                 s.nblk);
   if (any_null(k_seg, summ)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(k_seg)) return fail(HGA_ERR_INVALID_ARG, "k_seg must be 16-byte aligned");
-  cudaError_t e = hga::launch_block_summaries(s, k_seg, s.S, 0, at_block, s.nqb(), summ,
+  cudaError_t e = hga::launch_block_summaries(s, k_seg, s.S, 0, at_block, s.nsb(), summ,
                                               reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "segment summaries launch");
 }
@@ -789,7 +793,7 @@ hga_status hga_cache_segment(const hga_dims* dims, const void* k_seg, const void
   if (r != HGA_OK) return r;
   if (any_null(k_seg, v_seg, pool_k, pool_v, cache)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
   if (!cache_arrays_ok(cache)) return fail(HGA_ERR_INVALID_ARG, "block cache: NULL arrays or negative sizes");
-  const int nseg = s.nqb();
+  const int nseg = s.nsb();
   if (at_block < 0 || at_block + nseg > cache->host_capacity_blocks)
     return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the cache's %d", at_block, at_block + nseg,
                 cache->host_capacity_blocks);
@@ -877,7 +881,7 @@ hga_status hga_append_segment(const hga_dims* dims, const void* k_seg, const voi
   hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
-  const int nseg = s.nqb();
+  const int nseg = s.nsb();
   if (nseg > hga::kMaxQueryBlocks) return fail(HGA_ERR_SHAPE, "segment of %d blocks > %d", nseg, hga::kMaxQueryBlocks);
   if (any_null(k_seg, v_seg, summ)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(k_seg) || !aligned16(v_seg)) return fail(HGA_ERR_INVALID_ARG, "k_seg/v_seg must be 16-byte aligned");
@@ -964,7 +968,7 @@ hga_status hga_offload_segment(const hga_dims* dims, const void* k_seg, const vo
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
   if (any_null(k_seg, v_seg, host_k, host_v)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
-  const int nseg = s.nqb();
+  const int nseg = s.nsb();
   if (at_block < 0 || at_block + nseg > capacity_blocks)
     return fail(HGA_ERR_INVALID_ARG, "blocks [%d,%d) outside the tier's %d", at_block, at_block + nseg,
                 capacity_blocks);
@@ -989,7 +993,7 @@ hga_status hga_decode_select(const hga_dims* dims, int n_q, const void* q_new, c
   hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
-  if (n_q < 1 || n_q > s.blk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, block = %d]", n_q, s.blk);
+  if (n_q < 1 || n_q > s.qblk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, query block = %d]", n_q, s.qblk);
   if (s.nblk > hga::kMaxSelectBlocks)
     return fail(HGA_ERR_SHAPE, "n_hist_blocks %d > %d", s.nblk, hga::kMaxSelectBlocks);
   if (any_null(q_new, idx, ws) || (s.nblk > 0 && summ == nullptr)) return fail(HGA_ERR_INVALID_ARG, "NULL pointer");
@@ -1003,7 +1007,7 @@ hga_status hga_decode_select(const hga_dims* dims, int n_q, const void* q_new, c
 
 size_t hga_decode_workspace_size(const hga_dims* dims, int n_q) {
   hga::Shape s{};
-  if (check_dims(dims, &s) != HGA_OK || n_q < 1 || n_q > s.blk) return 0;
+  if (check_dims(dims, &s) != HGA_OK || n_q < 1 || n_q > s.qblk) return 0;
   const size_t attn = hga::decode_workspace_floats(s, n_q) * sizeof(float);
   const size_t select = (size_t)s.B * s.Hkv * (s.nblk > 0 ? s.nblk : 1) * sizeof(unsigned long long);
   return round256(attn > select ? attn : select);
@@ -1015,7 +1019,7 @@ hga_status hga_decode_attn(const hga_dims* dims, int n_q, int t0, const void* q_
   hga::Shape s{};
   hga_status r = check_dims(dims, &s);
   if (r != HGA_OK) return r;
-  if (n_q < 1 || n_q > s.blk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, block = %d]", n_q, s.blk);
+  if (n_q < 1 || n_q > s.qblk) return fail(HGA_ERR_SHAPE, "n_q %d outside [1, query block = %d]", n_q, s.qblk);
   if (t0 < 0 || t0 + n_q > s.S)
     return fail(HGA_ERR_SHAPE, "new tokens [%d, %d) outside the segment buffer of %d", t0, t0 + n_q, s.S);
   if (s.topk + (s.S + s.blk - 1) / s.blk > 512)

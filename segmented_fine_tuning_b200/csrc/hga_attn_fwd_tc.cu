@@ -364,7 +364,8 @@ __global__ void __launch_bounds__(384, 1)
 }  // namespace
 
 bool tc_supported(const Shape& s) {
-  return s.bf16 && (s.d == 128 || s.d == 64) && s.blk == kBM && (s.G() % 2) == 0 && s.topk <= kMaxTopk &&
+  return s.bf16 && (s.d == 128 || s.d == 64) && s.blk == kBM && s.qblk == kBM && (s.G() % 2) == 0 &&
+         s.topk <= kMaxTopk &&
          s.nqb() <= kMaxQueryBlocks;
 }
 

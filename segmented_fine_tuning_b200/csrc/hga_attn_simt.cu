@@ -50,6 +50,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 struct SimtArgs {
   int B, Hq, Hkv, d, blk, S, nkv, topk, nqb, G;
+  int qblk;     // query-block size (rows sharing one selection); blk = history block size
   float scale;  // 1/sqrt(d)
   const int32_t* idx;
   int* err;
@@ -58,7 +59,7 @@ struct SimtArgs {
 };
 
 __device__ __forceinline__ bool block_on(const SimtArgs& a, int b, int p) {
-  return !a.qmask || a.qmask[(size_t)b * a.nqb + p / a.blk];
+  return !a.qmask || a.qmask[(size_t)b * a.nqb + p / a.qblk];
 }
 
 // Key j of query block i: either history token (block idx, offset) or a
@@ -67,7 +68,7 @@ __device__ __forceinline__ bool block_on(const SimtArgs& a, int b, int p) {
 template <int DPL, typename T, typename F>
 __device__ __forceinline__ void for_each_key(const SimtArgs& a, int b, int h, int p, const T* ks, const T* kh,
                                              F&& f) {
-  const int i = p / a.blk;
+  const int i = p / a.qblk;
   const int32_t* sel = a.idx + (((size_t)b * a.Hkv + h) * a.nqb + i) * a.topk;
   const size_t hist_T = (size_t)a.nkv * a.blk;
   for (int r = 0; r < a.topk; ++r) {
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(256) dkdv_simt_kernel(SimtArgs a, const T* __r
 SimtArgs make_args(const Shape& s, int nkv, const int32_t* idx, int* err) {
   SimtArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.d = s.d; a.blk = s.blk; a.S = s.S; a.nkv = nkv; a.topk = s.topk;
-  a.nqb = s.nqb(); a.G = s.G(); a.scale = 1.0f / sqrtf((float)s.d); a.idx = idx; a.err = err;
+  a.nqb = s.nqb(); a.G = s.G(); a.qblk = s.qblk; a.scale = 1.0f / sqrtf((float)s.d); a.idx = idx; a.err = err;
   a.qmask = nullptr; a.gscale = 1.0f;
   return a;
 }

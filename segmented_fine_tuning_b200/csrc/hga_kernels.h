@@ -14,8 +14,10 @@ enum : int { kDevErrIndex = 1, kDevErrTimeout = 2 };
 struct Shape {
   int B, Hq, Hkv, d, blk, S, nblk, topk;
   bool bf16;
+  int qblk;  // query-block size (blk when the dims leave it 0)
   int G() const { return Hq / Hkv; }
-  int nqb() const { return S / blk; }
+  int nqb() const { return S / qblk; }  // query blocks of the segment
+  int nsb() const { return S / blk; }   // history blocks the finished segment becomes
 };
 
 // Largest K and history length the selection kernel handles in one CTA.

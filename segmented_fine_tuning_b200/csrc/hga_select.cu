@@ -669,7 +669,7 @@ cudaError_t launch_block_summaries(const Shape& s, const void* k_src, int T_src,
 
 cudaError_t launch_append_segment(const Shape& s, const void* k_seg, const void* v_seg, int dst_b0, float* summ,
                                   void* pool_k, void* pool_v, int pool_slots, const int32_t* slots, cudaStream_t st) {
-  const int nqb = s.nqb();
+  const int nqb = s.nsb();  // the segment's blocks
   if (nqb <= 0) return cudaSuccess;
   AppendSlots sl;
   for (int t = 0; t < kMaxQueryBlocks; ++t) sl.slot[t] = (pool_k && t < nqb) ? slots[t] : 0;
@@ -699,13 +699,13 @@ cudaError_t launch_select_topk(const Shape& s, const void* q, const float* summ,
     auto kern = select_kernel<__nv_bfloat16>;
     if ((e = smem_limit(reinterpret_cast<const void*>(kern), smem)) != cudaSuccess)
       return e;
-    kern<<<grid, kSelThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk,
+    kern<<<grid, kSelThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.qblk, s.nblk,
                                   s.topk, isd, idx, scores);
   } else {
     auto kern = select_kernel<float>;
     if ((e = smem_limit(reinterpret_cast<const void*>(kern), smem)) != cudaSuccess)
       return e;
-    kern<<<grid, kSelThreads, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.blk, s.nblk, s.topk,
+    kern<<<grid, kSelThreads, smem, st>>>(static_cast<const float*>(q), summ, s.S, s.Hq, s.Hkv, s.d, s.qblk, s.nblk, s.topk,
                                   isd, idx, scores);
   }
   return cudaGetLastError();

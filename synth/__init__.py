@@ -45,6 +45,7 @@ class Workload:
     structured_keys: bool = False
     dominant_frac: float = 0.0
     fwd_only: bool = False
+    qblk: int = 0  # query-block size; 0 = blk
 
     @property
     def T(self) -> int:
@@ -55,8 +56,12 @@ class Workload:
         return self.Hq // self.Hkv
 
     @property
+    def qb(self) -> int:
+        return self.qblk or self.blk
+
+    @property
     def nqb(self) -> int:
-        return self.S // self.blk
+        return self.S // self.qb
 
 
 # The five workloads of the HGA attention step.

@@ -9,7 +9,7 @@ from segmented_fine_tuning_b200 import Dims
 
 
 def dims_of(w: synth.Workload, nblk: int | None = None) -> Dims:
-    return Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk if nblk is None else nblk, w.topk, w.dtype)
+    return Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk if nblk is None else nblk, w.topk, w.dtype, w.qblk)
 
 
 def to_dev(t: synth.Tensor, device="cuda") -> torch.Tensor:

@@ -62,6 +62,8 @@ BAD_DIMS = [
     dict(topk=65),       # K <= 64
     dict(B=0),
     dict(n_hist_blocks=-1),
+    dict(q_block=48),                      # query-block size
+    dict(block=32, S=96, q_block=64),      # S % q_block
 ]
 
 

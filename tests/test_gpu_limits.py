@@ -26,7 +26,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _odims(w):
-    return oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk)
+    return oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.qblk)
 
 
 def _run(w, x, backward=True):

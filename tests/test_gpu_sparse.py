@@ -28,6 +28,8 @@ CASES = [
     (synth.Workload("sparse-tc-B2: B2 Hq4/Hkv2 S384 hist4 K2", 2, 4, 2, 128, 128, 384, 4, 2, "bf16", 112), 1),
     (synth.QWEN3_8B_LAYER, 4),
     (synth.TINY_F32, 2),
+    (synth.Workload("sparse-qblk64-blk128: Hq4/Hkv2 S384 hist4 K2", 1, 4, 2, 128, 128, 384, 4, 2, "bf16", 113,
+                    qblk=64), 2),
 ]
 
 
@@ -48,7 +50,7 @@ def test_sparse_backward_matches_oracle(w, k):
                         st.o, st.lse, dev["d_o"], mask.cuda(), scale, dq, dk, dv, st.ws)
     torch.cuda.synchronize()
     hga_device_status()
-    od = oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk)
+    od = oracle.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.qblk)
     idx = st.idx.cpu().numpy()
     ref = oracle.attn_bwd_sparse(od, x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx, x.d_o.f64,
                                  mask.numpy().astype(np.int8), scale)
@@ -60,7 +62,7 @@ def test_sparse_backward_matches_oracle(w, k):
     for b in range(w.B):
         for i in range(w.nqb):
             if not mask[b, i]:
-                assert np.all(dqh[b, i * w.blk:(i + 1) * w.blk] == 0.0)
+                assert np.all(dqh[b, i * w.qb:(i + 1) * w.qb] == 0.0)
     print(f"{w.name}: {k} of {w.nqb} query blocks, scale {scale}")
 
 
