@@ -109,6 +109,7 @@ _SIGNATURES = [
                                      ctypes.POINTER(ctypes.c_int), _P, _P, _P, _I]),
     ("hga_cache_segment", _I, [_D, _P, _P, _P, _P, _C, _I, _P]),
     ("hga_remap_idx", _I, [_D, _P, _P, _P, _P]),
+    ("hga_attn_uses_tensor_cores", _I, [_D, _I]),
     ("hga_append_segment", _I, [_D, _P, _P, _I, _P, _P, _P, _C, _P, _P, _I, _P, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
     ("hga_decode_select", _I, [_D, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -558,3 +559,11 @@ def spaco_sample_blocks(B: int, n_qblocks: int, k: int, generator: torch.Generat
         mask[b, torch.randperm(n_qblocks, generator=generator)[:k]] = 1
     scale = n_qblocks / k
     return mask, (min(scale, cap) if cap is not None else scale)
+
+
+def hga_attn_uses_tensor_cores(dims: Dims, n_kv_blocks: int) -> bool:
+    """True when the attention calls run these dims on the tcgen05 kernels."""
+    r = load_library().hga_attn_uses_tensor_cores(ctypes.byref(dims.c()), n_kv_blocks)
+    if r < 0:
+        raise ValueError(f"dims rejected by the library: {load_library().hga_last_error().decode()}")
+    return bool(r)

@@ -108,16 +108,17 @@ hga_status get_encoder(EncodeTiledFn* fn) {
   return HGA_OK;
 }
 
-// bf16 tensor [B, T, H, d] (d in {64, 128}) with a {64, 1, 128, 1} box (128
-// tokens x 64 channels = 128-byte rows), 128-byte swizzle.
-hga_status encode_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
+// bf16 tensor [B, T, H, d] (d in {64, 128}) with a {64, 1, rows, 1} box (rows
+// tokens x 64 channels = 128-byte rows; rows 128, or 64 for the history when
+// its blocks hold 64 tokens), 128-byte swizzle.
+hga_status encode_tokens(CUtensorMap* m, const void* base, int B, int T, int H, int d, int rows = 128) {
   EncodeTiledFn enc = nullptr;
   hga_status s = get_encoder(&enc);
   if (s != HGA_OK) return s;
   const cuuint64_t D = (cuuint64_t)d;
   const cuuint64_t dims[4] = {D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t strides[3] = {D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -167,6 +168,12 @@ hga_status check_attn_ptrs(const hga::Shape& s, int n_kv_blocks, const void* q, 
   return HGA_OK;
 }
 
+// The tensor-core kernels take the shape, and with 64-token history blocks
+// they pack two block indices of 15 bits into one tile entry.
+bool use_tc(const hga::Shape& s, int n_kv_blocks) {
+  return hga::tc_supported(s) && (s.blk != 64 || n_kv_blocks < 0x7FFF);
+}
+
 hga_status build_maps(const hga::Shape& s, int nkv, const void* q, const void* d_o, const void* ks, const void* vs,
                       const void* kh, const void* vh, hga::TcMaps* m) {
   hga_status r;
@@ -175,8 +182,11 @@ hga_status build_maps(const hga::Shape& s, int nkv, const void* q, const void* d
   if ((r = encode_tokens(&m->ks, ks, s.B, s.S, s.Hkv, s.d)) != HGA_OK) return r;
   if ((r = encode_tokens(&m->vs, vs, s.B, s.S, s.Hkv, s.d)) != HGA_OK) return r;
   // With no history the history maps are never read; point them at the segment.
-  if ((r = encode_tokens(&m->kh, nkv > 0 ? kh : ks, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv, s.d)) != HGA_OK) return r;
-  if ((r = encode_tokens(&m->vh, nkv > 0 ? vh : vs, s.B, nkv > 0 ? nkv * 128 : s.S, s.Hkv, s.d)) != HGA_OK) return r;
+  const int hr = nkv > 0 ? s.blk : 128;  // history box rows: one block
+  if ((r = encode_tokens(&m->kh, nkv > 0 ? kh : ks, s.B, nkv > 0 ? nkv * s.blk : s.S, s.Hkv, s.d, hr)) != HGA_OK)
+    return r;
+  if ((r = encode_tokens(&m->vh, nkv > 0 ? vh : vs, s.B, nkv > 0 ? nkv * s.blk : s.S, s.Hkv, s.d, hr)) != HGA_OK)
+    return r;
   return HGA_OK;
 }
 
@@ -307,7 +317,7 @@ hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, 
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (hga::tc_supported(s)) {
+  if (use_tc(s, n_kv_blocks)) {
     hga::TcMaps m;
     if ((r = build_maps(s, n_kv_blocks, q, nullptr, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
     e = hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, st);
@@ -391,7 +401,7 @@ hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const
   if (pre && (e = hga::launch_bwd_preprocess(s, o, d_o, Dr, st)) != cudaSuccess)
     return cuda_fail(e, "backward preprocess launch");
   if (!parts) return HGA_OK;
-  if (hga::tc_supported(s)) {
+  if (use_tc(s, n_kv_blocks)) {
     hga::TcMaps m;
     if ((r = build_maps(s, n_kv_blocks, q, d_o, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
     int dev = 0;
@@ -427,6 +437,12 @@ hga_status run_bwd(const hga_dims* dims, const void* q, const void* k_seg, const
 }  // namespace
 
 extern "C" {
+
+int hga_attn_uses_tensor_cores(const hga_dims* dims, int n_kv_blocks) {
+  hga::Shape s{};
+  if (check_dims(dims, &s) != HGA_OK || n_kv_blocks < 0) return -1;
+  return use_tc(s, n_kv_blocks) ? 1 : 0;
+}
 
 hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
                         const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, const void* o,

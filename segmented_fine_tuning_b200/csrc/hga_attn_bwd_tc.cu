@@ -43,6 +43,9 @@ constexpr int kB = 128;  // rows / keys per tile
 constexpr int kHalf = kB * 128;              // one 64-channel TMA box: 128 rows x 128 B
 constexpr int kSubRows = 64;                 // rows of a sub-tile
 constexpr int kSubOff = kSubRows * 128;      // byte offset of the second 64-row half inside a box
+// History tiles of 64-token blocks hold two blocks: tile = n0 | (n1 << 16),
+// n1 = kNoBlock when the tile's upper 64 keys have no block (an odd count).
+constexpr int kNoBlock = 0x7FFF;
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kLog2e = 1.4426950408889634f;
 // Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
@@ -75,6 +78,7 @@ struct BwdArgs {
   // qmask == nullptr and gscale == 1: the plain backward.
   const uint8_t* qmask;
   float gscale;
+  int hblk;  // history block tokens: 128 (one block per tile) or 64 (two per tile)
 };
 
 // ============================================================== dQ kernel
@@ -149,6 +153,19 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) ctl->tiles[nh + __popc(m & ((1u << lane) - 1u))] = n;
       nh += __popc(m);
     }
+    if (a.hblk == 64) {
+      // 64-token history blocks: two per 128-key tile (nh <= 64, so one pass)
+      __syncwarp();
+      const int np = (nh + 1) >> 1;
+      int packed = 0;
+      if (lane < np) {
+        const int n1 = (2 * lane + 1 < nh) ? ctl->tiles[2 * lane + 1] : kNoBlock;
+        packed = ctl->tiles[2 * lane] | (n1 << 16);
+      }
+      __syncwarp();
+      if (lane < np) ctl->tiles[lane] = packed;
+      nh = np;
+    }
     for (int jb = lane; jb <= i; jb += 32) ctl->tiles[nh + jb] = -(jb + 1);
     if (lane == 0) {
       ctl->nt = nh + i + 1;
@@ -185,19 +202,27 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; j < nt; ++j) {
         const int tile = ctl->tiles[j];
         const bool hist = tile >= 0;
-        const int row0 = (hist ? tile : (-tile - 1)) * kB;
+        const bool pair = hist && a.hblk == 64;
+        const int row0 = pair ? (tile & 0xFFFF) * 64 : (hist ? tile : (-tile - 1)) * kB;
+        // the upper half of a lone block's tile repeats it (finite values; its
+        // keys get P = 0 in the dS pass)
+        const int row1 = pair ? ((tile >> 16) == kNoBlock ? row0 : (tile >> 16) * 64) : 0;
         const int ks = j % kKStages, vs = j % kVStages;
         if (!mbar_wait(&ctl->k_empty[ks], ((j / kKStages) & 1) ^ 1, abort, a.err)) break;
         mbar_expect_tx(&ctl->k_full[ks], kTileBytes);
-        for (int hh = 0; hh < kBoxes; ++hh)
-          tma_load_4d(hist ? &tm_kh : &tm_ks, &ctl->k_full[ks], sK + ks * kTileBytes + hh * kHalf, hh * 64, kvh,
-                      row0, b);
+        for (int hh = 0; hh < kBoxes; ++hh) {
+          uint8_t* dst = sK + ks * kTileBytes + hh * kHalf;
+          tma_load_4d(hist ? &tm_kh : &tm_ks, &ctl->k_full[ks], dst, hh * 64, kvh, row0, b);
+          if (pair) tma_load_4d(&tm_kh, &ctl->k_full[ks], dst + kSubOff, hh * 64, kvh, row1, b);
+        }
         k_issued = j + 1;
         if (!mbar_wait(&ctl->v_empty[vs], ((j / kVStages) & 1) ^ 1, abort, a.err)) break;
         mbar_expect_tx(&ctl->v_full[vs], kTileBytes);
-        for (int hh = 0; hh < kBoxes; ++hh)
-          tma_load_4d(hist ? &tm_vh : &tm_vs, &ctl->v_full[vs], sV + vs * kTileBytes + hh * kHalf, hh * 64, kvh,
-                      row0, b);
+        for (int hh = 0; hh < kBoxes; ++hh) {
+          uint8_t* dst = sV + vs * kTileBytes + hh * kHalf;
+          tma_load_4d(hist ? &tm_vh : &tm_vs, &ctl->v_full[vs], dst, hh * 64, kvh, row0, b);
+          if (pair) tma_load_4d(&tm_vh, &ctl->v_full[vs], dst + kSubOff, hh * 64, kvh, row1, b);
+        }
         v_issued = j + 1;
       }
       volatile int no_abort = 0;
@@ -300,7 +325,13 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld64x2_wait(tmem + lane_off + kDqS + x * 128 + 64 * e, tmem + lane_off + kDqP + 64 * e, sd);
       tc_fence_before();
       mbar_arrive(&ctl->dp_free);  // dP(j) is in registers: the tensor core may overwrite it
-      const bool diag = (j == nt - 1);
+      // keys above `lim` get P = 0: the diagonal segment tile masks keys after
+      // the row's own position; a history tile holding one 64-token block
+      // masks its upper 64 keys
+      int lim = 127;
+      if (j == nt - 1) lim = r;
+      else if (a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) lim = 63;
+      const bool diag = lim < 127;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t pk[16];
@@ -311,8 +342,8 @@ __global__ void __launch_bounds__(320, 1)
                                 s2, nl);
           float2 pr = exp2_pair(x, (kBwdPolyPairs >> (xx >> 1)) & 1u);
           if (diag) {
-            pr.x = key <= r ? pr.x : 0.f;
-            pr.y = key + 1 <= r ? pr.y : 0.f;
+            pr.x = key <= lim ? pr.x : 0.f;
+            pr.y = key + 1 <= lim ? pr.y : 0.f;
           }
           const float2 ds = mul2(pr, sub2(make_float2(__uint_as_float(sd[64 + 32 * cc + xx]),
                                                       __uint_as_float(sd[64 + 32 * cc + xx + 1])),
@@ -613,7 +644,7 @@ cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
   a.scale = 1.0f / sqrtf((float)KD);
   a.sl2 = kLog2e * a.scale;
   a.idx = idx; a.lse = lse; a.Dr = Dr; a.dq = dq; a.dk = dk; a.dv = dv; a.err = err;
-  a.qmask = qmask; a.gscale = gscale;
+  a.qmask = qmask; a.gscale = gscale; a.hblk = s.blk;
   if (parts & kBwdDkdv) {
     // Per-head partials are added into the outputs: start from zero.
     const size_t kv_bytes = (size_t)s.B * s.S * s.Hkv * KD * sizeof(float);

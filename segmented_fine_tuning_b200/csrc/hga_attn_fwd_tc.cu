@@ -38,6 +38,10 @@ namespace {
 constexpr int kBM = 128;                      // query rows per tile
 constexpr int kBN = 128;                      // keys per tile
 constexpr int kHalf = kBM * 128;              // one 64-column TMA box: 128 rows x 128 bytes
+constexpr int kRowHalf = 64 * 128;            // byte offset of row 64 inside a box
+// History tiles of 64-token blocks hold two blocks: tile = n0 | (n1 << 16),
+// n1 = kNoBlock when the tile's upper 64 keys have no block (an odd count).
+constexpr int kNoBlock = 0x7FFF;
 constexpr int kStages = 5;                    // K/V ring slots
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -76,6 +80,7 @@ struct FwdArgs {
   float* lse;
   int* err;
   int withhold_kv;  // self test of the timeout path: the producer issues no K/V loads
+  int hblk;         // history block tokens: 128 (one block per tile) or 64 (two per tile)
 };
 
 template <int KD>
@@ -113,6 +118,19 @@ __global__ void __launch_bounds__(384, 1)
       const unsigned m = __ballot_sync(0xffffffffu, ok);
       if (ok) ctl->tiles[nh + __popc(m & ((1u << lane) - 1u))] = n;
       nh += __popc(m);
+    }
+    if (a.hblk == 64) {
+      // 64-token history blocks: two per 128-key tile (nh <= 64, so one pass)
+      __syncwarp();
+      const int np = (nh + 1) >> 1;
+      int packed = 0;
+      if (lane < np) {
+        const int n1 = (2 * lane + 1 < nh) ? ctl->tiles[2 * lane + 1] : kNoBlock;
+        packed = ctl->tiles[2 * lane] | (n1 << 16);
+      }
+      __syncwarp();
+      if (lane < np) ctl->tiles[lane] = packed;
+      nh = np;
     }
     for (int jb = lane; jb <= i; jb += 32) ctl->tiles[nh + jb] = -(jb + 1);
     if (lane == 0) {
@@ -158,7 +176,11 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < (a.withhold_kv ? 0 : nt); ++j) {
         const int tile = ctl->tiles[j];
         const bool hist = tile >= 0;
-        const int row0 = (hist ? tile : (-tile - 1)) * kBN;
+        const bool pair = hist && a.hblk == 64;
+        const int row0 = pair ? (tile & 0xFFFF) * 64 : (hist ? tile : (-tile - 1)) * kBN;
+        // the upper half of a lone block's tile repeats it (finite values; its
+        // keys are masked in the softmax)
+        const int row1 = pair ? ((tile >> 16) == kNoBlock ? row0 : (tile >> 16) * 64) : 0;
         bool ok = true;
         for (int w = 0; w < 2 && ok; ++w) {
           const int pos = 2 * j + w;
@@ -169,8 +191,11 @@ __global__ void __launch_bounds__(384, 1)
           }
           const CUtensorMap* m = hist ? (w ? &tm_vh : &tm_kh) : (w ? &tm_vs : &tm_ks);
           mbar_expect_tx(&ctl->kv_full[s], kTileBytes);
-          for (int hh = 0; hh < kBoxes; ++hh)
-            tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes + hh * kHalf, hh * 64, kvh, row0, b);
+          for (int hh = 0; hh < kBoxes; ++hh) {
+            uint8_t* dst = sRing + s * kTileBytes + hh * kHalf;
+            tma_load_4d(m, &ctl->kv_full[s], dst, hh * 64, kvh, row0, b);
+            if (pair) tma_load_4d(m, &ctl->kv_full[s], dst + kRowHalf, hh * 64, kvh, row1, b);
+          }
           issued = pos + 1;
         }
         if (!ok) break;
@@ -283,6 +308,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (e > r) v[e] = 0xFF800000u;  // -inf
+      } else if (a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) {
+        // a history tile holding one 64-token block: its upper 64 keys are masked
+#pragma unroll
+        for (int e = 64; e < 128; ++e) v[e] = 0xFF800000u;
       }
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -364,7 +393,7 @@ __global__ void __launch_bounds__(384, 1)
 }  // namespace
 
 bool tc_supported(const Shape& s) {
-  return s.bf16 && (s.d == 128 || s.d == 64) && s.blk == kBM && s.qblk == kBM && (s.G() % 2) == 0 &&
+  return s.bf16 && (s.d == 128 || s.d == 64) && (s.blk == kBM || s.blk == 64) && s.qblk == kBM && (s.G() % 2) == 0 &&
          s.topk <= kMaxTopk &&
          s.nqb() <= kMaxQueryBlocks;
 }
@@ -378,7 +407,7 @@ cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
   FwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
   a.sl2 = 1.4426950408889634f / sqrtf((float)KD);
-  a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err;
+  a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err; a.hblk = s.blk;
   a.withhold_kv = withhold_kv ? 1 : 0;
   const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
   fwd_tc_kernel<KD><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);

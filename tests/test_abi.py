@@ -184,3 +184,21 @@ def test_size_limits_rejected_on_host(lib):
     d = _dims(S=129 * 128, n_hist_blocks=129 * 128 // 128 + 1)
     assert lib.hga_append_segment(ctypes.byref(d), p, p, 0, p, None, None, None, None, None, 0, None, None) == 2
     assert "128" in lib.hga_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,nkv,want", [
+    (dict(), 4, 1),                                        # bf16, d128, block 128
+    (dict(d=64), 4, 1),                                    # head dim 64
+    (dict(block=64, q_block=128), 9, 1),                   # 64-token history blocks, two per tile
+    (dict(block=64, q_block=128, n_hist_blocks=40000, topk=4), 40000, 0),  # block indices past 15 bits
+    (dict(block=64), 9, 0),                                # 64-row query blocks: CUDA-core kernels
+    (dict(block=128, q_block=64), 4, 0),
+    (dict(dtype=0), 4, 0),                                 # fp32
+    (dict(Hq=6, Hkv=2), 4, 0),                             # odd group size
+    (dict(block=32, q_block=128), 4, 0),                   # 32-token history blocks
+    (dict(q_block=48), 4, -1),                             # rejected dims
+])
+def test_tensor_core_path_selection(lib, kw, nkv, want):
+    """Which kernels the attention calls use for a shape (host-only query)."""
+    d = _dims(**kw)
+    assert lib.hga_attn_uses_tensor_cores(ctypes.byref(d), nkv) == want, (kw, lib.hga_last_error())

@@ -30,6 +30,8 @@ CASES = [
     (synth.TINY_F32, 2),
     (synth.Workload("sparse-qblk64-blk128: Hq4/Hkv2 S384 hist4 K2", 1, 4, 2, 128, 128, 384, 4, 2, "bf16", 113,
                     qblk=64), 2),
+    (synth.Workload("sparse-tc-blk64: Hq4/Hkv2 S512 hist11 K5", 1, 4, 2, 128, 64, 512, 11, 5, "bf16", 114,
+                    qblk=128), 2),
 ]
 
 
