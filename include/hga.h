@@ -30,8 +30,9 @@
  *                     and the selection get no gradient.
  *
  * Notation: B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0, query head hq
- * uses KV head hq / (Hq/Hkv)), d head dim, `block` tokens per history block and
- * per query block, S segment tokens (S % block == 0), Nqb = S / block.
+ * uses KV head hq / (Hq/Hkv)), d head dim, `block` tokens per history block,
+ * q_block rows per query block (dims.q_block, 0 = block), S segment tokens
+ * (S % block == 0 and S % q_block == 0), Nqb = S / q_block.
  *
  * Layouts (row-major, token-major as QKV projections produce them):
  *   q, o, d_o           [B, S, Hq, d]          dtype
