@@ -294,7 +294,7 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
 /*
  * Decode step (article, Industry impact; fr edition, Impact: HGA also serves
  * generation and retrieval).  One step processes n_q new query tokens
- * (1 <= n_q <= block) at active-segment positions t0 .. t0+n_q-1; they form
+ * (1 <= n_q <= q_block) at active-segment positions t0 .. t0+n_q-1; they form
  * one partial query block.  Here dims->S is the CAPACITY of the active
  * segment's KV buffer (k_seg/v_seg [B, S, Hkv, d], positions 0 .. t0+n_q-1
  * already written by the caller, the new tokens' K/V included), and
@@ -307,7 +307,7 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
  *                lower n), ascending, then -1 up to topk.
  * q_new [B, n_q, Hq, d] dtype; summ as for hga_select_topk; idx [B, Hkv, topk]
  * int32; scores_or_null fp32 [B, Hkv, topk] (the selected blocks' scores,
- * -inf for padding).  With n_q = block and t0 a multiple of block this is
+ * -inf for padding).  With n_q = q_block and t0 a multiple of q_block this is
  * exactly hga_select_topk's result for that query block (up to fp32 rounding
  * of the mean near ties).  The blocks are scored in parallel into ws, then
  * selected per (b, KV head); ws as for hga_decode_attn (the same buffer may
@@ -320,11 +320,11 @@ HGA_API hga_status hga_attn_bwd_dq(const hga_dims* dims, const void* q, const vo
  *   o [B, n_q, Hq, d] dtype;  lse [B, Hq, n_q] fp32 (natural log)
  * ws: device scratch of at least hga_decode_workspace_size(dims, n_q) bytes
  * (16-byte aligned; contents need no initialisation), owned by the caller.
- * With n_q = block and t0 a multiple of block the result equals hga_attn_fwd's
+ * With n_q = q_block and t0 a multiple of q_block the result equals hga_attn_fwd's
  * rows of that query block.
  * A finished segment joins the history as in the prefill: hga_segment_summaries
  * appends its blocks' summaries, hga_offload_segment moves its K/V to the tier.
- * Errors: HGA_ERR_SHAPE (n_q outside [1, block], new tokens outside the
+ * Errors: HGA_ERR_SHAPE (n_q outside [1, q_block], new tokens outside the
  * buffer, n_hist_blocks > 4096 for the selection, topk + S/block > 512 for the
  * attention), HGA_ERR_INVALID_ARG (null
  * or misaligned pointers, short workspace); an idx entry outside
