@@ -63,7 +63,7 @@ def load_peaks():
 
 def workload_config(w: synth.Workload, l2_note: str):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "block": w.blk,
-            "segment_tokens": w.S, "history_blocks": w.nblk, "topk": w.topk, "l2": l2_note}
+            "q_block": w.qb, "segment_tokens": w.S, "history_blocks": w.nblk, "topk": w.topk, "l2": l2_note}
 
 
 # ---------------------------------------------------------------- ranks
@@ -93,7 +93,7 @@ def work_model(w: synth.Workload, keff_sum_per_head: float):
     dV); of those, the dQ kernel does dP and dQ for every pair, the dK/dV
     kernel dK and dV for segment pairs."""
     d = w.d
-    hist_pairs = keff_sum_per_head * w.blk * w.blk  # per head: sum_i K_eff(i) * blk rows * blk keys
+    hist_pairs = keff_sum_per_head * w.qb * w.blk  # per head: sum_i K_eff(i) * q_block rows * block keys
     seg_pairs = w.S * (w.S + 1) / 2
     H = w.Hq * w.B
     flops = {
@@ -210,7 +210,8 @@ def committed_traffic(kernel: str):
 
 # Device workloads of `--workload`: the headline layer step, and the two
 # parity workloads (dense-equivalence, 131K prefill forward) timed the same way.
-DEVICE_WORKLOADS = {"layer": synth.QWEN3_8B_LAYER, "dense": synth.DENSE_EQUIV, "prefill": synth.PREFILL_131K}
+DEVICE_WORKLOADS = {"layer": synth.QWEN3_8B_LAYER, "dense": synth.DENSE_EQUIV, "prefill": synth.PREFILL_131K,
+                    "layer64": synth.QWEN3_8B_LAYER64}
 
 
 def run_device(args, rank, world, device, w=None, steps=None):
@@ -219,7 +220,7 @@ def run_device(args, rank, world, device, w=None, steps=None):
 
     w = DEVICE_WORKLOADS[args.workload] if w is None else w
     steps = args.steps if steps is None else steps
-    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
+    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype, w.qblk)
     x = synth.draw(w)
     dev = {n: to_dev(getattr(x, n), device) for n in ("q", "k_seg", "v_seg", "k_hist", "v_hist", "d_o")}
     st = AttentionStep(D, device)
@@ -598,7 +599,7 @@ def run_decode(args, device):
     import segmented_fine_tuning_b200 as hga
     w = synth.DECODE_131K
     nq, t0 = 1, w.S - 1
-    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
+    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype, w.qblk)
     x = synth.draw_decode(w, nq, t0)
     dev = {n: to_dev(getattr(x, n), device) for n in ("k_seg", "v_seg", "k_hist", "v_hist")}
     qn = to_dev(x.extra["q_new"], device)
@@ -699,7 +700,7 @@ def run_tier(args, device):
     L2 flushed between steps); bytes are the algorithmic bytes moved."""
     import segmented_fine_tuning_b200 as hga
     w = synth.QWEN3_8B_LAYER
-    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype)
+    D = hga.Dims(w.B, w.Hq, w.Hkv, w.d, w.blk, w.S, w.nblk, w.topk, w.dtype, w.qblk)
     x = synth.draw(w)
     stream = torch.cuda.current_stream(device)
     copy_stream = torch.cuda.Stream(device)
@@ -888,13 +889,15 @@ def main():
                     help="device pool (cache) slots per layer for --workload segmented (default: the largest history)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the 131K-token prefill and dense-equivalence sub-measurements of the default (layer) run")
-    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode", "tier"), default="layer",
-                    help="layer: one Qwen3-8B-shaped layer step (the headline); segmented: the full 36-layer, "
+    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode", "tier", "layer64"),
+                    default="layer",
+                    help="layer: one Qwen3-8B-shaped layer step (the headline); layer64: the same layer with "
+                         "64-token history blocks under 128-row query blocks; segmented: the full 36-layer, "
                          "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
                          "the 131K prefill forward, device-timed only; decode: one new token at 131K context; "
                          "tier: the history-tier fetch, gather, remap and segment-append paths")
     args = ap.parse_args()
-    if args.workload in ("dense", "prefill", "decode", "tier"):
+    if args.workload in ("dense", "prefill", "decode", "tier", "layer64"):
         args.no_e2e = args.no_cpu_baseline = True
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3

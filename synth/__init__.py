@@ -72,6 +72,10 @@ DENSE_EQUIV = Workload("dense-equivalence: B1 Hq32/Hkv8 d128, hist 12x128, S512,
                        12, 12, "bf16", 3)
 PREFILL_131K = Workload("prefill-131k: B1 Hq32/Hkv8 d128, hist 992x128, S4096, K32, fwd only", 1, 32, 8, 128, 128,
                         4096, 992, 32, "bf16", 4, structured_keys=True, dominant_frac=0.01, fwd_only=True)
+# The layer with history blocks of 64 tokens under 128-row query blocks: the same history keys per query
+# block (32 x 64 = 16 x 128) and the same history length (224 x 64 = 112 x 128).
+QWEN3_8B_LAYER64 = Workload("qwen3-8b-layer-blk64: B1 Hq32/Hkv8 d128, hist 224x64, S2048, q_block 128, K32", 1, 32,
+                            8, 128, 64, 2048, 224, 32, "bf16", 6, structured_keys=True, qblk=128)
 
 WORKLOADS = {"tiny_f32": TINY_F32, "qwen3_8b_layer": QWEN3_8B_LAYER, "dense_equiv": DENSE_EQUIV,
              "prefill_131k": PREFILL_131K}
