@@ -211,7 +211,7 @@ def committed_traffic(kernel: str):
 # Device workloads of `--workload`: the headline layer step, and the two
 # parity workloads (dense-equivalence, 131K prefill forward) timed the same way.
 DEVICE_WORKLOADS = {"layer": synth.QWEN3_8B_LAYER, "dense": synth.DENSE_EQUIV, "prefill": synth.PREFILL_131K,
-                    "layer64": synth.QWEN3_8B_LAYER64}
+                    "layer64": synth.QWEN3_8B_LAYER64, "layer32": synth.QWEN3_8B_LAYER32}
 
 
 def run_device(args, rank, world, device, w=None, steps=None):
@@ -889,15 +889,17 @@ def main():
                     help="device pool (cache) slots per layer for --workload segmented (default: the largest history)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the 131K-token prefill and dense-equivalence sub-measurements of the default (layer) run")
-    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode", "tier", "layer64"),
+    ap.add_argument("--workload", choices=("layer", "segmented", "dense", "prefill", "decode", "tier", "layer64",
+                                           "layer32"),
                     default="layer",
                     help="layer: one Qwen3-8B-shaped layer step (the headline); layer64: the same layer with "
-                         "64-token history blocks under 128-row query blocks; segmented: the full 36-layer, "
+                         "64-token history blocks under 128-row query blocks; layer32: with 32-token history "
+                         "blocks and K 64; segmented: the full 36-layer, "
                          "8-segment pass with the pinned host tier; dense / prefill: the dense-equivalence step and "
                          "the 131K prefill forward, device-timed only; decode: one new token at 131K context; "
                          "tier: the history-tier fetch, gather, remap and segment-append paths")
     args = ap.parse_args()
-    if args.workload in ("dense", "prefill", "decode", "tier", "layer64"):
+    if args.workload in ("dense", "prefill", "decode", "tier", "layer64", "layer32"):
         args.no_e2e = args.no_cpu_baseline = True
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3

@@ -181,10 +181,12 @@ HGA_API hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void*
                         float* lse, hga_stream_t stream);
 
 /* 1 when hga_attn_fwd / hga_attn_bwd run these dims on the tcgen05
- * tensor-core kernels (bf16, d in {64, 128}, q_block 128, block 128 or 64 --
- * two 64-token history blocks per 128-key tile -- an even group size, K <= 64,
- * at most 128 query blocks), 0 when they run on the CUDA-core kernels, -1 for
- * dims the library rejects.  Host-only; no device work. */
+ * tensor-core kernels (bf16, d in {64, 128}, q_block 128, block 128, 64, 32
+ * or 16 -- 128/block selected history blocks per 128-key tile -- an even
+ * group size, K <= 64, at most 128 query blocks; with block 64 also
+ * n_kv_blocks < 32767, as a tile entry holds two 15-bit block indices), 0 when
+ * they run on the CUDA-core kernels, -1 for dims the library rejects.
+ * Host-only; no device work. */
 HGA_API int hga_attn_uses_tensor_cores(const hga_dims* dims, int n_kv_blocks);
 
 /* Bytes of device scratch hga_attn_bwd needs for these dims (256-byte

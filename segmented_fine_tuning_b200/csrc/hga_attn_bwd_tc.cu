@@ -46,6 +46,11 @@ constexpr int kSubOff = kSubRows * 128;      // byte offset of the second 64-row
 // History tiles of 64-token blocks hold two blocks: tile = n0 | (n1 << 16),
 // n1 = kNoBlock when the tile's upper 64 keys have no block (an odd count).
 constexpr int kNoBlock = 0x7FFF;
+// History blocks of 32 or 16 tokens run in the grouped instantiation of the
+// dQ kernel (kGrp): a tile holds g = 128 / block of them (four or eight), its
+// entry is s | (c << 16), the tile's blocks are hb[s .. s+c) with c <= g, and
+// the keys after the first c*block of a short last tile get P = 0.  Blocks of
+// 128 and 64 tokens keep the plain kernel.
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kLog2e = 1.4426950408889634f;
 // Pairs k (bit k) of every 32-column chunk whose 2^x goes to the FMA pipe
@@ -78,12 +83,13 @@ struct BwdArgs {
   // qmask == nullptr and gscale == 1: the plain backward.
   const uint8_t* qmask;
   float gscale;
-  int hblk;  // history block tokens: 128 (one block per tile) or 64 (two per tile)
+  int hblk;  // history block tokens: 128 (one block per tile), 64 (two), 32 or 16 (grouped)
 };
 
 // ============================================================== dQ kernel
 constexpr int kKStages = 3, kVStages = 2;
 
+template <bool kGrp>
 struct DqCtl {
   uint64_t qdo_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
@@ -94,11 +100,15 @@ struct DqCtl {
   uint32_t tmem;
   int abort;
   int nt;
-  int tiles[kMaxTiles];
+  int tiles[kMaxTiles];  // >= 0: history block, pair or group; < 0: segment block -(t+1)
+  int hb[kGrp ? kMaxTopk : 1];  // grouped: the valid selected history blocks, in idx order
 };
 // Head dim d in {64, 128}: a tile is 128 rows x d bf16 (d/64 TMA boxes).
-constexpr size_t dq_smem_bytes(int d) { return 1024 + (2 + kKStages + kVStages) * (kB * d * 2) + sizeof(DqCtl); }
-static_assert(dq_smem_bytes(128) <= 232448, "shared memory budget");
+template <bool kGrp>
+constexpr size_t dq_smem_bytes(int d) {
+  return 1024 + (2 + kKStages + kVStages) * (kB * d * 2) + sizeof(DqCtl<kGrp>);
+}
+static_assert(dq_smem_bytes<true>(128) <= 232448, "shared memory budget");
 
 // Tensor-memory columns of the dQ kernel: S double buffer, dP, dQ.
 constexpr uint32_t kDqS = 0, kDqP = 256, kDqAcc = 384;
@@ -108,7 +118,7 @@ constexpr uint32_t kDqS = 0, kDqP = 256, kDqAcc = 384;
 // and runs two tiles ahead.  dP has one buffer, but the dS pass releases it as
 // soon as it has loaded its columns (dp_free), so dP(j+1) is computed while
 // dS(j) is being formed; dQ(j) follows dS(j).
-template <int KD>
+template <int KD, bool kGrp>
 __global__ void __launch_bounds__(320, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
@@ -123,7 +133,7 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sDO = sm + kTileBytes;
   uint8_t* sK = sm + 2 * kTileBytes;
   uint8_t* sV = sK + kKStages * kTileBytes;
-  DqCtl* ctl = reinterpret_cast<DqCtl*>(sV + kVStages * kTileBytes);
+  DqCtl<kGrp>* ctl = reinterpret_cast<DqCtl<kGrp>*>(sV + kVStages * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_i = a.B * a.Hq;
@@ -150,10 +160,16 @@ __global__ void __launch_bounds__(320, 1)
       const bool ok = (n >= 0 && n < a.nkv);
       if (r < a.topk && !ok && n != -1) flag_error(a.err, kDevErrIndex);
       const unsigned m = __ballot_sync(0xffffffffu, ok);
-      if (ok) ctl->tiles[nh + __popc(m & ((1u << lane) - 1u))] = n;
+      if (ok) (kGrp ? ctl->hb : ctl->tiles)[nh + __popc(m & ((1u << lane) - 1u))] = n;
       nh += __popc(m);
     }
-    if (a.hblk == 64) {
+    if (kGrp) {
+      // g consecutive list entries per tile (the last one may be short)
+      const int g = kB / a.hblk;
+      const int nht = (nh + g - 1) / g;
+      for (int j = lane; j < nht; j += 32) ctl->tiles[j] = (j * g) | (min(g, nh - j * g) << 16);
+      nh = nht;
+    } else if (a.hblk == 64) {
       // 64-token history blocks: two per 128-key tile (nh <= 64, so one pass)
       __syncwarp();
       const int np = (nh + 1) >> 1;
@@ -192,7 +208,56 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (kGrp) {
+      // Grouped history tiles: the whole warp.  Lane 0 waits for each slot
+      // and arms it; lanes q < g then load block q of a history tile at once
+      // (lane 0 alone a segment tile).
+      const int g = kB / a.hblk;
+      if (lane == 0) {
+        mbar_expect_tx(&ctl->qdo_full, 2 * kTileBytes);
+        for (int hh = 0; hh < kBoxes; ++hh) {
+          tma_load_4d(&tm_q, &ctl->qdo_full, sQ + hh * kHalf, hh * 64, hq, i * kB, b);
+          tma_load_4d(&tm_do, &ctl->qdo_full, sDO + hh * kHalf, hh * 64, hq, i * kB, b);
+        }
+      }
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int tile = ctl->tiles[j];
+        const bool hist = tile >= 0;
+        // this lane's block of a history tile: a short tile repeats its last
+        // block (finite values; those keys get P = 0 in the dS pass)
+        const int row = hist ? ctl->hb[(tile & 0xFFFF) + min(lane, (tile >> 16) - 1)] * a.hblk : (-tile - 1) * kB;
+        const bool loads = hist ? lane < g : lane == 0;
+        const int sub = hist ? lane * a.hblk * 128 : 0;
+        const int ks = j % kKStages, vs = j % kVStages;
+        if (!mbar_wait_w(&ctl->k_empty[ks], ((j / kKStages) & 1) ^ 1, abort, a.err)) break;
+        if (lane == 0) mbar_expect_tx(&ctl->k_full[ks], kTileBytes);
+        __syncwarp();
+        if (loads)
+          for (int hh = 0; hh < kBoxes; ++hh)
+            tma_load_4d(hist ? &tm_kh : &tm_ks, &ctl->k_full[ks], sK + ks * kTileBytes + hh * kHalf + sub, hh * 64,
+                        kvh, row, b);
+        k_issued = j + 1;
+        if (!mbar_wait_w(&ctl->v_empty[vs], ((j / kVStages) & 1) ^ 1, abort, a.err)) break;
+        if (lane == 0) mbar_expect_tx(&ctl->v_full[vs], kTileBytes);
+        __syncwarp();
+        if (loads)
+          for (int hh = 0; hh < kBoxes; ++hh)
+            tma_load_4d(hist ? &tm_vh : &tm_vs, &ctl->v_full[vs], sV + vs * kTileBytes + hh * kHalf + sub, hh * 64,
+                        kvh, row, b);
+        v_issued = j + 1;
+      }
+      if (lane == 0) {
+        // Never leave the CTA with copies in flight (the slots' barriers
+        // count every lane's bytes).
+        volatile int no_abort = 0;
+        mbar_wait(&ctl->qdo_full, 0, &no_abort, a.err);
+        for (int j = k_issued > kKStages ? k_issued - kKStages : 0; j < k_issued; ++j)
+          mbar_wait(&ctl->k_full[j % kKStages], (j / kKStages) & 1, &no_abort, a.err);
+        for (int j = v_issued > kVStages ? v_issued - kVStages : 0; j < v_issued; ++j)
+          mbar_wait(&ctl->v_full[j % kVStages], (j / kVStages) & 1, &no_abort, a.err);
+      }
+    } else if (lane == 0) {
       mbar_expect_tx(&ctl->qdo_full, 2 * kTileBytes);
       for (int hh = 0; hh < kBoxes; ++hh) {
         tma_load_4d(&tm_q, &ctl->qdo_full, sQ + hh * kHalf, hh * 64, hq, i * kB, b);
@@ -327,10 +392,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&ctl->dp_free);  // dP(j) is in registers: the tensor core may overwrite it
       // keys above `lim` get P = 0: the diagonal segment tile masks keys after
       // the row's own position; a history tile holding one 64-token block
-      // masks its upper 64 keys
+      // masks its upper 64 keys, a short grouped tile the keys after its blocks
       int lim = 127;
       if (j == nt - 1) lim = r;
-      else if (a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) lim = 63;
+      else if (!kGrp && a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) lim = 63;
+      else if (kGrp && ctl->tiles[j] >= 0) lim = (ctl->tiles[j] >> 16) * a.hblk - 1;
       const bool diag = lim < 127;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -627,13 +693,13 @@ __global__ void __launch_bounds__(320, 1)
 
 }  // namespace
 
-template <int KD>
+template <int KD, bool kGrp>
 cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                        const float* Dr, float* dq, float* dk, float* dv, int parts, int* err, cudaStream_t st,
                        const uint8_t* qmask, float gscale) {
-  constexpr size_t dq_smem = dq_smem_bytes(KD), kv_smem = dkdv_smem_bytes(KD);
+  constexpr size_t dq_smem = dq_smem_bytes<kGrp>(KD), kv_smem = dkdv_smem_bytes(KD);
   cudaError_t e;
-  if ((e = smem_limit(reinterpret_cast<const void*>(dq_tc_kernel<KD>), dq_smem)) !=
+  if ((e = smem_limit(reinterpret_cast<const void*>(dq_tc_kernel<KD, kGrp>), dq_smem)) !=
       cudaSuccess)
     return e;
   if ((e = smem_limit(reinterpret_cast<const void*>(dkdv_tc_kernel<KD>), kv_smem)) !=
@@ -654,7 +720,7 @@ cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (parts & kBwdDq) {
-    dq_tc_kernel<KD><<<s.B * s.Hq * s.nqb(), 320, dq_smem, st>>>(m.q, m.d_o, m.ks, m.vs, m.kh, m.vh, a);
+    dq_tc_kernel<KD, kGrp><<<s.B * s.Hq * s.nqb(), 320, dq_smem, st>>>(m.q, m.d_o, m.ks, m.vs, m.kh, m.vh, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -663,8 +729,11 @@ cudaError_t launch_bwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
 cudaError_t launch_attn_bwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, const float* lse,
                                const float* Dr, float* dq, float* dk, float* dv, int parts, int* err,
                                cudaStream_t st, const uint8_t* qmask, float gscale) {
-  return s.d == 64 ? launch_bwd<64>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale)
-                   : launch_bwd<128>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale);
+  if (s.blk < 64)
+    return s.d == 64 ? launch_bwd<64, true>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale)
+                     : launch_bwd<128, true>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale);
+  return s.d == 64 ? launch_bwd<64, false>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale)
+                   : launch_bwd<128, false>(s, m, nkv, idx, lse, Dr, dq, dk, dv, parts, err, st, qmask, gscale);
 }
 
 }  // namespace hga

@@ -42,6 +42,11 @@ constexpr int kRowHalf = 64 * 128;            // byte offset of row 64 inside a 
 // History tiles of 64-token blocks hold two blocks: tile = n0 | (n1 << 16),
 // n1 = kNoBlock when the tile's upper 64 keys have no block (an odd count).
 constexpr int kNoBlock = 0x7FFF;
+// History blocks of 32 or 16 tokens run in the grouped instantiation
+// (kGrp): a tile holds g = 128 / block of them (four or eight), its entry is
+// s | (c << 16), the tile's blocks are hb[s .. s+c) with c <= g, and the keys
+// after the first c*block of a short last tile are masked.  Blocks of 128 and
+// 64 tokens keep the plain kernel.
 constexpr int kStages = 5;                    // K/V ring slots
 constexpr int kMaxTiles = kMaxTopk + kMaxQueryBlocks;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -54,6 +59,7 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units
 #endif
 constexpr uint32_t kFwdPolyPairs = HGA_FWD_POLY;
 
+template <bool kGrp>
 struct FwdCtl {
   uint64_t q_full;
   uint64_t kv_full[kStages];
@@ -65,12 +71,16 @@ struct FwdCtl {
   uint32_t tmem;
   int abort;
   int nt;
-  int tiles[kMaxTiles];  // >= 0: history block; < 0: segment block -(t+1)
+  int tiles[kMaxTiles];  // >= 0: history block, pair or group; < 0: segment block -(t+1)
+  int hb[kGrp ? kMaxTopk : 1];  // grouped: the valid selected history blocks, in idx order
 };
 
 // Head dim d in {64, 128}: a Q, K or V tile is 128 rows x d bf16 (d/64 boxes).
-constexpr size_t fwd_smem_bytes(int d) { return 1024 + 2 * (kBM * d * 2) + kStages * (kBM * d * 2) + sizeof(FwdCtl); }
-static_assert(fwd_smem_bytes(128) <= 232448, "shared memory budget");
+template <bool kGrp>
+constexpr size_t fwd_smem_bytes(int d) {
+  return 1024 + 2 * (kBM * d * 2) + kStages * (kBM * d * 2) + sizeof(FwdCtl<kGrp>);
+}
+static_assert(fwd_smem_bytes<true>(128) <= 232448, "shared memory budget");
 
 struct FwdArgs {
   int B, Hq, Hkv, S, nkv, topk, nqb, G;
@@ -80,10 +90,10 @@ struct FwdArgs {
   float* lse;
   int* err;
   int withhold_kv;  // self test of the timeout path: the producer issues no K/V loads
-  int hblk;         // history block tokens: 128 (one block per tile) or 64 (two per tile)
+  int hblk;         // history block tokens: 128 (one block per tile), 64 (two), 32 or 16 (grouped)
 };
 
-template <int KD>
+template <int KD, bool kGrp>
 __global__ void __launch_bounds__(384, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                   const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kh,
@@ -95,7 +105,7 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sQ = sm;                                // 2 Q tiles
   uint8_t* sRing = sm + 2 * kTileBytes;            // kStages K/V tiles
-  FwdCtl* ctl = reinterpret_cast<FwdCtl*>(sRing + kStages * kTileBytes);
+  FwdCtl<kGrp>* ctl = reinterpret_cast<FwdCtl<kGrp>*>(sRing + kStages * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Longest work first: query block i descending with blockIdx.
@@ -116,10 +126,16 @@ __global__ void __launch_bounds__(384, 1)
       const bool ok = (n >= 0 && n < a.nkv);
       if (r < a.topk && !ok && n != -1) flag_error(a.err, kDevErrIndex);
       const unsigned m = __ballot_sync(0xffffffffu, ok);
-      if (ok) ctl->tiles[nh + __popc(m & ((1u << lane) - 1u))] = n;
+      if (ok) (kGrp ? ctl->hb : ctl->tiles)[nh + __popc(m & ((1u << lane) - 1u))] = n;
       nh += __popc(m);
     }
-    if (a.hblk == 64) {
+    if (kGrp) {
+      // g consecutive list entries per tile (the last one may be short)
+      const int g = kBN / a.hblk;
+      const int nht = (nh + g - 1) / g;
+      for (int j = lane; j < nht; j += 32) ctl->tiles[j] = (j * g) | (min(g, nh - j * g) << 16);
+      nh = nht;
+    } else if (a.hblk == 64) {
       // 64-token history blocks: two per 128-key tile (nh <= 64, so one pass)
       __syncwarp();
       const int np = (nh + 1) >> 1;
@@ -162,7 +178,58 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (kGrp) {
+      // Grouped history tiles: the whole warp.  Lane 0 waits for each slot
+      // and arms it; lanes q < g then load block q of a history tile at once
+      // (lane 0 alone a segment tile).
+      const int g = kBN / a.hblk;
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_kh);
+        prefetch_tmap(&tm_vh);
+        prefetch_tmap(&tm_ks);
+        prefetch_tmap(&tm_vs);
+        mbar_expect_tx(&ctl->q_full, 2 * kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int hh = 0; hh < kBoxes; ++hh)
+            tma_load_4d(&tm_q, &ctl->q_full, sQ + t * kTileBytes + hh * kHalf, hh * 64, hq0 + t, i * kBM, b);
+      }
+      int issued = 0;
+      for (int j = 0; j < (a.withhold_kv ? 0 : nt); ++j) {
+        const int tile = ctl->tiles[j];
+        const bool hist = tile >= 0;
+        // this lane's block of a history tile: a short tile repeats its last
+        // block (finite values; those keys are masked in the softmax)
+        const int row = hist ? ctl->hb[(tile & 0xFFFF) + min(lane, (tile >> 16) - 1)] * a.hblk : (-tile - 1) * kBN;
+        const bool loads = hist ? lane < g : lane == 0;
+        const int sub = hist ? lane * a.hblk * 128 : 0;
+        bool ok = true;
+        for (int w = 0; w < 2; ++w) {
+          const int pos = 2 * j + w;
+          const int s = pos % kStages;
+          if (!mbar_wait_w(&ctl->kv_empty[s], ((pos / kStages) & 1) ^ 1, abort, a.err)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* m = hist ? (w ? &tm_vh : &tm_kh) : (w ? &tm_vs : &tm_ks);
+          if (lane == 0) mbar_expect_tx(&ctl->kv_full[s], kTileBytes);
+          __syncwarp();
+          if (loads)
+            for (int hh = 0; hh < kBoxes; ++hh)
+              tma_load_4d(m, &ctl->kv_full[s], sRing + s * kTileBytes + hh * kHalf + sub, hh * 64, kvh, row, b);
+          issued = pos + 1;
+        }
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        // Never leave the CTA with copies in flight (the slots' barriers
+        // count every lane's bytes).
+        volatile int no_abort = 0;
+        mbar_wait(&ctl->q_full, 0, &no_abort, a.err);
+        for (int pos = issued - kStages > 0 ? issued - kStages : 0; pos < issued; ++pos)
+          mbar_wait(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, &no_abort, a.err);
+      }
+    } else if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_kh);
       prefetch_tmap(&tm_vh);
@@ -308,10 +375,16 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (e > r) v[e] = 0xFF800000u;  // -inf
-      } else if (a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) {
+      } else if (!kGrp && a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) {
         // a history tile holding one 64-token block: its upper 64 keys are masked
 #pragma unroll
         for (int e = 64; e < 128; ++e) v[e] = 0xFF800000u;
+      } else if (kGrp && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) * a.hblk < kBN) {
+        // a short grouped history tile: the keys after its blocks are masked
+        const int nk = (ctl->tiles[j] >> 16) * a.hblk;
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+          if (e >= nk) v[e] = 0xFF800000u;
       }
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -393,16 +466,17 @@ __global__ void __launch_bounds__(384, 1)
 }  // namespace
 
 bool tc_supported(const Shape& s) {
-  return s.bf16 && (s.d == 128 || s.d == 64) && (s.blk == kBM || s.blk == 64) && s.qblk == kBM && (s.G() % 2) == 0 &&
+  return s.bf16 && (s.d == 128 || s.d == 64) && (s.blk == 128 || s.blk == 64 || s.blk == 32 || s.blk == 16) &&
+         s.qblk == kBM && (s.G() % 2) == 0 &&
          s.topk <= kMaxTopk &&
          s.nqb() <= kMaxQueryBlocks;
 }
 
-template <int KD>
+template <int KD, bool kGrp>
 cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse, int* err,
                        cudaStream_t st, bool withhold_kv) {
-  constexpr size_t smem = fwd_smem_bytes(KD);
-  cudaError_t e = smem_limit(reinterpret_cast<const void*>(fwd_tc_kernel<KD>), smem);
+  constexpr size_t smem = fwd_smem_bytes<kGrp>(KD);
+  cudaError_t e = smem_limit(reinterpret_cast<const void*>(fwd_tc_kernel<KD, kGrp>), smem);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
@@ -410,14 +484,17 @@ cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* 
   a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err; a.hblk = s.blk;
   a.withhold_kv = withhold_kv ? 1 : 0;
   const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
-  fwd_tc_kernel<KD><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
+  fwd_tc_kernel<KD, kGrp><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
                                int* err, cudaStream_t st, bool withhold_kv) {
-  return s.d == 64 ? launch_fwd<64>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
-                   : launch_fwd<128>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
+  if (s.blk < 64)
+    return s.d == 64 ? launch_fwd<64, true>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
+                     : launch_fwd<128, true>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
+  return s.d == 64 ? launch_fwd<64, false>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
+                   : launch_fwd<128, false>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
 }
 
 }  // namespace hga

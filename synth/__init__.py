@@ -76,6 +76,10 @@ PREFILL_131K = Workload("prefill-131k: B1 Hq32/Hkv8 d128, hist 992x128, S4096, K
 # block (32 x 64 = 16 x 128) and the same history length (224 x 64 = 112 x 128).
 QWEN3_8B_LAYER64 = Workload("qwen3-8b-layer-blk64: B1 Hq32/Hkv8 d128, hist 224x64, S2048, q_block 128, K32", 1, 32,
                             8, 128, 64, 2048, 224, 32, "bf16", 6, structured_keys=True, qblk=128)
+# The same with 32-token history blocks: K = 64 (the largest K) keeps 64 x 32 = 16 x 128 history keys per
+# query block over 448 x 32 = 112 x 128 history tokens.
+QWEN3_8B_LAYER32 = Workload("qwen3-8b-layer-blk32: B1 Hq32/Hkv8 d128, hist 448x32, S2048, q_block 128, K64", 1, 32,
+                            8, 128, 32, 2048, 448, 64, "bf16", 9, structured_keys=True, qblk=128)
 
 WORKLOADS = {"tiny_f32": TINY_F32, "qwen3_8b_layer": QWEN3_8B_LAYER, "dense_equiv": DENSE_EQUIV,
              "prefill_131k": PREFILL_131K}

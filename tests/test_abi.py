@@ -191,11 +191,14 @@ def test_size_limits_rejected_on_host(lib):
     (dict(d=64), 4, 1),                                    # head dim 64
     (dict(block=64, q_block=128), 9, 1),                   # 64-token history blocks, two per tile
     (dict(block=64, q_block=128, n_hist_blocks=40000, topk=4), 40000, 0),  # block indices past 15 bits
+    (dict(block=32, q_block=128, n_hist_blocks=40000, topk=4), 40000, 1),  # grouped tiles: no such limit
+    (dict(block=32, q_block=128), 4, 1),                   # 32-token history blocks, four per tile
+    (dict(block=16, q_block=128), 4, 1),                   # 16-token history blocks, eight per tile
     (dict(block=64), 9, 0),                                # 64-row query blocks: CUDA-core kernels
     (dict(block=128, q_block=64), 4, 0),
     (dict(dtype=0), 4, 0),                                 # fp32
     (dict(Hq=6, Hkv=2), 4, 0),                             # odd group size
-    (dict(block=32, q_block=128), 4, 0),                   # 32-token history blocks
+    (dict(block=32), 4, 0),                                # 32-row query blocks: CUDA-core kernels
     (dict(q_block=48), 4, -1),                             # rejected dims
 ])
 def test_tensor_core_path_selection(lib, kw, nkv, want):

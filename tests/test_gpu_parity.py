@@ -148,13 +148,21 @@ ATTN_CASES = [
     synth.Workload("tc-d64-B2-G2: B2 Hq4/Hkv2 d64 S256 hist3 K2", 2, 4, 2, 64, 128, 256, 3, 2, "bf16", 42),
     synth.Workload("simt-f32-d128-blk32", 1, 2, 2, 128, 32, 96, 6, 3, "f32", 37),
     # query blocks of another size than the history blocks (q_block != block); 128-row query blocks
-    # with 64-token history blocks run on the tensor-core kernels, two history blocks per 128-key tile
+    # with 64-, 32- or 16-token history blocks run on the tensor-core kernels, 128/block history
+    # blocks per 128-key tile (the last tile short when K valid blocks do not fill it)
     synth.Workload("qblk128-blk64: Hq4/Hkv2 S256 hist10 K3", 1, 4, 2, 128, 64, 256, 10, 3, "bf16", 43,
                    structured_keys=True, qblk=128),
     synth.Workload("tc-blk64-K4: Hq8/Hkv2 S384 hist12 K4", 1, 8, 2, 128, 64, 384, 12, 4, "bf16", 46, qblk=128),
     synth.Workload("tc-blk64-d64-B2: B2 Hq4/Hkv2 d64 S256 hist9 K5", 2, 4, 2, 64, 64, 256, 9, 5, "bf16", 47,
                    qblk=128),
     synth.Workload("tc-blk64-K>hist: Hq4/Hkv2 S256 hist3 K8", 1, 4, 2, 128, 64, 256, 3, 8, "bf16", 48, qblk=128),
+    synth.Workload("tc-blk32-K6: Hq4/Hkv2 S256 hist20 K6", 1, 4, 2, 128, 32, 256, 20, 6, "bf16", 49,
+                   structured_keys=True, qblk=128),
+    synth.Workload("tc-blk32-K>hist: Hq4/Hkv2 S256 hist3 K8", 1, 4, 2, 128, 32, 256, 3, 8, "bf16", 50, qblk=128),
+    synth.Workload("tc-blk16-d64-K11: Hq8/Hkv2 d64 S384 hist40 K11", 1, 8, 2, 64, 16, 384, 40, 11, "bf16", 51,
+                   qblk=128),
+    synth.Workload("tc-blk16-K64: B2 Hq4/Hkv2 S256 hist80 K64", 2, 4, 2, 128, 16, 256, 80, 64, "bf16", 52,
+                   structured_keys=True, qblk=128),
     synth.Workload("qblk64-blk128: B2 Hq4/Hkv2 d64 S256 hist5 K2", 2, 4, 2, 64, 128, 256, 5, 2, "bf16", 44, qblk=64),
     synth.Workload("qblk16-blk32-f32: Hq2/Hkv1 d64 S96 hist8 K3", 1, 2, 1, 64, 32, 96, 8, 3, "f32", 45, qblk=16),
 ]

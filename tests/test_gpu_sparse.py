@@ -32,6 +32,8 @@ CASES = [
                     qblk=64), 2),
     (synth.Workload("sparse-tc-blk64: Hq4/Hkv2 S512 hist11 K5", 1, 4, 2, 128, 64, 512, 11, 5, "bf16", 114,
                     qblk=128), 2),
+    (synth.Workload("sparse-tc-blk16: Hq4/Hkv2 S512 hist30 K13", 1, 4, 2, 128, 16, 512, 30, 13, "bf16", 115,
+                    qblk=128), 2),
 ]
 
 
