@@ -471,6 +471,12 @@ static_assert(dkdv_smem_bytes(128) <= 232448, "shared memory budget");
 
 // Tensor-memory columns of the dK/dV kernel.
 constexpr uint32_t kKvS = 0, kKvP = 128, kKvDK = 256, kKvDV = 384;
+// Row pitch (floats) of the fp32 dK/dV partials staged for the bulk
+// reduction; the two [128 x pitch] partials reuse the kernel's tile buffers.
+template <int KD>
+constexpr int kv_pad() { return KD + 4; }
+static_assert(2 * kB * kv_pad<128>() * 4 <= (2 + 2 * kQStages) * kB * 128 * 2, "partials fit the tile buffers");
+static_assert(2 * kB * kv_pad<64>() * 4 <= (2 + 2 * kQStages) * kB * 64 * 2, "partials fit the tile buffers");
 
 template <int KD>
 __global__ void __launch_bounds__(320, 1)
@@ -480,6 +486,7 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int kD = KD;
   constexpr int kTileBytes = kB * kD * 2;
   constexpr int kBoxes = kD / 64;
+  constexpr int kPad = kv_pad<KD>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sK = sm;
@@ -660,26 +667,41 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(&ctl->pds_full[h]);
     }
-    if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err))) {
+    const bool done = __all_sync(0xffffffffu, ok && mbar_wait(&ctl->dkv_full, 0, abort, a.err));
+    float* part = reinterpret_cast<float*>(sm);
+    if (done) {
       tc_fence_after();
-      // warpgroup e adds head-dim columns [e*d/2, (e+1)*d/2) of the key row
-      const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + (kD / 2) * e;
+      // This head's scaled dK, dV into the tile buffers (no copy or MMA reads
+      // them any more): part[t][row][col], rows padded to kPad floats so that
+      // the 32 rows of a warp fall in distinct banks; warpgroup e writes
+      // head-dim columns [e*d/2, (e+1)*d/2) of key row r.
       const float ks = a.scale * a.gscale, vsc = a.gscale;
 #pragma unroll
       for (int cc = 0; cc < kD / 64; ++cc) {
         uint32_t gk[32], gv[32];
         HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDK + (kD / 2) * e + 32 * cc, gk);
         HGA_TMEM_LD32_WAIT(tmem + lane_off + kKvDV + (kD / 2) * e + 32 * cc, gv);
-        float* pk4 = a.dk + off + 32 * cc;
-        float* pv4 = a.dv + off + 32 * cc;
+        float4* pk4 = reinterpret_cast<float4*>(part + r * kPad + (kD / 2) * e + 32 * cc);
+        float4* pv4 = reinterpret_cast<float4*>(part + (kB + r) * kPad + (kD / 2) * e + 32 * cc);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          red_add_v4(pk4 + 4 * x, __uint_as_float(gk[4 * x]) * ks, __uint_as_float(gk[4 * x + 1]) * ks,
-                     __uint_as_float(gk[4 * x + 2]) * ks, __uint_as_float(gk[4 * x + 3]) * ks);
-          red_add_v4(pv4 + 4 * x, __uint_as_float(gv[4 * x]) * vsc, __uint_as_float(gv[4 * x + 1]) * vsc,
-                     __uint_as_float(gv[4 * x + 2]) * vsc, __uint_as_float(gv[4 * x + 3]) * vsc);
+          pk4[x] = make_float4(__uint_as_float(gk[4 * x]) * ks, __uint_as_float(gk[4 * x + 1]) * ks,
+                               __uint_as_float(gk[4 * x + 2]) * ks, __uint_as_float(gk[4 * x + 3]) * ks);
+          pv4[x] = make_float4(__uint_as_float(gv[4 * x]) * vsc, __uint_as_float(gv[4 * x + 1]) * vsc,
+                               __uint_as_float(gv[4 * x + 2]) * vsc, __uint_as_float(gv[4 * x + 3]) * vsc);
         }
       }
+    }
+    // Every one of the 256 threads passes the barrier, whatever happened
+    // above; then thread (e, r) adds row r of dK (e = 0) or dV (e = 1) into
+    // the zeroed outputs on the bulk-copy engine.
+    fence_proxy_async_smem();
+    named_sync(1, 256);
+    if (done) {
+      float* out = (e ? a.dv : a.dk) + (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD;
+      bulk_reduce_add_f32(out, part + (e * kB + r) * kPad, kD * 4);
+      bulk_commit();
+      bulk_wait_read_all();  // the shared-memory source outlives the copy
     }
   }
 

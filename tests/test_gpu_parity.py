@@ -147,6 +147,11 @@ ATTN_CASES = [
                    structured_keys=True),
     synth.Workload("tc-d64-B2-G2: B2 Hq4/Hkv2 d64 S256 hist3 K2", 2, 4, 2, 64, 128, 256, 3, 2, "bf16", 42),
     synth.Workload("simt-f32-d128-blk32", 1, 2, 2, 128, 32, 96, 6, 3, "f32", 37),
+    # dK/dV: group sizes up to 8 sum the heads' parts in a thread-block cluster (8 and 6 here; 4 and 2
+    # above); 16 heads per KV head add theirs into zeroed outputs
+    synth.Workload("tc-G8: Hq16/Hkv2 d64 S256 hist5 K2", 1, 16, 2, 64, 128, 256, 5, 2, "bf16", 53),
+    synth.Workload("tc-G6: Hq12/Hkv2 S384 hist4 K2", 1, 12, 2, 128, 128, 384, 4, 2, "bf16", 54),
+    synth.Workload("tc-G16: Hq16/Hkv1 d64 S256 hist3 K2", 1, 16, 1, 64, 128, 256, 3, 2, "bf16", 55),
     # query blocks of another size than the history blocks (q_block != block); 128-row query blocks
     # with 64-, 32- or 16-token history blocks run on the tensor-core kernels, 128/block history
     # blocks per 128-key tile (the last tile short when K valid blocks do not fill it)
