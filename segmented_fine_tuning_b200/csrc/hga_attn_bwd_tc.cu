@@ -112,6 +112,9 @@ static_assert(dq_smem_bytes<true>(128) <= 232448, "shared memory budget");
 
 // Tensor-memory columns of the dQ kernel: S double buffer, dP, dQ.
 constexpr uint32_t kDqS = 0, kDqP = 256, kDqAcc = 384;
+// The dQ epilogue stages 2 x 128 half rows of d/2 + 4 floats in the tile buffers.
+static_assert(2 * kB * (128 / 2 + 4) * 4 <= (2 + kKStages + kVStages) * kB * 128 * 2, "dQ stage fits");
+static_assert(2 * kB * (64 / 2 + 4) * 4 <= (2 + kKStages + kVStages) * kB * 64 * 2, "dQ stage fits");
 
 // dQ kernel: full 128-key tiles (N = 128 products: half the shared-memory
 // re-reads of A per FLOP compared with 64-key halves).  S is double-buffered
@@ -425,18 +428,25 @@ __global__ void __launch_bounds__(320, 1)
     if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->dq_full, 0, abort, a.err))) {
       tc_fence_after();
       const float osc = a.scale * a.gscale;
-      // warpgroup e writes head-dim columns [e*d/2, (e+1)*d/2) of the row
-      float* out = a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + (kD / 2) * e;
+      // Warpgroup e's half row (head-dim columns [e*d/2, (e+1)*d/2)) goes
+      // through the freed tile buffers, rows padded to d/2 + 4 floats so that
+      // a warp's 32 rows fall in distinct banks, and out as one bulk copy
+      // (a warp's direct stores would each touch 32 rows).
+      float* stage = reinterpret_cast<float*>(sm) + (size_t)(e * kB + r) * (kD / 2 + 4);
 #pragma unroll
       for (int cc = 0; cc < kD / 64; ++cc) {
         uint32_t v[32];
         HGA_TMEM_LD32_WAIT(tmem + lane_off + kDqAcc + (kD / 2) * e + 32 * cc, v);
-        float4* dst = reinterpret_cast<float4*>(out + 32 * cc);
+        float4* dst = reinterpret_cast<float4*>(stage + 32 * cc);
 #pragma unroll
         for (int xx = 0; xx < 8; ++xx)
           dst[xx] = make_float4(__uint_as_float(v[4 * xx]) * osc, __uint_as_float(v[4 * xx + 1]) * osc,
                                 __uint_as_float(v[4 * xx + 2]) * osc, __uint_as_float(v[4 * xx + 3]) * osc);
       }
+      fence_proxy_async_smem();
+      bulk_store(a.dq + (((size_t)b * a.S + p) * a.Hq + hq) * kD + (kD / 2) * e, stage, (kD / 2) * 4);
+      bulk_commit();
+      bulk_wait_read_all();  // the shared-memory source outlives the copy
     }
   }
 
@@ -692,16 +702,15 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-    // Every one of the 256 threads passes the barrier, whatever happened
-    // above; then thread (e, r) adds row r of dK (e = 0) or dV (e = 1) into
-    // the zeroed outputs on the bulk-copy engine.
-    fence_proxy_async_smem();
-    named_sync(1, 256);
     if (done) {
-      float* out = (e ? a.dv : a.dk) + (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD;
-      bulk_reduce_add_f32(out, part + (e * kB + r) * kPad, kD * 4);
+      // Thread (e, r) adds the half rows it wrote into the zeroed outputs on
+      // the bulk-copy engine.
+      fence_proxy_async_smem();
+      const size_t off = (((size_t)b * a.S + (size_t)jb * kB + r) * a.Hkv + kvh) * kD + (kD / 2) * e;
+      bulk_reduce_add_f32(a.dk + off, part + r * kPad + (kD / 2) * e, (kD / 2) * 4);
+      bulk_reduce_add_f32(a.dv + off, part + (kB + r) * kPad + (kD / 2) * e, (kD / 2) * 4);
       bulk_commit();
-      bulk_wait_read_all();  // the shared-memory source outlives the copy
+      bulk_wait_read_all();  // the shared-memory source outlives the copies
     }
   }
 

@@ -81,6 +81,9 @@ constexpr size_t fwd_smem_bytes(int d) {
   return 1024 + 2 * (kBM * d * 2) + kStages * (kBM * d * 2) + sizeof(FwdCtl<kGrp>);
 }
 static_assert(fwd_smem_bytes<true>(128) <= 232448, "shared memory budget");
+// The O epilogue stages 2 x 128 rows of 2d + 16 bytes inside the Q tiles and ring slot 0.
+static_assert(2 * kBM * (2 * 128 + 16) <= 3 * kBM * 128 * 2, "O stage fits");
+static_assert(2 * kBM * (2 * 64 + 16) <= 3 * kBM * 64 * 2, "O stage fits");
 
 struct FwdArgs {
   int B, Hq, Hkv, S, nkv, topk, nqb, G;
@@ -435,12 +438,18 @@ __global__ void __launch_bounds__(384, 1)
       const float inv_l = 1.f / l;
       const int p = i * kBM + r;
       const int hq = hq0 + t;
-      __nv_bfloat16* orow = a.o + (((size_t)b * a.S + p) * a.Hq + hq) * kD;
+      // The row goes through shared memory, rows padded to 2d + 16 bytes so
+      // that a warp's 32 rows fall in distinct banks, and out as one bulk copy
+      // (a warp's direct stores would each touch 32 rows).  Head 0 stages in
+      // bytes [0, 128 (2d + 16)) -- the Q tiles, free once S_1 of the last
+      // tile is done, which o_full[0] implies; head 1 in the next 128 rows,
+      // reaching into ring slot 0 only after every MMA has finished.
+      uint8_t* stage = sm + (size_t)(t * kBM + r) * (2 * kD + 16);
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t ov[32];
         HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        uint4* dst = reinterpret_cast<uint4*>(stage + c * 64);
 #pragma unroll
         for (int qd = 0; qd < 4; ++qd) {
           uint4 w;
@@ -451,7 +460,11 @@ __global__ void __launch_bounds__(384, 1)
           dst[qd] = w;
         }
       }
+      fence_proxy_async_smem();
+      bulk_store(a.o + (((size_t)b * a.S + p) * a.Hq + hq) * kD, stage, kD * 2);
+      bulk_commit();
       a.lse[((size_t)b * a.Hq + hq) * a.S + p] = (m_ref + log2f(l)) * 0.6931471805599453f;
+      bulk_wait_read_all();  // the shared-memory source outlives the copy
     }
   }
 

@@ -413,17 +413,19 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
-// Named barrier `id` (1..15) for `nthreads` threads (a multiple of 32).
-__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Adds `bytes` (a multiple of 16) of fp32 from shared memory at `src` into
 // global memory at `dst` (both 16-byte aligned) on the bulk-copy engine, in
 // this thread's current bulk group.
 __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
   asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
                "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+// Copies `bytes` (a multiple of 16) from shared memory at `src` to global
+// memory at `dst` (both 16-byte aligned) on the bulk-copy engine, in this
+// thread's current bulk group.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)), "r"(bytes)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
