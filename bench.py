@@ -399,7 +399,7 @@ def run_e2e(args, ctx, device):
              "scratch": torch.empty(tuple(st.idx.shape), dtype=torch.int32).pin_memory(),
              "results": {"o": st.o, "lse": st.lse, "dq": st.dq, "dk": st.dk, "dv": st.dv}}
         r["out"] = {n: torch.empty(tuple(t.shape), dtype=t.dtype).pin_memory() for n, t in r["results"].items()}
-        r["ev"] = {e: torch.cuda.Event() for e in ("h2d", "comp", "d2h", "fetch")}
+        r["ev"] = {e: torch.cuda.Event() for e in ("q", "h2d", "comp", "d2h", "fetch")}
         r["ev"]["fetch"].record(fetch_stream)  # materialise the handle the C call records into
         sets.append(r)
     blk_bytes = w.blk * w.Hkv * w.d * 2 * 2  # K and V of one block
@@ -409,16 +409,20 @@ def run_e2e(args, ctx, device):
         r = sets[k % 2]
         h2d.wait_event(r["ev"]["comp"])  # step k-2 has consumed this set's inputs
         with torch.cuda.stream(h2d):
-            for n in host:
+            # Q first: the selection and the history fetch it drives need only Q, so they start while
+            # K, V and dO are still on the link
+            r["seg"]["q"].copy_(host["q"], non_blocking=True)
+            r["ev"]["q"].record(h2d)
+            for n in ("k_seg", "v_seg", "d_o"):
                 r["seg"][n].copy_(host[n], non_blocking=True)
         r["ev"]["h2d"].record(h2d)
 
     def select_and_fetch(k):
         # selection needs only this step's queries and the resident summaries, so it (and the history
-        # fetch it drives) runs as soon as the inputs land, while the previous step computes
+        # fetch it drives) runs as soon as Q lands, while the previous step computes
         r = sets[k % 2]
         st, seg = r["st"], r["seg"]
-        sel_stream.wait_event(r["ev"]["h2d"])
+        sel_stream.wait_event(r["ev"]["q"])
         sel_stream.wait_event(r["ev"]["comp"])  # step k-2 has finished with this set's idx and pool
         hga.hga_select_topk(D, seg["q"], st0.summ, st.idx, None, sel_stream)
         nu = hga.hga_fetch_blocks(D, tier_k, tier_v, D.n_hist_blocks, st.idx, r["scratch"], r["pool_k"],
