@@ -10,6 +10,6 @@ from ._binding import (  # noqa: F401
     hga_attn_bwd_workspace_size, hga_attn_fwd, hga_block_summaries, hga_cache_segment, hga_decode_attn,
     hga_decode_select, hga_decode_workspace_size,
     hga_device_status, hga_fetch_blocks, hga_gather_blocks_mapped, hga_fetch_blocks_cached, hga_offload_segment, hga_remap_idx, hga_segment_summaries, hga_select_topk, hga_selftest_attn_fwd_stalled,
-    hga_selftest_umma,
+    hga_selftest_umma, hga_set_forward_heads_per_cta,
     hga_status_string, load_library,
 )

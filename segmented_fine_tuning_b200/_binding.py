@@ -110,6 +110,7 @@ _SIGNATURES = [
     ("hga_cache_segment", _I, [_D, _P, _P, _P, _P, _C, _I, _P]),
     ("hga_remap_idx", _I, [_D, _P, _P, _P, _P]),
     ("hga_attn_uses_tensor_cores", _I, [_D, _I]),
+    ("hga_set_forward_heads_per_cta", _I, [_I]),
     ("hga_append_segment", _I, [_D, _P, _P, _I, _P, _P, _P, _C, _P, _P, _I, _P, _P]),
     ("hga_offload_segment", _I, [_D, _P, _P, _P, _P, _I, _I, _P]),
     ("hga_decode_select", _I, [_D, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -559,6 +560,11 @@ def spaco_sample_blocks(B: int, n_qblocks: int, k: int, generator: torch.Generat
         mask[b, torch.randperm(n_qblocks, generator=generator)[:k]] = 1
     scale = n_qblocks / k
     return mask, (min(scale, cap) if cap is not None else scale)
+
+
+def hga_set_forward_heads_per_cta(heads: int):
+    """Query heads per CTA of the tensor-core forward for later calls: 2, 1, or 0 (automatic)."""
+    _check(load_library().hga_set_forward_heads_per_cta(heads), "hga_set_forward_heads_per_cta")
 
 
 def hga_attn_uses_tensor_cores(dims: Dims, n_kv_blocks: int) -> bool:

@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <chrono>
 #include <memory>
 #include <mutex>
@@ -174,6 +175,18 @@ bool use_tc(const hga::Shape& s, int n_kv_blocks) {
   return hga::tc_supported(s) && (s.blk != 64 || n_kv_blocks < 0x7FFF);
 }
 
+// Query heads per CTA of the tensor-core forward: hga_set_forward_heads_per_cta
+// fixes it; by default a pair, unless the pairs' grid would leave SMs idle.
+std::atomic<int> g_fwd_heads{0};
+
+int fwd_heads_per_cta(const hga::Shape& s) {
+  const int forced = g_fwd_heads.load(std::memory_order_relaxed);
+  if (forced != 0) return forced;
+  int dev = 0, n_sm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  return (long long)s.B * s.Hkv * (s.G() / 2) * s.nqb() < n_sm ? 1 : 2;
+}
+
 hga_status build_maps(const hga::Shape& s, int nkv, const void* q, const void* d_o, const void* ks, const void* vs,
                       const void* kh, const void* vh, hga::TcMaps* m) {
   hga_status r;
@@ -320,7 +333,7 @@ hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, 
   if (use_tc(s, n_kv_blocks)) {
     hga::TcMaps m;
     if ((r = build_maps(s, n_kv_blocks, q, nullptr, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
-    e = hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, st);
+    e = hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, st, fwd_heads_per_cta(s));
   } else {
     e = hga::launch_attn_fwd_simt(s, q, k_seg, v_seg, k_hist, v_hist, n_kv_blocks, idx, o, lse, err, st);
   }
@@ -442,6 +455,12 @@ int hga_attn_uses_tensor_cores(const hga_dims* dims, int n_kv_blocks) {
   hga::Shape s{};
   if (check_dims(dims, &s) != HGA_OK || n_kv_blocks < 0) return -1;
   return use_tc(s, n_kv_blocks) ? 1 : 0;
+}
+
+hga_status hga_set_forward_heads_per_cta(int heads) {
+  if (heads < 0 || heads > 2) return fail(HGA_ERR_INVALID_ARG, "heads per CTA must be 0 (automatic), 1 or 2");
+  g_fwd_heads.store(heads, std::memory_order_relaxed);
+  return HGA_OK;
 }
 
 hga_status hga_attn_bwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
@@ -1066,7 +1085,8 @@ hga_status hga_selftest_attn_fwd_stalled(const hga_dims* dims, const void* q, co
   hga::TcMaps m;
   if ((r = build_maps(s, n_kv_blocks, q, nullptr, k_seg, v_seg, k_hist, v_hist, &m)) != HGA_OK) return r;
   cudaError_t e =
-      hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, reinterpret_cast<cudaStream_t>(stream), true);
+      hga::launch_attn_fwd_tc(s, m, n_kv_blocks, idx, o, lse, err, reinterpret_cast<cudaStream_t>(stream),
+                              fwd_heads_per_cta(s), true);
   return e == cudaSuccess ? HGA_OK : cuda_fail(e, "stalled forward launch");
 }
 

@@ -96,7 +96,7 @@ struct FwdArgs {
   int hblk;         // history block tokens: 128 (one block per tile), 64 (two), 32 or 16 (grouped)
 };
 
-template <int KD, bool kGrp>
+template <int KD, bool kGrp, bool kTwo>
 __global__ void __launch_bounds__(384, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ks,
                   const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_kh,
@@ -111,14 +111,17 @@ __global__ void __launch_bounds__(384, 1)
   FwdCtl<kGrp>* ctl = reinterpret_cast<FwdCtl<kGrp>*>(sRing + kStages * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // kTwo: a CTA serves a pair of query heads; otherwise one head (launches
+  // whose pairs would leave SMs idle), with the head-1 warps and products idle.
+  constexpr int kHeads = kTwo ? 2 : 1;
   // Longest work first: query block i descending with blockIdx.
-  const int npair = a.G >> 1;
-  const int per_i = a.B * a.Hkv * npair;
+  const int nunit = a.G / kHeads;
+  const int per_i = a.B * a.Hkv * nunit;
   const int i = a.nqb - 1 - (int)(blockIdx.x / per_i);
   const int rem = (int)(blockIdx.x % per_i);
-  const int b = rem / (a.Hkv * npair);
-  const int kvh = (rem / npair) % a.Hkv;
-  const int hq0 = kvh * a.G + 2 * (rem % npair);
+  const int b = rem / (a.Hkv * nunit);
+  const int kvh = (rem / nunit) % a.Hkv;
+  const int hq0 = kvh * a.G + kHeads * (rem % nunit);
 
   if (warp == 0) {
     const int32_t* row = a.idx + (((size_t)b * a.Hkv + kvh) * a.nqb + i) * a.topk;
@@ -192,8 +195,8 @@ __global__ void __launch_bounds__(384, 1)
         prefetch_tmap(&tm_vh);
         prefetch_tmap(&tm_ks);
         prefetch_tmap(&tm_vs);
-        mbar_expect_tx(&ctl->q_full, 2 * kTileBytes);
-        for (int t = 0; t < 2; ++t)
+        mbar_expect_tx(&ctl->q_full, kHeads * kTileBytes);
+        for (int t = 0; t < kHeads; ++t)
           for (int hh = 0; hh < kBoxes; ++hh)
             tma_load_4d(&tm_q, &ctl->q_full, sQ + t * kTileBytes + hh * kHalf, hh * 64, hq0 + t, i * kBM, b);
       }
@@ -238,8 +241,8 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(&tm_vh);
       prefetch_tmap(&tm_ks);
       prefetch_tmap(&tm_vs);
-      mbar_expect_tx(&ctl->q_full, 2 * kTileBytes);
-      for (int t = 0; t < 2; ++t)
+      mbar_expect_tx(&ctl->q_full, kHeads * kTileBytes);
+      for (int t = 0; t < kHeads; ++t)
         for (int hh = 0; hh < kBoxes; ++hh)
           tma_load_4d(&tm_q, &ctl->q_full, sQ + t * kTileBytes + hh * kHalf, hh * 64, hq0 + t, i * kBM, b);
       int issued = 0;
@@ -315,8 +318,10 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         issue_S(0, 0);
         umma_commit_w(&ctl->s_full[0]);
-        issue_S(1, 0);
-        umma_commit_w(&ctl->s_full[1]);
+        if (kTwo) {
+          issue_S(1, 0);
+          umma_commit_w(&ctl->s_full[1]);
+        }
         umma_commit_w(&ctl->kv_empty[0]);
         for (int j = 0; j < nt; ++j) {
           const int sV = (2 * j + 1) % kStages;
@@ -334,15 +339,19 @@ __global__ void __launch_bounds__(384, 1)
           } else {
             umma_commit_w(&ctl->o_full[0]);
           }
-          if (!mbar_wait_w(&ctl->p_full[1], j & 1, abort, a.err)) break;
-          tc_fence_after();
-          issue_PV(1, sV, j > 0);
+          if (kTwo) {
+            if (!mbar_wait_w(&ctl->p_full[1], j & 1, abort, a.err)) break;
+            tc_fence_after();
+            issue_PV(1, sV, j > 0);
+          }
           umma_commit_w(&ctl->kv_empty[sV]);
           if (more) {
-            issue_S(1, sK);
-            umma_commit_w(&ctl->s_full[1]);
+            if (kTwo) {
+              issue_S(1, sK);
+              umma_commit_w(&ctl->s_full[1]);
+            }
             umma_commit_w(&ctl->kv_empty[sK]);
-          } else {
+          } else if (kTwo) {
             umma_commit_w(&ctl->o_full[1]);
           }
         }
@@ -352,7 +361,7 @@ __global__ void __launch_bounds__(384, 1)
       volatile int no_abort = 0;
       mbar_wait_w(&ctl->mma_done, 0, &no_abort, a.err);
     }
-  } else if (warp < 8) {
+  } else if (warp < 4 * kHeads) {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;
@@ -485,29 +494,37 @@ bool tc_supported(const Shape& s) {
          s.nqb() <= kMaxQueryBlocks;
 }
 
-template <int KD, bool kGrp>
+template <int KD, bool kGrp, bool kTwo>
 cudaError_t launch_fwd(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse, int* err,
                        cudaStream_t st, bool withhold_kv) {
   constexpr size_t smem = fwd_smem_bytes<kGrp>(KD);
-  cudaError_t e = smem_limit(reinterpret_cast<const void*>(fwd_tc_kernel<KD, kGrp>), smem);
+  cudaError_t e = smem_limit(reinterpret_cast<const void*>(fwd_tc_kernel<KD, kGrp, kTwo>), smem);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.S = s.S; a.nkv = nkv; a.topk = s.topk; a.nqb = s.nqb(); a.G = s.G();
   a.sl2 = 1.4426950408889634f / sqrtf((float)KD);
   a.idx = idx; a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse; a.err = err; a.hblk = s.blk;
   a.withhold_kv = withhold_kv ? 1 : 0;
-  const int grid = s.B * s.Hkv * (s.G() / 2) * s.nqb();
-  fwd_tc_kernel<KD, kGrp><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
+  const int grid = s.B * s.Hkv * (s.G() / (kTwo ? 2 : 1)) * s.nqb();
+  fwd_tc_kernel<KD, kGrp, kTwo><<<grid, 384, smem, st>>>(m.q, m.ks, m.vs, m.kh, m.vh, a);
   return cudaGetLastError();
 }
 
+template <bool kGrp, bool kTwo>
+cudaError_t launch_fwd_d(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse, int* err,
+                         cudaStream_t st, bool withhold_kv) {
+  return s.d == 64 ? launch_fwd<64, kGrp, kTwo>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
+                   : launch_fwd<128, kGrp, kTwo>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
+}
+
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
-                               int* err, cudaStream_t st, bool withhold_kv) {
+                               int* err, cudaStream_t st, int heads_per_cta, bool withhold_kv) {
+  const bool two = heads_per_cta != 1;
   if (s.blk < 64)
-    return s.d == 64 ? launch_fwd<64, true>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
-                     : launch_fwd<128, true>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
-  return s.d == 64 ? launch_fwd<64, false>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
-                   : launch_fwd<128, false>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
+    return two ? launch_fwd_d<true, true>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
+               : launch_fwd_d<true, false>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
+  return two ? launch_fwd_d<false, true>(s, m, nkv, idx, o, lse, err, st, withhold_kv)
+             : launch_fwd_d<false, false>(s, m, nkv, idx, o, lse, err, st, withhold_kv);
 }
 
 }  // namespace hga

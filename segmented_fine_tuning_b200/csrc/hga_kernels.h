@@ -90,8 +90,11 @@ struct TcMaps {
 bool tc_supported(const Shape& s);
 // withhold_kv (self test only): the producer issues no K/V tile loads, so the
 // MMA warp's pipeline wait expires and the CTA takes its timeout path.
+// heads_per_cta: 2 (a CTA serves a pair of query heads sharing its K/V tiles)
+// or 1 (one head per CTA: twice the CTAs, for launches whose pairs would leave
+// SMs idle).
 cudaError_t launch_attn_fwd_tc(const Shape& s, const TcMaps& m, int nkv, const int32_t* idx, void* o, float* lse,
-                               int* err, cudaStream_t st, bool withhold_kv = false);
+                               int* err, cudaStream_t st, int heads_per_cta, bool withhold_kv = false);
 // qmask/gscale (sparse backward): only query blocks i with qmask[b*nqb + i] != 0
 // propagate gradient, and every gradient is multiplied by gscale; nullptr / 1
 // give the plain backward.

@@ -186,6 +186,16 @@ def test_size_limits_rejected_on_host(lib):
     assert "128" in lib.hga_last_error().decode()
 
 
+def test_forward_heads_per_cta_setter(lib):
+    """Host-only knob: 0, 1 and 2 are accepted, anything else is rejected."""
+    for h in (1, 2, 0):
+        assert lib.hga_set_forward_heads_per_cta(h) == 0
+    for h in (-1, 3):
+        assert lib.hga_set_forward_heads_per_cta(h) == 1
+        assert "heads per CTA" in lib.hga_last_error().decode()
+    assert lib.hga_set_forward_heads_per_cta(0) == 0
+
+
 @pytest.mark.parametrize("kw,nkv,want", [
     (dict(), 4, 1),                                        # bf16, d128, block 128
     (dict(d=64), 4, 1),                                    # head dim 64

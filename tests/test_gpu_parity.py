@@ -192,6 +192,28 @@ def test_attention_small(w):
     assert_close("dV", to_host(st.dv), dv_ref, ma, rl)
 
 
+@pytest.mark.parametrize("heads", [1, 2])
+@pytest.mark.parametrize("name", ["tc-K>hist", "tc-d64-B2-G2", "tc-blk64-K4", "tc-blk16-d64-K11", "tc-G6"])
+def test_forward_heads_per_cta(name, heads):
+    """The forward with one query head per CTA and with a pair per CTA (the
+    default picks by grid size), on the same tensor-core cases."""
+    from segmented_fine_tuning_b200 import hga_set_forward_heads_per_cta
+    w = next(c for c in ATTN_CASES if c.name.split(":")[0] == name)
+    x = synth.draw(w)
+    hga_set_forward_heads_per_cta(heads)
+    try:
+        st, _ = _gpu_step(w, x)
+    finally:
+        hga_set_forward_heads_per_cta(0)
+    od = _odims(w)
+    idx = st.idx.cpu().numpy()
+    args = (x.q.f64, x.k_seg.f64, x.v_seg.f64, x.k_hist.f64, x.v_hist.f64, idx)
+    o_ref, lse_ref = oracle.attn_fwd(od, *args)
+    ma, rl = _tols(w)
+    assert_close("O", to_host(st.o), o_ref, ma, rl)
+    assert_close("LSE", to_host(st.lse), lse_ref, ma, rl)
+
+
 def test_rescale_rows_diverge():
     """A history block late in the tile list dominates only the even query
     rows: their running maximum jumps mid-way (the O rescale path) while the
