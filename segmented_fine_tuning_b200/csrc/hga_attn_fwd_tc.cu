@@ -68,6 +68,7 @@ struct FwdCtl {
   uint64_t p_full[2];
   uint64_t o_full[2];
   uint64_t mma_done;
+  uint64_t x_full;  // split form: warpgroup 1's row statistics are in shared memory
   uint32_t tmem;
   int abort;
   int nt;
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(&ctl->o_full[t], 1);
       }
       mbar_init(&ctl->mma_done, 1);
+      mbar_init(&ctl->x_full, 128);
       fence_mbar_init();
     }
     __syncwarp();
@@ -291,8 +293,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);          // Q tiles, K-major
       const uint64_t dK = sdesc_sw128(smem_u32(sRing), 16, 1024);       // ring as K tiles, K-major
       const uint64_t dV = sdesc_sw128(smem_u32(sRing), kHalf, 1024);    // ring as V tiles, MN-major
-      auto issue_S = [=](int t, int s) {
-        const uint64_t a0 = dQ + sdesc_units(t * kTileBytes), b0 = dK + sdesc_units(s * kTileBytes);
+      auto issue_S = [=](int t, int s) {  // split form: both S buffers take the one Q tile
+        const uint64_t a0 = dQ + sdesc_units((kTwo ? t : 0) * kTileBytes), b0 = dK + sdesc_units(s * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = sdesc_units((kk >> 2) * kHalf + (kk & 3) * 32);
@@ -314,14 +316,12 @@ __global__ void __launch_bounds__(384, 1)
         return mbar_wait_w(&ctl->kv_full[pos % kStages], (pos / kStages) & 1, abort, a.err);
       };
       bool ok = mbar_wait_w(&ctl->q_full, 0, abort, a.err) && wait_full(0);
-      if (ok) {
+      if (ok && kTwo) {
         tc_fence_after();
         issue_S(0, 0);
         umma_commit_w(&ctl->s_full[0]);
-        if (kTwo) {
-          issue_S(1, 0);
-          umma_commit_w(&ctl->s_full[1]);
-        }
+        issue_S(1, 0);
+        umma_commit_w(&ctl->s_full[1]);
         umma_commit_w(&ctl->kv_empty[0]);
         for (int j = 0; j < nt; ++j) {
           const int sV = (2 * j + 1) % kStages;
@@ -339,20 +339,68 @@ __global__ void __launch_bounds__(384, 1)
           } else {
             umma_commit_w(&ctl->o_full[0]);
           }
-          if (kTwo) {
-            if (!mbar_wait_w(&ctl->p_full[1], j & 1, abort, a.err)) break;
-            tc_fence_after();
-            issue_PV(1, sV, j > 0);
-          }
+          if (!mbar_wait_w(&ctl->p_full[1], j & 1, abort, a.err)) break;
+          tc_fence_after();
+          issue_PV(1, sV, j > 0);
           umma_commit_w(&ctl->kv_empty[sV]);
           if (more) {
-            if (kTwo) {
-              issue_S(1, sK);
-              umma_commit_w(&ctl->s_full[1]);
-            }
+            issue_S(1, sK);
+            umma_commit_w(&ctl->s_full[1]);
             umma_commit_w(&ctl->kv_empty[sK]);
-          } else if (kTwo) {
+          } else {
             umma_commit_w(&ctl->o_full[1]);
+          }
+        }
+      } else if (ok) {
+        // Split form: warpgroup t takes tiles g = 2j + t of the one head (tile
+        // g's K at ring position 2g, V at 2g + 1); each slot is released after
+        // its one product.  Same order as the pair form: PV_0(j), S_0(j+1),
+        // PV_1(j), S_1(j+1).
+        const int n0 = (nt + 1) / 2, n1 = nt / 2;
+        tc_fence_after();
+        issue_S(0, 0);
+        umma_commit_w(&ctl->s_full[0]);
+        umma_commit_w(&ctl->kv_empty[0]);
+        if (n1 > 0) {
+          if (!wait_full(2)) ok = false;
+          if (ok) {
+            tc_fence_after();
+            issue_S(1, 2 % kStages);
+            umma_commit_w(&ctl->s_full[1]);
+            umma_commit_w(&ctl->kv_empty[2 % kStages]);
+          }
+        }
+        for (int j = 0; ok && j < n0; ++j) {
+          const int g0 = 2 * j, g1 = 2 * j + 1;
+          if (!wait_full(2 * g0 + 1)) break;
+          if (!mbar_wait_w(&ctl->p_full[0], j & 1, abort, a.err)) break;
+          tc_fence_after();
+          issue_PV(0, (2 * g0 + 1) % kStages, j > 0);
+          umma_commit_w(&ctl->kv_empty[(2 * g0 + 1) % kStages]);
+          if (j + 1 < n0) {
+            if (!wait_full(2 * (g0 + 2))) break;
+            tc_fence_after();
+            issue_S(0, (2 * (g0 + 2)) % kStages);
+            umma_commit_w(&ctl->s_full[0]);
+            umma_commit_w(&ctl->kv_empty[(2 * (g0 + 2)) % kStages]);
+          } else {
+            umma_commit_w(&ctl->o_full[0]);
+          }
+          if (j < n1) {
+            if (!wait_full(2 * g1 + 1)) break;
+            if (!mbar_wait_w(&ctl->p_full[1], j & 1, abort, a.err)) break;
+            tc_fence_after();
+            issue_PV(1, (2 * g1 + 1) % kStages, j > 0);
+            umma_commit_w(&ctl->kv_empty[(2 * g1 + 1) % kStages]);
+            if (j + 1 < n1) {
+              if (!wait_full(2 * (g1 + 2))) break;
+              tc_fence_after();
+              issue_S(1, (2 * (g1 + 2)) % kStages);
+              umma_commit_w(&ctl->s_full[1]);
+              umma_commit_w(&ctl->kv_empty[(2 * (g1 + 2)) % kStages]);
+            } else {
+              umma_commit_w(&ctl->o_full[1]);
+            }
           }
         }
       }
@@ -361,7 +409,7 @@ __global__ void __launch_bounds__(384, 1)
       volatile int no_abort = 0;
       mbar_wait_w(&ctl->mma_done, 0, &no_abort, a.err);
     }
-  } else if (warp < 4 * kHeads) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2, wq = warp & 3;
     const int r = wq * 32 + lane;
@@ -372,7 +420,10 @@ __global__ void __launch_bounds__(384, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     uint32_t v[128];
-    for (int j = 0; j < nt; ++j) {
+    // pair form: every tile for head t; split form: tiles g = 2j + t of the one head
+    const int ntt = kTwo ? nt : (nt + 1 - t) / 2;
+    for (int j = 0; j < ntt; ++j) {
+      const int g = kTwo ? j : 2 * j + t;  // the tile's position in the tile list
       // tcgen05.ld/st are warp-collective: every branch around them is
       // decided for the whole warp.
       if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[t], j & 1, abort, a.err))) {
@@ -382,18 +433,18 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       // The whole S row in one pass: 128 columns, one wait.
       tmem_ld128_wait(tS, v);
-      if (j == nt - 1) {
+      if (g == nt - 1) {
         // diagonal segment tile: keys after the query's own position are masked
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (e > r) v[e] = 0xFF800000u;  // -inf
-      } else if (!kGrp && a.hblk == 64 && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) == kNoBlock) {
+      } else if (!kGrp && a.hblk == 64 && ctl->tiles[g] >= 0 && (ctl->tiles[g] >> 16) == kNoBlock) {
         // a history tile holding one 64-token block: its upper 64 keys are masked
 #pragma unroll
         for (int e = 64; e < 128; ++e) v[e] = 0xFF800000u;
-      } else if (kGrp && ctl->tiles[j] >= 0 && (ctl->tiles[j] >> 16) * a.hblk < kBN) {
+      } else if (kGrp && ctl->tiles[g] >= 0 && (ctl->tiles[g] >> 16) * a.hblk < kBN) {
         // a short grouped history tile: the keys after its blocks are masked
-        const int nk = (ctl->tiles[j] >> 16) * a.hblk;
+        const int nk = (ctl->tiles[g] >> 16) * a.hblk;
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (e >= nk) v[e] = 0xFF800000u;
@@ -442,7 +493,63 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(&ctl->p_full[t]);
     }
-    if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->o_full[t], 0, abort, a.err))) {
+    // split form: warpgroup 1's row statistics go to the unused second Q tile
+    float* xs = reinterpret_cast<float*>(sm + 2 * kTileBytes - 1024);
+    if (!kTwo && t == 1) {
+      // Publish this row's (m, l) for warpgroup 0's merge (every thread
+      // arrives once, whatever happened; -inf / 0 when it has nothing).
+      const bool v1 = __all_sync(0xffffffffu, ok && (ntt == 0 || mbar_wait(&ctl->o_full[1], 0, abort, a.err)));
+      xs[r] = v1 && ntt > 0 ? m_ref : -INFINITY;
+      xs[kBM + r] = v1 && ntt > 0 ? l : 0.f;
+      mbar_arrive(&ctl->x_full);
+    } else if (!kTwo) {
+      // Warpgroup 0 merges the two partial states of the head:
+      // O = (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1), a_t = 2^(m_t - max(m_0, m_1)).
+      const bool with1 = nt / 2 > 0;
+      if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->o_full[0], 0, abort, a.err) &&
+                                      (!with1 || mbar_wait(&ctl->o_full[1], 0, abort, a.err)) &&
+                                      mbar_wait(&ctl->x_full, 0, abort, a.err))) {
+        tc_fence_after();
+        const float m1 = xs[r], l1 = xs[kBM + r];
+        const float mm = fmaxf(m_ref, m1);
+        const float a0 = ex2_approx(m_ref - mm), a1 = l1 > 0.f ? ex2_approx(m1 - mm) : 0.f;
+        const float lt = l * a0 + l1 * a1;
+        const float s0 = a0 / lt, s1 = a1 / lt;
+        const int p = i * kBM + r;
+        // staged and written as in the pair form (head 0's rows)
+        uint8_t* stage = sm + (size_t)r * (2 * kD + 16);
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t ov[32], ow[32];
+          HGA_TMEM_LD32_WAIT(tO + c * 32, ov);
+          if (with1) {
+            HGA_TMEM_LD32_WAIT(tO + 128 + c * 32, ow);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ow[e] = 0u;
+          }
+          uint4* dst = reinterpret_cast<uint4*>(stage + c * 64);
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              f[e] = __uint_as_float(ov[8 * qd + e]) * s0 + __uint_as_float(ow[8 * qd + e]) * s1;
+            uint4 w;
+            w.x = pack_bf16x2(f[0], f[1]);
+            w.y = pack_bf16x2(f[2], f[3]);
+            w.z = pack_bf16x2(f[4], f[5]);
+            w.w = pack_bf16x2(f[6], f[7]);
+            dst[qd] = w;
+          }
+        }
+        fence_proxy_async_smem();
+        bulk_store(a.o + (((size_t)b * a.S + p) * a.Hq + hq0) * kD, stage, kD * 2);
+        bulk_commit();
+        a.lse[((size_t)b * a.Hq + hq0) * a.S + p] = (mm + log2f(lt)) * 0.6931471805599453f;
+        bulk_wait_read_all();  // the shared-memory source outlives the copy
+      }
+    } else if (__all_sync(0xffffffffu, ok && mbar_wait(&ctl->o_full[t], 0, abort, a.err))) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const int p = i * kBM + r;
