@@ -19,9 +19,13 @@
 // state (running max m, sum l, unnormalised O) to the caller's workspace.  A
 // second kernel merges the chunks of every row: M = max m_c, L = sum l_c
 // 2^(m_c - M), O = sum O_c 2^(m_c - M) / L, LSE = (M + log2 L) ln 2.
+// For bf16 with at most 8 rows per KV head a streaming form of the chunk
+// kernel (decode_stream_kernel, below) takes the chunks instead.
 // The work is bound by HBM: the selected K/V blocks and the segment prefix
 // are read once.
 #include <float.h>
+
+#include <type_traits>
 
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
@@ -309,6 +313,208 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecArgs a, T*
   if (tid == 0) lse[((size_t)b * a.Hq + hq) * a.nq + u] = (M + log2f(L)) * 0.6931471805599453f;
 }
 
+// Streaming form of the chunk kernel for bf16 and at most kR (4 or 8) query
+// rows per KV head, the usual decode shape (G x n_q rows): one CTA of 8 warps
+// per (chunk, batch x KV head).  Half-warp w (0..15) takes keys w, w+16, ...
+// of the chunk; its 16 lanes split the head dimension (lane l holds channels
+// [l*D/16, (l+1)*D/16)).  K comes straight from global memory into registers
+// (all of a lane's pieces in flight at once) and meets the query rows held in
+// registers; a row's score is reduced over the 16 lanes by shuffles.  V is
+// staged in shared memory by cp.async from the start, so it lands while the
+// scores are formed.  After the chunk's softmax each half-warp accumulates
+// P V over its keys and the 16 half-warp partials are summed in shared
+// memory.  The chunk's (m, l, O) go to the same workspace as the general
+// kernel's, for the same merge.
+constexpr int kStreamThreads = 256;
+constexpr int kStreamKeysPerLane = 8;  // keys of a 128-key chunk per half-warp
+
+template <int KD, int kR>
+size_t stream_smem_bytes(int blk) {
+  return (size_t)blk * KD * 2 + (size_t)kR * blk * 4 + 2 * kR * 4 + (size_t)8 * kR * KD * 4;
+}
+
+template <int KD, int kR>
+__global__ void __launch_bounds__(kStreamThreads) decode_stream_kernel(const __nv_bfloat16* __restrict__ q_new,
+                                                                       const __nv_bfloat16* __restrict__ k_seg,
+                                                                       const __nv_bfloat16* __restrict__ v_seg,
+                                                                       const __nv_bfloat16* __restrict__ k_hist,
+                                                                       const __nv_bfloat16* __restrict__ v_hist,
+                                                                       const DecArgs a) {
+  constexpr int EL = KD / 16;  // channels per lane: 8 (16 bytes) or 4 (8 bytes)
+  extern __shared__ __align__(16) uint8_t dec_smem[];
+  const int blk = a.blk;
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(dec_smem);            // [blk][KD]
+  float* sS = reinterpret_cast<float*>(dec_smem + (size_t)blk * KD * 2);      // [kR][blk]
+  float* sM = sS + kR * blk;
+  float* sL = sM + kR;
+  float* sRed = sL + kR;                                                      // [8][kR][KD]
+
+  // KV head fastest in the grid: the Hkv CTAs of a chunk read its tokens'
+  // rows (all heads side by side in memory) together
+  const int c = blockIdx.y;
+  const int b = blockIdx.x / a.Hkv, h = blockIdx.x % a.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hw = warp * 2 + (lane >> 4), hl = lane & 15;
+  const int R = a.R;
+
+  const bool hist = c < a.topk;
+  const __nv_bfloat16* kb;
+  const __nv_bfloat16* vb;
+  int nk, pos0 = 0;
+  if (hist) {
+    int n = __ldg(a.idx + ((size_t)b * a.Hkv + h) * a.topk + c);
+    if (n < -1 || n >= a.nkv) {
+      if (tid == 0) flag_error(a.err, kDevErrIndex);
+      n = -1;
+    }
+    nk = n >= 0 ? blk : 0;
+    const size_t off = (((size_t)b * a.nkv * blk + (size_t)(n >= 0 ? n : 0) * blk) * a.Hkv + h) * KD;
+    kb = k_hist + off;
+    vb = v_hist + off;
+  } else {
+    pos0 = (c - a.topk) * blk;
+    nk = min(blk, a.t0 + a.nq - pos0);
+    const size_t off = (((size_t)b * a.S + pos0) * a.Hkv + h) * KD;
+    kb = k_seg + off;
+    vb = v_seg + off;
+  }
+  const size_t key_stride = (size_t)a.Hkv * KD;
+
+  // 1. V into shared memory (16-byte cp.async), K pieces into registers
+  for (int x = tid; x < nk * (KD / 8); x += kStreamThreads) {
+    const int j = x / (KD / 8), v = x % (KD / 8);
+    cp_async16(sV + (size_t)j * KD + v * 8, vb + j * key_stride + v * 8);
+  }
+  cp_async_commit();
+  using Piece = typename std::conditional<EL == 8, uint4, uint2>::type;
+  Piece kp[kStreamKeysPerLane];
+#pragma unroll
+  for (int kk = 0; kk < kStreamKeysPerLane; ++kk) {
+    const int j = hw + 16 * kk;
+    if (j < nk) kp[kk] = __ldg(reinterpret_cast<const Piece*>(kb + j * key_stride + hl * EL));
+    else kp[kk] = Piece{};
+  }
+  // this lane's channels of the query rows, in log2 units (rows >= R are zero)
+  float q[kR][EL];
+#pragma unroll
+  for (int r = 0; r < kR; ++r) {
+    const int g = r / a.nq, u = r % a.nq;
+    const __nv_bfloat16* src = q_new + (((size_t)b * a.nq + u) * a.Hq + h * a.G + g) * KD + hl * EL;
+#pragma unroll
+    for (int e = 0; e < EL; ++e) q[r][e] = r < R ? __bfloat162float(src[e]) * a.sl2 : 0.f;
+  }
+
+  // 2. scores: a half-warp per key, reduced over its 16 lanes
+#pragma unroll
+  for (int kk = 0; kk < kStreamKeysPerLane; ++kk) {
+    const int j = hw + 16 * kk;
+    float kv[EL];
+    if constexpr (EL == 8) {
+      DecElem<__nv_bfloat16>::unpack(kp[kk], kv);
+    } else {
+      const uint2 w = kp[kk];
+      kv[0] = __uint_as_float(w.x << 16); kv[1] = __uint_as_float(w.x & 0xFFFF0000u);
+      kv[2] = __uint_as_float(w.y << 16); kv[3] = __uint_as_float(w.y & 0xFFFF0000u);
+    }
+    float sc[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < EL; ++e) acc = fmaf(q[r][e], kv[e], acc);
+      sc[r] = acc;
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+      for (int r = 0; r < kR; ++r) sc[r] += __shfl_xor_sync(0xffffffffu, sc[r], o);
+    if (hl == 0 && j < blk) {
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
+        if (r < R) {
+          const int u = r % a.nq;
+          const bool visible = j < nk && (hist || pos0 + j <= a.t0 + u);
+          sS[r * blk + j] = visible ? sc[r] : -INFINITY;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. per row: max, probabilities 2^(s - m), sum (one warp per row)
+  for (int r = warp; r < R; r += kStreamThreads / 32) {
+    float m = -INFINITY;
+    for (int j = lane; j < blk; j += 32) m = fmaxf(m, sS[r * blk + j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int j = lane; j < blk; j += 32) {
+      const float p = (m == -INFINITY) ? 0.f : ex2_approx(sS[r * blk + j] - m);
+      sS[r * blk + j] = p;
+      l += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      sM[r] = m;
+      sL[r] = l;
+    }
+  }
+  cp_async_wait_group<0>();  // this thread's V copies have landed
+  __syncthreads();
+
+  // 4. P V over the half-warp's keys, then the two half-warps of a warp by a
+  //    shuffle and the 8 warps in shared memory
+  float o[kR][EL];
+#pragma unroll
+  for (int r = 0; r < kR; ++r)
+#pragma unroll
+    for (int e = 0; e < EL; ++e) o[r][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < kStreamKeysPerLane; ++kk) {
+    const int j = hw + 16 * kk;
+    if (j < nk) {
+      float vv[EL];
+      const Piece w = *reinterpret_cast<const Piece*>(sV + (size_t)j * KD + hl * EL);
+      if constexpr (EL == 8) {
+        DecElem<__nv_bfloat16>::unpack(w, vv);
+      } else {
+        vv[0] = __uint_as_float(w.x << 16); vv[1] = __uint_as_float(w.x & 0xFFFF0000u);
+        vv[2] = __uint_as_float(w.y << 16); vv[3] = __uint_as_float(w.y & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
+        const float pr = r < R ? sS[r * blk + j] : 0.f;  // the same address in all 16 lanes
+#pragma unroll
+        for (int e = 0; e < EL; ++e) o[r][e] = fmaf(pr, vv[e], o[r][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kR; ++r)
+#pragma unroll
+    for (int e = 0; e < EL; ++e) o[r][e] += __shfl_xor_sync(0xffffffffu, o[r][e], 16);
+  if (lane < 16) {
+#pragma unroll
+    for (int r = 0; r < kR; ++r)
+#pragma unroll
+      for (int e = 0; e < EL; ++e) sRed[((size_t)warp * kR + r) * KD + hl * EL + e] = o[r][e];
+  }
+  __syncthreads();
+  const size_t base = (((size_t)b * a.Hkv + h) * a.n_chunks + c) * a.R;
+  for (int x = tid; x < R * KD; x += kStreamThreads) {
+    const int r = x / KD, col = x % KD;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += sRed[((size_t)w * kR + r) * KD + col];
+    a.part_o[(base + r) * KD + col] = sum;
+  }
+  if (tid < R) {
+    a.part_ml[(base + tid) * 2] = sM[tid];
+    a.part_ml[(base + tid) * 2 + 1] = sL[tid];
+  }
+}
+
 }  // namespace
 
 size_t decode_workspace_floats(const Shape& s, int nq) {
@@ -331,7 +537,33 @@ cudaError_t launch_decode_attn(const Shape& s, int nq, int t0, const void* q_new
   a.part_o = ws + (size_t)s.B * s.Hkv * a.n_chunks * a.R * 2;
   const dim3 grid(a.n_chunks, (a.R + kDecRows - 1) / kDecRows, s.B * s.Hkv);
   cudaError_t e;
-  if (s.bf16) {
+  if (s.bf16 && a.R <= 8 && (s.d == 128 || s.d == 64) && s.blk <= 16 * kStreamKeysPerLane) {
+    // the usual decode shape: the streaming chunk kernel
+    const dim3 sgrid(s.B * s.Hkv, a.n_chunks);
+    const bool r4 = a.R <= 4;
+    const void* fn = s.d == 128 ? (r4 ? reinterpret_cast<const void*>(decode_stream_kernel<128, 4>)
+                                      : reinterpret_cast<const void*>(decode_stream_kernel<128, 8>))
+                                : (r4 ? reinterpret_cast<const void*>(decode_stream_kernel<64, 4>)
+                                      : reinterpret_cast<const void*>(decode_stream_kernel<64, 8>));
+    const size_t smem = s.d == 128 ? (r4 ? stream_smem_bytes<128, 4>(s.blk) : stream_smem_bytes<128, 8>(s.blk))
+                                   : (r4 ? stream_smem_bytes<64, 4>(s.blk) : stream_smem_bytes<64, 8>(s.blk));
+    if ((e = smem_limit(fn, smem)) != cudaSuccess) return e;
+    const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(q_new);
+    const __nv_bfloat16* ks = static_cast<const __nv_bfloat16*>(k_seg);
+    const __nv_bfloat16* vs = static_cast<const __nv_bfloat16*>(v_seg);
+    const __nv_bfloat16* kh = static_cast<const __nv_bfloat16*>(k_hist);
+    const __nv_bfloat16* vh = static_cast<const __nv_bfloat16*>(v_hist);
+    if (s.d == 128 && r4)
+      decode_stream_kernel<128, 4><<<sgrid, kStreamThreads, smem, st>>>(qn, ks, vs, kh, vh, a);
+    else if (s.d == 128)
+      decode_stream_kernel<128, 8><<<sgrid, kStreamThreads, smem, st>>>(qn, ks, vs, kh, vh, a);
+    else if (r4)
+      decode_stream_kernel<64, 4><<<sgrid, kStreamThreads, smem, st>>>(qn, ks, vs, kh, vh, a);
+    else
+      decode_stream_kernel<64, 8><<<sgrid, kStreamThreads, smem, st>>>(qn, ks, vs, kh, vh, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    decode_combine_kernel<__nv_bfloat16><<<s.B * s.Hkv * a.R, 128, 0, st>>>(a, static_cast<__nv_bfloat16*>(o), lse);
+  } else if (s.bf16) {
     const size_t smem = dec_smem_bytes<__nv_bfloat16>(s.blk, s.d);
     auto kp = decode_partial_kernel<__nv_bfloat16>;
     if ((e = smem_limit(reinterpret_cast<const void*>(kp), smem)) != cudaSuccess)

@@ -36,6 +36,12 @@ CASES = [
     (synth.Workload("dec-K>hist: hist2 K5", 1, 8, 2, 128, 128, 256, 2, 5, "bf16", 94), 1, 200),
     (synth.Workload("dec-f32-d64-blk64: Hq2/Hkv1 S256 hist16 K4", 1, 2, 1, 64, 64, 256, 16, 4, "f32", 95), 3, 100),
     (synth.Workload("dec-bf16-d64-blk32-G3", 1, 6, 2, 64, 32, 128, 7, 2, "bf16", 96), 4, 60),
+    # up to 8 rows per KV head (G x n_q) in bf16 take the streaming chunk kernel
+    (synth.Workload("dec-stream-d64-blk32: B2 Hq4/Hkv2 d64 S128 hist7 K3", 2, 4, 2, 64, 32, 128, 7, 3, "bf16", 97),
+     2, 60),
+    (synth.Workload("dec-stream-G8: Hq16/Hkv2 S256 hist6 K3", 1, 16, 2, 128, 128, 256, 6, 3, "bf16", 98), 1, 130),
+    (W_SMALL, 2, 126),       # 8 rows, the two tokens straddle the block boundary at 128
+    (synth.Workload("dec-stream-blk16: Hq8/Hkv2 S128 hist20 K6", 1, 8, 2, 128, 16, 128, 20, 6, "bf16", 99), 1, 90),
 ]
 
 
