@@ -1,5 +1,6 @@
 // Tensor-core (tcgen05) forward of the HGA attention step, bf16 in, fp32
-// accumulate, for d in {64, 128} and 128-token blocks.
+// accumulate, for d in {64, 128}, 128-row query blocks and history blocks of
+// 128, 64, 32 or 16 tokens.
 //
 // Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention
 // and Segmented Backpropagation in Practice", Background: each query block
@@ -10,13 +11,17 @@
 // heads of h.  Both heads share the KV head and the query block, hence the
 // same tile list: the K_eff selected history blocks followed by segment blocks
 // 0..i (the last one, the diagonal, is causally masked).  Every K/V tile that
-// TMA brings into shared memory feeds two 128x128x128 products.
+// TMA brings into shared memory feeds two 128x128x128 products.  Launches
+// whose pairs would leave SMs idle use the split form instead: one head per
+// CTA, its tiles alternating between the two softmax warpgroups (t takes
+// tiles 2j + t), which merge their partial states at the end.
 //
 // Roles (384 threads, 1 CTA per SM):
-//   warps 0-3   softmax for head 0 of the pair (one query row per thread)
-//   warps 4-7   softmax for head 1
+//   warps 0-3   softmax for head 0 of the pair (split form: the even tiles),
+//               one query row per thread
+//   warps 4-7   softmax for head 1 (split form: the odd tiles)
 //   warp  8     TMA producer: Q tiles once, then K_j, V_j into a 5-slot ring
-//   warp  9     MMA issuer (one thread): S_t = Q_t K_j^T, O_t += P_t V_j
+//   warp  9     MMA issuer (one elected lane): S_t = Q_t K_j^T, O_t += P_t V_j
 // Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns each, fp32.
 // The softmax writes P (bf16) back into the S columns it has just read, and
 // the PV product takes P straight from tensor memory.
