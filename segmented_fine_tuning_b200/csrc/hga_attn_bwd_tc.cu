@@ -1,5 +1,6 @@
 // Tensor-core (tcgen05) backward of the HGA attention step for the active
-// segment, bf16 in, fp32 accumulate, d in {64, 128}, 128-token blocks.
+// segment, bf16 in, fp32 accumulate, d in {64, 128}, 128-row query blocks
+// over history blocks of 128, 64, 32 or 16 tokens.
 //
 // Article: "Low-VRAM Long-Context Fine-Tuning: Hierarchical Global Attention
 // and Segmented Backpropagation in Practice", Background and (fr edition)
@@ -19,7 +20,8 @@
 // warpgroups, 64 key columns each) is written as bf16 over the S columns it
 // came from; dQ += dS K takes dS from tensor memory.  S runs two tiles ahead;
 // dP's buffer is released as soon as the dS pass has loaded it, so dP(j+1)
-// overlaps the dS math of tile j.
+// overlaps the dS math of tile j.  Each thread's dQ half row leaves through
+// shared memory as one bulk copy.
 //
 // Kernel 2 works in 64-query sub-tiles so that tensor memory holds two
 // sub-tiles of S^T and dP^T at once: while the CUDA cores turn sub-tile u into
@@ -31,8 +33,9 @@
 // halves, with the transposed products (keys in tensor-memory lanes):
 // S^T = K Q^T, dP^T = V dO^T (M 128 keys, N 64 queries), P^T and dS^T in
 // place as bf16, dV += P^T dO and dK += dS^T Q (K = 64 queries) accumulated
-// in tensor memory.  Each CTA adds its head's partial dK/dV to the fp32
-// outputs with vector reductions (red.global.add.v4.f32).
+// in tensor memory.  Each CTA adds its head's partial dK/dV to the zeroed fp32
+// outputs: the rows go through shared memory and each thread adds its half
+// rows with bulk reduce-adds (cp.reduce.async.bulk .add.f32).
 #include "hga_kernels.h"
 #include "hga_ptx.cuh"
 

@@ -406,13 +406,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Fire-and-forget vector float add to global memory (no value returned, so
-// consecutive reductions from one thread do not wait on each other).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 // Adds `bytes` (a multiple of 16) of fp32 from shared memory at `src` into
 // global memory at `dst` (both 16-byte aligned) on the bulk-copy engine, in
 // this thread's current bulk group.
