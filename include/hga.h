@@ -189,12 +189,14 @@ HGA_API hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void*
  * Host-only; no device work. */
 HGA_API int hga_attn_uses_tensor_cores(const hga_dims* dims, int n_kv_blocks);
 
-/* Query heads per CTA of the tensor-core forward, for every later call in the
- * process: 2 (a CTA serves a pair of query heads of one KV head, sharing each
- * K/V tile), 1 (one head per CTA: twice the CTAs), or 0 (the default: a pair,
- * unless B * Hkv * (G/2) * Nqb is below the device's SM count, then one).  The
- * results are the same either way; this is a throughput knob.  Host-only, no
- * device work; HGA_ERR_INVALID_ARG for other values. */
+/* Query heads per CTA of the tensor-core forward, for later calls from the
+ * calling thread (a per-thread setting, like hga_last_error): 2 (a CTA serves
+ * a pair of query heads of one KV head, sharing each K/V tile), 1 (one head
+ * per CTA, its tiles split over the CTA's two softmax warpgroups: twice the
+ * CTAs), or 0 (the default: a pair, unless B * Hkv * (G/2) * Nqb is below the
+ * device's SM count, then one).  The results are the same either way; this is
+ * a throughput knob.  Host-only, no device work; HGA_ERR_INVALID_ARG for other
+ * values. */
 HGA_API hga_status hga_set_forward_heads_per_cta(int heads);
 
 /* Bytes of device scratch hga_attn_bwd needs for these dims (256-byte

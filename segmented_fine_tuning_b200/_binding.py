@@ -563,7 +563,7 @@ def spaco_sample_blocks(B: int, n_qblocks: int, k: int, generator: torch.Generat
 
 
 def hga_set_forward_heads_per_cta(heads: int):
-    """Query heads per CTA of the tensor-core forward for later calls: 2, 1, or 0 (automatic)."""
+    """Query heads per CTA of the tensor-core forward for later calls from this thread: 2, 1, or 0 (automatic)."""
     _check(load_library().hga_set_forward_heads_per_cta(heads), "hga_set_forward_heads_per_cta")
 
 

@@ -9,7 +9,6 @@
 #include <string.h>
 
 #include <algorithm>
-#include <atomic>
 #include <chrono>
 #include <memory>
 #include <mutex>
@@ -176,11 +175,12 @@ bool use_tc(const hga::Shape& s, int n_kv_blocks) {
 }
 
 // Query heads per CTA of the tensor-core forward: hga_set_forward_heads_per_cta
-// fixes it; by default a pair, unless the pairs' grid would leave SMs idle.
-std::atomic<int> g_fwd_heads{0};
+// fixes it for the calling thread (like hga_last_error, per thread); by
+// default a pair, unless the pairs' grid would leave SMs idle.
+thread_local int g_fwd_heads = 0;
 
 int fwd_heads_per_cta(const hga::Shape& s) {
-  const int forced = g_fwd_heads.load(std::memory_order_relaxed);
+  const int forced = g_fwd_heads;
   if (forced != 0) return forced;
   int dev = 0, n_sm = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
@@ -459,7 +459,7 @@ int hga_attn_uses_tensor_cores(const hga_dims* dims, int n_kv_blocks) {
 
 hga_status hga_set_forward_heads_per_cta(int heads) {
   if (heads < 0 || heads > 2) return fail(HGA_ERR_INVALID_ARG, "heads per CTA must be 0 (automatic), 1 or 2");
-  g_fwd_heads.store(heads, std::memory_order_relaxed);
+  g_fwd_heads = heads;
   return HGA_OK;
 }
 
