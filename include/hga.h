@@ -172,9 +172,11 @@ HGA_API hga_status hga_select_topk(const hga_dims* dims, const void* q_seg, cons
  *   s_j = q.k_j / sqrt(d);  O = sum_j softmax(s)_j v_j;  lse = log sum_j exp(s_j)
  * k_hist/v_hist hold n_kv_blocks blocks: the history itself (n_kv_blocks =
  * n_hist_blocks) or a staging pool filled by hga_fetch_blocks (idx then holds
- * pool slots).  o has the input dtype; lse fp32.
- * Errors: HGA_ERR_INVALID_ARG, HGA_ERR_SHAPE (host checks); an idx entry
- * outside [-1, n_kv_blocks) is skipped and flags HGA_ERR_INDEX on the device.
+ * pool slots).  o has the input dtype; lse fp32.  q, k_seg, v_seg, k_hist,
+ * v_hist and o must start on a 16-byte boundary.
+ * Errors: HGA_ERR_INVALID_ARG (null or misaligned pointers), HGA_ERR_SHAPE
+ * (host checks); an idx entry outside [-1, n_kv_blocks) is skipped and flags
+ * HGA_ERR_INDEX on the device.
  */
 HGA_API hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, const void* v_seg,
                         const void* k_hist, const void* v_hist, int n_kv_blocks, const int32_t* idx, void* o,

@@ -326,6 +326,7 @@ hga_status hga_attn_fwd(const hga_dims* dims, const void* q, const void* k_seg, 
   if (r != HGA_OK) return r;
   if ((r = check_attn_ptrs(s, n_kv_blocks, q, k_seg, v_seg, k_hist, v_hist, idx)) != HGA_OK) return r;
   if (any_null(o, lse)) return fail(HGA_ERR_INVALID_ARG, "NULL output pointer");
+  if (!aligned16(o)) return fail(HGA_ERR_INVALID_ARG, "o must be 16-byte aligned");
   int* err = nullptr;
   if ((r = device_err_ptr(&err)) != HGA_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -83,6 +83,8 @@ def test_null_and_invalid_arguments(lib):
     assert lib.hga_attn_fwd(ctypes.byref(d), None, p, p, p, p, 4, p, p, p, None) == 1
     assert lib.hga_attn_fwd(ctypes.byref(d), p, p, p, None, p, 4, p, p, p, None) == 1   # history missing
     assert lib.hga_attn_fwd(ctypes.byref(d), ctypes.c_void_p(18), p, p, p, p, 4, p, p, p, None) == 1  # misaligned
+    assert lib.hga_attn_fwd(ctypes.byref(d), p, p, p, p, p, 4, p, ctypes.c_void_p(24), p, None) == 1  # o misaligned
+    assert "o must be 16-byte aligned" in lib.hga_last_error().decode()
     assert lib.hga_block_summaries(ctypes.byref(d), p, 0, 9, p, None) == 1   # range past n_hist_blocks
     assert lib.hga_block_summaries(ctypes.byref(d), p, 3, 1, p, None) == 1
     assert lib.hga_select_topk(ctypes.byref(_dims(n_hist_blocks=5000)), p, p, p, None, None) == 2
